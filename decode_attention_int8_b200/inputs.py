@@ -1,0 +1,238 @@
+"""Seeded synthetic workloads for q8-KV decode attention.
+
+This module only draws random inputs and lays them out; it holds none of the attention
+arithmetic. Both the CUDA path and the CPU oracle consume what it returns.
+
+Recipe (the five named workloads below, plus ``make_custom`` for test grids):
+  - q: fp32, iid N(0, 1), shape [B][n_q_heads][head_dim].
+  - K, V: fp32 drawn iid per element (N(0, 1), or Student-t with 3 degrees of freedom),
+    K optionally plus a per-(KV head, channel) bias held constant over tokens, then
+    quantised per (token, KV head) row: scale = max|x| / 127 (fp32), code =
+    clamp(round-half-even(x / scale), -127, 127); an all-zero row gets scale 1/127 and
+    codes 0. The pools are int8 [num_blocks][block_size][n_kv_heads][head_dim] with fp32
+    scales [num_blocks][block_size][n_kv_heads].
+  - block_table: int32 [B][max_blocks_per_seq]; sequence b owns ceil(L_b / block_size)
+    physical blocks, assigned in order ("identity") or from a random permutation of the
+    pool ("permutation"); unused entries are -1.
+  - softmax scale 1 / sqrt(head_dim) rounded to fp32.
+Random numbers come from numpy PCG64 streams keyed by (seed, stream, chunk), so a
+workload is identical whatever the thread count.
+"""
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field, replace
+
+import numpy as np
+
+# Stream identifiers of the PCG64 seed sequences.
+_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS = range(6)
+_CHUNK_SLOTS = 4096  # pool slots generated per independent random stream
+
+
+@dataclass(frozen=True)
+class Config:
+    name: str
+    B: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    seq_len: int | tuple  # fixed length, or ("uniform", lo, hi) inclusive
+    block_size: int
+    table: str  # "identity" | "permutation"
+    k_dist: str = "normal"  # "normal" | "student_t3"
+    v_dist: str = "normal"
+    k_bias_std: float = 0.0
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def group(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    @property
+    def max_seq_len(self) -> int:
+        return self.seq_len if isinstance(self.seq_len, int) else int(self.seq_len[2])
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return -(-self.max_seq_len // self.block_size)
+
+
+# The five workloads: shapes and distributions of long-context GQA decode over paged
+# int8 caches (head_dim 128, contexts 256 to 128K).
+CONFIGS = [
+    Config("tiny_mha", 1, 8, 8, 128, 256, 16, "identity", seed=0,
+           description="B=1, 8/8 heads, L=256, block 16, identity table"),
+    Config("gqa_batch", 16, 32, 8, 128, 4096, 64, "permutation", seed=1,
+           description="B=16, 32/8 heads, L=4096, block 64, permuted 1024-block pool"),
+    Config("long_context", 1, 32, 4, 128, 131072, 128, "permutation", k_bias_std=2.0, seed=2,
+           description="B=1, 32/4 heads, L=131072, block 128, K + per-channel N(0, 2^2) bias"),
+    Config("ragged_outliers", 64, 64, 8, 128, ("uniform", 1, 32768), 128, "permutation",
+           k_dist="student_t3", v_dist="student_t3", seed=3,
+           description="B=64, 64/8 heads, L~U[1,32768], block 128, Student-t(3) K/V"),
+    Config("bandwidth", 256, 32, 8, 128, 8192, 64, "permutation", seed=4,
+           description="B=256, 32/8 heads, L=8192, block 64, 32768-block pool"),
+]
+
+
+@dataclass
+class Workload:
+    cfg: Config
+    q: np.ndarray  # fp32 [B][Hq][D]
+    k: np.ndarray  # int8 [P][bs][Hk][D]
+    v: np.ndarray
+    ks: np.ndarray  # fp32 [P][bs][Hk]
+    vs: np.ndarray
+    block_table: np.ndarray  # int32 [B][max_blocks_per_seq]
+    seq_lens: np.ndarray  # int32 [B]
+    scale: float  # fp32 value
+    k32: np.ndarray | None = field(default=None, repr=False)
+    v32: np.ndarray | None = field(default=None, repr=False)
+
+    @property
+    def num_blocks(self) -> int:
+        return int(self.k.shape[0])
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_table.shape[1])
+
+    def algorithmic_bytes(self) -> int:
+        """Bytes one call must move: every valid (token, KV head) K row, V row and both
+        scales once, q read and out written (fp32), the used block-table entries and
+        seq_lens."""
+        c = self.cfg
+        L = self.seq_lens.astype(np.int64)
+        units = int(L.sum()) * c.n_kv_heads
+        nblk = int(((L + c.block_size - 1) // c.block_size).sum())
+        return (units * (2 * c.head_dim + 8) + c.B * c.n_q_heads * c.head_dim * 4 * 2
+                + 4 * nblk + 4 * c.B)
+
+
+def _rng(seed: int, stream: int, chunk: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, stream, chunk])))
+
+
+def _draw(rng: np.random.Generator, dist: str, shape) -> np.ndarray:
+    if dist == "normal":
+        return rng.standard_normal(shape, dtype=np.float32)
+    if dist == "student_t3":
+        return rng.standard_t(3.0, shape).astype(np.float32)
+    raise ValueError(f"unknown distribution {dist!r}")
+
+
+def quantize_rows(x: np.ndarray):
+    """Per-row int8 quantisation of the input data (the cache-writer's recipe):
+    scale = max|x| / 127, code = clamp(rne(x / scale), -127, 127); zero rows get
+    scale 1/127 and codes 0. All arithmetic in fp32."""
+    x = np.asarray(x, np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    zero = amax == 0
+    scale = np.where(zero, np.float32(1.0) / np.float32(127.0), amax / np.float32(127.0))
+    scale = scale.astype(np.float32)
+    codes = np.rint(x / scale[..., None])
+    codes = np.clip(codes, -127, 127).astype(np.int8)
+    codes[zero] = 0
+    return codes, scale
+
+
+def _fill_pool(seed, stream, dist, P, bs, Hk, D, bias, keep_fp32, threads):
+    """Generate one int8 pool and its scales chunk by chunk (deterministic per chunk)."""
+    slots = P * bs
+    codes = np.empty((slots, Hk, D), np.int8)
+    scales = np.empty((slots, Hk), np.float32)
+    raw = np.empty((slots, Hk, D), np.float32) if keep_fp32 else None
+    n_chunks = -(-slots // _CHUNK_SLOTS)
+
+    def work(i):
+        lo, hi = i * _CHUNK_SLOTS, min(slots, (i + 1) * _CHUNK_SLOTS)
+        x = _draw(_rng(seed, stream, i), dist, (hi - lo, Hk, D))
+        if bias is not None:
+            x += bias[None, :, :]
+        c, s = quantize_rows(x)
+        codes[lo:hi] = c
+        scales[lo:hi] = s
+        if raw is not None:
+            raw[lo:hi] = x
+
+    if threads > 1 and n_chunks > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(work, range(n_chunks)))
+    else:
+        for i in range(n_chunks):
+            work(i)
+    shape = (P, bs, Hk, D)
+    return (codes.reshape(shape), scales.reshape(P, bs, Hk),
+            None if raw is None else raw.reshape(shape))
+
+
+def _seq_lens(cfg: Config) -> np.ndarray:
+    if isinstance(cfg.seq_len, int):
+        return np.full(cfg.B, cfg.seq_len, np.int32)
+    kind, lo, hi = cfg.seq_len
+    if kind != "uniform":
+        raise ValueError(kind)
+    return _rng(cfg.seed, _S_LENS).integers(lo, hi + 1, size=cfg.B).astype(np.int32)
+
+
+def build_block_table(seq_lens, block_size, max_blocks_per_seq, table, num_blocks, rng):
+    """Assign ceil(L_b / block_size) distinct physical blocks to every sequence."""
+    need = (np.asarray(seq_lens, np.int64) + block_size - 1) // block_size
+    total = int(need.sum())
+    if total > num_blocks:
+        raise ValueError("pool too small")
+    if table == "identity":
+        order = np.arange(num_blocks, dtype=np.int64)
+    elif table == "permutation":
+        order = rng.permutation(num_blocks)
+    else:
+        raise ValueError(f"unknown table kind {table!r}")
+    bt = np.full((len(seq_lens), max_blocks_per_seq), -1, np.int32)
+    off = 0
+    for b, n in enumerate(need):
+        bt[b, :n] = order[off:off + n]
+        off += n
+    return bt
+
+
+def make_custom(B, n_q_heads, n_kv_heads, head_dim, seq_lens, block_size, *, table="permutation",
+                k_dist="normal", v_dist="normal", k_bias_std=0.0, seed=0, max_blocks_per_seq=None,
+                extra_blocks=0, keep_fp32=False, threads=None, name="custom") -> Workload:
+    """A workload with explicit per-sequence lengths (used by the test grids)."""
+    seq_lens = np.asarray(seq_lens, np.int32).reshape(B)
+    cfg = Config(name, B, n_q_heads, n_kv_heads, head_dim,
+                 int(seq_lens.max(initial=0)), block_size, table, k_dist, v_dist, k_bias_std,
+                 seed)
+    return _make(cfg, seq_lens, max_blocks_per_seq, extra_blocks, keep_fp32, threads)
+
+
+def make(cfg: Config | int, *, keep_fp32: bool = False, threads: int | None = None) -> Workload:
+    """The named workload ``cfg`` (a Config or an index into CONFIGS)."""
+    if isinstance(cfg, int):
+        cfg = CONFIGS[cfg]
+    return _make(cfg, _seq_lens(cfg), None, 0, keep_fp32, threads)
+
+
+def _make(cfg: Config, seq_lens, max_blocks_per_seq, extra_blocks, keep_fp32, threads):
+    threads = threads or min(32, os.cpu_count() or 1)
+    bs, Hk, D = cfg.block_size, cfg.n_kv_heads, cfg.head_dim
+    need = int(((seq_lens.astype(np.int64) + bs - 1) // bs).sum())
+    P = max(1, need + int(extra_blocks))
+    mbps = max_blocks_per_seq or max(1, -(-int(seq_lens.max(initial=0)) // bs))
+    q = _rng(cfg.seed, _S_Q).standard_normal((cfg.B, cfg.n_q_heads, D), dtype=np.float32)
+    bias = None
+    if cfg.k_bias_std:
+        bias = (_rng(cfg.seed, _S_BIAS).standard_normal((Hk, D), dtype=np.float32)
+                * np.float32(cfg.k_bias_std))
+    k, ks, k32 = _fill_pool(cfg.seed, _S_K, cfg.k_dist, P, bs, Hk, D, bias, keep_fp32, threads)
+    v, vs, v32 = _fill_pool(cfg.seed, _S_V, cfg.v_dist, P, bs, Hk, D, None, keep_fp32, threads)
+    bt = build_block_table(seq_lens, bs, mbps, cfg.table, P, _rng(cfg.seed, _S_TABLE))
+    scale = float(np.float32(1.0) / np.float32(math.sqrt(D)))
+    return Workload(cfg, q, k, v, ks, vs, bt, seq_lens.astype(np.int32), scale, k32, v32)
+
+
+def with_config(cfg: Config, **kw) -> Config:
+    return replace(cfg, **kw)

@@ -1,0 +1,449 @@
+/*
+ * q8kv_oracle.c -- plain single-threaded CPU oracle for q8-KV single-query decode
+ * attention. TEST INFRASTRUCTURE ONLY (see q8kv_oracle.h for what may call it).
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fPIC -shared (no -ffast-math, no
+ * FMA contraction: the fp32 Q quantisation must round every operation separately).
+ *
+ * Readings of the pages taken here (the garbled spots in the Kestrel-LLM walk-through,
+ * trdm.cn/news/511694, section 2):
+ *   - zero-block guard "if (qm 1e-6f) qm 1.0f" is read as  if (qm < 1e-6f) qm = 1.0f;
+ *   - the cast "(int8_t)clamp(q*iq, -128, 127)" is replaced by round-half-to-even, then
+ *     clamp to [-127, 127] (the rounding rule this library fixes);
+ *   - the K/V scale arrays hold the dequantisation multiplier itself (no extra 1/127)
+ *     and are indexed by the physical slot: scale[slot * n_kv_heads + kv_head];
+ *   - the running max starts at -infinity (the page's -1e9 gives the same result when
+ *     every score exceeds -1e9);
+ *   - on the new-maximum branch the token's own weight is exp(0) = 1;
+ *   - seq_len == 0 yields an all-zero output row.
+ */
+#include "q8kv_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Planted mistakes for the pin-strength test (tests/test_oracle_mutants.py): building
+ * with -DQ8KVO_MUTANT=n switches on mistake n; the default build has none. */
+#ifndef Q8KVO_MUTANT
+#define Q8KVO_MUTANT 0
+#endif
+#define MUT(n) (Q8KVO_MUTANT == (n))
+
+/* ---------------------------------------------------------------- Q quantisation */
+
+/* Round to nearest, ties to even, written out so that it does not depend on the
+ * floating-point environment. x is an fp32 value widened to double (exact). */
+static double round_half_even(double x)
+{
+    double f = floor(x);
+    double frac = x - f; /* exact: |x| < 2^24 here */
+    if (frac > 0.5)
+        return f + 1.0;
+    if (frac < 0.5)
+        return f;
+    return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+/* One 32-element block, walk-through section 2 part 1:
+ *   qm  = max |q_i|                      (fp32)
+ *   if qm < 1e-6: qm = 1                  (all-zero block -> codes 0)
+ *   qsc = qm * (1/127)                    (fp32)
+ *   iq  = 127 / qm                        (fp32, correctly rounded)
+ *   qi  = clamp(rne(q_i * iq), -127, 127) (product rounded to fp32 first) */
+static void quantize_block(const float *qb, int8_t *qi, float *qsc)
+{
+    float qm = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        float a = fabsf(qb[i]);
+        if (a > qm)
+            qm = a;
+    }
+    if (MUT(8) ? (qm <= 1e-6f) : (qm < 1e-6f))
+        qm = 1.0f;
+    *qsc = qm * (1.0f / 127.0f);
+    float iq = 127.0f / qm;
+    for (int i = 0; i < 32; ++i) {
+        float prod = qb[i] * iq;
+        double r = MUT(3) ? trunc((double)prod) : round_half_even((double)prod);
+        if (r > 127.0)
+            r = 127.0;
+        if (r < -127.0)
+            r = -127.0;
+        qi[i] = (int8_t)r;
+    }
+}
+
+int q8kvo_quantize_q(const float *q, long n, int8_t *qi, float *qsc)
+{
+    if (!q || !qi || !qsc || n < 0 || (n % 32) != 0)
+        return Q8KVO_EINVAL;
+    for (long i = 0; i < n; ++i)
+        if (!isfinite(q[i]))
+            return Q8KVO_EINVAL;
+    for (long b = 0; b < n / 32; ++b)
+        quantize_block(q + 32 * b, qi + 32 * b, qsc + b);
+    return Q8KVO_OK;
+}
+
+/* ---------------------------------------------------------------- cache access */
+
+static int check_cache(const q8kvo_cache *c)
+{
+    if (!c || !c->block_table || !c->seq_lens)
+        return Q8KVO_EINVAL;
+    if (c->B <= 0 || c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+        (c->head_dim % 32) != 0 || c->block_size <= 0 || c->max_blocks_per_seq <= 0 ||
+        c->num_blocks <= 0 || (c->n_q_heads % c->n_kv_heads) != 0 || !isfinite(c->scale))
+        return Q8KVO_EINVAL;
+    return Q8KVO_OK;
+}
+
+static int check_seq(const q8kvo_cache *c, int b, int h)
+{
+    if (b < 0 || b >= c->B || h < 0 || h >= c->n_q_heads)
+        return Q8KVO_EINVAL;
+    int L = c->seq_lens[b];
+    if (L < 0 || (long)L > (long)c->max_blocks_per_seq * c->block_size)
+        return Q8KVO_ERANGE;
+    int nblk = (L + c->block_size - 1) / c->block_size;
+    for (int i = 0; i < nblk; ++i) {
+        int p = c->block_table[(long)b * c->max_blocks_per_seq + i];
+        if (p < 0 || p >= c->num_blocks)
+            return Q8KVO_ERANGE;
+    }
+    return Q8KVO_OK;
+}
+
+/* Physical slot of token t of sequence b (beaiera.top, "Top-K index global mapping";
+ * Kestrel walk-through section 2 part 2: block t / kv_bs, offset t % kv_bs). */
+static long slot_of(const q8kvo_cache *c, int b, int t)
+{
+    long blk = c->block_table[(long)b * c->max_blocks_per_seq + t / c->block_size];
+    return blk * c->block_size + (MUT(5) ? (t + 1) % c->block_size : t % c->block_size);
+}
+
+/* GQA mapping of the llama2.c loop: kv_head = q_head / (n_q_heads / n_kv_heads). */
+static int kv_head_of(const q8kvo_cache *c, int h)
+{
+    return MUT(2) ? h % c->n_kv_heads : h / (c->n_q_heads / c->n_kv_heads);
+}
+
+/* Quantised query of (b, h): codes and per-block scales. */
+static int quantized_query(const q8kvo_cache *c, const float *q, int b, int h, int8_t *qi,
+                           float *qsc)
+{
+    const float *qh = q + ((long)b * c->n_q_heads + h) * c->head_dim;
+    return q8kvo_quantize_q(qh, c->head_dim, qi, qsc);
+}
+
+/* int32 dot of quant block j of the query with the same 32 channels of a K row. */
+static int32_t block_dot(const int8_t *qi, const int8_t *krow, int j)
+{
+    int32_t acc = 0;
+    for (int i = 0; i < 32; ++i)
+        acc += (int32_t)qi[32 * j + i] * (int32_t)krow[32 * j + (MUT(14) ? (i + 1) % 32 : i)];
+    return acc;
+}
+
+/* Score of token t: s = (sum_j dot_j * qsc_j) * ks * scale, in fp64 (section 2 part 2,
+ * "block scales put back": the integer dot is the skeleton, the float scales are
+ * applied while accumulating). */
+static double score_of(const q8kvo_cache *c, const int8_t *qi, const float *qsc, int b, int kvh,
+                       int t)
+{
+    long slot = slot_of(c, b, t);
+    const int8_t *krow = c->k + (slot * c->n_kv_heads + kvh) * (long)c->head_dim;
+    int nb = c->head_dim / 32;
+    double s = 0.0;
+    for (int j = 0; j < nb; ++j)
+        s += (double)block_dot(qi, krow, j) * (double)qsc[MUT(7) ? 0 : j];
+    double ks = MUT(1) ? 1.0 : (double)c->ks[slot * c->n_kv_heads + kvh];
+    return s * ks * (double)c->scale * (MUT(13) ? (double)c->scale : 1.0);
+}
+
+int q8kvo_block_dots(const q8kvo_cache *c, const float *q, int b, int h, int32_t *dots)
+{
+    int rc = check_cache(c);
+    if (rc)
+        return rc;
+    if (!c->k || !q || !dots)
+        return Q8KVO_EINVAL;
+    if ((rc = check_seq(c, b, h)))
+        return rc;
+    int D = c->head_dim, nb = D / 32, kvh = kv_head_of(c, h), L = c->seq_lens[b];
+    int8_t *qi = (int8_t *)malloc((size_t)D);
+    float *qsc = (float *)malloc(sizeof(float) * (size_t)nb);
+    if (!qi || !qsc) {
+        free(qi);
+        free(qsc);
+        return Q8KVO_ENOMEM;
+    }
+    rc = quantized_query(c, q, b, h, qi, qsc);
+    for (int t = 0; rc == Q8KVO_OK && t < L; ++t) {
+        long slot = slot_of(c, b, t);
+        const int8_t *krow = c->k + (slot * c->n_kv_heads + kvh) * (long)D;
+        for (int j = 0; j < nb; ++j)
+            dots[(long)t * nb + j] = block_dot(qi, krow, j);
+    }
+    free(qi);
+    free(qsc);
+    return rc;
+}
+
+int q8kvo_scores(const q8kvo_cache *c, const float *q, int b, int h, double *s)
+{
+    int rc = check_cache(c);
+    if (rc)
+        return rc;
+    if (!c->k || !c->ks || !q || !s)
+        return Q8KVO_EINVAL;
+    if ((rc = check_seq(c, b, h)))
+        return rc;
+    int D = c->head_dim, nb = D / 32, kvh = kv_head_of(c, h), L = c->seq_lens[b];
+    int8_t *qi = (int8_t *)malloc((size_t)D);
+    float *qsc = (float *)malloc(sizeof(float) * (size_t)nb);
+    if (!qi || !qsc) {
+        free(qi);
+        free(qsc);
+        return Q8KVO_ENOMEM;
+    }
+    rc = quantized_query(c, q, b, h, qi, qsc);
+    for (int t = 0; rc == Q8KVO_OK && t < L; ++t)
+        s[t] = score_of(c, qi, qsc, b, kvh, t);
+    free(qi);
+    free(qsc);
+    return rc;
+}
+
+/* ---------------------------------------------------------------- single pass */
+
+/* One (b, h), walk-through section 2 parts 1-3, token by token:
+ *   if s > M:  f = exp(M - s); S *= f; acc *= f; M = s; w = 1
+ *   else:      w = exp(s - M)
+ *   S += w;  acc[d] += w * vs * V[d]
+ * and finally out = acc / S. */
+static int decode_online_one(const q8kvo_cache *c, const float *q, int b, int h, double *out,
+                             double *m_trace, long *n_iter, int8_t *qi, float *qsc, double *acc)
+{
+    int D = c->head_dim, kvh = kv_head_of(c, h), L = c->seq_lens[b];
+    int rc = quantized_query(c, q, b, h, qi, qsc);
+    if (rc)
+        return rc;
+    double M = -INFINITY, S = 0.0;
+    for (int d = 0; d < D; ++d)
+        acc[d] = 0.0;
+    long iters = 0;
+    for (int t = 0; t < L; ++t) {
+        double s = score_of(c, qi, qsc, b, kvh, t);
+        double w;
+        if (s > M) {
+            double f = exp(M - s);
+            if (!MUT(10))
+                S *= f;
+            for (int d = 0; d < D && !MUT(4); ++d)
+                acc[d] *= f;
+            M = s;
+            w = 1.0;
+        } else {
+            w = exp(s - M);
+        }
+        S += w;
+        long slot = slot_of(c, b, t);
+        const int8_t *vrow = c->v + (slot * c->n_kv_heads + kvh) * (long)D;
+        double wv = w * (double)(MUT(6) ? c->ks : c->vs)[slot * c->n_kv_heads + kvh];
+        for (int d = 0; d < D; ++d)
+            acc[d] += wv * (double)vrow[d];
+        if (m_trace)
+            m_trace[t] = M;
+        ++iters;
+    }
+    for (int d = 0; d < D; ++d)
+        out[d] = (L > 0) ? acc[d] / S : 0.0;
+    if (n_iter)
+        *n_iter = iters;
+    return Q8KVO_OK;
+}
+
+static int scratch_alloc(int D, int8_t **qi, float **qsc, double **acc)
+{
+    *qi = (int8_t *)malloc((size_t)D);
+    *qsc = (float *)malloc(sizeof(float) * (size_t)(D / 32));
+    *acc = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!*qi || !*qsc || !*acc) {
+        free(*qi);
+        free(*qsc);
+        free(*acc);
+        return Q8KVO_ENOMEM;
+    }
+    return Q8KVO_OK;
+}
+
+static int check_q8(const q8kvo_cache *c, const float *q, const void *out)
+{
+    int rc = check_cache(c);
+    if (rc)
+        return rc;
+    if (!c->k || !c->v || !c->ks || !c->vs || !q || !out)
+        return Q8KVO_EINVAL;
+    return Q8KVO_OK;
+}
+
+int q8kvo_decode_online(const q8kvo_cache *c, const float *q, int b, int h, double *out,
+                        double *m_trace, long *n_iter)
+{
+    int rc = check_q8(c, q, out);
+    if (rc || (rc = check_seq(c, b, h)))
+        return rc;
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    rc = decode_online_one(c, q, b, h, out, m_trace, n_iter, qi, qsc, acc);
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
+int q8kvo_decode_all(const q8kvo_cache *c, const float *q, double *out)
+{
+    int rc = check_q8(c, q, out);
+    if (rc)
+        return rc;
+    for (int b = 0; b < c->B; ++b)
+        if ((rc = check_seq(c, b, 0)))
+            return rc;
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    for (int b = 0; b < c->B && rc == Q8KVO_OK; ++b)
+        for (int h = 0; h < c->n_q_heads && rc == Q8KVO_OK; ++h)
+            rc = decode_online_one(c, q, b, h, out + ((long)b * c->n_q_heads + h) * c->head_dim,
+                                   NULL, NULL, qi, qsc, acc);
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
+int q8kvo_decode_pairs(const q8kvo_cache *c, const float *q, const int32_t *pairs, long n,
+                       double *out)
+{
+    int rc = check_q8(c, q, out);
+    if (rc)
+        return rc;
+    if (!pairs || n < 0)
+        return Q8KVO_EINVAL;
+    for (long i = 0; i < n; ++i)
+        if ((rc = check_seq(c, pairs[2 * i], pairs[2 * i + 1])))
+            return rc;
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    for (long i = 0; i < n && rc == Q8KVO_OK; ++i)
+        rc = decode_online_one(c, q, pairs[2 * i], pairs[2 * i + 1], out + i * c->head_dim, NULL,
+                               NULL, qi, qsc, acc);
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
+/* ---------------------------------------------------------------- three pass */
+
+/* The naive form the walk-through (section 3) contrasts with, laid out like the
+ * llama2.c loop: all scores first, then the stable softmax (subtract the max,
+ * exponentiate, sum, divide), then the weighted sum of dequantised V. */
+int q8kvo_decode_threepass(const q8kvo_cache *c, const float *q, int b, int h, double *out)
+{
+    int rc = check_q8(c, q, out);
+    if (rc || (rc = check_seq(c, b, h)))
+        return rc;
+    int D = c->head_dim, kvh = kv_head_of(c, h), L = c->seq_lens[b];
+    for (int d = 0; d < D; ++d)
+        out[d] = 0.0;
+    if (L == 0)
+        return Q8KVO_OK;
+    double *s = (double *)malloc(sizeof(double) * (size_t)L);
+    if (!s)
+        return Q8KVO_ENOMEM;
+    rc = q8kvo_scores(c, q, b, h, s);
+    if (rc) {
+        free(s);
+        return rc;
+    }
+    double mx = s[0];
+    for (int t = 1; t < L; ++t)
+        if (s[t] > mx)
+            mx = s[t];
+    double sum = 0.0;
+    for (int t = 0; t < L; ++t) {
+        s[t] = exp(s[t] - mx);
+        sum += s[t];
+    }
+    for (int t = 0; t < L; ++t) {
+        long slot = slot_of(c, b, t);
+        const int8_t *vrow = c->v + (slot * c->n_kv_heads + kvh) * (long)D;
+        double a = s[t] / sum * (double)c->vs[slot * c->n_kv_heads + kvh];
+        for (int d = 0; d < D; ++d)
+            out[d] += a * (double)vrow[d];
+    }
+    free(s);
+    return Q8KVO_OK;
+}
+
+/* ---------------------------------------------------------------- unquantised */
+
+/* fp64 attention of the original fp32 q, K and V (no quantisation anywhere):
+ * s_t = scale * q . k_t, stable softmax, weighted V. */
+int q8kvo_attn_fp32(const q8kvo_cache *c, const float *q, const float *k32, const float *v32,
+                    int b, int h, double *out)
+{
+    int rc = check_cache(c);
+    if (rc)
+        return rc;
+    if (!q || !k32 || !v32 || !out)
+        return Q8KVO_EINVAL;
+    if ((rc = check_seq(c, b, h)))
+        return rc;
+    int D = c->head_dim, kvh = kv_head_of(c, h), L = c->seq_lens[b];
+    const float *qh = q + ((long)b * c->n_q_heads + h) * D;
+    for (int d = 0; d < D; ++d)
+        out[d] = 0.0;
+    if (L == 0)
+        return Q8KVO_OK;
+    double *s = (double *)malloc(sizeof(double) * (size_t)L);
+    if (!s)
+        return Q8KVO_ENOMEM;
+    double mx = -INFINITY;
+    for (int t = 0; t < L; ++t) {
+        long slot = slot_of(c, b, t);
+        const float *krow = k32 + (slot * c->n_kv_heads + kvh) * (long)D;
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d)
+            acc += (double)qh[d] * (double)krow[d];
+        s[t] = acc * (double)c->scale;
+        if (s[t] > mx)
+            mx = s[t];
+    }
+    double sum = 0.0;
+    for (int t = 0; t < L; ++t) {
+        s[t] = exp(s[t] - mx);
+        sum += s[t];
+    }
+    for (int t = 0; t < L; ++t) {
+        long slot = slot_of(c, b, t);
+        const float *vrow = v32 + (slot * c->n_kv_heads + kvh) * (long)D;
+        double a = s[t] / sum;
+        for (int d = 0; d < D; ++d)
+            out[d] += a * (double)vrow[d];
+    }
+    free(s);
+    return Q8KVO_OK;
+}

@@ -1,0 +1,109 @@
+/*
+ * q8kv_oracle.h -- plain, slow, single-threaded CPU oracle for q8-KV single-query
+ * decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path links, loads or calls this
+ * code; only the test suite, the smoke check and the benchmark's CPU-baseline leg do.
+ * It shares no source, header, table or helper with the CUDA library.
+ *
+ * What it computes follows the Kestrel-LLM walk-through "flash_attn_single_q_q8_neon"
+ * (trdm.cn/news/511694):
+ *   - section 2, part 1 ("Q quantised once"): Q -> int8 in 32-element blocks with a
+ *     max-abs/127 scale per block, a zero-block guard, and a clamp;
+ *   - section 2, part 2 ("online softmax running state"): per token, exact int8 block
+ *     dot products into int32, each block scaled by its Q scale, then by the
+ *     per-(token, KV head) K scale and the softmax scale; the running max M and sum S,
+ *     with the accumulator rescaled whenever M rises; V accumulated as int8 V times
+ *     (softmax weight x per-(token, head) V scale);
+ *   - section 2, part 3 ("normalise the output"): one division by S at the end;
+ *   - section 3 ("consequences of the change"): the naive variant that stores every
+ *     score first is functionally equivalent (used here as a cross-check).
+ * GQA head mapping kv_head = q_head / (n_q_heads / n_kv_heads) follows the llama2.c
+ * attention loop (aicoding.csdn.net, "attention core logic").
+ * The block-table -> slot mapping follows beaiera.top "deepseek-attention-div64",
+ * section "Top-K index global mapping": slot = block_table[b][t / bs] * bs + t % bs.
+ *
+ * Precision: the Q quantisation runs in IEEE fp32 (it decides integers, so it is done
+ * in the precision the GPU uses), everything after the int32 dots runs in fp64.
+ * Rounding of the quantised Q: round-half-to-even, then clamp to [-127, 127].
+ *
+ * Pinning: every function here is pinned by the -m "not gpu" tests to hand-derived
+ * golden cases, closed forms and library routines; see the test files named
+ * test_oracle_*.py.
+ */
+#ifndef Q8KV_ORACLE_H
+#define Q8KV_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes of every oracle call. */
+#define Q8KVO_OK 0
+#define Q8KVO_EINVAL 1   /* null pointer, bad size, or non-finite input */
+#define Q8KVO_ERANGE 2   /* seq_len or block-table entry outside the cache */
+#define Q8KVO_ENOMEM 3
+
+/* A paged q8 KV cache, exactly as the CUDA library receives it.
+ *   k, v     int8  [num_blocks][block_size][n_kv_heads][head_dim]
+ *   ks, vs   fp32  [num_blocks][block_size][n_kv_heads]   (dequant multipliers)
+ *   block_table int32 [B][max_blocks_per_seq]
+ *   seq_lens    int32 [B]
+ * All pointers are host pointers owned by the caller. */
+typedef struct {
+    const int8_t *k;
+    const int8_t *v;
+    const float *ks;
+    const float *vs;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    int B;
+    int n_q_heads;
+    int n_kv_heads;
+    int head_dim;
+    int block_size;
+    int max_blocks_per_seq;
+    int num_blocks;
+    float scale;
+} q8kvo_cache;
+
+/* Quantise n fp32 values (n a multiple of 32) block by block.
+ * qi[n] receives the int8 codes, qsc[n/32] the per-block fp32 scales. */
+int q8kvo_quantize_q(const float *q, long n, int8_t *qi, float *qsc);
+
+/* int32 dot product of each 32-element block of the quantised query of (b, h) with
+ * the K row of every token of sequence b: dots[t][j], t < seq_lens[b], j < head_dim/32. */
+int q8kvo_block_dots(const q8kvo_cache *c, const float *q, int b, int h, int32_t *dots);
+
+/* Scores s[t] (fp64, natural-log units) of (b, h), exactly as the online pass uses them. */
+int q8kvo_scores(const q8kvo_cache *c, const float *q, int b, int h, double *s);
+
+/* Single-pass online-softmax decode of one (b, h): out[head_dim] in fp64.
+ * m_trace (optional, length seq_lens[b]) receives M after each token;
+ * n_iter (optional) receives the number of token iterations executed. */
+int q8kvo_decode_online(const q8kvo_cache *c, const float *q, int b, int h,
+                        double *out, double *m_trace, long *n_iter);
+
+/* Naive three-pass variant (all scores, then max, then exp/sum, then weighted V). */
+int q8kvo_decode_threepass(const q8kvo_cache *c, const float *q, int b, int h, double *out);
+
+/* Online decode of every (b, h): out[B][n_q_heads][head_dim] (fp64). */
+int q8kvo_decode_all(const q8kvo_cache *c, const float *q, double *out);
+
+/* Online decode of n chosen (b, h) pairs: pairs[2*i] = b, pairs[2*i+1] = h;
+ * out[n][head_dim] (fp64). */
+int q8kvo_decode_pairs(const q8kvo_cache *c, const float *q, const int32_t *pairs, long n,
+                       double *out);
+
+/* Unquantised attention of one (b, h) in fp64 from fp32 q and fp32 K/V pools laid out
+ * like the int8 pools ([num_blocks][block_size][n_kv_heads][head_dim]); the q8 fields of
+ * c (k, v, ks, vs) are ignored. Used to report the error of q8 against fp32 attention. */
+int q8kvo_attn_fp32(const q8kvo_cache *c, const float *q, const float *k32, const float *v32,
+                    int b, int h, double *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
