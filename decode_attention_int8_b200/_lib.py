@@ -1,0 +1,194 @@
+"""ctypes binding of libq8kv.so (the C ABI in include/q8kv.h).
+
+Argument marshalling only: shapes and dtypes are read off torch tensors, device pointers
+and the current CUDA stream are passed through, and a non-OK status raises Q8KVError.
+Every step of the computation runs in the CUDA library; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+_lock = threading.Lock()
+_lib = None
+
+Q8KV_OK = 0
+DEVERR_SEQ_LEN = 0x1
+DEVERR_BLOCK_TABLE = 0x2
+DEVERR_TIMEOUT = 0x4
+
+EXPORTS = (
+    "q8kv_decode_attn",
+    "q8kv_workspace_bytes",
+    "q8kv_workspace_init",
+    "q8kv_decode_attn_ws",
+    "q8kv_debug_quantize_q",
+    "q8kv_debug_block_dots",
+    "q8kv_device_errors",
+    "q8kv_status_string",
+    "q8kv_last_cuda_error",
+    "q8kv_version",
+)
+
+
+class Q8KVError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = lib().q8kv_status_string(status).decode()
+        if status == 3:
+            msg += f" (cudaError {lib().q8kv_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} (status {status})")
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libq8kv.so, building it first when it is missing or older than its sources."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB
+            if not os.path.exists(path) or _build.stale():
+                _build.build()
+            L = ctypes.CDLL(path)
+            P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            sig = {
+                "q8kv_decode_attn": ([P] * 8 + [I] * 7 + [F, P], I),
+                "q8kv_workspace_bytes": ([I, I, I, I], Z),
+                "q8kv_workspace_init": ([P, Z, P], I),
+                "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
+                "q8kv_debug_quantize_q": ([P, P, P, I, I, P], I),
+                "q8kv_debug_block_dots": ([P, I] + [P] * 8 + [I] * 7 + [F, P], I),
+                "q8kv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
+                "q8kv_status_string": ([I], ctypes.c_char_p),
+                "q8kv_last_cuda_error": ([], I),
+                "q8kv_version": ([], I),
+            }
+            for name, (args, res) in sig.items():
+                fn = getattr(L, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = L
+    return _lib
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or t.dim() != ndim or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor with {ndim} dims, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens):
+    _need(out, "out", torch.float32, 3)
+    _need(q, "q", torch.float32, 3)
+    _need(k_blocks, "k_blocks", torch.int8, 4)
+    _need(v_blocks, "v_blocks", torch.int8, 4)
+    _need(kscale, "kscale", torch.float32, 3)
+    _need(vscale, "vscale", torch.float32, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    P, bs, Hk, Dk = k_blocks.shape
+    if tuple(out.shape) != (B, Hq, D) or Dk != D or tuple(v_blocks.shape) != (P, bs, Hk, D):
+        raise ValueError("q/out/k_blocks/v_blocks shapes disagree")
+    if tuple(kscale.shape) != (P, bs, Hk) or tuple(vscale.shape) != (P, bs, Hk):
+        raise ValueError("kscale/vscale must be [num_blocks][block_size][n_kv_heads]")
+    if block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table/seq_lens batch dimension disagrees with q")
+    return B, Hq, Hk, D, bs, int(block_table.shape[1]), P
+
+
+def _check(status: int, what: str):
+    if status != Q8KV_OK:
+        raise Q8KVError(status, what)
+
+
+def q8kv_decode_attn(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens, scale,
+                     stream=None):
+    """Decode attention into ``out`` with the library-managed workspace."""
+    geo = _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens)
+    _check(lib().q8kv_decode_attn(_ptr(out), _ptr(q), _ptr(k_blocks), _ptr(v_blocks),
+                                  _ptr(kscale), _ptr(vscale), _ptr(block_table), _ptr(seq_lens),
+                                  *geo, float(scale), _stream(stream)), "q8kv_decode_attn")
+    return out
+
+
+def q8kv_workspace_bytes(B: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
+    return int(lib().q8kv_workspace_bytes(B, n_q_heads, n_kv_heads, head_dim))
+
+
+def q8kv_workspace_init(workspace: torch.Tensor, stream=None):
+    _check(lib().q8kv_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "q8kv_workspace_init")
+
+
+def q8kv_decode_attn_ws(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens, scale,
+                        workspace, stream=None):
+    """Decode attention with a caller-owned (zero-initialised) workspace tensor."""
+    geo = _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check(lib().q8kv_decode_attn_ws(_ptr(out), _ptr(q), _ptr(k_blocks), _ptr(v_blocks),
+                                     _ptr(kscale), _ptr(vscale), _ptr(block_table),
+                                     _ptr(seq_lens), *geo, float(scale), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "q8kv_decode_attn_ws")
+    return out
+
+
+def q8kv_debug_quantize_q(qi, qsc, q, stream=None):
+    """int8 codes qi [..., D] and block scales qsc [..., D/32] of the fp32 rows of q [..., D]."""
+    D = q.shape[-1]
+    n_rows = q.numel() // D
+    for t, dt in ((qi, torch.int8), (qsc, torch.float32), (q, torch.float32)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q8kv_debug_quantize_q: bad tensor")
+    if qi.numel() != q.numel() or qsc.numel() != n_rows * (D // 32):
+        raise ValueError("q8kv_debug_quantize_q: size mismatch")
+    _check(lib().q8kv_debug_quantize_q(_ptr(qi), _ptr(qsc), _ptr(q), n_rows, D, _stream(stream)),
+           "q8kv_debug_quantize_q")
+
+
+def q8kv_debug_block_dots(dots, out, q, k_blocks, v_blocks, kscale, vscale, block_table,
+                          seq_lens, scale, stream=None):
+    """int32 block dots [B][Hq][max_len][D/32] from the decode kernel (and ``out``)."""
+    geo = _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens)
+    _need(dots, "dots", torch.int32, 4)
+    B, Hq, _, D, _, _, _ = geo
+    if dots.shape[0] != B or dots.shape[1] != Hq or dots.shape[3] != D // 32:
+        raise ValueError("dots must be [B][n_q_heads][max_seq_len][head_dim/32]")
+    _check(lib().q8kv_debug_block_dots(_ptr(dots), int(dots.shape[2]), _ptr(out), _ptr(q),
+                                       _ptr(k_blocks), _ptr(v_blocks), _ptr(kscale),
+                                       _ptr(vscale), _ptr(block_table), _ptr(seq_lens), *geo,
+                                       float(scale), _stream(stream)), "q8kv_debug_block_dots")
+
+
+def q8kv_device_errors(clear: bool = True) -> int:
+    flags = ctypes.c_uint(0)
+    _check(lib().q8kv_device_errors(ctypes.byref(flags), 1 if clear else 0), "q8kv_device_errors")
+    return int(flags.value)
+
+
+def q8kv_version() -> int:
+    return int(lib().q8kv_version())

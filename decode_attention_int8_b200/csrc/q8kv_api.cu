@@ -1,0 +1,512 @@
+// q8kv_api.cu -- the C ABI of include/q8kv.h: host-side argument checks, the tiling plan,
+// TMA descriptors, workspace management and kernel launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "q8kv.h"
+#include "q8kv_decode.cuh"
+#include "q8kv_qquant.cuh"
+
+namespace {
+
+using namespace q8kv;
+
+__device__ unsigned g_device_errors = 0;
+
+thread_local int t_last_cuda_error = 0;
+
+q8kv_status cuda_fail(cudaError_t e)
+{
+    t_last_cuda_error = static_cast<int>(e);
+    return Q8KV_ERR_CUDA;
+}
+
+#define Q8KV_CUDA(call)                                                                            \
+    do {                                                                                           \
+        cudaError_t e_ = (call);                                                                   \
+        if (e_ != cudaSuccess)                                                                     \
+            return cuda_fail(e_);                                                                  \
+    } while (0)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int smem_optin = 0;
+    unsigned *errors = nullptr;      // address of g_device_errors on this device
+    bool attr_set[2][2] = {{false, false}, {false, false}};
+    void *ws = nullptr;              // library-managed workspace
+    size_t ws_bytes = 0;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+q8kv_status device_info(DeviceInfo **out)
+{
+    int dev = 0;
+    Q8KV_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices)
+        return Q8KV_ERR_UNSUPPORTED;
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        Q8KV_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        Q8KV_CUDA(cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        void *addr = nullptr;
+        Q8KV_CUDA(cudaGetSymbolAddress(&addr, g_device_errors));
+        d.errors = static_cast<unsigned *>(addr);
+        d.ready = true;
+    }
+    *out = &d;
+    return Q8KV_OK;
+}
+
+q8kv_status encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn)
+{
+    if (!g_encode) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        Q8KV_CUDA(cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                                   cudaEnableDefault, &q));
+        if (q != cudaDriverEntryPointSuccess || !p)
+            return Q8KV_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    *fn = g_encode;
+    return Q8KV_OK;
+}
+
+struct Shape {
+    int B, Hq, Hk, D, bs, mbps, P;
+};
+
+// How the work is tiled for one shape on one device.
+struct Plan {
+    int G, slices, NT, HPC, nhc, pairs, subtiles, TT, box_tok, log2_box, n_boxes, n_stages;
+    int scale_bulk, heads_seg, scratch_stride, grid;
+    SmemLayout lay;
+    size_t smem_bytes;
+    size_t ws_seg_off, ws_grp_off, ws_part_off, ws_bytes;
+};
+
+bool is_pow2(int x)
+{
+    return x > 0 && (x & (x - 1)) == 0;
+}
+
+int ilog2(int x)
+{
+    int r = 0;
+    while ((1 << (r + 1)) <= x)
+        ++r;
+    return r;
+}
+
+size_t align256(size_t x)
+{
+    return (x + 255) & ~static_cast<size_t>(255);
+}
+
+// Head tiling only (what the workspace size depends on).
+q8kv_status plan_heads(int Hq, int Hk, int D, Plan &pl)
+{
+    if (Hq <= 0 || Hk <= 0 || D <= 0 || Hq % Hk != 0)
+        return Q8KV_ERR_INVALID_ARG;
+    if (D != kD)
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.G = Hq / Hk;
+    if (pl.G > 128)
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.slices = 1;
+    while (pl.slices * 16 < pl.G)
+        pl.slices *= 2;
+    pl.NT = (pl.G > 8) ? 2 : 1;
+    const int max_hpc = kConsumerWarps / pl.slices;
+    pl.HPC = 1;
+    while (pl.HPC * 2 <= max_hpc && Hk % (pl.HPC * 2) == 0)
+        pl.HPC *= 2;
+    pl.scale_bulk = (pl.HPC == Hk) ? 1 : 0;
+    if (!pl.scale_bulk && (pl.HPC < 4 || Hk % 4 != 0))
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.nhc = Hk / pl.HPC;
+    pl.pairs = pl.HPC * pl.slices;
+    pl.subtiles = kConsumerWarps / pl.pairs;
+    pl.TT = 16 * pl.subtiles;
+    pl.heads_seg = pl.HPC * pl.G;
+    pl.scratch_stride = 32 * 32 * pl.NT + 32;
+    return Q8KV_OK;
+}
+
+void plan_workspace(int B, int grid, Plan &pl)
+{
+    pl.ws_seg_off = 0;
+    pl.ws_grp_off = align256(sizeof(int) * (size_t)B * pl.nhc);
+    pl.ws_part_off = pl.ws_grp_off + align256(sizeof(int) * 2 * (size_t)grid);
+    pl.ws_bytes = pl.ws_part_off +
+                  align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * (kD + 2));
+}
+
+q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
+{
+    if (s.B <= 0 || s.bs <= 0 || s.mbps <= 0 || s.P <= 0)
+        return Q8KV_ERR_INVALID_ARG;
+    q8kv_status st = plan_heads(s.Hq, s.Hk, s.D, pl);
+    if (st != Q8KV_OK)
+        return st;
+    if (!is_pow2(s.bs) || s.bs < 16 || s.bs > 256)
+        return Q8KV_ERR_UNSUPPORTED;
+    if (s.B > 16384 || (long long)s.P * s.bs >= (1LL << 31) ||
+        (long long)s.mbps * s.bs >= (1LL << 31))
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.box_tok = pl.TT < s.bs ? pl.TT : s.bs;
+    pl.log2_box = ilog2(pl.box_tok);
+    pl.n_boxes = pl.TT / pl.box_tok;
+    const int scratch_floats = (pl.subtiles - 1) * pl.pairs * pl.scratch_stride;
+    pl.n_stages = 0;
+    for (int n = kMaxStages; n >= 2; --n) {
+        SmemLayout L = make_layout(pl.TT, pl.HPC, n, s.B, scratch_floats);
+        if ((size_t)L.total + 1024 <= (size_t)dev.smem_optin) {
+            pl.n_stages = n;
+            pl.lay = L;
+            break;
+        }
+    }
+    if (pl.n_stages == 0)
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.smem_bytes = (size_t)pl.lay.total + 1024;
+    const long long tiles_per_seq = ((long long)s.mbps * s.bs + pl.TT - 1) / pl.TT;
+    const long long tiles_max = (long long)s.B * pl.nhc * tiles_per_seq;
+    pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
+    plan_workspace(s.B, dev.sms, pl); // sized for the full grid so one size fits all calls
+    return Q8KV_OK;
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+q8kv_status encode_maps(const Shape &s, const Plan &pl, const int8_t *k, const int8_t *v,
+                        const float *ks, const float *vs, CUtensorMap *mk, CUtensorMap *mv,
+                        CUtensorMap *mks, CUtensorMap *mvs)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    q8kv_status st = encoder(&enc);
+    if (st != Q8KV_OK)
+        return st;
+    const cuuint64_t slots = (cuuint64_t)s.P * s.bs;
+    // K/V pool viewed as (channel, slot, kv head): the box lands in shared memory as
+    // [kv head][token][128 channels], 128-byte swizzled.
+    cuuint64_t dims[3] = {(cuuint64_t)kD, slots, (cuuint64_t)s.Hk};
+    cuuint64_t strides[2] = {(cuuint64_t)s.Hk * kD, (cuuint64_t)kD};
+    cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)pl.box_tok, (cuuint32_t)pl.HPC};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t *>(k), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return Q8KV_ERR_UNSUPPORTED;
+    r = enc(mv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t *>(v), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return Q8KV_ERR_UNSUPPORTED;
+    std::memset(mks, 0, sizeof(*mks));
+    std::memset(mvs, 0, sizeof(*mvs));
+    if (!pl.scale_bulk) {
+        cuuint64_t sd[2] = {(cuuint64_t)s.Hk, slots};
+        cuuint64_t ss[1] = {(cuuint64_t)s.Hk * 4};
+        cuuint32_t sb[2] = {(cuuint32_t)pl.HPC, (cuuint32_t)pl.box_tok};
+        cuuint32_t se[2] = {1, 1};
+        r = enc(mks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(ks), sd, ss, sb, se,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return Q8KV_ERR_UNSUPPORTED;
+        r = enc(mvs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(vs), sd, ss, sb, se,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return Q8KV_ERR_UNSUPPORTED;
+    }
+    return Q8KV_OK;
+}
+
+struct Call {
+    float *out;
+    const float *q;
+    const int8_t *k, *v;
+    const float *ks, *vs;
+    const int32_t *bt, *lens;
+    Shape s;
+    float scale;
+    int32_t *dots;
+    int dots_max_len;
+};
+
+q8kv_status check_call(const Call &c)
+{
+    if (!c.out || !c.q || !c.k || !c.v || !c.ks || !c.vs || !c.bt || !c.lens)
+        return Q8KV_ERR_INVALID_ARG;
+    if (c.s.B <= 0 || c.s.Hq <= 0 || c.s.Hk <= 0 || c.s.D <= 0 || c.s.bs <= 0 || c.s.mbps <= 0 ||
+        c.s.P <= 0 || c.s.Hq % c.s.Hk != 0 || c.s.D % 32 != 0)
+        return Q8KV_ERR_INVALID_ARG;
+    if (!std::isfinite(c.scale))
+        return Q8KV_ERR_INVALID_ARG;
+    if (!aligned16(c.out) || !aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) ||
+        !aligned16(c.ks) || !aligned16(c.vs))
+        return Q8KV_ERR_INVALID_ARG;
+    return Q8KV_OK;
+}
+
+template <int NT, bool kDump>
+q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl,
+                          const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mks,
+                          const CUtensorMap &mvs, cudaStream_t stream)
+{
+    auto fn = decode_kernel<NT, kDump>;
+    if (!dev.attr_set[NT - 1][kDump ? 1 : 0]) {
+        Q8KV_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev.smem_optin));
+        dev.attr_set[NT - 1][kDump ? 1 : 0] = true;
+    }
+    fn<<<pl.grid, kThreads, pl.smem_bytes, stream>>>(p, mk, mv, mks, mvs);
+    Q8KV_CUDA(cudaGetLastError());
+    return Q8KV_OK;
+}
+
+q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaStream_t stream)
+{
+    q8kv_status st = check_call(c);
+    if (st != Q8KV_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        st = device_info(&dev);
+    }
+    if (st != Q8KV_OK)
+        return st;
+    Plan pl;
+    st = make_plan(c.s, *dev, pl);
+    if (st != Q8KV_OK)
+        return st;
+    if (managed_ws) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (dev->ws_bytes < pl.ws_bytes) {
+            if (dev->ws) {
+                Q8KV_CUDA(cudaFree(dev->ws));
+                dev->ws = nullptr;
+                dev->ws_bytes = 0;
+            }
+            Q8KV_CUDA(cudaMalloc(&dev->ws, pl.ws_bytes));
+            Q8KV_CUDA(cudaMemsetAsync(dev->ws, 0, pl.ws_bytes, stream));
+            dev->ws_bytes = pl.ws_bytes;
+        }
+        ws = dev->ws;
+        ws_bytes = dev->ws_bytes;
+    }
+    if (!ws || ws_bytes < pl.ws_bytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return Q8KV_ERR_WORKSPACE;
+
+    CUtensorMap mk, mv, mks, mvs;
+    st = encode_maps(c.s, pl, c.k, c.v, c.ks, c.vs, &mk, &mv, &mks, &mvs);
+    if (st != Q8KV_OK)
+        return st;
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    p.out = c.out;
+    p.q = c.q;
+    p.block_table = c.bt;
+    p.seq_lens = c.lens;
+    p.kscale = c.ks;
+    p.vscale = c.vs;
+    p.seg_counters = reinterpret_cast<int *>(w + pl.ws_seg_off);
+    p.grp_counters = reinterpret_cast<int *>(w + pl.ws_grp_off);
+    p.partials = reinterpret_cast<float *>(w + pl.ws_part_off);
+    p.errors = dev->errors;
+    p.dbg_dots = c.dots;
+    p.dbg_max_len = c.dots_max_len;
+    p.B = c.s.B;
+    p.Hq = c.s.Hq;
+    p.Hk = c.s.Hk;
+    p.G = pl.G;
+    p.bs = c.s.bs;
+    p.mbps = c.s.mbps;
+    p.num_blocks = c.s.P;
+    p.HPC = pl.HPC;
+    p.nhc = pl.nhc;
+    p.slices = pl.slices;
+    p.pairs = pl.pairs;
+    p.subtiles = pl.subtiles;
+    p.TT = pl.TT;
+    p.box_tok = pl.box_tok;
+    p.log2_box = pl.log2_box;
+    p.n_boxes = pl.n_boxes;
+    p.n_stages = pl.n_stages;
+    p.scale_bulk = pl.scale_bulk;
+    p.heads_seg = pl.heads_seg;
+    p.scratch_stride = pl.scratch_stride;
+    p.scale_log2 = (float)((double)c.scale * 1.4426950408889634);
+    p.lay = pl.lay;
+
+    const bool dump = c.dots != nullptr;
+    if (pl.NT == 1)
+        return dump ? launch_kernel<1, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
+                    : launch_kernel<1, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
+    return dump ? launch_kernel<2, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
+                : launch_kernel<2, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
+}
+
+} // namespace
+
+extern "C" {
+
+q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
+                             const int8_t *v_blocks, const float *kscale, const float *vscale,
+                             const int32_t *block_table, const int32_t *seq_lens, int B,
+                             int n_q_heads, int n_kv_heads, int head_dim, int kv_block_size,
+                             int max_blocks_per_seq, int num_kv_blocks, float scale,
+                             cudaStream_t stream)
+{
+    Call c{out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+           Shape{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
+                 num_kv_blocks},
+           scale, nullptr, 0};
+    return run(c, nullptr, 0, true, stream);
+}
+
+size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim)
+{
+    if (B <= 0)
+        return 0;
+    Plan pl;
+    if (plan_heads(n_q_heads, n_kv_heads, head_dim, pl) != Q8KV_OK)
+        return 0;
+    DeviceInfo *dev = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (device_info(&dev) != Q8KV_OK)
+            return 0;
+    }
+    plan_workspace(B, dev->sms, pl);
+    return pl.ws_bytes;
+}
+
+q8kv_status q8kv_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (!workspace || workspace_bytes == 0)
+        return Q8KV_ERR_INVALID_ARG;
+    Q8KV_CUDA(cudaMemsetAsync(workspace, 0, workspace_bytes, stream));
+    return Q8KV_OK;
+}
+
+q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_blocks,
+                                const int8_t *v_blocks, const float *kscale,
+                                const float *vscale, const int32_t *block_table,
+                                const int32_t *seq_lens, int B, int n_q_heads, int n_kv_heads,
+                                int head_dim, int kv_block_size, int max_blocks_per_seq,
+                                int num_kv_blocks, float scale, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream)
+{
+    Call c{out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+           Shape{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
+                 num_kv_blocks},
+           scale, nullptr, 0};
+    return run(c, workspace, workspace_bytes, false, stream);
+}
+
+q8kv_status q8kv_debug_quantize_q(int8_t *qi, float *qsc, const float *q, int n_rows,
+                                  int head_dim, cudaStream_t stream)
+{
+    if (!qi || !qsc || !q || n_rows <= 0 || head_dim <= 0 || head_dim % 32 != 0)
+        return Q8KV_ERR_INVALID_ARG;
+    if (!aligned16(q) || (reinterpret_cast<uintptr_t>(qi) & 7u) != 0)
+        return Q8KV_ERR_INVALID_ARG;
+    const long long n_blocks = (long long)n_rows * (head_dim / 32);
+    const long long threads = n_blocks * 4;
+    const int tpb = 256;
+    const long long grid = (threads + tpb - 1) / tpb;
+    if (grid > 0x7fffffffLL)
+        return Q8KV_ERR_UNSUPPORTED;
+    qquant_debug_kernel<<<(unsigned)grid, tpb, 0, stream>>>(qi, qsc, q, n_blocks);
+    Q8KV_CUDA(cudaGetLastError());
+    return Q8KV_OK;
+}
+
+q8kv_status q8kv_debug_block_dots(int32_t *dots, int max_seq_len, float *out, const float *q,
+                                  const int8_t *k_blocks, const int8_t *v_blocks,
+                                  const float *kscale, const float *vscale,
+                                  const int32_t *block_table, const int32_t *seq_lens, int B,
+                                  int n_q_heads, int n_kv_heads, int head_dim,
+                                  int kv_block_size, int max_blocks_per_seq, int num_kv_blocks,
+                                  float scale, cudaStream_t stream)
+{
+    if (!dots || max_seq_len <= 0)
+        return Q8KV_ERR_INVALID_ARG;
+    if ((long long)max_seq_len < (long long)max_blocks_per_seq * kv_block_size)
+        return Q8KV_ERR_INVALID_ARG; // a valid seq_len could exceed the dots buffer
+    Call c{out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+           Shape{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
+                 num_kv_blocks},
+           scale, dots, max_seq_len};
+    return run(c, nullptr, 0, true, stream);
+}
+
+q8kv_status q8kv_device_errors(unsigned *flags, int clear)
+{
+    if (!flags)
+        return Q8KV_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    q8kv_status st;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        st = device_info(&dev);
+    }
+    if (st != Q8KV_OK)
+        return st;
+    Q8KV_CUDA(cudaDeviceSynchronize());
+    Q8KV_CUDA(cudaMemcpy(flags, dev->errors, sizeof(unsigned), cudaMemcpyDeviceToHost));
+    if (clear)
+        Q8KV_CUDA(cudaMemset(dev->errors, 0, sizeof(unsigned)));
+    return Q8KV_OK;
+}
+
+const char *q8kv_status_string(q8kv_status status)
+{
+    switch (status) {
+    case Q8KV_OK:
+        return "ok";
+    case Q8KV_ERR_INVALID_ARG:
+        return "invalid argument";
+    case Q8KV_ERR_UNSUPPORTED:
+        return "unsupported shape";
+    case Q8KV_ERR_CUDA:
+        return "CUDA error";
+    case Q8KV_ERR_WORKSPACE:
+        return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int q8kv_last_cuda_error(void)
+{
+    return t_last_cuda_error;
+}
+
+int q8kv_version(void)
+{
+    return 100;
+}
+
+} // extern "C"

@@ -1,0 +1,972 @@
+// q8kv_decode.cuh -- the q8-KV single-query decode-attention kernel for sm_100a.
+//
+// What it computes (Kestrel-LLM walk-through "flash_attn_single_q_q8_neon",
+// trdm.cn/news/511694, section 2 parts 1-3): per (sequence b, query head h) quantise q
+// to int8 in 32-element blocks, take exact int32 block dot products with every int8 K
+// row of the sequence, scale them by the Q block scale, the per-(token, KV head) K scale
+// and the softmax scale, fold the scores into an online softmax (running max M, running
+// sum S, accumulator rescaled when M rises), accumulate int8 V times weight times the
+// per-(token, KV head) V scale, and divide by S once at the end.
+//
+// How (B200 design, none of it from the pages):
+//  * One persistent CTA per SM. The work is the flat list of "tiles" (TT tokens x HPC KV
+//    heads of one sequence), ordered sequence-major; CTA i takes a contiguous 1/grid
+//    share of it, so load balance does not depend on how ragged the batch is. The list
+//    is indexed through a per-sequence prefix sum every CTA builds in shared memory.
+//  * Warp 8 is the producer: it resolves block-table entries 32 tiles at a time and
+//    streams K and V tiles with TMA (3-D tensor maps, 128-byte swizzle, evict-first L2
+//    policy) and the scales with bulk copies into an n-stage ring guarded by mbarriers.
+//  * Warps 0-7 consume: each owns (KV head, 16-head slice of its query group, 16-token
+//    subtile). QK is an int8 tensor-core MMA (m16n8k32, one MMA per 32-channel quant
+//    block, so each MMA result is exactly one int32 block dot). PV is an f16 MMA
+//    (m16n8k16) on exact f16 copies of the int8 V codes with the fp32 weights split into
+//    hi + lo f16 halves (about 22 significant bits), pre-scaled by a power of two that
+//    tracks the largest V scale seen so the halves stay in the f16 normal range.
+//  * The online softmax runs per 16-token subtile in base 2; per-warp states are merged
+//    in shared memory, and CTAs that share a sequence merge their partial (M, S, acc)
+//    through the workspace with a two-level last-arriver log-sum-exp combine (no waiting
+//    on other CTAs, counters reset by the last arriver).
+#pragma once
+
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "q8kv_ptx.cuh"
+#include "q8kv_qquant.cuh"
+
+namespace q8kv {
+
+constexpr int kD = 128;             // head_dim handled by this kernel
+constexpr int kNB = kD / 32;        // quant blocks per head
+constexpr int kConsumerWarps = 8;   // warps 0-7
+constexpr int kProducerWarp = 8;    // warp 8
+constexpr int kThreads = 9 * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kMaxBoxes = 8;        // TMA boxes per stage
+constexpr int kGroupFanIn = 8;      // contributors merged per first-level combine
+constexpr int kMaxStages = 8;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
+constexpr int kEMin = 15;           // smallest biased exponent used for the V-scale window
+
+// Device-side error bits (match Q8KV_DEVERR_* in q8kv.h).
+constexpr unsigned kErrSeqLen = 0x1u;
+constexpr unsigned kErrBlockTable = 0x2u;
+constexpr unsigned kErrTimeout = 0x4u;
+
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a)
+{
+    return (x + a - 1) / a * a;
+}
+
+// Shared-memory carve-up, computed identically on host and device.
+struct SmemLayout {
+    uint32_t stage_bytes; // one ring slot: K | V | kscale | vscale
+    uint32_t off_k, off_v, off_ks, off_vs; // within a slot
+    uint32_t off_full, off_empty, off_mask, off_misc, off_prefix, off_scratch;
+    uint32_t total; // bytes from the 1024-aligned base
+};
+
+__host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages, int B,
+                                                  int scratch_floats)
+{
+    SmemLayout L;
+    const uint32_t kv = (uint32_t)(TT * HPC * kD);
+    const uint32_t sc = align_up((uint32_t)(TT * HPC * 4), 128);
+    L.off_k = 0;
+    L.off_v = kv;
+    L.off_ks = 2 * kv;
+    L.off_vs = 2 * kv + sc;
+    L.stage_bytes = align_up(2 * kv + 2 * sc, 1024);
+    uint32_t o = (uint32_t)n_stages * L.stage_bytes;
+    L.off_full = o;
+    o += 8 * kMaxStages;
+    L.off_empty = o;
+    o += 8 * kMaxStages;
+    L.off_mask = o;
+    o += 4 * kMaxStages;
+    L.off_misc = o;
+    o += 64;
+    L.off_prefix = o;
+    o = align_up(o + 4u * (uint32_t)(B + 1), 16);
+    L.off_scratch = o;
+    o += 4u * (uint32_t)scratch_floats;
+    L.total = o;
+    return L;
+}
+
+struct DecodeParams {
+    float *out;
+    const float *q;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    const float *kscale;
+    const float *vscale;
+    float *partials;     // [2 * grid][heads_seg][kD + 2]
+    int *seg_counters;   // [B * nhc]
+    int *grp_counters;   // [2 * grid]
+    unsigned *errors;    // device error word
+    int32_t *dbg_dots;   // [B][Hq][dbg_max_len][kNB] (debug instantiation only)
+    int dbg_max_len;
+    int B, Hq, Hk, G;
+    int bs, mbps, num_blocks;
+    int HPC, nhc, slices, pairs, subtiles, TT, box_tok, log2_box, n_boxes, n_stages;
+    int scale_bulk;      // 1: scales by contiguous bulk copy (HPC == Hk); 0: 2-D tensor map
+    int heads_seg;       // query heads per segment (HPC * G)
+    int scratch_stride;  // floats per (subtile, pair) merge region
+    float scale_log2;    // softmax scale * log2(e)
+    SmemLayout lay;
+};
+
+__device__ __forceinline__ void consumer_bar()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+
+__device__ __forceinline__ float ldcg_f(const float *p)
+{
+    return __ldcg(p);
+}
+
+__device__ __forceinline__ float4 ldcg_f4(const float *p)
+{
+    return __ldcg(reinterpret_cast<const float4 *>(p));
+}
+
+// CTA owning flat tile x when N tiles are split over g CTAs ([i*N/g, (i+1)*N/g)).
+__device__ __forceinline__ int cta_of_tile(long long x, long long N, int g)
+{
+    return (int)(((x + 1) * g - 1) / N);
+}
+
+__device__ __forceinline__ long long cta_start(int i, long long N, int g)
+{
+    return (long long)i * N / g;
+}
+
+// Merge partial (M, S, acc) slots into either the output rows of (b, hc) or one slot.
+// slot_k(k) gives the slot index of the k-th input. Called by all consumer threads.
+template <typename SlotFn>
+__device__ void merge_slots(const DecodeParams &p, int n_in, SlotFn slot_k, bool to_out, int b,
+                            int hc, int dest_slot, int ctid)
+{
+    const int H = p.heads_seg;
+    const size_t stride = (size_t)H * (kD + 2);
+    for (int u = ctid; u < H * (kD / 4); u += kConsumerThreads) {
+        const int hl = u / (kD / 4), d4 = u % (kD / 4);
+        float mx = -INFINITY;
+        for (int k = 0; k < n_in; ++k)
+            mx = fmaxf(mx, ldcg_f(p.partials + slot_k(k) * stride + (size_t)H * kD + hl));
+        float ssum = 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < n_in; ++k) {
+            const float *base = p.partials + slot_k(k) * stride;
+            const float mk = ldcg_f(base + (size_t)H * kD + hl);
+            const float f = (mk == -INFINITY) ? 0.f : exp2f(mk - mx);
+            ssum += f * ldcg_f(base + (size_t)H * kD + H + hl);
+            const float4 v = ldcg_f4(base + (size_t)hl * kD + d4 * 4);
+            a.x += f * v.x;
+            a.y += f * v.y;
+            a.z += f * v.z;
+            a.w += f * v.w;
+        }
+        if (to_out) {
+            const float inv = ssum > 0.f ? 1.0f / ssum : 0.f;
+            const long long h = (long long)hc * H + hl;
+            float4 o = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+            *reinterpret_cast<float4 *>(p.out + ((long long)b * p.Hq + h) * kD + d4 * 4) = o;
+        } else {
+            float *base = p.partials + (size_t)dest_slot * stride;
+            __syncwarp();
+            *reinterpret_cast<float4 *>(base + (size_t)hl * kD + d4 * 4) = a;
+            if (d4 == 0) {
+                base[(size_t)H * kD + hl] = mx;
+                base[(size_t)H * kD + H + hl] = ssum;
+            }
+        }
+    }
+}
+
+// Per-sequence tile prefix: prefix[b + 1] = sum over b' <= b of nhc * ceil(L_b' / TT).
+__device__ void build_prefix(const DecodeParams &p, int *prefix, volatile int *wsum, int tid,
+                             int warp, int lane)
+{
+    const int cap = p.mbps * p.bs;
+    int carry = 0;
+    for (int base = 0; base < p.B; base += kThreads) {
+        const int b = base + tid;
+        int v = 0;
+        if (b < p.B) {
+            int L = p.seq_lens[b];
+            if (L < 0 || L > cap) {
+                atomicOr(p.errors, kErrSeqLen);
+                L = L < 0 ? 0 : cap;
+            }
+            v = ((L + p.TT - 1) / p.TT) * p.nhc;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(kFullMask, v, o);
+            if (lane >= o)
+                v += t;
+        }
+        if (lane == 31)
+            wsum[warp] = v;
+        __syncthreads();
+        int off = carry, total = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            const int ws = wsum[w];
+            if (w < warp)
+                off += ws;
+            total += ws;
+        }
+        if (b < p.B)
+            prefix[b + 1] = off + v;
+        carry += total;
+        __syncthreads();
+    }
+    if (tid == 0)
+        prefix[0] = 0;
+}
+
+__device__ __forceinline__ int clamp_len(int L, int cap)
+{
+    return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// ------------------------------------------------------------------ producer warp
+
+__device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                        const CUtensorMap *tmKs, const CUtensorMap *tmVs, uint8_t *smem,
+                        const int *prefix, long long t0, long long t1, int lane)
+{
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
+    int *mask = reinterpret_cast<int *>(smem + p.lay.off_mask);
+    const uint64_t pol = l2_policy_evict_first();
+    const int cap = p.mbps * p.bs;
+    const uint32_t kv_box = (uint32_t)(p.box_tok * p.HPC * kD);
+    const uint32_t sc_box = (uint32_t)(p.box_tok * p.HPC * 4);
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, issued_par = 0;
+    bool aborted = false;
+
+    for (long long xb = t0; xb < t1 && !aborted; xb += 32) {
+        const long long x = xb + lane;
+        int hc = 0;
+        int slot[kMaxBoxes];
+#pragma unroll
+        for (int bx = 0; bx < kMaxBoxes; ++bx)
+            slot[bx] = -1;
+        if (x < t1) {
+            int lo = 0, hi = p.B - 1; // largest b with prefix[b] <= x
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (prefix[mid] <= x)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            const int b = lo;
+            const int pre = prefix[b];
+            const int ntb = (prefix[b + 1] - pre) / p.nhc;
+            const int local = (int)(x - pre);
+            hc = local / ntb;
+            const int lt = local - hc * ntb;
+            const int tok0 = lt * p.TT;
+            const int L = clamp_len(__ldg(p.seq_lens + b), cap);
+#pragma unroll
+            for (int bx = 0; bx < kMaxBoxes; ++bx) {
+                const int tk = tok0 + bx * p.box_tok;
+                if (bx < p.n_boxes && tk < L) {
+                    const int ph = __ldg(p.block_table + (long long)b * p.mbps + tk / p.bs);
+                    if (ph >= 0 && ph < p.num_blocks)
+                        slot[bx] = ph * p.bs + (tk % p.bs);
+                    else
+                        atomicOr(p.errors, kErrBlockTable);
+                }
+            }
+        }
+        const int n = (int)((t1 - xb) < 32 ? (t1 - xb) : 32);
+        for (int i = 0; i < n; ++i) {
+            const int hci = __shfl_sync(kFullMask, hc, i);
+            int sl[kMaxBoxes];
+#pragma unroll
+            for (int bx = 0; bx < kMaxBoxes; ++bx)
+                sl[bx] = __shfl_sync(kFullMask, slot[bx], i);
+            int ok = 1;
+            if (lane == 0) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, globaltimer_ns() + kWaitLimitNs)) {
+                    ok = 0;
+                    atomicOr(p.errors, kErrTimeout);
+                } else {
+                    uint32_t bytes = 0;
+                    int loaded = 0;
+#pragma unroll
+                    for (int bx = 0; bx < kMaxBoxes; ++bx)
+                        if (bx < p.n_boxes && sl[bx] >= 0) {
+                            bytes += 2 * (kv_box + sc_box);
+                            loaded |= 1 << bx;
+                        }
+                    // which boxes hold data; published by the release of the arrive below
+                    mask[stage] = loaded;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    uint8_t *sb = smem + (size_t)stage * p.lay.stage_bytes;
+#pragma unroll
+                    for (int bx = 0; bx < kMaxBoxes; ++bx) {
+                        if (bx < p.n_boxes && sl[bx] >= 0) {
+                            tma_load_3d(sb + p.lay.off_k + bx * kv_box, tmK, &full[stage], 0, sl[bx],
+                                        hci * p.HPC, pol);
+                            tma_load_3d(sb + p.lay.off_v + bx * kv_box, tmV, &full[stage], 0, sl[bx],
+                                        hci * p.HPC, pol);
+                            if (p.scale_bulk) {
+                                const long long e0 = (long long)sl[bx] * p.Hk;
+                                bulk_load(sb + p.lay.off_ks + bx * sc_box, p.kscale + e0, sc_box,
+                                          &full[stage], pol);
+                                bulk_load(sb + p.lay.off_vs + bx * sc_box, p.vscale + e0, sc_box,
+                                          &full[stage], pol);
+                            } else {
+                                tma_load_2d(sb + p.lay.off_ks + bx * sc_box, tmKs, &full[stage],
+                                            hci * p.HPC, sl[bx], pol);
+                                tma_load_2d(sb + p.lay.off_vs + bx * sc_box, tmVs, &full[stage],
+                                            hci * p.HPC, sl[bx], pol);
+                            }
+                        }
+                    }
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                }
+            }
+            ok = __shfl_sync(kFullMask, ok, 0);
+            if (!ok) {
+                aborted = true;
+                break;
+            }
+            if (++stage == p.n_stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+    // Every copy this warp issued must have landed before the CTA may exit.
+    if (lane == 0) {
+        for (int s = 0; s < p.n_stages; ++s)
+            if ((issued >> s) & 1u)
+                mbar_wait(&full[s], (issued_par >> s) & 1u, globaltimer_ns() + kWaitLimitNs);
+    }
+}
+
+// ------------------------------------------------------------------ consumer warps
+
+template <int NT>
+struct WarpState {
+    float acc[NT][8][4]; // PV accumulator fragments (columns = heads, rows = channels)
+    float M[NT];         // running max (base 2) of this lane's QK row head
+    float S[NT];         // this lane's share of the running sum
+    int E;               // V-scale exponent window (biased exponent of max V scale seen)
+    uint32_t qa[kNB][4]; // int8 A fragments of the quantised query heads
+    float qs[NT][kNB];   // Q block scales of rows g and g + 8
+};
+
+template <int NT>
+__device__ __forceinline__ void load_query(const DecodeParams &p, WarpState<NT> &st, int b, int hc,
+                                           int kl, int slice, int g, int c)
+{
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (r >= NT) {
+#pragma unroll
+            for (int j = 0; j < kNB; ++j) {
+                st.qa[j][1] = 0u;
+                st.qa[j][3] = 0u;
+            }
+            continue;
+        }
+        const int hg = slice * 16 + r * 8 + g;
+        const bool valid = hg < p.G;
+        const float *qrow =
+            p.q + ((long long)b * p.Hq + (long long)(hc * p.HPC + kl) * p.G + hg) * kD;
+        float v[kNB][8];
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+            if (valid) {
+                x0 = __ldg(reinterpret_cast<const float4 *>(qrow + 32 * j + 8 * c));
+                x1 = __ldg(reinterpret_cast<const float4 *>(qrow + 32 * j + 8 * c + 4));
+            }
+            v[j][0] = x0.x;
+            v[j][1] = x0.y;
+            v[j][2] = x0.z;
+            v[j][3] = x0.w;
+            v[j][4] = x1.x;
+            v[j][5] = x1.y;
+            v[j][6] = x1.z;
+            v[j][7] = x1.w;
+        }
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            uint32_t lo, hi;
+            quantize_block_quad(v[j], lo, hi, st.qs[r][j]);
+            // MMA k positions 4c..4c+3 and 16+4c..16+4c+3 carry channels 8c..8c+7 of the
+            // block; the K operand uses the same assignment, so each MMA is one block dot.
+            st.qa[j][r == 0 ? 0 : 1] = lo;
+            st.qa[j][r == 0 ? 2 : 3] = hi;
+        }
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void reset_state(WarpState<NT> &st)
+{
+#pragma unroll
+    for (int pv = 0; pv < NT; ++pv) {
+        st.M[pv] = -INFINITY;
+        st.S[pv] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                st.acc[pv][i][k] = 0.f;
+    }
+    st.E = kEMin;
+}
+
+// Per-thread shared-memory offsets that are the same for every stage.
+struct ThreadOffsets {
+    uint32_t k[2][kNB]; // K fragment loads (QK n-tile, quant block)
+    uint32_t v[4];      // V rows 2c, 2c+1, 2c+8, 2c+9 (channel chunk g)
+    uint32_t s[2][2];   // scale of tokens nt*8 + 2c + e
+    int tok[2][2];      // stage-local token index of (nt, e)
+};
+
+__device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int kl, int ts, int g,
+                                                      int c)
+{
+    ThreadOffsets o;
+    const int lb = p.log2_box, bt = p.box_tok, H = p.HPC;
+    auto row_kv = [&](int tok) { return ((tok >> lb) * H + kl) * bt + (tok & (bt - 1)); };
+    auto row_sc = [&](int tok) { return ((tok >> lb) * bt + (tok & (bt - 1))) * H + kl; };
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int r = row_kv(ts * 16 + nt * 8 + g);
+#pragma unroll
+        for (int j = 0; j < kNB; ++j)
+            o.k[nt][j] = p.lay.off_k + r * 128 + ((((2 * j) | (c >> 1)) ^ (r & 7)) << 4) +
+                         ((c & 1) << 3);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int tok = ts * 16 + nt * 8 + 2 * c + e;
+            o.tok[nt][e] = tok;
+            o.s[nt][e] = 4 * row_sc(tok);
+        }
+    }
+#pragma unroll
+    for (int qv = 0; qv < 4; ++qv) {
+        const int t = 2 * c + (qv & 1) + (qv >> 1) * 8;
+        const int r = row_kv(ts * 16 + t);
+        o.v[qv] = p.lay.off_v + r * 128 + ((g ^ (r & 7)) << 4);
+    }
+    return o;
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// One stage (16 tokens of one KV head for this warp).
+template <int NT, bool kDump>
+__device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<NT> &st,
+                                              const ThreadOffsets &o, uint32_t sbase, int nvalid,
+                                              int loaded, int b, int hc, int kl, int slice,
+                                              int tok0, int g, int c)
+{
+    // ---- scores: int8 MMA per quant block, exact int32 block dots
+    float s[NT][2][2];
+#pragma unroll
+    for (int r = 0; r < NT; ++r)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+            s[r][nt][0] = s[r][nt][1] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            const uint2 kk = lds64(sbase + o.k[nt][j]);
+            int d[4];
+            mma_s8_16832(d, st.qa[j][0], st.qa[j][1], st.qa[j][2], st.qa[j][3], kk.x, kk.y);
+            if constexpr (kDump) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = q >> 1, e = q & 1;
+                    const int hg = slice * 16 + r * 8 + g;
+                    const int tl = o.tok[nt][e];
+                    if (hg < p.G && tl < nvalid && ((loaded >> (tl >> p.log2_box)) & 1)) {
+                        const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
+                        p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) * kNB +
+                                   j] = d[q];
+                    }
+                }
+            }
+            s[0][nt][0] += (float)d[0] * st.qs[0][j];
+            s[0][nt][1] += (float)d[1] * st.qs[0][j];
+            if constexpr (NT == 2) {
+                s[NT - 1][nt][0] += (float)d[2] * st.qs[NT - 1][j];
+                s[NT - 1][nt][1] += (float)d[3] * st.qs[NT - 1][j];
+            }
+        }
+    }
+    // ---- per-token K and V scales; masking of tokens past the sequence end
+    float kss[2][2], vsv[2][2];
+    bool val[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            val[nt][e] = o.tok[nt][e] < nvalid && ((loaded >> (o.tok[nt][e] >> p.log2_box)) & 1);
+            kss[nt][e] = lds_f32(sbase + p.lay.off_ks + o.s[nt][e]) * p.scale_log2;
+            const float vv = lds_f32(sbase + p.lay.off_vs + o.s[nt][e]);
+            vsv[nt][e] = val[nt][e] ? vv : 0.f;
+        }
+    // ---- online softmax (base 2), blockwise over the 16 tokens
+    float alpha[NT];
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float v = val[nt][e] ? s[r][nt][e] * kss[nt][e] : -INFINITY;
+                s[r][nt][e] = v;
+                m = fmaxf(m, v);
+            }
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
+        const float mn = fmaxf(st.M[r], m);
+        const float ms = (mn == -INFINITY) ? 0.f : mn;
+        alpha[r] = exp2f(st.M[r] - ms);
+        st.M[r] = mn;
+        float ws = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float w = exp2f(s[r][nt][e] - ms);
+                s[r][nt][e] = w;
+                ws += w;
+            }
+        st.S[r] = st.S[r] * alpha[r] + ws;
+    }
+    // ---- V-scale window: weights are scaled by 2^(141 - E) so that w * vs < 2^15
+    float vm = fmaxf(fmaxf(vsv[0][0], vsv[0][1]), fmaxf(vsv[1][0], vsv[1][1]));
+    vm = fmaxf(vm, __shfl_xor_sync(kFullMask, vm, 1));
+    vm = fmaxf(vm, __shfl_xor_sync(kFullMask, vm, 2));
+    const int et = max(kEMin, (int)(__float_as_uint(vm) >> 23));
+    int de = 0;
+    if (et > st.E) {
+        de = et - st.E;
+        st.E = et;
+    }
+    const float mult = exp2i(141 - st.E);
+    const float shrink = exp2i(-min(de, 126));
+    // ---- weights as split f16 B operands (column n = head g, k = token)
+    uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float p0 = s[r][nt][0] * (vsv[nt][0] * mult);
+            const float p1 = s[r][nt][1] * (vsv[nt][1] * mult);
+            const __half2 h = __floats2half2_rn(p0, p1);
+            const float r0 = p0 - __low2float(h), r1 = p1 - __high2float(h);
+            bh[r][nt] = *reinterpret_cast<const uint32_t *>(&h);
+            bl[r][nt] = pack_f16x2(r0, r1);
+        }
+    }
+    // ---- rescale the accumulator when M rose or the V-scale window moved
+#pragma unroll
+    for (int pv = 0; pv < NT; ++pv) {
+        const float fr = alpha[pv] * shrink;
+        const float f0 = __shfl_sync(kFullMask, fr, 8 * c);
+        const float f1 = __shfl_sync(kFullMask, fr, 8 * c + 4);
+        if (__any_sync(kFullMask, (f0 != 1.f) || (f1 != 1.f))) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                st.acc[pv][i][0] *= f0;
+                st.acc[pv][i][1] *= f1;
+                st.acc[pv][i][2] *= f0;
+                st.acc[pv][i][3] *= f1;
+            }
+        }
+    }
+    // ---- PV: rows = channels 16g + 2i (+1), k = tokens, columns = heads
+    const uint4 R0 = lds128(sbase + o.v[0]);
+    const uint4 R1 = lds128(sbase + o.v[1]);
+    const uint4 R2 = lds128(sbase + o.v[2]);
+    const uint4 R3 = lds128(sbase + o.v[3]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t w0 = word_of(R0, i >> 1), w1 = word_of(R1, i >> 1);
+        const uint32_t w2 = word_of(R2, i >> 1), w3 = word_of(R3, i >> 1);
+        const uint32_t sl = (i & 1) ? 0x0602u : 0x0400u;
+        const uint32_t sh = (i & 1) ? 0x0703u : 0x0501u;
+        const uint32_t a0 = s8pair_to_f16x2(prmt(w0, w1, sl));
+        const uint32_t a1 = s8pair_to_f16x2(prmt(w0, w1, sh));
+        const uint32_t a2 = s8pair_to_f16x2(prmt(w2, w3, sl));
+        const uint32_t a3 = s8pair_to_f16x2(prmt(w2, w3, sh));
+#pragma unroll
+        for (int pv = 0; pv < NT; ++pv) {
+            mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, bh[pv][0], bh[pv][1]);
+            mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, bl[pv][0], bl[pv][1]);
+        }
+    }
+}
+
+// Write the 16 channels 16g..16g+15 of column head (pv, col) scaled by f.
+template <int NT>
+__device__ __forceinline__ void store_row16(float *dst, const WarpState<NT> &st, int pv, int q,
+                                            float f)
+{
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float4 v = make_float4(st.acc[pv][i][q] * f, st.acc[pv][i][q + 2] * f,
+                                     st.acc[pv][i + 1][q] * f, st.acc[pv][i + 1][q + 2] * f);
+        *reinterpret_cast<float4 *>(dst + 2 * i) = v;
+    }
+}
+
+// End of a segment (all of this CTA's tiles of sequence b, head chunk hc).
+template <int NT>
+__device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8_t *smem, int b,
+                                 int hc, int kl, int slice, int pair, int ts, int g, int c,
+                                 int ctid, const int *prefix, long long t0, long long t1,
+                                 long long N, int gcta)
+{
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + p.lay.off_misc);
+    // complete this lane's row sums
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 1);
+        st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 2);
+    }
+    // undo the V-scale window: acc back to true units
+    const float unscale = exp2i(st.E - 141);
+#pragma unroll
+    for (int pv = 0; pv < NT; ++pv)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                st.acc[pv][i][k] *= unscale;
+
+    // merge the token subtiles of each (KV head, slice) pair inside the CTA
+    if (p.subtiles > 1) {
+        float *scr = reinterpret_cast<float *>(smem + p.lay.off_scratch);
+        const int lane = g * 4 + c;
+        if (ts > 0) {
+            float *reg = scr + (size_t)((ts - 1) * p.pairs + pair) * p.scratch_stride;
+#pragma unroll
+            for (int pv = 0; pv < NT; ++pv)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        reg[lane * (32 * NT) + (pv * 8 + i) * 4 + k] = st.acc[pv][i][k];
+            if (c == 0) {
+#pragma unroll
+                for (int r = 0; r < NT; ++r) {
+                    reg[32 * 32 * NT + r * 8 + g] = st.M[r];
+                    reg[32 * 32 * NT + 16 + r * 8 + g] = st.S[r];
+                }
+            }
+        }
+        consumer_bar();
+        if (ts == 0) {
+            for (int k = 1; k < p.subtiles; ++k) {
+                const float *reg = scr + (size_t)((k - 1) * p.pairs + pair) * p.scratch_stride;
+#pragma unroll
+                for (int pv = 0; pv < NT; ++pv) {
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int col = 2 * c + q;
+                        const float mm = __shfl_sync(kFullMask, st.M[pv], 4 * col);
+                        const float mo = reg[32 * 32 * NT + pv * 8 + col];
+                        const float mn = fmaxf(mm, mo);
+                        const float fa = (mm == -INFINITY) ? 0.f : exp2f(mm - mn);
+                        const float fo = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            st.acc[pv][i][q] = st.acc[pv][i][q] * fa +
+                                               reg[lane * (32 * NT) + (pv * 8 + i) * 4 + q] * fo;
+                            st.acc[pv][i][q + 2] =
+                                st.acc[pv][i][q + 2] * fa +
+                                reg[lane * (32 * NT) + (pv * 8 + i) * 4 + q + 2] * fo;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < NT; ++r) {
+                    const float mo = reg[32 * 32 * NT + r * 8 + g];
+                    const float so = reg[32 * 32 * NT + 16 + r * 8 + g];
+                    const float mn = fmaxf(st.M[r], mo);
+                    const float fa = (st.M[r] == -INFINITY) ? 0.f : exp2f(st.M[r] - mn);
+                    const float fo = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+                    st.S[r] = st.S[r] * fa + so * fo;
+                    st.M[r] = mn;
+                }
+            }
+        }
+        consumer_bar();
+    }
+
+    const int pre = prefix[b];
+    const int ntb = (prefix[b + 1] - pre) / p.nhc;
+    const long long seg0 = pre + (long long)hc * ntb, seg1 = seg0 + ntb;
+    const bool complete = seg0 >= t0 && seg1 <= t1;
+    if (complete) {
+        if (ts == 0) {
+#pragma unroll
+            for (int pv = 0; pv < NT; ++pv)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int col = 2 * c + q;
+                    const float sc = __shfl_sync(kFullMask, st.S[pv], 4 * col);
+                    const int hg = slice * 16 + pv * 8 + col;
+                    if (hg < p.G) {
+                        const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
+                        float *dst = p.out + ((long long)b * p.Hq + h) * kD + 16 * g;
+                        store_row16(dst, st, pv, q, sc > 0.f ? 1.0f / sc : 0.f);
+                    }
+                }
+        }
+        return;
+    }
+
+    // partial: this CTA's share of the segment goes to its workspace slot
+    const int me = blockIdx.x;
+    const int which = (seg0 <= t0) ? 0 : 1;
+    const int H = p.heads_seg;
+    const size_t stride = (size_t)H * (kD + 2);
+    if (ts == 0) {
+        float *slotp = p.partials + (size_t)(2 * me + which) * stride;
+#pragma unroll
+        for (int pv = 0; pv < NT; ++pv)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int hg = slice * 16 + pv * 8 + 2 * c + q;
+                if (hg < p.G)
+                    store_row16(slotp + (size_t)(kl * p.G + hg) * kD + 16 * g, st, pv, q, 1.0f);
+            }
+        if (c == 0) {
+#pragma unroll
+            for (int r = 0; r < NT; ++r) {
+                const int hg = slice * 16 + r * 8 + g;
+                if (hg < p.G) {
+                    slotp[(size_t)H * kD + kl * p.G + hg] = st.M[r];
+                    slotp[(size_t)H * kD + H + kl * p.G + hg] = st.S[r];
+                }
+            }
+        }
+    }
+    __threadfence();
+    consumer_bar();
+
+    const int first = cta_of_tile(seg0, N, gcta), last = cta_of_tile(seg1 - 1, N, gcta);
+    const int n = last - first + 1;
+    auto which_of = [&](int i) { return (seg0 <= cta_start(i, N, gcta)) ? 0 : 1; };
+    int *segc = p.seg_counters + (long long)b * p.nhc + hc;
+    if (n <= kGroupFanIn) {
+        if (ctid == 0)
+            misc[1] = (atomicAdd(segc, 1) == n - 1) ? 1 : 0;
+        consumer_bar();
+        const bool last_in = misc[1] != 0;
+        consumer_bar();
+        if (last_in) {
+            __threadfence();
+            merge_slots(p, n, [&](int k) { return (size_t)(2 * (first + k) + which_of(first + k)); },
+                        true, b, hc, 0, ctid);
+            if (ctid == 0)
+                *segc = 0;
+        }
+        return;
+    }
+    const int ngroups = (n + kGroupFanIn - 1) / kGroupFanIn;
+    const int leader = first + ((me - first) / kGroupFanIn) * kGroupFanIn;
+    const int gsize = min(kGroupFanIn, last + 1 - leader);
+    const int lslot = 2 * leader + which_of(leader);
+    if (ctid == 0)
+        misc[1] = (atomicAdd(p.grp_counters + lslot, 1) == gsize - 1) ? 1 : 0;
+    consumer_bar();
+    const bool grp_last = misc[1] != 0;
+    consumer_bar();
+    if (!grp_last)
+        return;
+    __threadfence();
+    merge_slots(p, gsize, [&](int k) { return (size_t)(2 * (leader + k) + which_of(leader + k)); },
+                false, b, hc, lslot, ctid);
+    __threadfence();
+    consumer_bar();
+    if (ctid == 0) {
+        p.grp_counters[lslot] = 0;
+        misc[1] = (atomicAdd(segc, 1) == ngroups - 1) ? 1 : 0;
+    }
+    consumer_bar();
+    const bool seg_last = misc[1] != 0;
+    consumer_bar();
+    if (seg_last) {
+        __threadfence();
+        merge_slots(p, ngroups,
+                    [&](int k) {
+                        const int ld = first + k * kGroupFanIn;
+                        return (size_t)(2 * ld + which_of(ld));
+                    },
+                    true, b, hc, 0, ctid);
+        if (ctid == 0)
+            *segc = 0;
+    }
+}
+
+// The consumer's view of the flat tile list: which sequence / head chunk tile x is.
+// Consumers derive it from the prefix sums themselves, so their control flow (and every
+// named barrier they take) never depends on data arriving.
+struct SegCursor {
+    int b, hc, ntb, L;
+    long long seg0, seg1;
+};
+
+__device__ __forceinline__ void cursor_at(const DecodeParams &p, const int *prefix, long long x,
+                                          SegCursor &cu)
+{
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= x)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    cu.b = lo;
+    const int pre = prefix[lo];
+    cu.ntb = (prefix[lo + 1] - pre) / p.nhc;
+    cu.hc = (int)((x - pre) / cu.ntb);
+    cu.seg0 = pre + (long long)cu.hc * cu.ntb;
+    cu.seg1 = cu.seg0 + cu.ntb;
+    cu.L = clamp_len(__ldg(p.seq_lens + lo), p.mbps * p.bs);
+}
+
+template <int NT, bool kDump>
+__device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix, long long t0,
+                        long long t1, long long N, int gcta, int warp, int lane)
+{
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
+    const int pair = warp % p.pairs, ts = warp / p.pairs;
+    const int kl = pair / p.slices, slice = pair % p.slices;
+    const int g = lane >> 2, c = lane & 3;
+    const ThreadOffsets o = make_offsets(p, kl, ts, g, c);
+    const uint32_t sm0 = smem_addr(smem);
+    WarpState<NT> st;
+    reset_state(st);
+#pragma unroll
+    for (int j = 0; j < kNB; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            st.qa[j][k] = 0u;
+#pragma unroll
+    for (int r = 0; r < NT; ++r)
+#pragma unroll
+        for (int j = 0; j < kNB; ++j)
+            st.qs[r][j] = 0.f;
+
+    SegCursor cu;
+    cursor_at(p, prefix, t0, cu);
+    bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
+    int stage = 0;
+    uint32_t phase = 0;
+    for (long long x = t0; x < t1; ++x) {
+        if (x >= cu.seg1)
+            cursor_at(p, prefix, x, cu);
+        const bool seg_first = x == (cu.seg0 > t0 ? cu.seg0 : t0);
+        const bool seg_last = x + 1 == (cu.seg1 < t1 ? cu.seg1 : t1);
+        const int tok0 = (int)(x - cu.seg0) * p.TT;
+        const int nvalid = min(p.TT, cu.L - tok0);
+        if (seg_first) {
+            load_query(p, st, cu.b, cu.hc, kl, slice, g, c);
+            reset_state(st);
+        }
+        if (!dead && !mbar_wait(&full[stage], phase, globaltimer_ns() + kWaitLimitNs)) {
+            dead = true;
+            atomicOr(p.errors, kErrTimeout);
+        }
+        if (!dead) {
+            const int loaded = reinterpret_cast<volatile int *>(smem + p.lay.off_mask)[stage];
+            process_stage<NT, kDump>(p, st, o, sm0 + (uint32_t)stage * p.lay.stage_bytes, nvalid,
+                                     loaded, cu.b, cu.hc, kl, slice, tok0, g, c);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[stage]);
+        }
+        if (seg_last)
+            finalize_segment(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c, warp * 32 + lane,
+                             prefix, t0, t1, N, gcta);
+        if (++stage == p.n_stages) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
+template <int NT, bool kDump>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKs,
+                  const __grid_constant__ CUtensorMap tmVs)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
+    int *prefix = reinterpret_cast<int *>(smem + p.lay.off_prefix);
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + p.lay.off_misc);
+
+    if (tid == 0) {
+        for (int s = 0; s < p.n_stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        if (!p.scale_bulk) {
+            tma_prefetch_desc(&tmKs);
+            tma_prefetch_desc(&tmVs);
+        }
+    }
+    build_prefix(p, prefix, misc + 2, tid, warp, lane);
+    __syncthreads();
+
+    const long long N = prefix[p.B];
+    // rows of empty sequences are zero
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+        if (prefix[b + 1] != prefix[b])
+            continue;
+        float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
+        for (int i = tid; i < p.Hq * kD / 4; i += kThreads)
+            row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int gcta = (int)(N < (long long)gridDim.x ? N : (long long)gridDim.x);
+    if ((int)blockIdx.x >= gcta)
+        return;
+    const long long t0 = cta_start(blockIdx.x, N, gcta), t1 = cta_start(blockIdx.x + 1, N, gcta);
+    if (warp == kProducerWarp)
+        produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
+    else
+        consume<NT, kDump>(p, smem, prefix, t0, t1, N, gcta, warp, lane);
+}
+
+} // namespace q8kv

@@ -1,0 +1,162 @@
+/*
+ * q8kv.h -- C ABI of the q8-KV single-query decode-attention library for NVIDIA B200
+ * (sm_100a). Shared library: decode_attention_int8_b200/libq8kv.so.
+ *
+ * The operation (Kestrel-LLM walk-through "flash_attn_single_q_q8_neon",
+ * trdm.cn/news/511694, section 2 parts 1-3): for every batch entry b and query head h,
+ *   1. quantise q[b][h] once to int8 in 32-element blocks: qm = max|q| (if qm < 1e-6 then
+ *      qm = 1), qsc_j = qm * fl(1/127), code = clamp(round-half-to-even(q * fl(127/qm)),
+ *      -127, 127), all in IEEE fp32;
+ *   2. for every token t < seq_lens[b], with kv = h / (n_q_heads / n_kv_heads) (the GQA
+ *      mapping of the llama2.c loop, aicoding.csdn.net, "attention core logic") and
+ *      slot = block_table[b][t / kv_block_size] * kv_block_size + t % kv_block_size
+ *      (beaiera.top "deepseek-attention-div64", "Top-K index global mapping"):
+ *        dot_j = sum over the 32 channels of block j of code * K[slot][kv]   (int32, exact)
+ *        s_t   = (sum_j dot_j * qsc_j) * kscale[slot][kv] * scale
+ *   3. out[b][h] = sum_t exp(s_t - M) * vscale[slot][kv] * V[slot][kv] / sum_t exp(s_t - M),
+ *      computed in one pass with a running max M and running sum S (online softmax) and
+ *      one division at the end.
+ * The scan is split over the sequence across thread blocks (flash-decoding) and the
+ * pieces are merged with a log-sum-exp combine inside the same launch; the result equals
+ * the single pass up to fp32 rounding order.
+ *
+ * Layouts (all row-major, C order):
+ *   q            fp32  [B][n_q_heads][head_dim]
+ *   out          fp32  [B][n_q_heads][head_dim]
+ *   k_blocks     int8  [num_kv_blocks][kv_block_size][n_kv_heads][head_dim]
+ *   v_blocks     int8  same shape as k_blocks
+ *   kscale       fp32  [num_kv_blocks][kv_block_size][n_kv_heads]  (dequant multipliers:
+ *   vscale       fp32  same shape                                   value = code * scale)
+ *   block_table  int32 [B][max_blocks_per_seq]  physical block of each logical block;
+ *                      entries past ceil(seq_lens[b] / kv_block_size) are never read
+ *   seq_lens     int32 [B]
+ * The same block table indexes both pools and both scale arrays; scales are indexed by
+ * the physical slot.
+ *
+ * Pointers: device pointers owned by the caller; the library never frees or retains
+ * them. q, out, k_blocks, v_blocks, kscale, vscale must be 16-byte aligned (any torch or
+ * cudaMalloc allocation is).
+ *
+ * Asynchrony: every call enqueues work on `stream` (NULL = legacy default stream) and
+ * returns without synchronising. Q8KV_OK means the work was enqueued; faults surface at
+ * the caller's next synchronisation.
+ *
+ * Errors: argument checks run on the host before any launch and return
+ * Q8KV_ERR_INVALID_ARG or Q8KV_ERR_UNSUPPORTED without touching the GPU. Data that only
+ * the device can see is checked in the kernel without trapping: a seq_len below 0 is
+ * treated as 0, one above max_blocks_per_seq * kv_block_size is clamped, a block-table
+ * entry outside [0, num_kv_blocks) makes the kernel skip that block's tokens; each of
+ * these sets a bit in a device-side error word that q8kv_device_errors() reads.
+ *
+ * Supported shapes of the decode kernel: head_dim 128; kv_block_size a multiple of 16 in
+ * [16, 256]; n_q_heads a multiple of n_kv_heads with group n_q_heads / n_kv_heads <= 128;
+ * n_kv_heads <= 8, or a multiple of 4; B <= 16384; num_kv_blocks * kv_block_size < 2^31.
+ * Other shapes return Q8KV_ERR_UNSUPPORTED.
+ */
+#ifndef Q8KV_H
+#define Q8KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    Q8KV_OK = 0,
+    Q8KV_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad alignment, ... */
+    Q8KV_ERR_UNSUPPORTED = 2, /* valid arguments outside the shapes the kernels handle */
+    Q8KV_ERR_CUDA = 3,        /* a CUDA runtime call failed: see q8kv_last_cuda_error() */
+    Q8KV_ERR_WORKSPACE = 4    /* workspace null or smaller than q8kv_workspace_bytes() */
+} q8kv_status;
+
+/* Device-side error bits reported by q8kv_device_errors(). */
+#define Q8KV_DEVERR_SEQ_LEN 0x1u     /* a seq_len was negative or too long (clamped)     */
+#define Q8KV_DEVERR_BLOCK_TABLE 0x2u /* a block-table entry was outside the pool (skipped) */
+#define Q8KV_DEVERR_TIMEOUT 0x4u     /* a pipeline wait ran past its limit (kernel gave up) */
+
+/*
+ * Decode attention with a library-managed workspace (one per device, grown on demand
+ * under a lock, zero-initialised; the first call on a device, or a call that needs a
+ * larger workspace, allocates and so must not happen during stream capture). Calls that
+ * run concurrently on different streams of one device must use q8kv_decode_attn_ws with
+ * separate workspaces.
+ *
+ *   out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens: see the layouts above
+ *   B                  batch size (> 0)
+ *   n_q_heads          query heads (> 0, a multiple of n_kv_heads)
+ *   n_kv_heads         KV heads (> 0)
+ *   head_dim           channels per head (128)
+ *   kv_block_size      tokens per physical block
+ *   max_blocks_per_seq row stride of block_table; seq_lens[b] <= max_blocks_per_seq *
+ *                      kv_block_size
+ *   num_kv_blocks      physical blocks in each pool (bounds every block-table entry)
+ *   scale              softmax scale (finite; 1/sqrt(head_dim) in standard attention,
+ *                      beaiera.top "deepseek-attention-div64", "derivation of the scale")
+ */
+q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
+                             const int8_t *v_blocks, const float *kscale, const float *vscale,
+                             const int32_t *block_table, const int32_t *seq_lens, int B,
+                             int n_q_heads, int n_kv_heads, int head_dim, int kv_block_size,
+                             int max_blocks_per_seq, int num_kv_blocks, float scale,
+                             cudaStream_t stream);
+
+/* Bytes of workspace q8kv_decode_attn_ws needs for these sizes on the current device
+ * (0 if the sizes are invalid or unsupported). */
+size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim);
+
+/* Zero a caller-owned workspace (required once before its first use; the kernels leave
+ * it zeroed again after every complete call). */
+q8kv_status q8kv_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Same as q8kv_decode_attn with a caller-owned workspace (device memory of at least
+ * q8kv_workspace_bytes() bytes, 256-byte aligned, zeroed once by q8kv_workspace_init).
+ * The call allocates nothing. Calls that overlap on the GPU must not share a workspace. */
+q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_blocks,
+                                const int8_t *v_blocks, const float *kscale,
+                                const float *vscale, const int32_t *block_table,
+                                const int32_t *seq_lens, int B, int n_q_heads, int n_kv_heads,
+                                int head_dim, int kv_block_size, int max_blocks_per_seq,
+                                int num_kv_blocks, float scale, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
+/* Debug: the Q quantisation alone (step 1) on n_rows rows of head_dim fp32 values
+ * (head_dim a multiple of 32). qi int8 [n_rows][head_dim], qsc fp32
+ * [n_rows][head_dim / 32]. Uses the device routine the decode kernel uses. */
+q8kv_status q8kv_debug_quantize_q(int8_t *qi, float *qsc, const float *q, int n_rows,
+                                  int head_dim, cudaStream_t stream);
+
+/* Debug: the int32 block dot products of step 2, produced by the decode kernel itself
+ * (same staging and tensor-core fragments) and written out as
+ * dots int32 [B][n_q_heads][max_seq_len][head_dim / 32]; entries of tokens at or past
+ * seq_lens[b] are left untouched. max_seq_len must be >= every seq_lens[b]. Also writes
+ * `out` like q8kv_decode_attn. Uses the library-managed workspace. */
+q8kv_status q8kv_debug_block_dots(int32_t *dots, int max_seq_len, float *out, const float *q,
+                                  const int8_t *k_blocks, const int8_t *v_blocks,
+                                  const float *kscale, const float *vscale,
+                                  const int32_t *block_table, const int32_t *seq_lens, int B,
+                                  int n_q_heads, int n_kv_heads, int head_dim,
+                                  int kv_block_size, int max_blocks_per_seq, int num_kv_blocks,
+                                  float scale, cudaStream_t stream);
+
+/* Read (and, if clear != 0, reset) the device-side error word of the current device.
+ * Synchronises the device. */
+q8kv_status q8kv_device_errors(unsigned *flags, int clear);
+
+/* Static description of a status code. */
+const char *q8kv_status_string(q8kv_status status);
+
+/* The cudaError_t of the last failing CUDA call made by this library on this thread
+ * (0 if none). */
+int q8kv_last_cuda_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int q8kv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
