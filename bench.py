@@ -1,0 +1,392 @@
+"""Benchmark of q8-KV single-query decode attention on B200.
+
+One step = one q8kv_decode_attn call over one batch of the workload (the whole hot path:
+Q quantisation, paged K/V streaming, int8 block dots, online softmax, V accumulation,
+split combine), through the C ABI. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl reference]
+
+Metric: effective KV bandwidth = algorithmic bytes of one call / time per call, where the
+algorithmic bytes are every valid (token, KV head) K row, V row and both scales once, plus
+q read and out written in fp32, the used block-table entries and seq_lens.
+
+Timing: the KV pool is rotated over enough copies that their total exceeds 4x the L2 size,
+so every call streams from HBM; W untimed calls, then K calls bracketed by a barrier and a
+device synchronisation, timed with CUDA events on the launching stream; the maximum over
+ranks is reported. Under torchrun every rank runs its own copy of the workload on its own
+GPU (independent sequences, no collective on the data path): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "q8-KV decode attention: µs/call and effective KV GB/s (% of B200 HBM peak)"
+UNIT = "GB/s"
+DEFAULT_CONFIG = 1  # the batched GQA decode workload the metric is quoted on
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAK_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_PEAK_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples of one GPU while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def workload_config(w, n_copies, extra):
+    c = w.cfg
+    lens = w.seq_lens
+    d = {"workload": c.name, "B": c.B, "n_q_heads": c.n_q_heads, "n_kv_heads": c.n_kv_heads,
+         "head_dim": c.head_dim, "kv_block_size": c.block_size,
+         "seq_len": int(lens.max()) if lens.min() == lens.max() else
+         f"ragged {int(lens.min())}..{int(lens.max())} (sum {int(lens.sum())})",
+         "num_kv_blocks": w.num_blocks, "algorithmic_bytes": w.algorithmic_bytes(),
+         "l2": f"inputs larger than L2: KV pool rotated over {n_copies} copies "
+               f"({n_copies * (w.k.nbytes + w.v.nbytes + w.ks.nbytes + w.vs.nbytes) / 1e6:.0f} MB"
+               f" > {L2_BYTES / 1e6:.0f} MB L2)"}
+    d.update(extra)
+    return d
+
+
+def cpu_baseline(w, min_seconds=10.0):
+    """The oracle as it stands, single-threaded, on whole passes over the workload."""
+    import oracle
+
+    cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
+                              w.cfg.n_q_heads, w.scale)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_all(cache, w.q)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds:
+            break
+    gbs = w.algorithmic_bytes() * reps / dt / 1e9
+    return {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"whole workload ({w.cfg.B} sequences x {w.cfg.n_q_heads} heads), "
+                      f"{reps} passes, {dt:.1f} s, single-threaded C oracle"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, on this arm's workload and metric."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from decode_attention_int8_b200 import inputs
+    import numpy as np
+    import oracle
+
+    w = inputs.make(args.config)
+    cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
+                              w.cfg.n_q_heads, w.scale)
+    B, Hq = w.cfg.B, w.cfg.n_q_heads
+    pairs_all = [(b, h) for b in range(B) for h in range(Hq) if w.seq_lens[b] > 0]
+    # time one pair to size a step so that the whole run takes about two minutes
+    t = time.perf_counter()
+    oracle.decode_pairs(cache, w.q, pairs_all[:1])
+    per_pair = max(time.perf_counter() - t, 1e-5)
+    budget = min(2.0, 120.0 / max(1, args.steps + args.warmup))
+    n_pairs = int(max(1, min(len(pairs_all), budget / per_pair)))
+    rng = np.random.default_rng(0)
+
+    def step(i):
+        # a random sample of (sequence, head) rows; the workload's algorithmic bytes are
+        # counted pro rata to the rows done
+        sel = rng.choice(len(pairs_all), n_pairs, replace=False)
+        oracle.decode_pairs(cache, w.q, [pairs_all[j] for j in sel])
+        return n_pairs
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    done = 0
+    for i in range(args.steps):
+        done += step(i)
+    dt = time.perf_counter() - t0
+    frac = done / len(pairs_all)
+    gbs = w.algorithmic_bytes() * frac / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.cfg.name, "B": B, "n_q_heads": Hq,
+                       "n_kv_heads": w.cfg.n_kv_heads, "head_dim": w.cfg.head_dim,
+                       "kv_block_size": w.cfg.block_size},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{n_pairs} random (sequence, head) rows per step of "
+                                       f"{len(pairs_all)}; bytes counted pro rata"},
+            "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    world, rank, local = dist_env()
+    import numpy as np
+    import torch
+
+    import decode_attention_int8_b200 as q8
+    from decode_attention_int8_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    w = inputs.make(args.config)
+    lib = q8.lib()
+    algo = w.algorithmic_bytes()
+    pool_bytes = w.k.nbytes + w.v.nbytes + w.ks.nbytes + w.vs.nbytes
+    n_copies = max(2, math.ceil(4 * L2_BYTES / pool_bytes) + 1) if pool_bytes < 8 * L2_BYTES else 1
+    n_copies = min(n_copies, 64)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    q = t(w.q)
+    bt = t(w.block_table)
+    lens = t(w.seq_lens)
+    pools = [(t(w.k), t(w.v), t(w.ks), t(w.vs)) for _ in range(n_copies)]
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    c = w.cfg
+    geo = (c.B, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block_size, w.max_blocks_per_seq,
+           w.num_blocks)
+    P = lambda x: ctypes.c_void_p(x.data_ptr())
+    argsets = [(P(out), P(q), P(k), P(v), P(ks), P(vs), P(bt), P(lens), *geo,
+                ctypes.c_float(w.scale), sp) for (k, v, ks, vs) in pools]
+    fn = lib.q8kv_decode_attn
+
+    def call(i):
+        st = fn(*argsets[i % n_copies])
+        if st != 0:
+            raise q8.Q8KVError(st, "q8kv_decode_attn")
+
+    # warm-up (also sizes the library workspace outside the timed region)
+    for i in range(max(args.warmup, 1)):
+        call(i)
+    torch.cuda.synchronize(dev)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    # timed region: per-call CUDA events on the launching stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        call(i)
+        ends[i].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t_begin.elapsed_time(t_end)
+    per_call = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kernel_ms = statistics.fmean(per_call)
+    if pg is not None:
+        tt = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    value = algo * world / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the C ABI with host buffers: per step copy q / block table /
+    # seq_lens from pinned host memory, decode, copy out back (the KV cache stays resident)
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(w.q).pin_memory()
+        hbt = torch.from_numpy(w.block_table).pin_memory()
+        hlens = torch.from_numpy(w.seq_lens).pin_memory()
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        e2e_steps = max(10, min(args.steps, 2000))
+        for i in range(3):
+            q.copy_(hq, non_blocking=True)
+            call(i)
+            hout.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            q.copy_(hq, non_blocking=True)
+            bt.copy_(hbt, non_blocking=True)
+            lens.copy_(hlens, non_blocking=True)
+            call(i)
+            hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        if pg is not None:
+            tt = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": round(algo * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+               "h2d_bytes_per_step": int(w.q.nbytes + w.block_table.nbytes + w.seq_lens.nbytes),
+               "d2h_bytes_per_step": int(w.q.nbytes), "us_per_step": round(e2e_ms * 1e3, 3),
+               "steps": e2e_steps}
+
+    peak, peak_kind = measured_peak()
+    achieved = algo / (kernel_ms * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                tinfo = json.load(f)
+            ent = tinfo.get(c.name)
+            if ent and ent.get("kernel_source_hash") == source_hash():
+                traffic = ent["bytes_per_launch"]
+        except Exception:
+            traffic = None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "us_per_call": round(ms_per_step * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+        "config": workload_config(w, n_copies, {"parallelism": f"replicas{world}"}),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
+                     "traffic": traffic, "kernel": "q8kv::decode_kernel",
+                     "kernel_us": round(kernel_ms * 1e3, 3)},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def source_hash() -> str:
+    """Hash of the kernel sources (traffic figures are valid only for the exact kernel)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_attention_int8_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -141,17 +141,20 @@ q8kv_status plan_heads(int Hq, int Hk, int D, Plan &pl)
     pl.subtiles = kConsumerWarps / pl.pairs;
     pl.TT = 16 * pl.subtiles;
     pl.heads_seg = pl.HPC * pl.G;
-    pl.scratch_stride = 32 * 32 * pl.NT + 32;
+    pl.scratch_stride = 32 * 32 * pl.NT + 48; // acc fragments + M, S, A of 16 heads
     return Q8KV_OK;
 }
 
-void plan_workspace(int B, int grid, Plan &pl)
+// Workspace: segment counters and group counters (2 per CTA each, at fixed offsets that do
+// not depend on the shape, so a workspace can serve calls of any shape), then the partial
+// slots (2 per CTA).
+void plan_workspace(int grid, Plan &pl)
 {
     pl.ws_seg_off = 0;
-    pl.ws_grp_off = align256(sizeof(int) * (size_t)B * pl.nhc);
+    pl.ws_grp_off = align256(sizeof(int) * 2 * (size_t)grid);
     pl.ws_part_off = pl.ws_grp_off + align256(sizeof(int) * 2 * (size_t)grid);
     pl.ws_bytes = pl.ws_part_off +
-                  align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * (kD + 2));
+                  align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * (kD + kSlotExtra));
 }
 
 q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
@@ -185,7 +188,7 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     const long long tiles_per_seq = ((long long)s.mbps * s.bs + pl.TT - 1) / pl.TT;
     const long long tiles_max = (long long)s.B * pl.nhc * tiles_per_seq;
     pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
-    plan_workspace(s.B, dev.sms, pl); // sized for the full grid so one size fits all calls
+    plan_workspace(dev.sms, pl); // sized for the full grid so one size fits all calls
     return Q8KV_OK;
 }
 
@@ -399,7 +402,7 @@ size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim)
         if (device_info(&dev) != Q8KV_OK)
             return 0;
     }
-    plan_workspace(B, dev->sms, pl);
+    plan_workspace(dev->sms, pl);
     return pl.ws_bytes;
 }
 

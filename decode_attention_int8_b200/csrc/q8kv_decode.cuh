@@ -20,12 +20,15 @@
 //    subtile). QK is an int8 tensor-core MMA (m16n8k32, one MMA per 32-channel quant
 //    block, so each MMA result is exactly one int32 block dot). PV is an f16 MMA
 //    (m16n8k16) on exact f16 copies of the int8 V codes with the fp32 weights split into
-//    hi + lo f16 halves (about 22 significant bits), pre-scaled by a power of two that
-//    tracks the largest V scale seen so the halves stay in the f16 normal range.
-//  * The online softmax runs per 16-token subtile in base 2; per-warp states are merged
-//    in shared memory, and CTAs that share a sequence merge their partial (M, S, acc)
-//    through the workspace with a two-level last-arriver log-sum-exp combine (no waiting
-//    on other CTAs, counters reset by the last arriver).
+//    hi + lo f16 halves (about 22 significant bits).
+//  * The online softmax runs per 16-token subtile in base 2. The denominator S keeps the
+//    softmax running max M; the V accumulator keeps its own running max A of
+//    (score + log2 V scale), so the weight * V scale that enters the f16 halves is at
+//    most 2^15 and the largest one is at least 2^14 (full f16 precision whatever the
+//    spread of the V scales). Both are ordinary online maxima: rescale when they rise.
+//  * Per-warp states are merged in shared memory, and CTAs that share a sequence merge
+//    their partial (M, S, A, acc) through the workspace with a two-level last-arriver
+//    log-sum-exp combine (no waiting on other CTAs, counters reset by the last arriver).
 #pragma once
 
 #include <cuda.h>
@@ -47,7 +50,8 @@ constexpr int kMaxBoxes = 8;        // TMA boxes per stage
 constexpr int kGroupFanIn = 8;      // contributors merged per first-level combine
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
-constexpr int kEMin = 15;           // smallest biased exponent used for the V-scale window
+constexpr int kSlotExtra = 3;       // per-head M, S, A after the kD accumulator floats
+constexpr float kVExpLimit = 100.f; // V-scale exponents are clamped to [-100, 100]
 
 // Device-side error bits (match Q8KV_DEVERR_* in q8kv.h).
 constexpr unsigned kErrSeqLen = 0x1u;
@@ -102,9 +106,9 @@ struct DecodeParams {
     const int32_t *seq_lens;
     const float *kscale;
     const float *vscale;
-    float *partials;     // [2 * grid][heads_seg][kD + 2]
-    int *seg_counters;   // [B * nhc]
-    int *grp_counters;   // [2 * grid]
+    float *partials;     // [2 * grid slots] x heads_seg x (kD acc | M | S | A)
+    int *seg_counters;   // [2 * grid], indexed by the slot of a segment's first contributor
+    int *grp_counters;   // [2 * grid], indexed by the slot of a group leader
     unsigned *errors;    // device error word
     int32_t *dbg_dots;   // [B][Hq][dbg_max_len][kNB] (debug instantiation only)
     int dbg_max_len;
@@ -144,44 +148,51 @@ __device__ __forceinline__ long long cta_start(int i, long long N, int g)
     return (long long)i * N / g;
 }
 
-// Merge partial (M, S, acc) slots into either the output rows of (b, hc) or one slot.
+// Merge partial (M, S, A, acc) slots into either the output rows of (b, hc) or one slot.
 // slot_k(k) gives the slot index of the k-th input. Called by all consumer threads.
+// Slot layout: acc [H][kD] (units 2^-A), then M [H], S [H], A [H] (base-2 logs).
 template <typename SlotFn>
 __device__ void merge_slots(const DecodeParams &p, int n_in, SlotFn slot_k, bool to_out, int b,
                             int hc, int dest_slot, int ctid)
 {
     const int H = p.heads_seg;
-    const size_t stride = (size_t)H * (kD + 2);
+    const size_t stride = (size_t)H * (kD + kSlotExtra);
+    const size_t oM = (size_t)H * kD, oS = oM + H, oA = oS + H;
     for (int u = ctid; u < H * (kD / 4); u += kConsumerThreads) {
         const int hl = u / (kD / 4), d4 = u % (kD / 4);
-        float mx = -INFINITY;
-        for (int k = 0; k < n_in; ++k)
-            mx = fmaxf(mx, ldcg_f(p.partials + slot_k(k) * stride + (size_t)H * kD + hl));
+        float mx = -INFINITY, ax = -INFINITY;
+        for (int k = 0; k < n_in; ++k) {
+            const float *base = p.partials + slot_k(k) * stride;
+            mx = fmaxf(mx, ldcg_f(base + oM + hl));
+            ax = fmaxf(ax, ldcg_f(base + oA + hl));
+        }
         float ssum = 0.f;
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < n_in; ++k) {
             const float *base = p.partials + slot_k(k) * stride;
-            const float mk = ldcg_f(base + (size_t)H * kD + hl);
-            const float f = (mk == -INFINITY) ? 0.f : exp2f(mk - mx);
-            ssum += f * ldcg_f(base + (size_t)H * kD + H + hl);
+            const float mk = ldcg_f(base + oM + hl), ak = ldcg_f(base + oA + hl);
+            const float fs = (mk == -INFINITY) ? 0.f : exp2f(mk - mx);
+            const float fa = (ak == -INFINITY) ? 0.f : exp2f(ak - ax);
+            ssum += fs * ldcg_f(base + oS + hl);
             const float4 v = ldcg_f4(base + (size_t)hl * kD + d4 * 4);
-            a.x += f * v.x;
-            a.y += f * v.y;
-            a.z += f * v.z;
-            a.w += f * v.w;
+            a.x += fa * v.x;
+            a.y += fa * v.y;
+            a.z += fa * v.z;
+            a.w += fa * v.w;
         }
         if (to_out) {
-            const float inv = ssum > 0.f ? 1.0f / ssum : 0.f;
+            const float f = ssum > 0.f ? exp2f(ax - mx) / ssum : 0.f;
             const long long h = (long long)hc * H + hl;
-            float4 o = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+            float4 o = make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
             *reinterpret_cast<float4 *>(p.out + ((long long)b * p.Hq + h) * kD + d4 * 4) = o;
         } else {
             float *base = p.partials + (size_t)dest_slot * stride;
             __syncwarp();
             *reinterpret_cast<float4 *>(base + (size_t)hl * kD + d4 * 4) = a;
             if (d4 == 0) {
-                base[(size_t)H * kD + hl] = mx;
-                base[(size_t)H * kD + H + hl] = ssum;
+                base[oM + hl] = mx;
+                base[oS + hl] = ssum;
+                base[oA + hl] = ax;
             }
         }
     }
@@ -361,9 +372,9 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
 template <int NT>
 struct WarpState {
     float acc[NT][8][4]; // PV accumulator fragments (columns = heads, rows = channels)
-    float M[NT];         // running max (base 2) of this lane's QK row head
-    float S[NT];         // this lane's share of the running sum
-    int E;               // V-scale exponent window (biased exponent of max V scale seen)
+    float M[NT];         // softmax running max (base 2) of this lane's QK row head
+    float S[NT];         // this lane's share of the running sum (units 2^-M)
+    float A[NT];         // accumulator running max of score + log2(V scale) - 14
     uint32_t qa[kNB][4]; // int8 A fragments of the quantised query heads
     float qs[NT][kNB];   // Q block scales of rows g and g + 8
 };
@@ -422,13 +433,13 @@ __device__ __forceinline__ void reset_state(WarpState<NT> &st)
     for (int pv = 0; pv < NT; ++pv) {
         st.M[pv] = -INFINITY;
         st.S[pv] = 0.f;
+        st.A[pv] = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 st.acc[pv][i][k] = 0.f;
     }
-    st.E = kEMin;
 }
 
 // Per-thread shared-memory offsets that are the same for every stage.
@@ -517,7 +528,7 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
         }
     }
     // ---- per-token K and V scales; masking of tokens past the sequence end
-    float kss[2][2], vsv[2][2];
+    float kss[2][2], vsv[2][2], vex[2][2];
     bool val[2][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -527,12 +538,18 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
             kss[nt][e] = lds_f32(sbase + p.lay.off_ks + o.s[nt][e]) * p.scale_log2;
             const float vv = lds_f32(sbase + p.lay.off_vs + o.s[nt][e]);
             vsv[nt][e] = val[nt][e] ? vv : 0.f;
+            // floor(log2 |vs|) from the exponent field, clamped to [-100, 100]
+            const float ex = (float)((int)((__float_as_uint(vv) >> 23) & 0xffu) - 127);
+            vex[nt][e] = fminf(fmaxf(ex, -kVExpLimit), kVExpLimit);
         }
-    // ---- online softmax (base 2), blockwise over the 16 tokens
-    float alpha[NT];
+    // ---- online softmax (base 2), blockwise over the 16 tokens. M: running max of the
+    // scores (denominator). A: running max of score + log2(vs) - 14 (numerator), so that
+    // every weight * vs * 2^(M - A) entering the f16 MMA is below 2^15.
+    float alpha_a[NT];
+    uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
     for (int r = 0; r < NT; ++r) {
-        float m = -INFINITY;
+        float m = -INFINITY, a = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -540,56 +557,46 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
                 const float v = val[nt][e] ? s[r][nt][e] * kss[nt][e] : -INFINITY;
                 s[r][nt][e] = v;
                 m = fmaxf(m, v);
+                a = fmaxf(a, v + vex[nt][e]);
             }
         m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
         m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
+        a = fmaxf(a, __shfl_xor_sync(kFullMask, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(kFullMask, a, 2));
         const float mn = fmaxf(st.M[r], m);
+        const float an = fmaxf(st.A[r], a - 14.f);
         const float ms = (mn == -INFINITY) ? 0.f : mn;
-        alpha[r] = exp2f(st.M[r] - ms);
+        const float as = (an == -INFINITY) ? 0.f : an;
+        const float alpha_s = exp2f(st.M[r] - ms);
+        alpha_a[r] = exp2f(st.A[r] - as);
         st.M[r] = mn;
+        st.A[r] = an;
+        const float cvs = exp2f(ms - as); // 2^(M - A), within [2^-86, 2^114]
         float ws = 0.f;
+        float pw[2][2];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const float w = exp2f(s[r][nt][e] - ms);
-                s[r][nt][e] = w;
                 ws += w;
+                pw[nt][e] = w * (vsv[nt][e] * cvs);
             }
-        st.S[r] = st.S[r] * alpha[r] + ws;
-    }
-    // ---- V-scale window: weights are scaled by 2^(141 - E) so that w * vs < 2^15
-    float vm = fmaxf(fmaxf(vsv[0][0], vsv[0][1]), fmaxf(vsv[1][0], vsv[1][1]));
-    vm = fmaxf(vm, __shfl_xor_sync(kFullMask, vm, 1));
-    vm = fmaxf(vm, __shfl_xor_sync(kFullMask, vm, 2));
-    const int et = max(kEMin, (int)(__float_as_uint(vm) >> 23));
-    int de = 0;
-    if (et > st.E) {
-        de = et - st.E;
-        st.E = et;
-    }
-    const float mult = exp2i(141 - st.E);
-    const float shrink = exp2i(-min(de, 126));
-    // ---- weights as split f16 B operands (column n = head g, k = token)
-    uint32_t bh[NT][2], bl[NT][2];
-#pragma unroll
-    for (int r = 0; r < NT; ++r) {
+        st.S[r] = st.S[r] * alpha_s + ws;
+        // weights as split f16 B operands (column n = head g, k = token)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            const float p0 = s[r][nt][0] * (vsv[nt][0] * mult);
-            const float p1 = s[r][nt][1] * (vsv[nt][1] * mult);
-            const __half2 h = __floats2half2_rn(p0, p1);
-            const float r0 = p0 - __low2float(h), r1 = p1 - __high2float(h);
+            const __half2 h = __floats2half2_rn(pw[nt][0], pw[nt][1]);
+            const float r0 = pw[nt][0] - __low2float(h), r1 = pw[nt][1] - __high2float(h);
             bh[r][nt] = *reinterpret_cast<const uint32_t *>(&h);
             bl[r][nt] = pack_f16x2(r0, r1);
         }
     }
-    // ---- rescale the accumulator when M rose or the V-scale window moved
+    // ---- rescale the accumulator columns whose A rose
 #pragma unroll
     for (int pv = 0; pv < NT; ++pv) {
-        const float fr = alpha[pv] * shrink;
-        const float f0 = __shfl_sync(kFullMask, fr, 8 * c);
-        const float f1 = __shfl_sync(kFullMask, fr, 8 * c + 4);
+        const float f0 = __shfl_sync(kFullMask, alpha_a[pv], 8 * c);
+        const float f1 = __shfl_sync(kFullMask, alpha_a[pv], 8 * c + 4);
         if (__any_sync(kFullMask, (f0 != 1.f) || (f1 != 1.f))) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -650,15 +657,6 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
         st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 1);
         st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 2);
     }
-    // undo the V-scale window: acc back to true units
-    const float unscale = exp2i(st.E - 141);
-#pragma unroll
-    for (int pv = 0; pv < NT; ++pv)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                st.acc[pv][i][k] *= unscale;
 
     // merge the token subtiles of each (KV head, slice) pair inside the CTA
     if (p.subtiles > 1) {
@@ -678,6 +676,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
                 for (int r = 0; r < NT; ++r) {
                     reg[32 * 32 * NT + r * 8 + g] = st.M[r];
                     reg[32 * 32 * NT + 16 + r * 8 + g] = st.S[r];
+                    reg[32 * 32 * NT + 32 + r * 8 + g] = st.A[r];
                 }
             }
         }
@@ -690,11 +689,11 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         const int col = 2 * c + q;
-                        const float mm = __shfl_sync(kFullMask, st.M[pv], 4 * col);
-                        const float mo = reg[32 * 32 * NT + pv * 8 + col];
-                        const float mn = fmaxf(mm, mo);
-                        const float fa = (mm == -INFINITY) ? 0.f : exp2f(mm - mn);
-                        const float fo = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+                        const float am = __shfl_sync(kFullMask, st.A[pv], 4 * col);
+                        const float ao = reg[32 * 32 * NT + 32 + pv * 8 + col];
+                        const float an = fmaxf(am, ao);
+                        const float fa = (am == -INFINITY) ? 0.f : exp2f(am - an);
+                        const float fo = (ao == -INFINITY) ? 0.f : exp2f(ao - an);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             st.acc[pv][i][q] = st.acc[pv][i][q] * fa +
@@ -709,11 +708,13 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
                 for (int r = 0; r < NT; ++r) {
                     const float mo = reg[32 * 32 * NT + r * 8 + g];
                     const float so = reg[32 * 32 * NT + 16 + r * 8 + g];
+                    const float ao = reg[32 * 32 * NT + 32 + r * 8 + g];
                     const float mn = fmaxf(st.M[r], mo);
                     const float fa = (st.M[r] == -INFINITY) ? 0.f : exp2f(st.M[r] - mn);
                     const float fo = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
                     st.S[r] = st.S[r] * fa + so * fo;
                     st.M[r] = mn;
+                    st.A[r] = fmaxf(st.A[r], ao);
                 }
             }
         }
@@ -732,11 +733,13 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
                 for (int q = 0; q < 2; ++q) {
                     const int col = 2 * c + q;
                     const float sc = __shfl_sync(kFullMask, st.S[pv], 4 * col);
+                    const float mc = __shfl_sync(kFullMask, st.M[pv], 4 * col);
+                    const float ac = __shfl_sync(kFullMask, st.A[pv], 4 * col);
                     const int hg = slice * 16 + pv * 8 + col;
                     if (hg < p.G) {
                         const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
                         float *dst = p.out + ((long long)b * p.Hq + h) * kD + 16 * g;
-                        store_row16(dst, st, pv, q, sc > 0.f ? 1.0f / sc : 0.f);
+                        store_row16(dst, st, pv, q, sc > 0.f ? exp2f(ac - mc) / sc : 0.f);
                     }
                 }
         }
@@ -747,7 +750,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
     const int me = blockIdx.x;
     const int which = (seg0 <= t0) ? 0 : 1;
     const int H = p.heads_seg;
-    const size_t stride = (size_t)H * (kD + 2);
+    const size_t stride = (size_t)H * (kD + kSlotExtra);
     if (ts == 0) {
         float *slotp = p.partials + (size_t)(2 * me + which) * stride;
 #pragma unroll
@@ -765,6 +768,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
                 if (hg < p.G) {
                     slotp[(size_t)H * kD + kl * p.G + hg] = st.M[r];
                     slotp[(size_t)H * kD + H + kl * p.G + hg] = st.S[r];
+                    slotp[(size_t)H * kD + 2 * H + kl * p.G + hg] = st.A[r];
                 }
             }
         }
@@ -775,7 +779,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
     const int first = cta_of_tile(seg0, N, gcta), last = cta_of_tile(seg1 - 1, N, gcta);
     const int n = last - first + 1;
     auto which_of = [&](int i) { return (seg0 <= cta_start(i, N, gcta)) ? 0 : 1; };
-    int *segc = p.seg_counters + (long long)b * p.nhc + hc;
+    int *segc = p.seg_counters + 2 * first + which_of(first);
     if (n <= kGroupFanIn) {
         if (ctid == 0)
             misc[1] = (atomicAdd(segc, 1) == n - 1) ? 1 : 0;
