@@ -154,7 +154,7 @@ void plan_workspace(int grid, Plan &pl)
     pl.ws_grp_off = align256(sizeof(int) * 2 * (size_t)grid);
     pl.ws_part_off = pl.ws_grp_off + align256(sizeof(int) * 2 * (size_t)grid);
     pl.ws_bytes = pl.ws_part_off +
-                  align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * (kD + kSlotExtra));
+                  align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * kSlotRow);
 }
 
 q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
@@ -169,13 +169,18 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     if (s.B > 16384 || (long long)s.P * s.bs >= (1LL << 31) ||
         (long long)s.mbps * s.bs >= (1LL << 31))
         return Q8KV_ERR_UNSUPPORTED;
+    const long long tiles_per_seq = ((long long)s.mbps * s.bs + pl.TT - 1) / pl.TT;
+    const long long tiles_max = (long long)s.B * pl.nhc * tiles_per_seq;
+    if (tiles_max >= (1LL << 31))
+        return Q8KV_ERR_UNSUPPORTED; // tile indices are 32-bit
+    pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
     pl.box_tok = pl.TT < s.bs ? pl.TT : s.bs;
     pl.log2_box = ilog2(pl.box_tok);
     pl.n_boxes = pl.TT / pl.box_tok;
     const int scratch_floats = (pl.subtiles - 1) * pl.pairs * pl.scratch_stride;
     pl.n_stages = 0;
     for (int n = kMaxStages; n >= 2; --n) {
-        SmemLayout L = make_layout(pl.TT, pl.HPC, n, s.B, scratch_floats);
+        SmemLayout L = make_layout(pl.TT, pl.HPC, n, s.B, scratch_floats, pl.grid);
         if ((size_t)L.total + 1024 <= (size_t)dev.smem_optin) {
             pl.n_stages = n;
             pl.lay = L;
@@ -185,9 +190,6 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     if (pl.n_stages == 0)
         return Q8KV_ERR_UNSUPPORTED;
     pl.smem_bytes = (size_t)pl.lay.total + 1024;
-    const long long tiles_per_seq = ((long long)s.mbps * s.bs + pl.TT - 1) / pl.TT;
-    const long long tiles_max = (long long)s.B * pl.nhc * tiles_per_seq;
-    pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
     plan_workspace(dev.sms, pl); // sized for the full grid so one size fits all calls
     return Q8KV_OK;
 }
@@ -197,7 +199,7 @@ bool aligned16(const void *p)
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
-q8kv_status encode_maps(const Shape &s, const Plan &pl, const int8_t *k, const int8_t *v,
+q8kv_status encode_maps_uncached(const Shape &s, const Plan &pl, const int8_t *k, const int8_t *v,
                         const float *ks, const float *vs, CUtensorMap *mk, CUtensorMap *mv,
                         CUtensorMap *mks, CUtensorMap *mvs)
 {
@@ -240,6 +242,57 @@ q8kv_status encode_maps(const Shape &s, const Plan &pl, const int8_t *k, const i
         if (r != CUDA_SUCCESS)
             return Q8KV_ERR_UNSUPPORTED;
     }
+    return Q8KV_OK;
+}
+
+// Tensor maps depend only on the pool pointers and the tiling; repeated calls on the same
+// cache reuse them (a small round-robin cache, guarded by g_mutex).
+struct MapKey {
+    const void *k, *v, *ks, *vs;
+    int Hk, bs, P, HPC, box_tok, scale_bulk;
+    bool operator==(const MapKey &o) const
+    {
+        return k == o.k && v == o.v && ks == o.ks && vs == o.vs && Hk == o.Hk && bs == o.bs &&
+               P == o.P && HPC == o.HPC && box_tok == o.box_tok && scale_bulk == o.scale_bulk;
+    }
+};
+
+struct MapEntry {
+    bool used = false;
+    MapKey key{};
+    CUtensorMap mk, mv, mks, mvs;
+};
+
+constexpr int kMapCache = 16;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+
+q8kv_status encode_maps(const Shape &s, const Plan &pl, const int8_t *k, const int8_t *v,
+                        const float *ks, const float *vs, CUtensorMap *mk, CUtensorMap *mv,
+                        CUtensorMap *mks, CUtensorMap *mvs)
+{
+    const MapKey key{k, v, ks, vs, s.Hk, s.bs, s.P, pl.HPC, pl.box_tok, pl.scale_bulk};
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (auto &e : g_maps) {
+        if (e.used && e.key == key) {
+            *mk = e.mk;
+            *mv = e.mv;
+            *mks = e.mks;
+            *mvs = e.mvs;
+            return Q8KV_OK;
+        }
+    }
+    q8kv_status st = encode_maps_uncached(s, pl, k, v, ks, vs, mk, mv, mks, mvs);
+    if (st != Q8KV_OK)
+        return st;
+    MapEntry &e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.used = true;
+    e.key = key;
+    e.mk = *mk;
+    e.mv = *mv;
+    e.mks = *mks;
+    e.mvs = *mvs;
     return Q8KV_OK;
 }
 

@@ -47,10 +47,10 @@ constexpr int kProducerWarp = 8;    // warp 8
 constexpr int kThreads = 9 * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMaxBoxes = 8;        // TMA boxes per stage
-constexpr int kGroupFanIn = 8;      // contributors merged per first-level combine
+constexpr int kGroupFanIn = 16;     // contributors merged per first-level combine
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
-constexpr int kSlotExtra = 3;       // per-head M, S, A after the kD accumulator floats
+constexpr int kSlotRow = kD + 4;    // per-head partial: kD accumulator floats, M, S, A, pad
 constexpr float kVExpLimit = 100.f; // V-scale exponents are clamped to [-100, 100]
 
 // Device-side error bits (match Q8KV_DEVERR_* in q8kv.h).
@@ -67,12 +67,12 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a)
 struct SmemLayout {
     uint32_t stage_bytes; // one ring slot: K | V | kscale | vscale
     uint32_t off_k, off_v, off_ks, off_vs; // within a slot
-    uint32_t off_full, off_empty, off_mask, off_misc, off_prefix, off_scratch;
+    uint32_t off_full, off_empty, off_mbar, off_mask, off_misc, off_cstart, off_prefix, off_scratch;
     uint32_t total; // bytes from the 1024-aligned base
 };
 
 __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages, int B,
-                                                  int scratch_floats)
+                                                  int scratch_floats, int grid)
 {
     SmemLayout L;
     const uint32_t kv = (uint32_t)(TT * HPC * kD);
@@ -87,10 +87,14 @@ __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages,
     o += 8 * kMaxStages;
     L.off_empty = o;
     o += 8 * kMaxStages;
+    L.off_mbar = o;
+    o += 8;
     L.off_mask = o;
     o += 4 * kMaxStages;
     L.off_misc = o;
     o += 64;
+    L.off_cstart = o;
+    o = align_up(o + 4u * (uint32_t)(grid + 1), 16);
     L.off_prefix = o;
     o = align_up(o + 4u * (uint32_t)(B + 1), 16);
     L.off_scratch = o;
@@ -106,7 +110,7 @@ struct DecodeParams {
     const int32_t *seq_lens;
     const float *kscale;
     const float *vscale;
-    float *partials;     // [2 * grid slots] x heads_seg x (kD acc | M | S | A)
+    float *partials;     // [2 * grid slots] x heads_seg x kSlotRow (kD acc, M, S, A, pad)
     int *seg_counters;   // [2 * grid], indexed by the slot of a segment's first contributor
     int *grp_counters;   // [2 * grid], indexed by the slot of a group leader
     unsigned *errors;    // device error word
@@ -137,64 +141,117 @@ __device__ __forceinline__ float4 ldcg_f4(const float *p)
     return __ldcg(reinterpret_cast<const float4 *>(p));
 }
 
-// CTA owning flat tile x when N tiles are split over g CTAs ([i*N/g, (i+1)*N/g)).
-__device__ __forceinline__ int cta_of_tile(long long x, long long N, int g)
+// CTA owning flat tile x: the largest i with cstart[i] <= x, where cstart[i] = i * N / g
+// (the table every CTA builds once, so no 64-bit division runs after the prologue).
+__device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
 {
-    return (int)(((x + 1) * g - 1) / N);
+    int lo = 0, hi = g - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cstart[mid] <= x)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
 }
 
-__device__ __forceinline__ long long cta_start(int i, long long N, int g)
-{
-    return (long long)i * N / g;
-}
-
-// Merge partial (M, S, A, acc) slots into either the output rows of (b, hc) or one slot.
-// slot_k(k) gives the slot index of the k-th input. Called by all consumer threads.
-// Slot layout: acc [H][kD] (units 2^-A), then M [H], S [H], A [H] (base-2 logs).
+// Merge n_in partial (M, S, A, acc) slots into either the output rows of (b, hc) or one
+// slot. slot_k(k) gives the slot index of the k-th input. A slot holds heads_seg rows of
+// kSlotRow floats: acc [kD] (units 2^-A), then M, S, A (base-2 logs, S in units 2^-M).
+// Runs after the main loop, when the stage ring is idle: one thread pulls every input row
+// of a chunk of heads into the ring with bulk copies (one round trip to L2), then all
+// consumer threads combine from shared memory. Called by all consumer threads.
 template <typename SlotFn>
-__device__ void merge_slots(const DecodeParams &p, int n_in, SlotFn slot_k, bool to_out, int b,
-                            int hc, int dest_slot, int ctid)
+__device__ void merge_slots(const DecodeParams &p, uint8_t *smem, uint32_t &mphase, int n_in,
+                            SlotFn slot_k, bool to_out, int b, int hc, int dest_slot, int ctid)
 {
     const int H = p.heads_seg;
-    const size_t stride = (size_t)H * (kD + kSlotExtra);
-    const size_t oM = (size_t)H * kD, oS = oM + H, oA = oS + H;
-    for (int u = ctid; u < H * (kD / 4); u += kConsumerThreads) {
-        const int hl = u / (kD / 4), d4 = u % (kD / 4);
-        float mx = -INFINITY, ax = -INFINITY;
-        for (int k = 0; k < n_in; ++k) {
-            const float *base = p.partials + slot_k(k) * stride;
-            mx = fmaxf(mx, ldcg_f(base + oM + hl));
-            ax = fmaxf(ax, ldcg_f(base + oA + hl));
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + p.lay.off_mbar);
+    float *buf = reinterpret_cast<float *>(smem);
+    const uint32_t row_bytes = kSlotRow * 4;
+    const uint32_t ring = (uint32_t)p.n_stages * p.lay.stage_bytes;
+    int hch = (int)(ring / ((uint32_t)n_in * row_bytes));
+    hch = hch < 1 ? 1 : (hch > H ? H : hch);
+    for (int h0 = 0; h0 < H; h0 += hch) {
+        const int hn = (H - h0) < hch ? (H - h0) : hch;
+        if (ctid == 0) {
+            // the partials were written by other CTAs through the generic proxy
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            mbar_arrive_expect_tx(mbar, (uint32_t)n_in * hn * row_bytes);
+            for (int k = 0; k < n_in; ++k)
+                bulk_load_plain(buf + (size_t)k * hn * kSlotRow,
+                                p.partials + ((size_t)slot_k(k) * H + h0) * kSlotRow,
+                                (uint32_t)hn * row_bytes, mbar);
         }
-        float ssum = 0.f;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < n_in; ++k) {
-            const float *base = p.partials + slot_k(k) * stride;
-            const float mk = ldcg_f(base + oM + hl), ak = ldcg_f(base + oA + hl);
-            const float fs = (mk == -INFINITY) ? 0.f : exp2f(mk - mx);
-            const float fa = (ak == -INFINITY) ? 0.f : exp2f(ak - ax);
-            ssum += fs * ldcg_f(base + oS + hl);
-            const float4 v = ldcg_f4(base + (size_t)hl * kD + d4 * 4);
-            a.x += fa * v.x;
-            a.y += fa * v.y;
-            a.z += fa * v.z;
-            a.w += fa * v.w;
-        }
-        if (to_out) {
-            const float f = ssum > 0.f ? exp2f(ax - mx) / ssum : 0.f;
-            const long long h = (long long)hc * H + hl;
-            float4 o = make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
-            *reinterpret_cast<float4 *>(p.out + ((long long)b * p.Hq + h) * kD + d4 * 4) = o;
-        } else {
-            float *base = p.partials + (size_t)dest_slot * stride;
+        if (!mbar_wait(mbar, mphase, kWaitLimitNs))
+            atomicOr(p.errors, kErrTimeout);
+        mphase ^= 1u;
+        // per head: maxima over the inputs, then each input's two factors (written over its
+        // M and S words) and the combined S (written over input 0's pad word)
+        const int warp = ctid >> 5, lane = ctid & 31;
+        for (int hl = warp; hl < hn; hl += kConsumerWarps) {
+            float m = -INFINITY, a = -INFINITY, sv = 0.f;
+            float *row = nullptr;
+            if (lane < n_in) {
+                row = buf + ((size_t)lane * hn + hl) * kSlotRow;
+                m = row[kD];
+                sv = row[kD + 1];
+                a = row[kD + 2];
+            }
+            float mx = m, ax = a;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, o));
+                ax = fmaxf(ax, __shfl_xor_sync(kFullMask, ax, o));
+            }
+            const float fs = (m == -INFINITY) ? 0.f : exp2f(m - mx);
+            const float fa = (a == -INFINITY) ? 0.f : exp2f(a - ax);
+            float ssum = fs * sv;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1)
+                ssum += __shfl_xor_sync(kFullMask, ssum, o);
             __syncwarp();
-            *reinterpret_cast<float4 *>(base + (size_t)hl * kD + d4 * 4) = a;
-            if (d4 == 0) {
-                base[oM + hl] = mx;
-                base[oS + hl] = ssum;
-                base[oA + hl] = ax;
+            if (row) {
+                row[kD] = fa; // factor of this input's accumulator
+                if (lane == 0) {
+                    row[kD + 1] = mx;
+                    row[kD + 2] = ax;
+                    row[kD + 3] = ssum;
+                }
             }
         }
+        consumer_bar();
+        for (int u = ctid; u < hn * (kD / 4); u += kConsumerThreads) {
+            const int hl = u / (kD / 4), d4 = u % (kD / 4);
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < kGroupFanIn; ++k) {
+                if (k < n_in) {
+                    const float *row = buf + ((size_t)k * hn + hl) * kSlotRow;
+                    const float fa = row[kD];
+                    const float4 v = *reinterpret_cast<const float4 *>(row + d4 * 4);
+                    a.x += fa * v.x;
+                    a.y += fa * v.y;
+                    a.z += fa * v.z;
+                    a.w += fa * v.w;
+                }
+            }
+            const float4 hdr = *reinterpret_cast<const float4 *>(buf + (size_t)hl * kSlotRow + kD);
+            const float mx = hdr.y, ax = hdr.z, ssum = hdr.w;
+            if (to_out) {
+                const float f = ssum > 0.f ? exp2f(ax - mx) / ssum : 0.f;
+                const int h = hc * H + h0 + hl;
+                float4 o = make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
+                *reinterpret_cast<float4 *>(p.out + ((long long)b * p.Hq + h) * kD + d4 * 4) = o;
+            } else {
+                float *row = p.partials + ((size_t)dest_slot * H + h0 + hl) * kSlotRow;
+                *reinterpret_cast<float4 *>(row + d4 * 4) = a;
+                if (d4 == 0)
+                    *reinterpret_cast<float4 *>(row + kD) = make_float4(mx, ssum, ax, 0.f);
+            }
+        }
+        consumer_bar(); // the ring is refilled for the next chunk
     }
 }
 
@@ -249,7 +306,7 @@ __device__ __forceinline__ int clamp_len(int L, int cap)
 
 __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUtensorMap *tmV,
                         const CUtensorMap *tmKs, const CUtensorMap *tmVs, uint8_t *smem,
-                        const int *prefix, long long t0, long long t1, int lane)
+                        const int *prefix, int t0, int t1, int lane)
 {
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
@@ -262,8 +319,8 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     uint32_t phase = 0, issued = 0, issued_par = 0;
     bool aborted = false;
 
-    for (long long xb = t0; xb < t1 && !aborted; xb += 32) {
-        const long long x = xb + lane;
+    for (int xb = t0; xb < t1 && !aborted; xb += 32) {
+        const int x = xb + lane;
         int hc = 0;
         int slot[kMaxBoxes];
 #pragma unroll
@@ -281,7 +338,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
             const int b = lo;
             const int pre = prefix[b];
             const int ntb = (prefix[b + 1] - pre) / p.nhc;
-            const int local = (int)(x - pre);
+            const int local = x - pre;
             hc = local / ntb;
             const int lt = local - hc * ntb;
             const int tok0 = lt * p.TT;
@@ -298,7 +355,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                 }
             }
         }
-        const int n = (int)((t1 - xb) < 32 ? (t1 - xb) : 32);
+        const int n = (t1 - xb) < 32 ? (t1 - xb) : 32;
         for (int i = 0; i < n; ++i) {
             const int hci = __shfl_sync(kFullMask, hc, i);
             int sl[kMaxBoxes];
@@ -307,7 +364,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                 sl[bx] = __shfl_sync(kFullMask, slot[bx], i);
             int ok = 1;
             if (lane == 0) {
-                if (!mbar_wait(&empty[stage], phase ^ 1u, globaltimer_ns() + kWaitLimitNs)) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, kWaitLimitNs)) {
                     ok = 0;
                     atomicOr(p.errors, kErrTimeout);
                 } else {
@@ -363,7 +420,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     if (lane == 0) {
         for (int s = 0; s < p.n_stages; ++s)
             if ((issued >> s) & 1u)
-                mbar_wait(&full[s], (issued_par >> s) & 1u, globaltimer_ns() + kWaitLimitNs);
+                mbar_wait(&full[s], (issued_par >> s) & 1u, kWaitLimitNs);
     }
 }
 
@@ -519,11 +576,12 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
                     }
                 }
             }
-            s[0][nt][0] += (float)d[0] * st.qs[0][j];
-            s[0][nt][1] += (float)d[1] * st.qs[0][j];
+            // |dot| <= 32 * 127 * 127 < 2^22: exact conversion
+            s[0][nt][0] += small_int_to_float(d[0]) * st.qs[0][j];
+            s[0][nt][1] += small_int_to_float(d[1]) * st.qs[0][j];
             if constexpr (NT == 2) {
-                s[NT - 1][nt][0] += (float)d[2] * st.qs[NT - 1][j];
-                s[NT - 1][nt][1] += (float)d[3] * st.qs[NT - 1][j];
+                s[NT - 1][nt][0] += small_int_to_float(d[2]) * st.qs[NT - 1][j];
+                s[NT - 1][nt][1] += small_int_to_float(d[3]) * st.qs[NT - 1][j];
             }
         }
     }
@@ -539,8 +597,7 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
             const float vv = lds_f32(sbase + p.lay.off_vs + o.s[nt][e]);
             vsv[nt][e] = val[nt][e] ? vv : 0.f;
             // floor(log2 |vs|) from the exponent field, clamped to [-100, 100]
-            const float ex = (float)((int)((__float_as_uint(vv) >> 23) & 0xffu) - 127);
-            vex[nt][e] = fminf(fmaxf(ex, -kVExpLimit), kVExpLimit);
+            vex[nt][e] = fminf(fmaxf(exponent_as_float(vv), -kVExpLimit), kVExpLimit);
         }
     // ---- online softmax (base 2), blockwise over the 16 tokens. M: running max of the
     // scores (denominator). A: running max of score + log2(vs) - 14 (numerator), so that
@@ -643,14 +700,20 @@ __device__ __forceinline__ void store_row16(float *dst, const WarpState<NT> &st,
     }
 }
 
+// Segments of this CTA that other CTAs share (at most two), combined after the main loop.
+struct Pending {
+    struct Seg {
+        int b, hc, seg0, seg1;
+    } seg[2];
+    int n;
+};
+
 // End of a segment (all of this CTA's tiles of sequence b, head chunk hc).
 template <int NT>
 __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8_t *smem, int b,
                                  int hc, int kl, int slice, int pair, int ts, int g, int c,
-                                 int ctid, const int *prefix, long long t0, long long t1,
-                                 long long N, int gcta)
+                                 int ctid, const int *prefix, int t0, int t1, Pending &pend)
 {
-    volatile int *misc = reinterpret_cast<volatile int *>(smem + p.lay.off_misc);
     // complete this lane's row sums
 #pragma unroll
     for (int r = 0; r < NT; ++r) {
@@ -723,7 +786,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
 
     const int pre = prefix[b];
     const int ntb = (prefix[b + 1] - pre) / p.nhc;
-    const long long seg0 = pre + (long long)hc * ntb, seg1 = seg0 + ntb;
+    const int seg0 = pre + hc * ntb, seg1 = seg0 + ntb;
     const bool complete = seg0 >= t0 && seg1 <= t1;
     if (complete) {
         if (ts == 0) {
@@ -746,88 +809,120 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
         return;
     }
 
-    // partial: this CTA's share of the segment goes to its workspace slot
-    const int me = blockIdx.x;
+    // partial: this CTA's share of the segment goes to its workspace slot; the cross-CTA
+    // combine runs after the main loop (combine_pending)
     const int which = (seg0 <= t0) ? 0 : 1;
     const int H = p.heads_seg;
-    const size_t stride = (size_t)H * (kD + kSlotExtra);
     if (ts == 0) {
-        float *slotp = p.partials + (size_t)(2 * me + which) * stride;
+        float *slotp = p.partials + (size_t)(2 * blockIdx.x + which) * H * kSlotRow;
 #pragma unroll
         for (int pv = 0; pv < NT; ++pv)
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int hg = slice * 16 + pv * 8 + 2 * c + q;
                 if (hg < p.G)
-                    store_row16(slotp + (size_t)(kl * p.G + hg) * kD + 16 * g, st, pv, q, 1.0f);
+                    store_row16(slotp + (size_t)(kl * p.G + hg) * kSlotRow + 16 * g, st, pv, q,
+                                1.0f);
             }
         if (c == 0) {
 #pragma unroll
             for (int r = 0; r < NT; ++r) {
                 const int hg = slice * 16 + r * 8 + g;
-                if (hg < p.G) {
-                    slotp[(size_t)H * kD + kl * p.G + hg] = st.M[r];
-                    slotp[(size_t)H * kD + H + kl * p.G + hg] = st.S[r];
-                    slotp[(size_t)H * kD + 2 * H + kl * p.G + hg] = st.A[r];
-                }
+                if (hg < p.G)
+                    *reinterpret_cast<float4 *>(slotp + (size_t)(kl * p.G + hg) * kSlotRow + kD) =
+                        make_float4(st.M[r], st.S[r], st.A[r], 0.f);
             }
         }
     }
+    pend.seg[pend.n].b = b;
+    pend.seg[pend.n].hc = hc;
+    pend.seg[pend.n].seg0 = seg0;
+    pend.seg[pend.n].seg1 = seg1;
+    ++pend.n;
+}
+
+// Cross-CTA combine of this CTA's partial segments (at most two: the one it started in
+// and the one it ended in). Every contributor bumps a counter; the last one to arrive
+// merges (for more than kGroupFanIn contributors: per group of kGroupFanIn, then the
+// groups). Counters live in the workspace and are reset by the last arriver, so no CTA
+// ever waits for another.
+__device__ void combine_pending(const DecodeParams &p, uint8_t *smem, const Pending &pend,
+                                const int *cstart, int gcta, int ctid)
+{
+    if (pend.n == 0)
+        return;
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + p.lay.off_misc);
+    uint32_t mphase = 0;
     __threadfence();
     consumer_bar();
-
-    const int first = cta_of_tile(seg0, N, gcta), last = cta_of_tile(seg1 - 1, N, gcta);
-    const int n = last - first + 1;
-    auto which_of = [&](int i) { return (seg0 <= cta_start(i, N, gcta)) ? 0 : 1; };
-    int *segc = p.seg_counters + 2 * first + which_of(first);
-    if (n <= kGroupFanIn) {
-        if (ctid == 0)
-            misc[1] = (atomicAdd(segc, 1) == n - 1) ? 1 : 0;
+    int first[2], last[2], n[2], ctr[2];
+    int *cnt[2];
+    for (int i = 0; i < pend.n; ++i) {
+        const Pending::Seg &sg = pend.seg[i];
+        first[i] = cta_of_tile(cstart, gcta, sg.seg0);
+        last[i] = cta_of_tile(cstart, gcta, sg.seg1 - 1);
+        n[i] = last[i] - first[i] + 1;
+        const int f = first[i];
+        if (n[i] <= kGroupFanIn) {
+            cnt[i] = p.seg_counters + 2 * f + ((sg.seg0 <= cstart[f]) ? 0 : 1);
+            ctr[i] = n[i];
+        } else {
+            const int leader = f + (((int)blockIdx.x - f) / kGroupFanIn) * kGroupFanIn;
+            cnt[i] = p.grp_counters + 2 * leader + ((sg.seg0 <= cstart[leader]) ? 0 : 1);
+            ctr[i] = min(kGroupFanIn, last[i] + 1 - leader);
+        }
+    }
+    if (ctid == 0) {
+        int tk[2] = {0, 0};
+        for (int i = 0; i < pend.n; ++i)
+            tk[i] = atomicAdd(cnt[i], 1);
+        for (int i = 0; i < pend.n; ++i)
+            misc[1 + i] = (tk[i] == ctr[i] - 1) ? 1 : 0;
+    }
+    consumer_bar();
+    int is_last[2] = {misc[1], pend.n > 1 ? misc[2] : 0};
+    consumer_bar();
+    for (int i = 0; i < pend.n; ++i) {
+        if (!is_last[i])
+            continue;
+        const Pending::Seg &sg = pend.seg[i];
+        const int f = first[i];
+        auto which_of = [&](int c) { return (sg.seg0 <= cstart[c]) ? 0 : 1; };
+        __threadfence();
+        if (n[i] <= kGroupFanIn) {
+            merge_slots(p, smem, mphase, n[i], [&](int k) { return 2 * (f + k) + which_of(f + k); },
+                        true, sg.b, sg.hc, 0, ctid);
+            if (ctid == 0)
+                *cnt[i] = 0;
+            continue;
+        }
+        const int leader = f + (((int)blockIdx.x - f) / kGroupFanIn) * kGroupFanIn;
+        const int lslot = 2 * leader + which_of(leader);
+        merge_slots(p, smem, mphase, ctr[i],
+                    [&](int k) { return 2 * (leader + k) + which_of(leader + k); }, false, sg.b,
+                    sg.hc, lslot, ctid);
+        __threadfence();
         consumer_bar();
-        const bool last_in = misc[1] != 0;
+        const int ngroups = (n[i] + kGroupFanIn - 1) / kGroupFanIn;
+        int *segc = p.seg_counters + 2 * f + which_of(f);
+        if (ctid == 0) {
+            *cnt[i] = 0;
+            misc[3] = (atomicAdd(segc, 1) == ngroups - 1) ? 1 : 0;
+        }
         consumer_bar();
-        if (last_in) {
+        const bool seg_last = misc[3] != 0;
+        consumer_bar();
+        if (seg_last) {
             __threadfence();
-            merge_slots(p, n, [&](int k) { return (size_t)(2 * (first + k) + which_of(first + k)); },
-                        true, b, hc, 0, ctid);
+            merge_slots(p, smem, mphase, ngroups,
+                        [&](int k) {
+                            const int ld = f + k * kGroupFanIn;
+                            return 2 * ld + which_of(ld);
+                        },
+                        true, sg.b, sg.hc, 0, ctid);
             if (ctid == 0)
                 *segc = 0;
         }
-        return;
-    }
-    const int ngroups = (n + kGroupFanIn - 1) / kGroupFanIn;
-    const int leader = first + ((me - first) / kGroupFanIn) * kGroupFanIn;
-    const int gsize = min(kGroupFanIn, last + 1 - leader);
-    const int lslot = 2 * leader + which_of(leader);
-    if (ctid == 0)
-        misc[1] = (atomicAdd(p.grp_counters + lslot, 1) == gsize - 1) ? 1 : 0;
-    consumer_bar();
-    const bool grp_last = misc[1] != 0;
-    consumer_bar();
-    if (!grp_last)
-        return;
-    __threadfence();
-    merge_slots(p, gsize, [&](int k) { return (size_t)(2 * (leader + k) + which_of(leader + k)); },
-                false, b, hc, lslot, ctid);
-    __threadfence();
-    consumer_bar();
-    if (ctid == 0) {
-        p.grp_counters[lslot] = 0;
-        misc[1] = (atomicAdd(segc, 1) == ngroups - 1) ? 1 : 0;
-    }
-    consumer_bar();
-    const bool seg_last = misc[1] != 0;
-    consumer_bar();
-    if (seg_last) {
-        __threadfence();
-        merge_slots(p, ngroups,
-                    [&](int k) {
-                        const int ld = first + k * kGroupFanIn;
-                        return (size_t)(2 * ld + which_of(ld));
-                    },
-                    true, b, hc, 0, ctid);
-        if (ctid == 0)
-            *segc = 0;
     }
 }
 
@@ -835,11 +930,10 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
 // Consumers derive it from the prefix sums themselves, so their control flow (and every
 // named barrier they take) never depends on data arriving.
 struct SegCursor {
-    int b, hc, ntb, L;
-    long long seg0, seg1;
+    int b, hc, ntb, L, seg0, seg1;
 };
 
-__device__ __forceinline__ void cursor_at(const DecodeParams &p, const int *prefix, long long x,
+__device__ __forceinline__ void cursor_at(const DecodeParams &p, const int *prefix, int x,
                                           SegCursor &cu)
 {
     int lo = 0, hi = p.B - 1;
@@ -853,15 +947,15 @@ __device__ __forceinline__ void cursor_at(const DecodeParams &p, const int *pref
     cu.b = lo;
     const int pre = prefix[lo];
     cu.ntb = (prefix[lo + 1] - pre) / p.nhc;
-    cu.hc = (int)((x - pre) / cu.ntb);
-    cu.seg0 = pre + (long long)cu.hc * cu.ntb;
+    cu.hc = (x - pre) / cu.ntb;
+    cu.seg0 = pre + cu.hc * cu.ntb;
     cu.seg1 = cu.seg0 + cu.ntb;
     cu.L = clamp_len(__ldg(p.seq_lens + lo), p.mbps * p.bs);
 }
 
 template <int NT, bool kDump>
-__device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix, long long t0,
-                        long long t1, long long N, int gcta, int warp, int lane)
+__device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
+                        const int *cstart, int t0, int t1, int gcta, int warp, int lane)
 {
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
@@ -883,23 +977,25 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         for (int j = 0; j < kNB; ++j)
             st.qs[r][j] = 0.f;
 
+    Pending pend;
+    pend.n = 0;
     SegCursor cu;
     cursor_at(p, prefix, t0, cu);
     bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
     int stage = 0;
     uint32_t phase = 0;
-    for (long long x = t0; x < t1; ++x) {
+    for (int x = t0; x < t1; ++x) {
         if (x >= cu.seg1)
             cursor_at(p, prefix, x, cu);
         const bool seg_first = x == (cu.seg0 > t0 ? cu.seg0 : t0);
         const bool seg_last = x + 1 == (cu.seg1 < t1 ? cu.seg1 : t1);
-        const int tok0 = (int)(x - cu.seg0) * p.TT;
+        const int tok0 = (x - cu.seg0) * p.TT;
         const int nvalid = min(p.TT, cu.L - tok0);
         if (seg_first) {
             load_query(p, st, cu.b, cu.hc, kl, slice, g, c);
             reset_state(st);
         }
-        if (!dead && !mbar_wait(&full[stage], phase, globaltimer_ns() + kWaitLimitNs)) {
+        if (!dead && !mbar_wait(&full[stage], phase, kWaitLimitNs)) {
             dead = true;
             atomicOr(p.errors, kErrTimeout);
         }
@@ -913,12 +1009,13 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         }
         if (seg_last)
             finalize_segment(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c, warp * 32 + lane,
-                             prefix, t0, t1, N, gcta);
+                             prefix, t0, t1, pend);
         if (++stage == p.n_stages) {
             stage = 0;
             phase ^= 1u;
         }
     }
+    combine_pending(p, smem, pend, cstart, gcta, warp * 32 + lane);
 }
 
 template <int NT, bool kDump>
@@ -941,6 +1038,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
+        mbar_init(reinterpret_cast<uint64_t *>(smem + p.lay.off_mbar), 1);
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -954,7 +1052,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     build_prefix(p, prefix, misc + 2, tid, warp, lane);
     __syncthreads();
 
-    const long long N = prefix[p.B];
+    const int N = prefix[p.B];
+    int *cstart = reinterpret_cast<int *>(smem + p.lay.off_cstart);
     // rows of empty sequences are zero
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
         if (prefix[b + 1] != prefix[b])
@@ -963,14 +1062,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = tid; i < p.Hq * kD / 4; i += kThreads)
             row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const int gcta = (int)(N < (long long)gridDim.x ? N : (long long)gridDim.x);
+    const int gcta = N < (int)gridDim.x ? N : (int)gridDim.x;
+    for (int i = tid; i <= gcta; i += kThreads)
+        cstart[i] = (int)((long long)i * N / gcta);
+    __syncthreads();
     if ((int)blockIdx.x >= gcta)
         return;
-    const long long t0 = cta_start(blockIdx.x, N, gcta), t1 = cta_start(blockIdx.x + 1, N, gcta);
+    const int t0 = cstart[blockIdx.x], t1 = cstart[blockIdx.x + 1];
     if (warp == kProducerWarp)
         produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
     else
-        consume<NT, kDump>(p, smem, prefix, t0, t1, N, gcta, warp, lane);
+        consume<NT, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
 }
 
 } // namespace q8kv

@@ -61,17 +61,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, giving up at `deadline_ns`
-// (%globaltimer). Returns false on time-out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline_ns)
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+                 : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete, giving up after `limit_ns` of
+// %globaltimer time (read only every 64 polls, so waiting costs almost no issue slots).
+// Returns false on time-out.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() > deadline_ns)
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_hint(bar, parity, 100000u))
+            return true;
+        if ((it & 63u) == 0u && globaltimer_ns() - t0 > limit_ns)
             return false;
     }
-    return true;
 }
 
 // ---------------------------------------------------------------- TMA
@@ -122,6 +137,16 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
                  : "memory");
 }
 
+// Contiguous bulk copy global -> shared without an L2 policy.
+__device__ __forceinline__ void bulk_load_plain(void *dst, const void *src, uint32_t bytes,
+                                                uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
 // ---------------------------------------------------------------- shared-memory loads
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr)
@@ -153,7 +178,7 @@ __device__ __forceinline__ float lds_f32(uint32_t addr)
 __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1)
 {
-    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, "
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, "
                  "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
                  : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
@@ -163,7 +188,7 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t 
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
                                               uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1)
 {
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
                  "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
                  : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -195,6 +220,21 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
 {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Exact int32 -> fp32 for |x| < 2^22 without the conversion unit: the integer is added
+// to the bit pattern of 1.5 * 2^23 (unit spacing) and 1.5 * 2^23 is subtracted.
+__device__ __forceinline__ float small_int_to_float(int x)
+{
+    return __int_as_float(x + 0x4B400000) - 12582912.0f;
+}
+
+// floor(log2 |v|) of a normal fp32 value, as fp32, from its exponent field (no conversion
+// unit): the field is placed in the mantissa of 2^23 and 2^23 + 127 is subtracted.
+__device__ __forceinline__ float exponent_as_float(float v)
+{
+    const uint32_t e = (__float_as_uint(v) >> 23) & 0xffu;
+    return __uint_as_float(0x4B000000u | e) - 8388735.0f;
 }
 
 // Exact power of two 2^e as fp32 for e in [-126, 127].
