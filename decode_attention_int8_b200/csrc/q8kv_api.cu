@@ -41,7 +41,7 @@ struct DeviceInfo {
     int sms = 0;
     int smem_optin = 0;
     unsigned *errors = nullptr;      // address of g_device_errors on this device
-    bool attr_set[2][2] = {{false, false}, {false, false}};
+    bool attr_set[3][2] = {{false, false}, {false, false}, {false, false}};
     void *ws = nullptr;              // library-managed workspace
     size_t ws_bytes = 0;
 };
@@ -139,7 +139,7 @@ q8kv_status plan_heads(int Hq, int Hk, int D, Plan &pl)
     pl.nhc = Hk / pl.HPC;
     pl.pairs = pl.HPC * pl.slices;
     pl.subtiles = kConsumerWarps / pl.pairs;
-    pl.TT = 16 * pl.subtiles;
+    pl.TT = 16 * kSub * pl.subtiles;
     pl.heads_seg = pl.HPC * pl.G;
     pl.scratch_stride = 32 * 32 * pl.NT + 48; // acc fragments + M, S, A of 16 heads
     return Q8KV_OK;
@@ -323,16 +323,23 @@ q8kv_status check_call(const Call &c)
     return Q8KV_OK;
 }
 
-template <int NT, bool kDump>
+template <int NT, bool kPack, bool kDump>
 q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl,
                           const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mks,
                           const CUtensorMap &mvs, cudaStream_t stream)
 {
-    auto fn = decode_kernel<NT, kDump>;
-    if (!dev.attr_set[NT - 1][kDump ? 1 : 0]) {
+    auto fn = decode_kernel<NT, kPack, kDump>;
+    const int variant = kPack ? 2 : NT - 1;
+    if (!dev.attr_set[variant][kDump ? 1 : 0]) {
+        // the setmaxnreg split in the kernel assumes exactly kLaunchRegs registers per thread
+        // at launch; anything else could leave a warpgroup waiting for registers forever
+        cudaFuncAttributes attr;
+        Q8KV_CUDA(cudaFuncGetAttributes(&attr, fn));
+        if (attr.numRegs != kLaunchRegs)
+            return Q8KV_ERR_UNSUPPORTED;
         Q8KV_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        dev.smem_optin));
-        dev.attr_set[NT - 1][kDump ? 1 : 0] = true;
+        dev.attr_set[variant][kDump ? 1 : 0] = true;
     }
     fn<<<pl.grid, kThreads, pl.smem_bytes, stream>>>(p, mk, mv, mks, mvs);
     Q8KV_CUDA(cudaGetLastError());
@@ -417,11 +424,14 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.lay = pl.lay;
 
     const bool dump = c.dots != nullptr;
+    if (pl.G <= 4) // heads fill at most half of the 8 MMA columns: pack the split halves
+        return dump ? launch_kernel<1, true, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
+                    : launch_kernel<1, true, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
     if (pl.NT == 1)
-        return dump ? launch_kernel<1, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
-                    : launch_kernel<1, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
-    return dump ? launch_kernel<2, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
-                : launch_kernel<2, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
+        return dump ? launch_kernel<1, false, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
+                    : launch_kernel<1, false, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
+    return dump ? launch_kernel<2, false, true>(*dev, p, pl, mk, mv, mks, mvs, stream)
+                : launch_kernel<2, false, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
 }
 
 } // namespace

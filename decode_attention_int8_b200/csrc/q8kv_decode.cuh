@@ -42,16 +42,24 @@ namespace q8kv {
 
 constexpr int kD = 128;             // head_dim handled by this kernel
 constexpr int kNB = kD / 32;        // quant blocks per head
-constexpr int kConsumerWarps = 8;   // warps 0-7
-constexpr int kProducerWarp = 8;    // warp 8
-constexpr int kThreads = 9 * 32;
+constexpr int kConsumerWarps = 8;   // warps 0-7 (two warpgroups)
+constexpr int kProducerWarp = 8;    // warp 8 (its warpgroup, warps 8-11, gives registers away)
+constexpr int kThreads = 12 * 32;
+constexpr int kLaunchRegs = 168;    // per-thread registers at launch (65536 / 384, rounded)
+constexpr int kProducerRegs = 56;   // after setmaxnreg.dec (producer warpgroup)
+constexpr int kConsumerRegs = 224;  // after setmaxnreg.inc (consumer warpgroups)
+static_assert(4 * 32 * kProducerRegs + 8 * 32 * kConsumerRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr int kSub = 2;             // 16-token subtiles per consumer warp per stage
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kMaxBoxes = 8;        // TMA boxes per stage
+constexpr int kMaxBoxes = 16;       // TMA boxes per stage
 constexpr int kGroupFanIn = 16;     // contributors merged per first-level combine
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
 constexpr int kSlotRow = kD + 4;    // per-head partial: kD accumulator floats, M, S, A, pad
 constexpr float kVExpLimit = 100.f; // V-scale exponents are clamped to [-100, 100]
+constexpr int kDotBias = 0x4B400000;    // bit pattern of 1.5 * 2^23
+constexpr float kDotBiasF = 12582912.0f; // 1.5 * 2^23
 
 // Device-side error bits (match Q8KV_DEVERR_* in q8kv.h).
 constexpr unsigned kErrSeqLen = 0x1u;
@@ -67,7 +75,8 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a)
 struct SmemLayout {
     uint32_t stage_bytes; // one ring slot: K | V | kscale | vscale
     uint32_t off_k, off_v, off_ks, off_vs; // within a slot
-    uint32_t off_full, off_empty, off_mbar, off_mask, off_misc, off_cstart, off_prefix, off_scratch;
+    uint32_t off_full, off_empty, off_mbar, off_mask, off_misc, off_slots, off_ptab, off_cstart,
+        off_prefix, off_scratch;
     uint32_t total; // bytes from the 1024-aligned base
 };
 
@@ -93,6 +102,10 @@ __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages,
     o += 4 * kMaxStages;
     L.off_misc = o;
     o += 64;
+    L.off_slots = o;
+    o += 4 * 32;
+    L.off_ptab = o; // producer: physical slot of every box of the next 32 tiles
+    o += 4 * 32 * kMaxBoxes;
     L.off_cstart = o;
     o = align_up(o + 4u * (uint32_t)(grid + 1), 16);
     L.off_prefix = o;
@@ -156,51 +169,58 @@ __device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
     return lo;
 }
 
-// Merge n_in partial (M, S, A, acc) slots into either the output rows of (b, hc) or one
-// slot. slot_k(k) gives the slot index of the k-th input. A slot holds heads_seg rows of
+// Merge n_in partial (M, S, A, acc) slots, listed in shared memory (slots[0..n_in)), into
+// either the output rows of (b, hc) or the slot dest_slot. A slot holds heads_seg rows of
 // kSlotRow floats: acc [kD] (units 2^-A), then M, S, A (base-2 logs, S in units 2^-M).
 // Runs after the main loop, when the stage ring is idle: one thread pulls every input row
 // of a chunk of heads into the ring with bulk copies (one round trip to L2), then all
-// consumer threads combine from shared memory. Called by all consumer threads.
-template <typename SlotFn>
-__device__ void merge_slots(const DecodeParams &p, uint8_t *smem, uint32_t &mphase, int n_in,
-                            SlotFn slot_k, bool to_out, int b, int hc, int dest_slot, int ctid)
+// consumer threads combine from shared memory. The code is kept small and rolled: it runs
+// once per call, so its instruction fetches are cold. Called by all consumer threads.
+__device__ __noinline__ void merge_slots(const DecodeParams &p, uint8_t *smem, uint32_t &mphase,
+                                         int n_in, bool to_out, int b, int hc, int dest_slot,
+                                         int ctid)
 {
     const int H = p.heads_seg;
+    const int *slots = reinterpret_cast<const int *>(smem + p.lay.off_slots);
     uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + p.lay.off_mbar);
     float *buf = reinterpret_cast<float *>(smem);
     const uint32_t row_bytes = kSlotRow * 4;
     const uint32_t ring = (uint32_t)p.n_stages * p.lay.stage_bytes;
     int hch = (int)(ring / ((uint32_t)n_in * row_bytes));
     hch = hch < 1 ? 1 : (hch > H ? H : hch);
+    const int warp = ctid >> 5, lane = ctid & 31;
     for (int h0 = 0; h0 < H; h0 += hch) {
         const int hn = (H - h0) < hch ? (H - h0) : hch;
-        if (ctid == 0) {
-            // the partials were written by other CTAs through the generic proxy
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            mbar_arrive_expect_tx(mbar, (uint32_t)n_in * hn * row_bytes);
-            for (int k = 0; k < n_in; ++k)
-                bulk_load_plain(buf + (size_t)k * hn * kSlotRow,
-                                p.partials + ((size_t)slot_k(k) * H + h0) * kSlotRow,
+        // lanes of warp 0 issue one bulk copy each (the partials were written by other CTAs
+        // through the generic proxy, hence the proxy fence)
+        if (warp == 0) {
+            if (lane == 0) {
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                mbar_arrive_expect_tx(mbar, (uint32_t)n_in * hn * row_bytes);
+            }
+            __syncwarp();
+            if (lane < n_in) {
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                bulk_load_plain(buf + (size_t)lane * hn * kSlotRow,
+                                p.partials + ((size_t)slots[lane] * H + h0) * kSlotRow,
                                 (uint32_t)hn * row_bytes, mbar);
+            }
         }
         if (!mbar_wait(mbar, mphase, kWaitLimitNs))
             atomicOr(p.errors, kErrTimeout);
         mphase ^= 1u;
-        // per head: maxima over the inputs, then each input's two factors (written over its
-        // M and S words) and the combined S (written over input 0's pad word)
-        const int warp = ctid >> 5, lane = ctid & 31;
+        // per head (one warp, one lane per input): the maxima, each input's accumulator
+        // factor (written over its M word), and the merged M, A, S (written over input 0's
+        // S, A and pad words)
         for (int hl = warp; hl < hn; hl += kConsumerWarps) {
             float m = -INFINITY, a = -INFINITY, sv = 0.f;
-            float *row = nullptr;
+            float *row = buf + ((size_t)lane * hn + hl) * kSlotRow;
             if (lane < n_in) {
-                row = buf + ((size_t)lane * hn + hl) * kSlotRow;
                 m = row[kD];
                 sv = row[kD + 1];
                 a = row[kD + 2];
             }
             float mx = m, ax = a;
-#pragma unroll
             for (int o = 16; o >= 1; o >>= 1) {
                 mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, o));
                 ax = fmaxf(ax, __shfl_xor_sync(kFullMask, ax, o));
@@ -208,47 +228,41 @@ __device__ void merge_slots(const DecodeParams &p, uint8_t *smem, uint32_t &mpha
             const float fs = (m == -INFINITY) ? 0.f : exp2f(m - mx);
             const float fa = (a == -INFINITY) ? 0.f : exp2f(a - ax);
             float ssum = fs * sv;
-#pragma unroll
             for (int o = 16; o >= 1; o >>= 1)
                 ssum += __shfl_xor_sync(kFullMask, ssum, o);
             __syncwarp();
-            if (row) {
-                row[kD] = fa; // factor of this input's accumulator
-                if (lane == 0) {
-                    row[kD + 1] = mx;
-                    row[kD + 2] = ax;
-                    row[kD + 3] = ssum;
-                }
+            if (lane < n_in)
+                row[kD] = fa;
+            if (lane == 0) {
+                row[kD + 1] = mx;
+                row[kD + 2] = ax;
+                row[kD + 3] = ssum;
             }
         }
         consumer_bar();
         for (int u = ctid; u < hn * (kD / 4); u += kConsumerThreads) {
             const int hl = u / (kD / 4), d4 = u % (kD / 4);
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < kGroupFanIn; ++k) {
-                if (k < n_in) {
-                    const float *row = buf + ((size_t)k * hn + hl) * kSlotRow;
-                    const float fa = row[kD];
-                    const float4 v = *reinterpret_cast<const float4 *>(row + d4 * 4);
-                    a.x += fa * v.x;
-                    a.y += fa * v.y;
-                    a.z += fa * v.z;
-                    a.w += fa * v.w;
-                }
+            const float *row = buf + (size_t)hl * kSlotRow;
+            for (int k = 0; k < n_in; ++k, row += (size_t)hn * kSlotRow) {
+                const float fa = row[kD];
+                const float4 v = *reinterpret_cast<const float4 *>(row + d4 * 4);
+                a.x += fa * v.x;
+                a.y += fa * v.y;
+                a.z += fa * v.z;
+                a.w += fa * v.w;
             }
             const float4 hdr = *reinterpret_cast<const float4 *>(buf + (size_t)hl * kSlotRow + kD);
-            const float mx = hdr.y, ax = hdr.z, ssum = hdr.w;
             if (to_out) {
-                const float f = ssum > 0.f ? exp2f(ax - mx) / ssum : 0.f;
+                const float f = hdr.w > 0.f ? exp2f(hdr.z - hdr.y) / hdr.w : 0.f;
                 const int h = hc * H + h0 + hl;
                 float4 o = make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
                 *reinterpret_cast<float4 *>(p.out + ((long long)b * p.Hq + h) * kD + d4 * 4) = o;
             } else {
-                float *row = p.partials + ((size_t)dest_slot * H + h0 + hl) * kSlotRow;
-                *reinterpret_cast<float4 *>(row + d4 * 4) = a;
+                float *drow = p.partials + ((size_t)dest_slot * H + h0 + hl) * kSlotRow;
+                *reinterpret_cast<float4 *>(drow + d4 * 4) = a;
                 if (d4 == 0)
-                    *reinterpret_cast<float4 *>(row + kD) = make_float4(mx, ssum, ax, 0.f);
+                    *reinterpret_cast<float4 *>(drow + kD) = make_float4(hdr.y, hdr.w, hdr.z, 0.f);
             }
         }
         consumer_bar(); // the ring is refilled for the next chunk
@@ -319,13 +333,11 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     uint32_t phase = 0, issued = 0, issued_par = 0;
     bool aborted = false;
 
+    int *ptab = reinterpret_cast<int *>(smem + p.lay.off_ptab);
     for (int xb = t0; xb < t1 && !aborted; xb += 32) {
+        // lane l resolves tile xb + l: its head chunk and the physical slot of every box
         const int x = xb + lane;
         int hc = 0;
-        int slot[kMaxBoxes];
-#pragma unroll
-        for (int bx = 0; bx < kMaxBoxes; ++bx)
-            slot[bx] = -1;
         if (x < t1) {
             int lo = 0, hi = p.B - 1; // largest b with prefix[b] <= x
             while (lo < hi) {
@@ -343,36 +355,34 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
             const int lt = local - hc * ntb;
             const int tok0 = lt * p.TT;
             const int L = clamp_len(__ldg(p.seq_lens + b), cap);
-#pragma unroll
-            for (int bx = 0; bx < kMaxBoxes; ++bx) {
+            for (int bx = 0; bx < p.n_boxes; ++bx) {
                 const int tk = tok0 + bx * p.box_tok;
-                if (bx < p.n_boxes && tk < L) {
+                int sl = -1;
+                if (tk < L) {
                     const int ph = __ldg(p.block_table + (long long)b * p.mbps + tk / p.bs);
                     if (ph >= 0 && ph < p.num_blocks)
-                        slot[bx] = ph * p.bs + (tk % p.bs);
+                        sl = ph * p.bs + (tk % p.bs);
                     else
                         atomicOr(p.errors, kErrBlockTable);
                 }
+                ptab[lane * kMaxBoxes + bx] = sl;
             }
         }
+        __syncwarp();
         const int n = (t1 - xb) < 32 ? (t1 - xb) : 32;
         for (int i = 0; i < n; ++i) {
             const int hci = __shfl_sync(kFullMask, hc, i);
-            int sl[kMaxBoxes];
-#pragma unroll
-            for (int bx = 0; bx < kMaxBoxes; ++bx)
-                sl[bx] = __shfl_sync(kFullMask, slot[bx], i);
             int ok = 1;
             if (lane == 0) {
                 if (!mbar_wait(&empty[stage], phase ^ 1u, kWaitLimitNs)) {
                     ok = 0;
                     atomicOr(p.errors, kErrTimeout);
                 } else {
+                    const int *sl = ptab + i * kMaxBoxes;
                     uint32_t bytes = 0;
                     int loaded = 0;
-#pragma unroll
-                    for (int bx = 0; bx < kMaxBoxes; ++bx)
-                        if (bx < p.n_boxes && sl[bx] >= 0) {
+                    for (int bx = 0; bx < p.n_boxes; ++bx)
+                        if (sl[bx] >= 0) {
                             bytes += 2 * (kv_box + sc_box);
                             loaded |= 1 << bx;
                         }
@@ -380,25 +390,25 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                     mask[stage] = loaded;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     uint8_t *sb = smem + (size_t)stage * p.lay.stage_bytes;
-#pragma unroll
-                    for (int bx = 0; bx < kMaxBoxes; ++bx) {
-                        if (bx < p.n_boxes && sl[bx] >= 0) {
-                            tma_load_3d(sb + p.lay.off_k + bx * kv_box, tmK, &full[stage], 0, sl[bx],
-                                        hci * p.HPC, pol);
-                            tma_load_3d(sb + p.lay.off_v + bx * kv_box, tmV, &full[stage], 0, sl[bx],
-                                        hci * p.HPC, pol);
-                            if (p.scale_bulk) {
-                                const long long e0 = (long long)sl[bx] * p.Hk;
-                                bulk_load(sb + p.lay.off_ks + bx * sc_box, p.kscale + e0, sc_box,
-                                          &full[stage], pol);
-                                bulk_load(sb + p.lay.off_vs + bx * sc_box, p.vscale + e0, sc_box,
-                                          &full[stage], pol);
-                            } else {
-                                tma_load_2d(sb + p.lay.off_ks + bx * sc_box, tmKs, &full[stage],
-                                            hci * p.HPC, sl[bx], pol);
-                                tma_load_2d(sb + p.lay.off_vs + bx * sc_box, tmVs, &full[stage],
-                                            hci * p.HPC, sl[bx], pol);
-                            }
+                    for (int bx = 0; bx < p.n_boxes; ++bx) {
+                        const int slot = sl[bx];
+                        if (slot < 0)
+                            continue;
+                        tma_load_3d(sb + p.lay.off_k + bx * kv_box, tmK, &full[stage], 0, slot,
+                                    hci * p.HPC, pol);
+                        tma_load_3d(sb + p.lay.off_v + bx * kv_box, tmV, &full[stage], 0, slot,
+                                    hci * p.HPC, pol);
+                        if (p.scale_bulk) {
+                            const long long e0 = (long long)slot * p.Hk;
+                            bulk_load(sb + p.lay.off_ks + bx * sc_box, p.kscale + e0, sc_box,
+                                      &full[stage], pol);
+                            bulk_load(sb + p.lay.off_vs + bx * sc_box, p.vscale + e0, sc_box,
+                                      &full[stage], pol);
+                        } else {
+                            tma_load_2d(sb + p.lay.off_ks + bx * sc_box, tmKs, &full[stage],
+                                        hci * p.HPC, slot, pol);
+                            tma_load_2d(sb + p.lay.off_vs + bx * sc_box, tmVs, &full[stage],
+                                        hci * p.HPC, slot, pol);
                         }
                     }
                     issued |= 1u << stage;
@@ -415,6 +425,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                 phase ^= 1u;
             }
         }
+        __syncwarp(); // the table is rewritten for the next 32 tiles
     }
     // Every copy this warp issued must have landed before the CTA may exit.
     if (lane == 0) {
@@ -436,10 +447,21 @@ struct WarpState {
     float qs[NT][kNB];   // Q block scales of rows g and g + 8
 };
 
+// Quantise this warp's query heads into int8 A fragments. Row g (and g + 8 when NT == 2)
+// holds head slice * 16 + g (+ 8). In packed mode (group <= 4) rows g and g + 4 both hold
+// head g & 3: the duplicate rows produce the same weights, which feed the low halves of the
+// split PV operand (columns 4-7) while rows 0-3 feed the high halves (columns 0-3).
 template <int NT>
-__device__ __forceinline__ void load_query(const DecodeParams &p, WarpState<NT> &st, int b, int hc,
-                                           int kl, int slice, int g, int c)
+struct QueryFrag {
+    uint32_t qa[kNB][4];
+    float qs[NT][kNB];
+};
+
+template <int NT, bool kPack>
+__device__ __forceinline__ QueryFrag<NT> load_query(const DecodeParams &p, int b, int hc, int kl,
+                                                 int slice, int g, int c)
 {
+    QueryFrag<NT> st;
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         if (r >= NT) {
@@ -450,7 +472,7 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, WarpState<NT> 
             }
             continue;
         }
-        const int hg = slice * 16 + r * 8 + g;
+        const int hg = kPack ? (g & 3) : slice * 16 + r * 8 + g;
         const bool valid = hg < p.G;
         const float *qrow =
             p.q + ((long long)b * p.Hq + (long long)(hc * p.HPC + kl) * p.G + hg) * kD;
@@ -481,6 +503,7 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, WarpState<NT> 
             st.qa[j][r == 0 ? 2 : 3] = hi;
         }
     }
+    return st;
 }
 
 template <int NT>
@@ -499,12 +522,13 @@ __device__ __forceinline__ void reset_state(WarpState<NT> &st)
     }
 }
 
-// Per-thread shared-memory offsets that are the same for every stage.
+// Per-thread shared-memory offsets that are the same for every stage. Subtile u of a
+// warp covers stage tokens ts * 16 * kSub + 16 * u + [0, 16).
 struct ThreadOffsets {
-    uint32_t k[2][kNB]; // K fragment loads (QK n-tile, quant block)
-    uint32_t v[4];      // V rows 2c, 2c+1, 2c+8, 2c+9 (channel chunk g)
-    uint32_t s[2][2];   // scale of tokens nt*8 + 2c + e
-    int tok[2][2];      // stage-local token index of (nt, e)
+    uint32_t k[kSub][2][kNB]; // K fragment loads (subtile, QK n-tile, quant block)
+    uint32_t v[kSub][4];      // V rows 2c, 2c+1, 2c+8, 2c+9 (channel chunk g)
+    uint32_t s[kSub][2][2];   // scale of tokens nt*8 + 2c + e
+    int tok[kSub][2][2];      // stage-local token index of (u, nt, e)
 };
 
 __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int kl, int ts, int g,
@@ -515,24 +539,28 @@ __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int
     auto row_kv = [&](int tok) { return ((tok >> lb) * H + kl) * bt + (tok & (bt - 1)); };
     auto row_sc = [&](int tok) { return ((tok >> lb) * bt + (tok & (bt - 1))) * H + kl; };
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int r = row_kv(ts * 16 + nt * 8 + g);
+    for (int u = 0; u < kSub; ++u) {
+        const int t0 = (ts * kSub + u) * 16;
 #pragma unroll
-        for (int j = 0; j < kNB; ++j)
-            o.k[nt][j] = p.lay.off_k + r * 128 + ((((2 * j) | (c >> 1)) ^ (r & 7)) << 4) +
-                         ((c & 1) << 3);
+        for (int nt = 0; nt < 2; ++nt) {
+            const int r = row_kv(t0 + nt * 8 + g);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int tok = ts * 16 + nt * 8 + 2 * c + e;
-            o.tok[nt][e] = tok;
-            o.s[nt][e] = 4 * row_sc(tok);
+            for (int j = 0; j < kNB; ++j)
+                o.k[u][nt][j] = p.lay.off_k + r * 128 + ((((2 * j) | (c >> 1)) ^ (r & 7)) << 4) +
+                                ((c & 1) << 3);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int tok = t0 + nt * 8 + 2 * c + e;
+                o.tok[u][nt][e] = tok;
+                o.s[u][nt][e] = 4 * row_sc(tok);
+            }
         }
-    }
 #pragma unroll
-    for (int qv = 0; qv < 4; ++qv) {
-        const int t = 2 * c + (qv & 1) + (qv >> 1) * 8;
-        const int r = row_kv(ts * 16 + t);
-        o.v[qv] = p.lay.off_v + r * 128 + ((g ^ (r & 7)) << 4);
+        for (int qv = 0; qv < 4; ++qv) {
+            const int t = 2 * c + (qv & 1) + (qv >> 1) * 8;
+            const int r = row_kv(t0 + t);
+            o.v[u][qv] = p.lay.off_v + r * 128 + ((g ^ (r & 7)) << 4);
+        }
     }
     return o;
 }
@@ -542,83 +570,110 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
-// One stage (16 tokens of one KV head for this warp).
-template <int NT, bool kDump>
+// One stage: kSub 16-token subtiles of one KV head for this warp, folded into the online
+// softmax as one block. kMasked: some tokens of the stage are past the sequence end or in a
+// block that was not loaded.
+template <int NT, bool kPack, bool kDump, bool kMasked>
 __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<NT> &st,
-                                              const ThreadOffsets &o, uint32_t sbase, int nvalid,
-                                              int loaded, int b, int hc, int kl, int slice,
-                                              int tok0, int g, int c)
+                                              const ThreadOffsets &o, const uint8_t *sb,
+                                              int nvalid, int loaded, int b, int hc, int kl,
+                                              int slice, int tok0, int g, int c)
 {
-    // ---- scores: int8 MMA per quant block, exact int32 block dots
-    float s[NT][2][2];
+    // ---- V rows first: their int8 -> f16 conversion overlaps the softmax chain below
+    uint4 R[kSub][4];
+#pragma unroll
+    for (int u = 0; u < kSub; ++u)
+#pragma unroll
+        for (int qv = 0; qv < 4; ++qv)
+            R[u][qv] = *reinterpret_cast<const uint4 *>(sb + o.v[u][qv]);
+    // ---- scores: int8 MMA per quant block, exact int32 block dots. The accumulator
+    // starts at the bit pattern of 1.5 * 2^23, so each result read as fp32 is
+    // 1.5 * 2^23 + dot exactly (|dot| <= 32 * 127 * 127 < 2^22).
+    float s[NT][kSub][2][2];
 #pragma unroll
     for (int r = 0; r < NT; ++r)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-            s[r][nt][0] = s[r][nt][1] = 0.f;
+        for (int u = 0; u < kSub; ++u)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < 2; ++nt)
+                s[r][u][nt][0] = s[r][u][nt][1] = 0.f;
 #pragma unroll
-        for (int j = 0; j < kNB; ++j) {
-            const uint2 kk = lds64(sbase + o.k[nt][j]);
-            int d[4];
-            mma_s8_16832(d, st.qa[j][0], st.qa[j][1], st.qa[j][2], st.qa[j][3], kk.x, kk.y);
-            if constexpr (kDump) {
+    for (int u = 0; u < kSub; ++u) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = q >> 1, e = q & 1;
-                    const int hg = slice * 16 + r * 8 + g;
-                    const int tl = o.tok[nt][e];
-                    if (hg < p.G && tl < nvalid && ((loaded >> (tl >> p.log2_box)) & 1)) {
-                        const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
-                        p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) * kNB +
-                                   j] = d[q];
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int j = 0; j < kNB; ++j) {
+                const uint2 kk = *reinterpret_cast<const uint2 *>(sb + o.k[u][nt][j]);
+                int d[4];
+                mma_s8_16832_biased(d, st.qa[j][0], NT == 2 ? st.qa[j][1] : 0u, st.qa[j][2],
+                                    NT == 2 ? st.qa[j][3] : 0u, kk.x, kk.y);
+                if constexpr (kDump) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = q >> 1, e = q & 1;
+                        const int hg = kPack ? g : slice * 16 + r * 8 + g;
+                        const bool row_ok = kPack ? (r == 0 && g < 4) : (r < NT);
+                        const int tl = o.tok[u][nt][e];
+                        if (row_ok && hg < p.G && tl < nvalid &&
+                            ((loaded >> (tl >> p.log2_box)) & 1)) {
+                            const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
+                            p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) *
+                                           kNB +
+                                       j] = d[q] - kDotBias;
+                        }
                     }
                 }
-            }
-            // |dot| <= 32 * 127 * 127 < 2^22: exact conversion
-            s[0][nt][0] += small_int_to_float(d[0]) * st.qs[0][j];
-            s[0][nt][1] += small_int_to_float(d[1]) * st.qs[0][j];
-            if constexpr (NT == 2) {
-                s[NT - 1][nt][0] += small_int_to_float(d[2]) * st.qs[NT - 1][j];
-                s[NT - 1][nt][1] += small_int_to_float(d[3]) * st.qs[NT - 1][j];
+                s[0][u][nt][0] += (__int_as_float(d[0]) - kDotBiasF) * st.qs[0][j];
+                s[0][u][nt][1] += (__int_as_float(d[1]) - kDotBiasF) * st.qs[0][j];
+                if constexpr (NT == 2) {
+                    s[NT - 1][u][nt][0] += (__int_as_float(d[2]) - kDotBiasF) * st.qs[NT - 1][j];
+                    s[NT - 1][u][nt][1] += (__int_as_float(d[3]) - kDotBiasF) * st.qs[NT - 1][j];
+                }
             }
         }
     }
     // ---- per-token K and V scales; masking of tokens past the sequence end
-    float kss[2][2], vsv[2][2], vex[2][2];
-    bool val[2][2];
+    float kss[kSub][2][2], vsv[kSub][2][2], vex[kSub][2][2];
+    bool val[kSub][2][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            val[nt][e] = o.tok[nt][e] < nvalid && ((loaded >> (o.tok[nt][e] >> p.log2_box)) & 1);
-            kss[nt][e] = lds_f32(sbase + p.lay.off_ks + o.s[nt][e]) * p.scale_log2;
-            const float vv = lds_f32(sbase + p.lay.off_vs + o.s[nt][e]);
-            vsv[nt][e] = val[nt][e] ? vv : 0.f;
-            // floor(log2 |vs|) from the exponent field, clamped to [-100, 100]
-            vex[nt][e] = fminf(fmaxf(exponent_as_float(vv), -kVExpLimit), kVExpLimit);
-        }
-    // ---- online softmax (base 2), blockwise over the 16 tokens. M: running max of the
-    // scores (denominator). A: running max of score + log2(vs) - 14 (numerator), so that
-    // every weight * vs * 2^(M - A) entering the f16 MMA is below 2^15.
-    float alpha_a[NT];
-    uint32_t bh[NT][2], bl[NT][2];
-#pragma unroll
-    for (int r = 0; r < NT; ++r) {
-        float m = -INFINITY, a = -INFINITY;
+    for (int u = 0; u < kSub; ++u)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const float v = val[nt][e] ? s[r][nt][e] * kss[nt][e] : -INFINITY;
-                s[r][nt][e] = v;
-                m = fmaxf(m, v);
-                a = fmaxf(a, v + vex[nt][e]);
+                const int tl = o.tok[u][nt][e];
+                val[u][nt][e] = !kMasked || (tl < nvalid && ((loaded >> (tl >> p.log2_box)) & 1));
+                kss[u][nt][e] =
+                    *reinterpret_cast<const float *>(sb + p.lay.off_ks + o.s[u][nt][e]) *
+                    p.scale_log2;
+                const float vv =
+                    *reinterpret_cast<const float *>(sb + p.lay.off_vs + o.s[u][nt][e]);
+                vsv[u][nt][e] = val[u][nt][e] ? vv : 0.f;
+                // floor(log2 |vs|) from the exponent field, clamped to [-100, 100]
+                vex[u][nt][e] = fminf(fmaxf(exponent_as_float(vv), -kVExpLimit), kVExpLimit);
             }
+    // ---- online softmax (base 2), blockwise over the stage's tokens. M: running max of the
+    // scores (denominator). A: running max of score + log2(vs) - 14 (numerator), so that
+    // every weight * vs * 2^(M - A) entering the f16 MMA is below 2^15.
+    float alpha_a[NT];
+    uint32_t bh[NT][kSub][2], bl[NT][kSub][2];
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        float m = -INFINITY, a = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float v = val[u][nt][e] ? s[r][u][nt][e] * kss[u][nt][e] : -INFINITY;
+                    s[r][u][nt][e] = v;
+                    m = fmaxf(m, v);
+                    a = fmaxf(a, v + vex[u][nt][e]);
+                }
         m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
         a = fmaxf(a, __shfl_xor_sync(kFullMask, a, 1));
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
         a = fmaxf(a, __shfl_xor_sync(kFullMask, a, 2));
         const float mn = fmaxf(st.M[r], m);
         const float an = fmaxf(st.A[r], a - 14.f);
@@ -630,26 +685,30 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
         st.A[r] = an;
         const float cvs = exp2f(ms - as); // 2^(M - A), within [2^-86, 2^114]
         float ws = 0.f;
-        float pw[2][2];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int u = 0; u < kSub; ++u) {
+            float pw[2][2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float w = exp2f(s[r][nt][e] - ms);
-                ws += w;
-                pw[nt][e] = w * (vsv[nt][e] * cvs);
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float w = exp2f(s[r][u][nt][e] - ms);
+                    ws += w;
+                    pw[nt][e] = w * (vsv[u][nt][e] * cvs);
+                }
+            // weights as split f16 B operands (column n = head g, k = token)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const __half2 h = __floats2half2_rn(pw[nt][0], pw[nt][1]);
+                const float r0 = pw[nt][0] - __low2float(h), r1 = pw[nt][1] - __high2float(h);
+                bh[r][u][nt] = *reinterpret_cast<const uint32_t *>(&h);
+                bl[r][u][nt] = pack_f16x2(r0, r1);
             }
-        st.S[r] = st.S[r] * alpha_s + ws;
-        // weights as split f16 B operands (column n = head g, k = token)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const __half2 h = __floats2half2_rn(pw[nt][0], pw[nt][1]);
-            const float r0 = pw[nt][0] - __low2float(h), r1 = pw[nt][1] - __high2float(h);
-            bh[r][nt] = *reinterpret_cast<const uint32_t *>(&h);
-            bl[r][nt] = pack_f16x2(r0, r1);
         }
+        st.S[r] = st.S[r] * alpha_s + ws;
     }
-    // ---- rescale the accumulator columns whose A rose
+    // ---- rescale the accumulator columns whose A rose (in packed mode rows 4-7 repeat
+    // rows 0-3, so the source lane of column col carries head col & 3 either way)
 #pragma unroll
     for (int pv = 0; pv < NT; ++pv) {
         const float f0 = __shfl_sync(kFullMask, alpha_a[pv], 8 * c);
@@ -664,25 +723,32 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
             }
         }
     }
-    // ---- PV: rows = channels 16g + 2i (+1), k = tokens, columns = heads
-    const uint4 R0 = lds128(sbase + o.v[0]);
-    const uint4 R1 = lds128(sbase + o.v[1]);
-    const uint4 R2 = lds128(sbase + o.v[2]);
-    const uint4 R3 = lds128(sbase + o.v[3]);
+    // ---- PV: rows = channels 16g + 2i (+1), k = tokens, columns = heads (packed mode:
+    // columns 0-3 high halves of heads 0-3, columns 4-7 their low halves)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t w0 = word_of(R0, i >> 1), w1 = word_of(R1, i >> 1);
-        const uint32_t w2 = word_of(R2, i >> 1), w3 = word_of(R3, i >> 1);
-        const uint32_t sl = (i & 1) ? 0x0602u : 0x0400u;
-        const uint32_t sh = (i & 1) ? 0x0703u : 0x0501u;
-        const uint32_t a0 = s8pair_to_f16x2(prmt(w0, w1, sl));
-        const uint32_t a1 = s8pair_to_f16x2(prmt(w0, w1, sh));
-        const uint32_t a2 = s8pair_to_f16x2(prmt(w2, w3, sl));
-        const uint32_t a3 = s8pair_to_f16x2(prmt(w2, w3, sh));
+    for (int u = 0; u < kSub; ++u) {
+        uint32_t b0[NT], b1[NT];
 #pragma unroll
         for (int pv = 0; pv < NT; ++pv) {
-            mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, bh[pv][0], bh[pv][1]);
-            mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, bl[pv][0], bl[pv][1]);
+            b0[pv] = (kPack && g >= 4) ? bl[pv][u][0] : bh[pv][u][0];
+            b1[pv] = (kPack && g >= 4) ? bl[pv][u][1] : bh[pv][u][1];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t w0 = word_of(R[u][0], i >> 1), w1 = word_of(R[u][1], i >> 1);
+            const uint32_t w2 = word_of(R[u][2], i >> 1), w3 = word_of(R[u][3], i >> 1);
+            const uint32_t sl = (i & 1) ? 0x0602u : 0x0400u;
+            const uint32_t sh = (i & 1) ? 0x0703u : 0x0501u;
+            const uint32_t a0 = s8pair_to_f16x2(prmt(w0, w1, sl));
+            const uint32_t a1 = s8pair_to_f16x2(prmt(w0, w1, sh));
+            const uint32_t a2 = s8pair_to_f16x2(prmt(w2, w3, sl));
+            const uint32_t a3 = s8pair_to_f16x2(prmt(w2, w3, sh));
+#pragma unroll
+            for (int pv = 0; pv < NT; ++pv) {
+                mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, b0[pv], b1[pv]);
+                if constexpr (!kPack)
+                    mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, bl[pv][u][0], bl[pv][u][1]);
+            }
         }
     }
 }
@@ -709,8 +775,9 @@ struct Pending {
 };
 
 // End of a segment (all of this CTA's tiles of sequence b, head chunk hc).
-template <int NT>
-__device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8_t *smem, int b,
+template <int NT, bool kPack>
+__device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st,
+                                                 uint8_t *smem, int b,
                                  int hc, int kl, int slice, int pair, int ts, int g, int c,
                                  int ctid, const int *prefix, int t0, int t1, Pending &pend)
 {
@@ -784,6 +851,15 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
         consumer_bar();
     }
 
+    // packed mode: column col + 4 holds the low half of column col's head
+    if constexpr (kPack) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                st.acc[0][i][k] += __shfl_xor_sync(kFullMask, st.acc[0][i][k], 2);
+    }
+    const bool col_lane = !kPack || c < 2; // lanes whose columns are real heads
     const int pre = prefix[b];
     const int ntb = (prefix[b + 1] - pre) / p.nhc;
     const int seg0 = pre + hc * ntb, seg1 = seg0 + ntb;
@@ -799,7 +875,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
                     const float mc = __shfl_sync(kFullMask, st.M[pv], 4 * col);
                     const float ac = __shfl_sync(kFullMask, st.A[pv], 4 * col);
                     const int hg = slice * 16 + pv * 8 + col;
-                    if (hg < p.G) {
+                    if (col_lane && hg < p.G) {
                         const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
                         float *dst = p.out + ((long long)b * p.Hq + h) * kD + 16 * g;
                         store_row16(dst, st, pv, q, sc > 0.f ? exp2f(ac - mc) / sc : 0.f);
@@ -820,7 +896,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int hg = slice * 16 + pv * 8 + 2 * c + q;
-                if (hg < p.G)
+                if (col_lane && hg < p.G)
                     store_row16(slotp + (size_t)(kl * p.G + hg) * kSlotRow + 16 * g, st, pv, q,
                                 1.0f);
             }
@@ -828,7 +904,7 @@ __device__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st, uint8
 #pragma unroll
             for (int r = 0; r < NT; ++r) {
                 const int hg = slice * 16 + r * 8 + g;
-                if (hg < p.G)
+                if ((!kPack || g < 4) && hg < p.G)
                     *reinterpret_cast<float4 *>(slotp + (size_t)(kl * p.G + hg) * kSlotRow + kD) =
                         make_float4(st.M[r], st.S[r], st.A[r], 0.f);
             }
@@ -887,20 +963,24 @@ __device__ void combine_pending(const DecodeParams &p, uint8_t *smem, const Pend
             continue;
         const Pending::Seg &sg = pend.seg[i];
         const int f = first[i];
+        int *slots = reinterpret_cast<int *>(smem + p.lay.off_slots);
         auto which_of = [&](int c) { return (sg.seg0 <= cstart[c]) ? 0 : 1; };
         __threadfence();
         if (n[i] <= kGroupFanIn) {
-            merge_slots(p, smem, mphase, n[i], [&](int k) { return 2 * (f + k) + which_of(f + k); },
-                        true, sg.b, sg.hc, 0, ctid);
+            if (ctid < n[i])
+                slots[ctid] = 2 * (f + ctid) + which_of(f + ctid);
+            consumer_bar();
+            merge_slots(p, smem, mphase, n[i], true, sg.b, sg.hc, 0, ctid);
             if (ctid == 0)
                 *cnt[i] = 0;
             continue;
         }
         const int leader = f + (((int)blockIdx.x - f) / kGroupFanIn) * kGroupFanIn;
         const int lslot = 2 * leader + which_of(leader);
-        merge_slots(p, smem, mphase, ctr[i],
-                    [&](int k) { return 2 * (leader + k) + which_of(leader + k); }, false, sg.b,
-                    sg.hc, lslot, ctid);
+        if (ctid < ctr[i])
+            slots[ctid] = 2 * (leader + ctid) + which_of(leader + ctid);
+        consumer_bar();
+        merge_slots(p, smem, mphase, ctr[i], false, sg.b, sg.hc, lslot, ctid);
         __threadfence();
         consumer_bar();
         const int ngroups = (n[i] + kGroupFanIn - 1) / kGroupFanIn;
@@ -914,12 +994,10 @@ __device__ void combine_pending(const DecodeParams &p, uint8_t *smem, const Pend
         consumer_bar();
         if (seg_last) {
             __threadfence();
-            merge_slots(p, smem, mphase, ngroups,
-                        [&](int k) {
-                            const int ld = f + k * kGroupFanIn;
-                            return 2 * ld + which_of(ld);
-                        },
-                        true, sg.b, sg.hc, 0, ctid);
+            if (ctid < ngroups)
+                slots[ctid] = 2 * (f + ctid * kGroupFanIn) + which_of(f + ctid * kGroupFanIn);
+            consumer_bar();
+            merge_slots(p, smem, mphase, ngroups, true, sg.b, sg.hc, 0, ctid);
             if (ctid == 0)
                 *segc = 0;
         }
@@ -933,9 +1011,9 @@ struct SegCursor {
     int b, hc, ntb, L, seg0, seg1;
 };
 
-__device__ __forceinline__ void cursor_at(const DecodeParams &p, const int *prefix, int x,
-                                          SegCursor &cu)
+__device__ __forceinline__ SegCursor cursor_at(const DecodeParams &p, const int *prefix, int x)
 {
+    SegCursor cu;
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -951,9 +1029,10 @@ __device__ __forceinline__ void cursor_at(const DecodeParams &p, const int *pref
     cu.seg0 = pre + cu.hc * cu.ntb;
     cu.seg1 = cu.seg0 + cu.ntb;
     cu.L = clamp_len(__ldg(p.seq_lens + lo), p.mbps * p.bs);
+    return cu;
 }
 
-template <int NT, bool kDump>
+template <int NT, bool kPack, bool kDump>
 __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                         const int *cstart, int t0, int t1, int gcta, int warp, int lane)
 {
@@ -963,7 +1042,6 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
     const int kl = pair / p.slices, slice = pair % p.slices;
     const int g = lane >> 2, c = lane & 3;
     const ThreadOffsets o = make_offsets(p, kl, ts, g, c);
-    const uint32_t sm0 = smem_addr(smem);
     WarpState<NT> st;
     reset_state(st);
 #pragma unroll
@@ -979,46 +1057,56 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
 
     Pending pend;
     pend.n = 0;
-    SegCursor cu;
-    cursor_at(p, prefix, t0, cu);
     bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
     int stage = 0;
     uint32_t phase = 0;
-    for (int x = t0; x < t1; ++x) {
-        if (x >= cu.seg1)
-            cursor_at(p, prefix, x, cu);
-        const bool seg_first = x == (cu.seg0 > t0 ? cu.seg0 : t0);
-        const bool seg_last = x + 1 == (cu.seg1 < t1 ? cu.seg1 : t1);
-        const int tok0 = (x - cu.seg0) * p.TT;
-        const int nvalid = min(p.TT, cu.L - tok0);
-        if (seg_first) {
-            load_query(p, st, cu.b, cu.hc, kl, slice, g, c);
+    // Outer loop: one segment (this CTA's tiles of one sequence and head chunk) per pass.
+    // The inner loop over the segment's tiles holds only wait / compute / release, so the
+    // hot code stays small enough for the instruction cache.
+    for (int x = t0; x < t1;) {
+        const SegCursor cu = cursor_at(p, prefix, x);
+        const int x_end = cu.seg1 < t1 ? cu.seg1 : t1;
+        {
+            const QueryFrag<NT> qf = load_query<NT, kPack>(p, cu.b, cu.hc, kl, slice, g, c);
+#pragma unroll
+            for (int j = 0; j < kNB; ++j) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    st.qa[j][k] = qf.qa[j][k];
+#pragma unroll
+                for (int r = 0; r < NT; ++r)
+                    st.qs[r][j] = qf.qs[r][j];
+            }
             reset_state(st);
         }
-        if (!dead && !mbar_wait(&full[stage], phase, kWaitLimitNs)) {
-            dead = true;
-            atomicOr(p.errors, kErrTimeout);
+        for (; x < x_end; ++x) {
+            const int tok0 = (x - cu.seg0) * p.TT;
+            const int nvalid = min(p.TT, cu.L - tok0);
+            if (!dead && !mbar_wait(&full[stage], phase, kWaitLimitNs)) {
+                dead = true;
+                atomicOr(p.errors, kErrTimeout);
+            }
+            if (!dead) {
+                const int loaded = reinterpret_cast<volatile int *>(smem + p.lay.off_mask)[stage];
+                const uint8_t *sb = smem + (size_t)stage * p.lay.stage_bytes;
+                process_stage<NT, kPack, kDump, true>(p, st, o, sb, nvalid, loaded, cu.b, cu.hc,
+                                                      kl, slice, tok0, g, c);
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[stage]);
+            }
+            if (++stage == p.n_stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
         }
-        if (!dead) {
-            const int loaded = reinterpret_cast<volatile int *>(smem + p.lay.off_mask)[stage];
-            process_stage<NT, kDump>(p, st, o, sm0 + (uint32_t)stage * p.lay.stage_bytes, nvalid,
-                                     loaded, cu.b, cu.hc, kl, slice, tok0, g, c);
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[stage]);
-        }
-        if (seg_last)
-            finalize_segment(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c, warp * 32 + lane,
-                             prefix, t0, t1, pend);
-        if (++stage == p.n_stages) {
-            stage = 0;
-            phase ^= 1u;
-        }
+        finalize_segment<NT, kPack>(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c,
+                                    warp * 32 + lane, prefix, t0, t1, pend);
     }
     combine_pending(p, smem, pend, cstart, gcta, warp * 32 + lane);
 }
 
-template <int NT, bool kDump>
+template <int NT, bool kPack, bool kDump>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKs,
@@ -1063,16 +1151,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const int gcta = N < (int)gridDim.x ? N : (int)gridDim.x;
-    for (int i = tid; i <= gcta; i += kThreads)
-        cstart[i] = (int)((long long)i * N / gcta);
+    {
+        const int qn = N / (gcta > 0 ? gcta : 1), rn = N - qn * (gcta > 0 ? gcta : 1);
+        for (int i = tid; i <= gcta; i += kThreads)
+            cstart[i] = i * qn + (i * rn) / gcta; // == floor(i * N / gcta)
+    }
     __syncthreads();
     if ((int)blockIdx.x >= gcta)
         return;
     const int t0 = cstart[blockIdx.x], t1 = cstart[blockIdx.x + 1];
-    if (warp == kProducerWarp)
-        produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
-    else
-        consume<NT, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
+    // Warp specialisation: the producer warpgroup hands most of its registers to the two
+    // consumer warpgroups (the sums match the launch allocation, checked by static_assert).
+    if (warp >= kConsumerWarps) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        if (warp == kProducerWarp)
+            produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+        consume<NT, kPack, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
+    }
 }
 
 } // namespace q8kv
