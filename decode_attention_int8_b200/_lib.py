@@ -27,6 +27,7 @@ EXPORTS = (
     "q8kv_workspace_bytes",
     "q8kv_workspace_init",
     "q8kv_decode_attn_ws",
+    "q8kv_decode_attn_static",
     "q8kv_debug_quantize_q",
     "q8kv_debug_block_dots",
     "q8kv_device_errors",
@@ -64,6 +65,7 @@ def lib():
                 "q8kv_workspace_bytes": ([I, I, I, I], Z),
                 "q8kv_workspace_init": ([P, Z, P], I),
                 "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
+                "q8kv_decode_attn_static": ([P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_debug_quantize_q": ([P, P, P, I, I, P], I),
                 "q8kv_debug_block_dots": ([P, I] + [P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
@@ -154,6 +156,19 @@ def q8kv_decode_attn_ws(out, q, k_blocks, v_blocks, kscale, vscale, block_table,
                                      _ptr(seq_lens), *geo, float(scale), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(),
                                      _stream(stream)), "q8kv_decode_attn_ws")
+    return out
+
+
+def q8kv_decode_attn_static(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+                            scale, stream=None):
+    """Decode attention with the library's fixed per-device scratch array (no allocation).
+
+    Calls that may overlap on the GPU race on that array; order them on one stream."""
+    geo = _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens)
+    _check(lib().q8kv_decode_attn_static(_ptr(out), _ptr(q), _ptr(k_blocks), _ptr(v_blocks),
+                                         _ptr(kscale), _ptr(vscale), _ptr(block_table),
+                                         _ptr(seq_lens), *geo, float(scale), _stream(stream)),
+           "q8kv_decode_attn_static")
     return out
 
 

@@ -436,6 +436,55 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
 
 } // namespace
 
+// Scratch of q8kv_decode_attn_static: split-KV counters and partial results at the same
+// offsets as a caller-owned workspace. A file-scope device array rather than an allocation,
+// so that a call of that entry point never allocates: its callers are ones that must not
+// allocate while serving (a pool allocator owns all device memory, or the step cannot take
+// cudaMalloc's latency or cudaFree's device-wide synchronisation). One instance exists per
+// device; calls that may overlap on the GPU share it and therefore race.
+static __device__ __align__(256) unsigned char g_static_scratch[Q8KV_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+struct StaticScratch {
+    bool ready = false;
+    void *ptr = nullptr;
+};
+
+StaticScratch g_static[kMaxDevices];
+
+// Set-up, once per device, with that device current: look up the array's address on this
+// device and zero its counter region on `stream` (the partial slots need no initial value).
+q8kv_status static_scratch(void **out, cudaStream_t stream)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo *dev = nullptr;
+    q8kv_status st = device_info(&dev);
+    if (st != Q8KV_OK)
+        return st;
+    int d = 0;
+    Q8KV_CUDA(cudaGetDevice(&d));
+    StaticScratch &sc = g_static[d];
+    if (!sc.ready) {
+        void *ptr = nullptr;
+        Q8KV_CUDA(cudaGetSymbolAddress((void **)&ptr, g_static_scratch));
+        if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 255u) != 0)
+            return Q8KV_ERR_WORKSPACE;
+        Plan pl;
+        pl.heads_seg = 0;
+        plan_workspace(dev->sms, pl); // counters end where the partial slots begin
+        if (pl.ws_part_off > Q8KV_STATIC_SCRATCH_BYTES)
+            return Q8KV_ERR_WORKSPACE;
+        Q8KV_CUDA(cudaMemsetAsync(ptr, 0, pl.ws_part_off, stream));
+        sc.ptr = ptr;
+        sc.ready = true;
+    }
+    *out = sc.ptr;
+    return Q8KV_OK;
+}
+
+} // namespace
+
 extern "C" {
 
 q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
@@ -490,6 +539,45 @@ q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_bloc
                  num_kv_blocks},
            scale, nullptr, 0};
     return run(c, workspace, workspace_bytes, false, stream);
+}
+
+q8kv_status q8kv_decode_attn_static(float *out, const float *q, const int8_t *k_blocks,
+                                    const int8_t *v_blocks, const float *kscale,
+                                    const float *vscale, const int32_t *block_table,
+                                    const int32_t *seq_lens, int B, int n_q_heads,
+                                    int n_kv_heads, int head_dim, int kv_block_size,
+                                    int max_blocks_per_seq, int num_kv_blocks, float scale,
+                                    cudaStream_t stream)
+{
+    Call c{out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+           Shape{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
+                 num_kv_blocks},
+           scale, nullptr, 0};
+    q8kv_status st = check_call(c); // argument errors before any CUDA call
+    if (st != Q8KV_OK)
+        return st;
+    // Unsupported shapes, and shapes whose workspace exceeds the array, are rejected here,
+    // before set-up enqueues anything.
+    {
+        DeviceInfo *dev = nullptr;
+        {
+            std::lock_guard<std::mutex> lock(g_mutex);
+            st = device_info(&dev);
+        }
+        if (st != Q8KV_OK)
+            return st;
+        Plan pl;
+        st = make_plan(c.s, *dev, pl);
+        if (st != Q8KV_OK)
+            return st;
+        if (pl.ws_bytes > Q8KV_STATIC_SCRATCH_BYTES)
+            return Q8KV_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    st = static_scratch(&scratch, stream);
+    if (st != Q8KV_OK)
+        return st;
+    return run(c, scratch, Q8KV_STATIC_SCRATCH_BYTES, false, stream);
 }
 
 q8kv_status q8kv_debug_quantize_q(int8_t *qi, float *qsc, const float *q, int n_rows,

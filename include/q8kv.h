@@ -123,6 +123,52 @@ q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_bloc
                                 int num_kv_blocks, float scale, void *workspace,
                                 size_t workspace_bytes, cudaStream_t stream);
 
+/* Size of the scratch array that q8kv_decode_attn_static uses (12 MiB per device). */
+#define Q8KV_STATIC_SCRATCH_BYTES (12u * 1024u * 1024u)
+
+/*
+ * Same as q8kv_decode_attn, but the call allocates no device memory at all: the split-KV
+ * counters and partial results live in a fixed device array inside the library,
+ * Q8KV_STATIC_SCRATCH_BYTES bytes per device. None of the source pages has a counterpart
+ * to this entry point; they describe the computation, not where its scratch lives.
+ *
+ * Who needs it: a caller that must not allocate while it serves requests. Examples are a
+ * server whose pool allocator hands out all device memory at start-up (a cudaMalloc then
+ * fails, or takes memory the pool had counted on), and a timed decode step that cannot
+ * afford the device-wide synchronisation of cudaFree or the latency of a first cudaMalloc.
+ * q8kv_decode_attn allocates on its first call per device and again when a shape needs a
+ * larger workspace; q8kv_decode_attn_ws makes the caller allocate one.
+ *
+ * Set-up: the first call on each device (with that device current) looks up the array's
+ * address and enqueues a zeroing of its counter region on `stream`. Later calls do
+ * neither. Make that first call before any stream capture begins.
+ *
+ * Zero state: the counter region at the start of the array (two int arrays of 2 entries
+ * per SM, each padded to 256 bytes) must be zero when a call starts. Set-up zeroes it and every complete call leaves it zero.
+ * After a call that set Q8KV_DEVERR_TIMEOUT the counters are undefined and results of
+ * later calls of this entry point in the same process are not reliable. The partial
+ * results need no initial value.
+ *
+ * Races: every call on one device uses the same array. Two calls that may run at the
+ * same time on the GPU (different streams with no ordering between them, or threads
+ * issuing to different streams) corrupt each other's results. Order them on one stream,
+ * or use q8kv_decode_attn_ws with one workspace per stream. Calls of the other entry
+ * points never touch this array.
+ *
+ * Errors: as q8kv_decode_attn, plus Q8KV_ERR_WORKSPACE (and nothing enqueued) when the
+ * shape needs more than Q8KV_STATIC_SCRATCH_BYTES, i.e. when q8kv_workspace_bytes() for
+ * it is larger. On a 148-SM B200 that happens when one tile covers more than 80 query
+ * heads (a tile holds up to 8 KV heads and all their query heads): n_q_heads 128 with
+ * n_kv_heads 8 or 1 is rejected, 64 with 8 fits.
+ */
+q8kv_status q8kv_decode_attn_static(float *out, const float *q, const int8_t *k_blocks,
+                                    const int8_t *v_blocks, const float *kscale,
+                                    const float *vscale, const int32_t *block_table,
+                                    const int32_t *seq_lens, int B, int n_q_heads,
+                                    int n_kv_heads, int head_dim, int kv_block_size,
+                                    int max_blocks_per_seq, int num_kv_blocks, float scale,
+                                    cudaStream_t stream);
+
 /* Debug: the Q quantisation alone (step 1) on n_rows rows of head_dim fp32 values
  * (head_dim a multiple of 32). qi int8 [n_rows][head_dim], qsc fp32
  * [n_rows][head_dim / 32]. Uses the device routine the decode kernel uses. */
