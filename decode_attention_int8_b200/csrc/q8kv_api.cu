@@ -10,12 +10,15 @@
 #include <mutex>
 
 #include "q8kv.h"
+#include "q8kv_combine.cuh"
 #include "q8kv_decode.cuh"
 #include "q8kv_qquant.cuh"
 
 namespace {
 
 using namespace q8kv;
+
+static_assert(kCombineSlotRow == kSlotRow, "partial row layout differs between the kernels");
 
 __device__ unsigned g_device_errors = 0;
 
@@ -94,7 +97,7 @@ struct Plan {
     int scale_bulk, heads_seg, scratch_stride, grid;
     SmemLayout lay;
     size_t smem_bytes;
-    size_t ws_seg_off, ws_grp_off, ws_part_off, ws_bytes;
+    size_t ws_desc_off, ws_part_off, ws_bytes;
 };
 
 bool is_pow2(int x)
@@ -145,14 +148,12 @@ q8kv_status plan_heads(int Hq, int Hk, int D, Plan &pl)
     return Q8KV_OK;
 }
 
-// Workspace: segment counters and group counters (2 per CTA each, at fixed offsets that do
-// not depend on the shape, so a workspace can serve calls of any shape), then the partial
-// slots (2 per CTA).
+// Workspace: the split-segment descriptors (2 per CTA, rewritten by every call, so no part
+// of the workspace needs an initial value), then the partial slots (2 per CTA).
 void plan_workspace(int grid, Plan &pl)
 {
-    pl.ws_seg_off = 0;
-    pl.ws_grp_off = align256(sizeof(int) * 2 * (size_t)grid);
-    pl.ws_part_off = pl.ws_grp_off + align256(sizeof(int) * 2 * (size_t)grid);
+    pl.ws_desc_off = 0;
+    pl.ws_part_off = align256(sizeof(int4) * 2 * (size_t)grid);
     pl.ws_bytes = pl.ws_part_off +
                   align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * kSlotRow);
 }
@@ -174,6 +175,8 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     if (tiles_max >= (1LL << 31))
         return Q8KV_ERR_UNSUPPORTED; // tile indices are 32-bit
     pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
+    if (2 * pl.grid > kCombineMaxDesc)
+        return Q8KV_ERR_UNSUPPORTED;
     pl.box_tok = pl.TT < s.bs ? pl.TT : s.bs;
     pl.log2_box = ilog2(pl.box_tok);
     pl.n_boxes = pl.TT / pl.box_tok;
@@ -341,8 +344,33 @@ q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl
                                        dev.smem_optin));
         dev.attr_set[variant][kDump ? 1 : 0] = true;
     }
-    fn<<<pl.grid, kThreads, pl.smem_bytes, stream>>>(p, mk, mv, mks, mvs);
-    Q8KV_CUDA(cudaGetLastError());
+    // Both kernels allow programmatic dependent launch: each may be scheduled while the
+    // kernel before it on the stream drains, and waits for it (griddepcontrol.wait) before
+    // touching global memory.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    Q8KV_CUDA(cudaLaunchKernelEx(&cfg, fn, p, mk, mv, mks, mvs));
+
+    CombineParams cp;
+    cp.out = p.out;
+    cp.partials = p.partials;
+    cp.desc = p.split_desc;
+    cp.n_desc = 2 * pl.grid;
+    cp.Hq = p.Hq;
+    cp.heads_seg = p.heads_seg;
+    cudaLaunchConfig_t cc = cfg;
+    cc.gridDim = dim3((unsigned)dev.sms);
+    cc.blockDim = dim3(kCombineThreads);
+    cc.dynamicSmemBytes = 0;
+    Q8KV_CUDA(cudaLaunchKernelEx(&cc, combine_kernel, cp));
     return Q8KV_OK;
 }
 
@@ -371,7 +399,6 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
                 dev->ws_bytes = 0;
             }
             Q8KV_CUDA(cudaMalloc(&dev->ws, pl.ws_bytes));
-            Q8KV_CUDA(cudaMemsetAsync(dev->ws, 0, pl.ws_bytes, stream));
             dev->ws_bytes = pl.ws_bytes;
         }
         ws = dev->ws;
@@ -394,8 +421,7 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.seq_lens = c.lens;
     p.kscale = c.ks;
     p.vscale = c.vs;
-    p.seg_counters = reinterpret_cast<int *>(w + pl.ws_seg_off);
-    p.grp_counters = reinterpret_cast<int *>(w + pl.ws_grp_off);
+    p.split_desc = reinterpret_cast<int4 *>(w + pl.ws_desc_off);
     p.partials = reinterpret_cast<float *>(w + pl.ws_part_off);
     p.errors = dev->errors;
     p.dbg_dots = c.dots;
@@ -454,8 +480,9 @@ struct StaticScratch {
 StaticScratch g_static[kMaxDevices];
 
 // Set-up, once per device, with that device current: look up the array's address on this
-// device and zero its counter region on `stream` (the partial slots need no initial value).
-q8kv_status static_scratch(void **out, cudaStream_t stream)
+// device. No part of the scratch needs an initial value (every call rewrites the
+// split-segment descriptors before the partial slots they point to are read).
+q8kv_status static_scratch(void **out)
 {
     std::lock_guard<std::mutex> lock(g_mutex);
     DeviceInfo *dev = nullptr;
@@ -470,12 +497,6 @@ q8kv_status static_scratch(void **out, cudaStream_t stream)
         Q8KV_CUDA(cudaGetSymbolAddress((void **)&ptr, g_static_scratch));
         if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 255u) != 0)
             return Q8KV_ERR_WORKSPACE;
-        Plan pl;
-        pl.heads_seg = 0;
-        plan_workspace(dev->sms, pl); // counters end where the partial slots begin
-        if (pl.ws_part_off > Q8KV_STATIC_SCRATCH_BYTES)
-            return Q8KV_ERR_WORKSPACE;
-        Q8KV_CUDA(cudaMemsetAsync(ptr, 0, pl.ws_part_off, stream));
         sc.ptr = ptr;
         sc.ready = true;
     }
@@ -574,7 +595,7 @@ q8kv_status q8kv_decode_attn_static(float *out, const float *q, const int8_t *k_
             return Q8KV_ERR_WORKSPACE;
     }
     void *scratch = nullptr;
-    st = static_scratch(&scratch, stream);
+    st = static_scratch(&scratch);
     if (st != Q8KV_OK)
         return st;
     return run(c, scratch, Q8KV_STATIC_SCRATCH_BYTES, false, stream);

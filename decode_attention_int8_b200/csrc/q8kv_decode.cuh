@@ -26,9 +26,11 @@
 //    (score + log2 V scale), so the weight * V scale that enters the f16 halves is at
 //    most 2^15 and the largest one is at least 2^14 (full f16 precision whatever the
 //    spread of the V scales). Both are ordinary online maxima: rescale when they rise.
-//  * Per-warp states are merged in shared memory, and CTAs that share a sequence merge
-//    their partial (M, S, A, acc) through the workspace with a two-level last-arriver
-//    log-sum-exp combine (no waiting on other CTAs, counters reset by the last arriver).
+//  * Per-warp states are merged in shared memory. A segment that one CTA covers whole is
+//    normalised and written out here; a CTA that covers only part of one leaves its
+//    partial (M, S, A, acc) in the workspace, and the first contributor records the
+//    segment in a descriptor for the log-sum-exp combine kernel (q8kv_combine.cuh) that
+//    runs next on the stream. No CTA ever waits for another.
 #pragma once
 
 #include <cuda.h>
@@ -53,7 +55,6 @@ static_assert(4 * 32 * kProducerRegs + 8 * 32 * kConsumerRegs <= kThreads * kLau
 constexpr int kSub = 2;             // 16-token subtiles per consumer warp per stage
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMaxBoxes = 16;       // TMA boxes per stage
-constexpr int kGroupFanIn = 16;     // contributors merged per first-level combine
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
 constexpr int kSlotRow = kD + 4;    // per-head partial: kD accumulator floats, M, S, A, pad
@@ -124,8 +125,7 @@ struct DecodeParams {
     const float *kscale;
     const float *vscale;
     float *partials;     // [2 * grid slots] x heads_seg x kSlotRow (kD acc, M, S, A, pad)
-    int *seg_counters;   // [2 * grid], indexed by the slot of a segment's first contributor
-    int *grp_counters;   // [2 * grid], indexed by the slot of a group leader
+    int4 *split_desc;    // [2 * grid] {b, hc, contributors, first slot}; rewritten every call
     unsigned *errors;    // device error word
     int32_t *dbg_dots;   // [B][Hq][dbg_max_len][kNB] (debug instantiation only)
     int dbg_max_len;
@@ -167,106 +167,6 @@ __device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
             hi = mid - 1;
     }
     return lo;
-}
-
-// Merge n_in partial (M, S, A, acc) slots, listed in shared memory (slots[0..n_in)), into
-// either the output rows of (b, hc) or the slot dest_slot. A slot holds heads_seg rows of
-// kSlotRow floats: acc [kD] (units 2^-A), then M, S, A (base-2 logs, S in units 2^-M).
-// Runs after the main loop, when the stage ring is idle: one thread pulls every input row
-// of a chunk of heads into the ring with bulk copies (one round trip to L2), then all
-// consumer threads combine from shared memory. The code is kept small and rolled: it runs
-// once per call, so its instruction fetches are cold. Called by all consumer threads.
-__device__ __noinline__ void merge_slots(const DecodeParams &p, uint8_t *smem, uint32_t &mphase,
-                                         int n_in, bool to_out, int b, int hc, int dest_slot,
-                                         int ctid)
-{
-    const int H = p.heads_seg;
-    const int *slots = reinterpret_cast<const int *>(smem + p.lay.off_slots);
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + p.lay.off_mbar);
-    float *buf = reinterpret_cast<float *>(smem);
-    const uint32_t row_bytes = kSlotRow * 4;
-    const uint32_t ring = (uint32_t)p.n_stages * p.lay.stage_bytes;
-    int hch = (int)(ring / ((uint32_t)n_in * row_bytes));
-    hch = hch < 1 ? 1 : (hch > H ? H : hch);
-    const int warp = ctid >> 5, lane = ctid & 31;
-    for (int h0 = 0; h0 < H; h0 += hch) {
-        const int hn = (H - h0) < hch ? (H - h0) : hch;
-        // lanes of warp 0 issue one bulk copy each (the partials were written by other CTAs
-        // through the generic proxy, hence the proxy fence)
-        if (warp == 0) {
-            if (lane == 0) {
-                asm volatile("fence.proxy.async.global;" ::: "memory");
-                mbar_arrive_expect_tx(mbar, (uint32_t)n_in * hn * row_bytes);
-            }
-            __syncwarp();
-            if (lane < n_in) {
-                asm volatile("fence.proxy.async.global;" ::: "memory");
-                bulk_load_plain(buf + (size_t)lane * hn * kSlotRow,
-                                p.partials + ((size_t)slots[lane] * H + h0) * kSlotRow,
-                                (uint32_t)hn * row_bytes, mbar);
-            }
-        }
-        if (!mbar_wait(mbar, mphase, kWaitLimitNs))
-            atomicOr(p.errors, kErrTimeout);
-        mphase ^= 1u;
-        // per head (one warp, one lane per input): the maxima, each input's accumulator
-        // factor (written over its M word), and the merged M, A, S (written over input 0's
-        // S, A and pad words)
-        for (int hl = warp; hl < hn; hl += kConsumerWarps) {
-            float m = -INFINITY, a = -INFINITY, sv = 0.f;
-            float *row = buf + ((size_t)lane * hn + hl) * kSlotRow;
-            if (lane < n_in) {
-                m = row[kD];
-                sv = row[kD + 1];
-                a = row[kD + 2];
-            }
-            float mx = m, ax = a;
-            for (int o = 16; o >= 1; o >>= 1) {
-                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, o));
-                ax = fmaxf(ax, __shfl_xor_sync(kFullMask, ax, o));
-            }
-            const float fs = (m == -INFINITY) ? 0.f : exp2f(m - mx);
-            const float fa = (a == -INFINITY) ? 0.f : exp2f(a - ax);
-            float ssum = fs * sv;
-            for (int o = 16; o >= 1; o >>= 1)
-                ssum += __shfl_xor_sync(kFullMask, ssum, o);
-            __syncwarp();
-            if (lane < n_in)
-                row[kD] = fa;
-            if (lane == 0) {
-                row[kD + 1] = mx;
-                row[kD + 2] = ax;
-                row[kD + 3] = ssum;
-            }
-        }
-        consumer_bar();
-        for (int u = ctid; u < hn * (kD / 4); u += kConsumerThreads) {
-            const int hl = u / (kD / 4), d4 = u % (kD / 4);
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-            const float *row = buf + (size_t)hl * kSlotRow;
-            for (int k = 0; k < n_in; ++k, row += (size_t)hn * kSlotRow) {
-                const float fa = row[kD];
-                const float4 v = *reinterpret_cast<const float4 *>(row + d4 * 4);
-                a.x += fa * v.x;
-                a.y += fa * v.y;
-                a.z += fa * v.z;
-                a.w += fa * v.w;
-            }
-            const float4 hdr = *reinterpret_cast<const float4 *>(buf + (size_t)hl * kSlotRow + kD);
-            if (to_out) {
-                const float f = hdr.w > 0.f ? exp2f(hdr.z - hdr.y) / hdr.w : 0.f;
-                const int h = hc * H + h0 + hl;
-                float4 o = make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
-                *reinterpret_cast<float4 *>(p.out + ((long long)b * p.Hq + h) * kD + d4 * 4) = o;
-            } else {
-                float *drow = p.partials + ((size_t)dest_slot * H + h0 + hl) * kSlotRow;
-                *reinterpret_cast<float4 *>(drow + d4 * 4) = a;
-                if (d4 == 0)
-                    *reinterpret_cast<float4 *>(drow + kD) = make_float4(hdr.y, hdr.w, hdr.z, 0.f);
-            }
-        }
-        consumer_bar(); // the ring is refilled for the next chunk
-    }
 }
 
 // Per-sequence tile prefix: prefix[b + 1] = sum over b' <= b of nhc * ceil(L_b' / TT).
@@ -766,20 +666,13 @@ __device__ __forceinline__ void store_row16(float *dst, const WarpState<NT> &st,
     }
 }
 
-// Segments of this CTA that other CTAs share (at most two), combined after the main loop.
-struct Pending {
-    struct Seg {
-        int b, hc, seg0, seg1;
-    } seg[2];
-    int n;
-};
-
 // End of a segment (all of this CTA's tiles of sequence b, head chunk hc).
 template <int NT, bool kPack>
 __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st,
                                                  uint8_t *smem, int b,
                                  int hc, int kl, int slice, int pair, int ts, int g, int c,
-                                 int ctid, const int *prefix, int t0, int t1, Pending &pend)
+                                 int ctid, const int *prefix, const int *cstart, int gcta,
+                                 int t0, int t1)
 {
     // complete this lane's row sums
 #pragma unroll
@@ -885,8 +778,9 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
         return;
     }
 
-    // partial: this CTA's share of the segment goes to its workspace slot; the cross-CTA
-    // combine runs after the main loop (combine_pending)
+    // partial: this CTA's share of the segment goes to its workspace slot (0: the segment
+    // this CTA's range starts in, 1: the one it ends in); the first contributor describes
+    // the segment for the combine kernel
     const int which = (seg0 <= t0) ? 0 : 1;
     const int H = p.heads_seg;
     if (ts == 0) {
@@ -910,97 +804,10 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
             }
         }
     }
-    pend.seg[pend.n].b = b;
-    pend.seg[pend.n].hc = hc;
-    pend.seg[pend.n].seg0 = seg0;
-    pend.seg[pend.n].seg1 = seg1;
-    ++pend.n;
-}
-
-// Cross-CTA combine of this CTA's partial segments (at most two: the one it started in
-// and the one it ended in). Every contributor bumps a counter; the last one to arrive
-// merges (for more than kGroupFanIn contributors: per group of kGroupFanIn, then the
-// groups). Counters live in the workspace and are reset by the last arriver, so no CTA
-// ever waits for another.
-__device__ void combine_pending(const DecodeParams &p, uint8_t *smem, const Pending &pend,
-                                const int *cstart, int gcta, int ctid)
-{
-    if (pend.n == 0)
-        return;
-    volatile int *misc = reinterpret_cast<volatile int *>(smem + p.lay.off_misc);
-    uint32_t mphase = 0;
-    __threadfence();
-    consumer_bar();
-    int first[2], last[2], n[2], ctr[2];
-    int *cnt[2];
-    for (int i = 0; i < pend.n; ++i) {
-        const Pending::Seg &sg = pend.seg[i];
-        first[i] = cta_of_tile(cstart, gcta, sg.seg0);
-        last[i] = cta_of_tile(cstart, gcta, sg.seg1 - 1);
-        n[i] = last[i] - first[i] + 1;
-        const int f = first[i];
-        if (n[i] <= kGroupFanIn) {
-            cnt[i] = p.seg_counters + 2 * f + ((sg.seg0 <= cstart[f]) ? 0 : 1);
-            ctr[i] = n[i];
-        } else {
-            const int leader = f + (((int)blockIdx.x - f) / kGroupFanIn) * kGroupFanIn;
-            cnt[i] = p.grp_counters + 2 * leader + ((sg.seg0 <= cstart[leader]) ? 0 : 1);
-            ctr[i] = min(kGroupFanIn, last[i] + 1 - leader);
-        }
-    }
-    if (ctid == 0) {
-        int tk[2] = {0, 0};
-        for (int i = 0; i < pend.n; ++i)
-            tk[i] = atomicAdd(cnt[i], 1);
-        for (int i = 0; i < pend.n; ++i)
-            misc[1 + i] = (tk[i] == ctr[i] - 1) ? 1 : 0;
-    }
-    consumer_bar();
-    int is_last[2] = {misc[1], pend.n > 1 ? misc[2] : 0};
-    consumer_bar();
-    for (int i = 0; i < pend.n; ++i) {
-        if (!is_last[i])
-            continue;
-        const Pending::Seg &sg = pend.seg[i];
-        const int f = first[i];
-        int *slots = reinterpret_cast<int *>(smem + p.lay.off_slots);
-        auto which_of = [&](int c) { return (sg.seg0 <= cstart[c]) ? 0 : 1; };
-        __threadfence();
-        if (n[i] <= kGroupFanIn) {
-            if (ctid < n[i])
-                slots[ctid] = 2 * (f + ctid) + which_of(f + ctid);
-            consumer_bar();
-            merge_slots(p, smem, mphase, n[i], true, sg.b, sg.hc, 0, ctid);
-            if (ctid == 0)
-                *cnt[i] = 0;
-            continue;
-        }
-        const int leader = f + (((int)blockIdx.x - f) / kGroupFanIn) * kGroupFanIn;
-        const int lslot = 2 * leader + which_of(leader);
-        if (ctid < ctr[i])
-            slots[ctid] = 2 * (leader + ctid) + which_of(leader + ctid);
-        consumer_bar();
-        merge_slots(p, smem, mphase, ctr[i], false, sg.b, sg.hc, lslot, ctid);
-        __threadfence();
-        consumer_bar();
-        const int ngroups = (n[i] + kGroupFanIn - 1) / kGroupFanIn;
-        int *segc = p.seg_counters + 2 * f + which_of(f);
-        if (ctid == 0) {
-            *cnt[i] = 0;
-            misc[3] = (atomicAdd(segc, 1) == ngroups - 1) ? 1 : 0;
-        }
-        consumer_bar();
-        const bool seg_last = misc[3] != 0;
-        consumer_bar();
-        if (seg_last) {
-            __threadfence();
-            if (ctid < ngroups)
-                slots[ctid] = 2 * (f + ctid * kGroupFanIn) + which_of(f + ctid * kGroupFanIn);
-            consumer_bar();
-            merge_slots(p, smem, mphase, ngroups, true, sg.b, sg.hc, 0, ctid);
-            if (ctid == 0)
-                *segc = 0;
-        }
+    if (ctid == 0 && seg0 >= t0) {
+        const int last = cta_of_tile(cstart, gcta, seg1 - 1);
+        const int slot = 2 * (int)blockIdx.x + which;
+        p.split_desc[slot] = make_int4(b, hc, last - (int)blockIdx.x + 1, slot);
     }
 }
 
@@ -1055,8 +862,6 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         for (int j = 0; j < kNB; ++j)
             st.qs[r][j] = 0.f;
 
-    Pending pend;
-    pend.n = 0;
     bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
     int stage = 0;
     uint32_t phase = 0;
@@ -1101,9 +906,8 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
             }
         }
         finalize_segment<NT, kPack>(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c,
-                                    warp * 32 + lane, prefix, t0, t1, pend);
+                                    warp * 32 + lane, prefix, cstart, gcta, t0, t1);
     }
-    combine_pending(p, smem, pend, cstart, gcta, warp * 32 + lane);
 }
 
 template <int NT, bool kPack, bool kDump>
@@ -1136,6 +940,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmKs);
             tma_prefetch_desc(&tmVs);
         }
+    }
+    // Everything above touches only shared memory and kernel parameters; from here on the
+    // previous kernel on the stream (another call's combine, which reads the workspace, or
+    // a producer of the inputs) must be complete.
+    grid_dep_wait();
+    grid_dep_launch();
+    if (tid == 0) { // no split segment recorded yet in this CTA's descriptor slots
+        p.split_desc[2 * blockIdx.x] = make_int4(0, 0, 0, 0);
+        p.split_desc[2 * blockIdx.x + 1] = make_int4(0, 0, 0, 0);
     }
     build_prefix(p, prefix, misc + 2, tid, warp, lane);
     __syncthreads();

@@ -19,6 +19,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Wait until the grid this one depends on (the previous kernel on the stream, when both
+// were launched with programmatic stream serialisation) has completed and its memory is
+// visible. A no-op for an ordinary launch.
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel on the stream to be scheduled (it still waits in grid_dep_wait for
+// this grid to complete before it touches memory).
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarriers
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)

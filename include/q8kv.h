@@ -17,8 +17,11 @@
  *      computed in one pass with a running max M and running sum S (online softmax) and
  *      one division at the end.
  * The scan is split over the sequence across thread blocks (flash-decoding) and the
- * pieces are merged with a log-sum-exp combine inside the same launch; the result equals
- * the single pass up to fp32 rounding order.
+ * pieces are merged by a log-sum-exp combine kernel launched right after the decode
+ * kernel on the same stream; the result equals the single pass up to fp32 rounding order.
+ * Both kernels use programmatic dependent launch: each may be scheduled while the kernel
+ * before it on the stream drains, and waits for that kernel to complete before it reads
+ * or writes global memory.
  *
  * Layouts (all row-major, C order):
  *   q            fp32  [B][n_q_heads][head_dim]
@@ -108,13 +111,13 @@ q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
  * (0 if the sizes are invalid or unsupported). */
 size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim);
 
-/* Zero a caller-owned workspace (required once before its first use; the kernels leave
- * it zeroed again after every complete call). */
+/* Zero a caller-owned workspace. Optional: no part of the workspace needs an initial value
+ * (every call rewrites the bookkeeping it reads). */
 q8kv_status q8kv_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Same as q8kv_decode_attn with a caller-owned workspace (device memory of at least
- * q8kv_workspace_bytes() bytes, 256-byte aligned, zeroed once by q8kv_workspace_init).
- * The call allocates nothing. Calls that overlap on the GPU must not share a workspace. */
+ * q8kv_workspace_bytes() bytes, 256-byte aligned, any contents). The call allocates
+ * nothing. Calls that overlap on the GPU must not share a workspace. */
 q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_blocks,
                                 const int8_t *v_blocks, const float *kscale,
                                 const float *vscale, const int32_t *block_table,
@@ -140,14 +143,12 @@ q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_bloc
  * larger workspace; q8kv_decode_attn_ws makes the caller allocate one.
  *
  * Set-up: the first call on each device (with that device current) looks up the array's
- * address and enqueues a zeroing of its counter region on `stream`. Later calls do
- * neither. Make that first call before any stream capture begins.
+ * address (cudaGetSymbolAddress) and the kernels' attributes; later calls reuse them.
+ * Make that first call before any stream capture begins.
  *
- * Zero state: the counter region at the start of the array (two int arrays of 2 entries
- * per SM, each padded to 256 bytes) must be zero when a call starts. Set-up zeroes it and every complete call leaves it zero.
- * After a call that set Q8KV_DEVERR_TIMEOUT the counters are undefined and results of
- * later calls of this entry point in the same process are not reliable. The partial
- * results need no initial value.
+ * Initial state: nothing in the array needs to start at zero. Every call first rewrites
+ * the split-segment descriptors (2 per CTA), then the partial results they point to, and
+ * the combine kernel reads only what the same call wrote.
  *
  * Races: every call on one device uses the same array. Two calls that may run at the
  * same time on the GPU (different streams with no ordering between them, or threads
