@@ -18,7 +18,10 @@
 // and waits for its completion before reading anything). The work is the list of units
 // (segment, query head, 32-channel quarter), split evenly over the CTAs; a CTA processes
 // up to 32 units at a time, giving each unit 32 / units-in-batch rows of 8 threads that
-// stride over the unit's inputs, so short and long input lists both keep loads in flight.
+// stride over the unit's inputs. A thread issues the loads of up to 8 inputs at once, so a
+// unit usually costs one round trip to L2 whatever its input count; maxima are taken
+// before any rescaling, so no exponential waits on another, and the rows of a unit are
+// merged through shared memory the same way.
 #pragma once
 
 #include <cstdint>
@@ -40,38 +43,37 @@ struct CombineParams {
     int Hq, heads_seg;
 };
 
-__device__ __forceinline__ float group_max(float v, int width)
-{
-    for (int o = (width < 32 ? width : 32) >> 1; o >= 1; o >>= 1)
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
-__device__ __forceinline__ float group_sum(float v, int width)
-{
-    for (int o = (width < 32 ? width : 32) >> 1; o >= 1; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
+constexpr int kCombineBatchIn = 8; // inputs a thread loads at once
 
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const __grid_constant__ CombineParams p)
 {
-    __shared__ int list[kCombineMaxDesc];
+    __shared__ int4 sdesc[kCombineMaxDesc];
     __shared__ int wcount[kCombineThreads / 32];
-    __shared__ float red[3][kCombineThreads / 32];
-    __shared__ float4 part[32][8];
+    __shared__ float4 part_acc[32][8];
+    __shared__ float2 part_ma[32];
+    __shared__ float part_s[32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the decode kernel's partials and descriptors are complete and visible after this
     grid_dep_wait();
     grid_dep_launch();
 
-    // compact list of the descriptors that start a split segment (same order in every CTA)
+    // compact copy of the descriptors that start a split segment (same order in every
+    // CTA); all descriptor loads are issued before the first is used
+    constexpr int kDescPerThread = kCombineMaxDesc / kCombineThreads;
+    int4 dv[kDescPerThread];
+#pragma unroll
+    for (int k = 0; k < kDescPerThread; ++k) {
+        const int i = k * kCombineThreads + tid;
+        dv[k] = i < p.n_desc ? __ldcg(&p.desc[i]) : make_int4(0, 0, 0, 0);
+    }
     int nvalid = 0;
-    for (int base = 0; base < p.n_desc; base += kCombineThreads) {
-        const int i = base + tid;
-        const bool v = i < p.n_desc && __ldcg(&p.desc[i].z) > 0;
+#pragma unroll
+    for (int k = 0; k < kDescPerThread; ++k) {
+        if (k * kCombineThreads >= p.n_desc)
+            break;
+        const bool v = dv[k].z > 0;
         const unsigned m = __ballot_sync(0xffffffffu, v);
         if (lane == 0)
             wcount[warp] = __popc(m);
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(kCombineThreads)
             total += wcount[w];
         }
         if (v)
-            list[off + __popc(m & ((1u << lane) - 1u))] = i;
+            sdesc[off + __popc(m & ((1u << lane) - 1u))] = dv[k];
         nvalid += total;
         __syncthreads();
     }
@@ -99,8 +101,7 @@ __global__ void __launch_bounds__(kCombineThreads)
         int upow = 1;
         while (upow < U)
             upow <<= 1;
-        const int IG = 32 / upow;        // input-group rows per unit
-        const int width = IG * 8;        // threads per unit (contiguous, aligned)
+        const int IG = 32 / upow; // rows per unit; row ig takes inputs ig, ig + IG, ...
         const int u = row / IG, ig = row % IG;
         const bool active = u < U;
         int b = 0, hc = 0, n = 0, first = 0, hl = 0, q = 0;
@@ -110,87 +111,89 @@ __global__ void __launch_bounds__(kCombineThreads)
             const int rem = (int)(unit - (long long)d * per_seg);
             hl = rem / (128 / kCombineQuarter);
             q = rem % (128 / kCombineQuarter);
-            const int4 ds = __ldcg(&p.desc[list[d]]);
+            const int4 ds = sdesc[d];
             b = ds.x;
             hc = ds.y;
             n = ds.z;
             first = ds.w;
         }
-        auto slot_of = [&](int i) { return i == 0 ? first : 2 * ((first >> 1) + i); };
-        auto header = [&](int i) {
-            return __ldcg(reinterpret_cast<const float4 *>(
-                p.partials + ((size_t)slot_of(i) * H + hl) * kCombineSlotRow + 128));
-        };
-        // maxima of M and A over the unit's inputs
-        float mx = -INFINITY, ax = -INFINITY;
-        for (int i = ig * 8 + fl; i < n; i += width) {
-            const float4 h = header(i);
-            mx = fmaxf(mx, h.x);
-            ax = fmaxf(ax, h.z);
-        }
-        mx = group_max(mx, width);
-        ax = group_max(ax, width);
-        if (width > 32) { // all threads agree on width, so the barriers are uniform
-            if (lane == 0) {
-                red[0][warp] = mx;
-                red[1][warp] = ax;
+        // this row's inputs: per chunk of kCombineBatchIn, all loads first, then the
+        // maxima, then the rescaled sums (no chain of dependent exponentials)
+        float m = -INFINITY, a = -INFINITY, s = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = ig; i0 < n; i0 += kCombineBatchIn * IG) {
+            float4 hd[kCombineBatchIn], x[kCombineBatchIn];
+#pragma unroll
+            for (int k = 0; k < kCombineBatchIn; ++k) {
+                const int i = i0 + k * IG;
+                hd[k] = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+                x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < n) {
+                    const int slot = i == 0 ? first : 2 * ((first >> 1) + i);
+                    const float *rp = p.partials + ((size_t)slot * H + hl) * kCombineSlotRow;
+                    hd[k] = __ldcg(reinterpret_cast<const float4 *>(rp + 128));
+                    x[k] = __ldcg(reinterpret_cast<const float4 *>(rp + q * kCombineQuarter + 4 * fl));
+                }
             }
-            __syncthreads();
-            const int w0 = (u * width) >> 5, nw = width >> 5;
-            mx = -INFINITY;
-            ax = -INFINITY;
-            for (int w = 0; w < nw && active; ++w) {
-                mx = fmaxf(mx, red[0][w0 + w]);
-                ax = fmaxf(ax, red[1][w0 + w]);
+            float mn = m, an = a;
+#pragma unroll
+            for (int k = 0; k < kCombineBatchIn; ++k) {
+                mn = fmaxf(mn, hd[k].x);
+                an = fmaxf(an, hd[k].z);
             }
-            __syncthreads();
+            const float fo = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+            const float go = (a == -INFINITY) ? 0.f : exp2f(a - an);
+            s *= fo;
+            acc = make_float4(acc.x * go, acc.y * go, acc.z * go, acc.w * go);
+#pragma unroll
+            for (int k = 0; k < kCombineBatchIn; ++k) {
+                const float fm = (hd[k].x == -INFINITY) ? 0.f : exp2f(hd[k].x - mn);
+                const float ga = (hd[k].z == -INFINITY) ? 0.f : exp2f(hd[k].z - an);
+                s += hd[k].y * fm;
+                acc.x += x[k].x * ga;
+                acc.y += x[k].y * ga;
+                acc.z += x[k].z * ga;
+                acc.w += x[k].w * ga;
+            }
+            m = mn;
+            a = an;
         }
-        // S = sum_i S_i 2^(M_i - mx)
-        float ssum = 0.f;
-        for (int i = ig * 8 + fl; i < n; i += width) {
-            const float4 h = header(i);
-            if (h.x != -INFINITY)
-                ssum += h.y * exp2f(h.x - mx);
-        }
-        ssum = group_sum(ssum, width);
-        if (width > 32) {
-            if (lane == 0)
-                red[2][warp] = ssum;
-            __syncthreads();
-            const int w0 = (u * width) >> 5, nw = width >> 5;
-            ssum = 0.f;
-            for (int w = 0; w < nw && active; ++w)
-                ssum += red[2][w0 + w];
-        }
-        // accumulators: row ig of the unit takes inputs ig, ig + IG, ...
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i = ig; i < n; i += IG) {
-            const size_t r = ((size_t)slot_of(i) * H + hl) * kCombineSlotRow;
-            const float ai = __ldcg(p.partials + r + 130);
-            const float f = (ai == -INFINITY) ? 0.f : exp2f(ai - ax);
-            const float4 x = __ldcg(reinterpret_cast<const float4 *>(
-                p.partials + r + q * kCombineQuarter + 4 * fl));
-            a.x += f * x.x;
-            a.y += f * x.y;
-            a.z += f * x.z;
-            a.w += f * x.w;
-        }
-        part[row][fl] = a;
+        // merge the unit's rows: maxima first, then every row rescales its own piece, then
+        // row 0 of the unit adds them up
+        if (fl == 0)
+            part_ma[row] = make_float2(m, a);
+        __syncthreads();
+        const int r0 = u * IG;
+        float um = -INFINITY, ua = -INFINITY;
+        if (active)
+            for (int k = 0; k < IG; ++k) {
+                const float2 o = part_ma[r0 + k];
+                um = fmaxf(um, o.x);
+                ua = fmaxf(ua, o.y);
+            }
+        const float fr = (m == -INFINITY) ? 0.f : exp2f(m - um);
+        const float gr = (a == -INFINITY) ? 0.f : exp2f(a - ua);
+        part_acc[row][fl] = make_float4(acc.x * gr, acc.y * gr, acc.z * gr, acc.w * gr);
+        if (fl == 0)
+            part_s[row] = s * fr;
         __syncthreads();
         if (active && ig == 0) {
+            float4 t = part_acc[r0][fl];
+            float st = part_s[r0];
             for (int k = 1; k < IG; ++k) {
-                const float4 o = part[row + k][fl];
-                a.x += o.x;
-                a.y += o.y;
-                a.z += o.z;
-                a.w += o.w;
+                const float4 o = part_acc[r0 + k][fl];
+                t.x += o.x;
+                t.y += o.y;
+                t.z += o.z;
+                t.w += o.w;
+                st += part_s[r0 + k];
             }
-            const float f = ssum > 0.f ? exp2f(ax - mx) / ssum : 0.f;
+            const float f = st > 0.f ? exp2f(ua - um) / st : 0.f;
             float *dst = p.out + ((long long)b * p.Hq + (long long)hc * H + hl) * 128 +
                          q * kCombineQuarter + 4 * fl;
-            *reinterpret_cast<float4 *>(dst) = make_float4(a.x * f, a.y * f, a.z * f, a.w * f);
+            *reinterpret_cast<float4 *>(dst) = make_float4(t.x * f, t.y * f, t.z * f, t.w * f);
         }
-        __syncthreads(); // part[] is reused by the next batch
+        __syncthreads(); // part_* are reused by the next batch
     }
 }
 

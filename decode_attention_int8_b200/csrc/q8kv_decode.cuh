@@ -681,7 +681,8 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
         st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 2);
     }
 
-    // merge the token subtiles of each (KV head, slice) pair inside the CTA
+    // merge the token subtiles of each (KV head, slice) pair inside the CTA (the scratch
+    // holds accumulator element e of lane l at e * 32 + l: conflict-free bank access)
     if (p.subtiles > 1) {
         float *scr = reinterpret_cast<float *>(smem + p.lay.off_scratch);
         const int lane = g * 4 + c;
@@ -693,7 +694,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        reg[lane * (32 * NT) + (pv * 8 + i) * 4 + k] = st.acc[pv][i][k];
+                        reg[((pv * 8 + i) * 4 + k) * 32 + lane] = st.acc[pv][i][k];
             if (c == 0) {
 #pragma unroll
                 for (int r = 0; r < NT; ++r) {
@@ -720,10 +721,10 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             st.acc[pv][i][q] = st.acc[pv][i][q] * fa +
-                                               reg[lane * (32 * NT) + (pv * 8 + i) * 4 + q] * fo;
+                                               reg[((pv * 8 + i) * 4 + q) * 32 + lane] * fo;
                             st.acc[pv][i][q + 2] =
                                 st.acc[pv][i][q + 2] * fa +
-                                reg[lane * (32 * NT) + (pv * 8 + i) * 4 + q + 2] * fo;
+                                reg[((pv * 8 + i) * 4 + q + 2) * 32 + lane] * fo;
                         }
                     }
                 }
