@@ -37,6 +37,7 @@ UNIT = "GB/s"
 DEFAULT_CONFIG = 1  # the batched GQA decode workload the metric is quoted on
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAK_GBS = 6650.0
+LAUNCHES_PER_CALL = 2  # decode kernel + split combine kernel
 
 
 def parse():
@@ -56,6 +57,22 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def reduce_max(x: float, pg, device) -> float:
+    """Maximum of a per-rank time over all ranks (the slowest rank bounds the job)."""
+    if pg is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the workload."""
+    return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
 
 
 def measured_peak():
@@ -78,6 +95,7 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.window = None
 
     def start(self):
         try:
@@ -92,7 +110,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self, t0: float, t1: float):
+        """Keep only the samples taken between host times t0 and t1 (the timed region)."""
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
@@ -105,7 +127,11 @@ class ClockSampler:
         self.thread.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.window is not None:
+            inside = [(t, ln) for t, ln in lines if self.window[0] <= t <= self.window[1]]
+            lines = inside if inside else lines
+        for _, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -279,6 +305,7 @@ def main():
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
+    host_t0 = time.monotonic()
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_begin.record(stream)
@@ -288,17 +315,17 @@ def main():
         ends[i].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    host_t1 = time.monotonic()
     barrier()
+    time.sleep(0.15)  # let the sampler deliver the last in-window line
+    sampler.mark(host_t0, host_t1)
     clocks = sampler.stop()
     total_ms = t_begin.elapsed_time(t_end)
     per_call = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     kernel_ms = statistics.fmean(per_call)
-    if pg is not None:
-        tt = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = reduce_max(total_ms, pg, dev)
     ms_per_step = total_ms / args.steps
-    value = algo * world / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbs(algo, world, ms_per_step)
 
     # end to end through the C ABI with host buffers: per step copy q / block table /
     # seq_lens from pinned host memory, decode, copy out back (the KV cache stays resident)
@@ -327,11 +354,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1) / e2e_steps
-        if pg is not None:
-            tt = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": round(algo * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+        e2e_ms = reduce_max(e2e_ms, pg, dev)
+        e2e = {"value": round(whole_job_gbs(algo, world, e2e_ms), 2), "unit": UNIT,
                "h2d_bytes_per_step": int(w.q.nbytes + w.block_table.nbytes + w.seq_lens.nbytes),
                "d2h_bytes_per_step": int(w.q.nbytes), "us_per_step": round(e2e_ms * 1e3, 3),
                "steps": e2e_steps}
@@ -358,9 +382,10 @@ def main():
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
-                     "traffic": traffic, "kernel": "q8kv::decode_kernel",
+                     "traffic": traffic,
+                     "kernel": "q8kv::decode_kernel + q8kv::combine_kernel (one call)",
                      "kernel_us": round(kernel_ms * 1e3, 3)},
-        "gpu_launches": args.steps,
+        "gpu_launches": LAUNCHES_PER_CALL * args.steps,
         "clocks": clocks,
     }
     if e2e is not None:
