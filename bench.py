@@ -363,16 +363,15 @@ def main():
     peak, peak_kind = measured_peak()
     achieved = algo / (kernel_ms * 1e-3) / 1e9
     traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    tpath = os.path.join(ROOT, "profiles", "traffic.txt")
     if os.path.exists(tpath):
-        try:
-            with open(tpath) as f:
-                tinfo = json.load(f)
-            ent = tinfo.get(c.name)
-            if ent and ent.get("kernel_source_hash") == source_hash():
-                traffic = ent["bytes_per_launch"]
-        except Exception:
-            traffic = None
+        h = source_hash()
+        with open(tpath) as f:
+            for ln in f:
+                parts = ln.split()
+                if len(parts) == 3 and not ln.startswith("#") and parts[0] == c.name \
+                        and parts[1] == h:
+                    traffic = int(parts[2])
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),

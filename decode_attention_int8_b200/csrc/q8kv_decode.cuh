@@ -607,34 +607,25 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
         }
         st.S[r] = st.S[r] * alpha_s + ws;
     }
-    // ---- rescale the accumulator columns whose A rose (in packed mode rows 4-7 repeat
-    // rows 0-3, so the source lane of column col carries head col & 3 either way)
+    // ---- rescale factors of the accumulator columns (in packed mode rows 4-7 repeat rows
+    // 0-3, so the source lane of column col carries head col & 3 either way)
+    float f0[NT], f1[NT];
 #pragma unroll
     for (int pv = 0; pv < NT; ++pv) {
-        const float f0 = __shfl_sync(kFullMask, alpha_a[pv], 8 * c);
-        const float f1 = __shfl_sync(kFullMask, alpha_a[pv], 8 * c + 4);
-        if (__any_sync(kFullMask, (f0 != 1.f) || (f1 != 1.f))) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                st.acc[pv][i][0] *= f0;
-                st.acc[pv][i][1] *= f1;
-                st.acc[pv][i][2] *= f0;
-                st.acc[pv][i][3] *= f1;
-            }
-        }
+        f0[pv] = __shfl_sync(kFullMask, alpha_a[pv], 8 * c);
+        f1[pv] = __shfl_sync(kFullMask, alpha_a[pv], 8 * c + 4);
     }
     // ---- PV: rows = channels 16g + 2i (+1), k = tokens, columns = heads (packed mode:
-    // columns 0-3 high halves of heads 0-3, columns 4-7 their low halves)
+    // columns 0-3 high halves of heads 0-3, columns 4-7 their low halves). The stage's
+    // products are summed in a fresh tensor-core accumulator and folded into the running
+    // one with one round-to-nearest FFMA (which also applies the rescale factor): the
+    // tensor-core accumulation does not round to nearest, so chaining every stage of a
+    // long scan through it would let its error grow with the scan length.
 #pragma unroll
-    for (int u = 0; u < kSub; ++u) {
-        uint32_t b0[NT], b1[NT];
+    for (int i = 0; i < 8; ++i) {
+        float d[NT][4];
 #pragma unroll
-        for (int pv = 0; pv < NT; ++pv) {
-            b0[pv] = (kPack && g >= 4) ? bl[pv][u][0] : bh[pv][u][0];
-            b1[pv] = (kPack && g >= 4) ? bl[pv][u][1] : bh[pv][u][1];
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int u = 0; u < kSub; ++u) {
             const uint32_t w0 = word_of(R[u][0], i >> 1), w1 = word_of(R[u][1], i >> 1);
             const uint32_t w2 = word_of(R[u][2], i >> 1), w3 = word_of(R[u][3], i >> 1);
             const uint32_t sl = (i & 1) ? 0x0602u : 0x0400u;
@@ -645,10 +636,22 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
             const uint32_t a3 = s8pair_to_f16x2(prmt(w2, w3, sh));
 #pragma unroll
             for (int pv = 0; pv < NT; ++pv) {
-                mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, b0[pv], b1[pv]);
+                const uint32_t b0 = (kPack && g >= 4) ? bl[pv][u][0] : bh[pv][u][0];
+                const uint32_t b1 = (kPack && g >= 4) ? bl[pv][u][1] : bh[pv][u][1];
+                if (u == 0)
+                    mma_f16_16816_zero_c(d[pv], a0, a1, a2, a3, b0, b1);
+                else
+                    mma_f16_16816(d[pv], a0, a1, a2, a3, b0, b1);
                 if constexpr (!kPack)
-                    mma_f16_16816(st.acc[pv][i], a0, a1, a2, a3, bl[pv][u][0], bl[pv][u][1]);
+                    mma_f16_16816(d[pv], a0, a1, a2, a3, bl[pv][u][0], bl[pv][u][1]);
             }
+        }
+#pragma unroll
+        for (int pv = 0; pv < NT; ++pv) {
+            st.acc[pv][i][0] = fmaf(st.acc[pv][i][0], f0[pv], d[pv][0]);
+            st.acc[pv][i][1] = fmaf(st.acc[pv][i][1], f1[pv], d[pv][1]);
+            st.acc[pv][i][2] = fmaf(st.acc[pv][i][2], f0[pv], d[pv][2]);
+            st.acc[pv][i][3] = fmaf(st.acc[pv][i][3], f1[pv], d[pv][3]);
         }
     }
 }

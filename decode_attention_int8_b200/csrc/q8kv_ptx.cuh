@@ -222,6 +222,17 @@ __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D(16x8 f32) = A(16x16 f16, row) * B(16x8 f16, col), accumulator input zero.
+__device__ __forceinline__ void mma_f16_16816_zero_c(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                     uint32_t a2, uint32_t a3, uint32_t b0,
+                                                     uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
 // ---------------------------------------------------------------- bit tricks
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
