@@ -192,6 +192,16 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     }
     if (pl.n_stages == 0)
         return Q8KV_ERR_UNSUPPORTED;
+    // The quantised query of each CTA's second segment is prepared in the prologue when the
+    // buffer fits next to the stages (it never costs a stage).
+    {
+        const uint32_t rows = pl.G <= 4 ? 4u : 8u * (uint32_t)pl.NT;
+        const uint32_t need = (uint32_t)pl.pairs * rows * kQRowBytes;
+        if ((size_t)pl.lay.off_qbuf + need + 1024 <= (size_t)dev.smem_optin) {
+            pl.lay.qbuf_rows = rows;
+            pl.lay.total = pl.lay.off_qbuf + need;
+        }
+    }
     pl.smem_bytes = (size_t)pl.lay.total + 1024;
     plan_workspace(dev.sms, pl); // sized for the full grid so one size fits all calls
     return Q8KV_OK;

@@ -48,17 +48,32 @@ constexpr int kConsumerWarps = 8;   // warps 0-7 (two warpgroups)
 constexpr int kProducerWarp = 8;    // warp 8 (its warpgroup, warps 8-11, gives registers away)
 constexpr int kThreads = 12 * 32;
 constexpr int kLaunchRegs = 168;    // per-thread registers at launch (65536 / 384, rounded)
-constexpr int kProducerRegs = 56;   // after setmaxnreg.dec (producer warpgroup)
-constexpr int kConsumerRegs = 224;  // after setmaxnreg.inc (consumer warpgroups)
-static_assert(4 * 32 * kProducerRegs + 8 * 32 * kConsumerRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
+// Per-thread registers after setmaxnreg: the producer warpgroup gives registers to the two
+// consumer warpgroups. One 8-row query tile (NT == 1) fits in 200 consumer registers with
+// 96 left to the producer (no spills); the packed path's int32 PV accumulators need 216, and
+// two query tiles 224.
+template <int NT, bool kPack>
+struct RegSplit {
+    static constexpr int producer = kPack ? 72 : (NT == 1 ? 96 : 56);
+    static constexpr int consumer = kPack ? 216 : (NT == 1 ? 200 : 224);
+    static_assert(4 * 32 * producer + 8 * 32 * consumer <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+};
 constexpr int kSub = 2;             // 16-token subtiles per consumer warp per stage
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMaxBoxes = 16;       // TMA boxes per stage
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
 constexpr int kSlotRow = kD + 4;    // per-head partial: kD accumulator floats, M, S, A, pad
-constexpr float kVExpLimit = 100.f; // V-scale exponents are clamped to [-100, 100]
+constexpr uint32_t kScaleGap = 1024; // bytes from a stage's K scales to its V scales (>= TT*HPC*4)
+// Work split: a segment that starts in the middle of a CTA's range costs that CTA about
+// three tiles' time (the finished segment's accumulators are folded, reduced and written
+// and the next query is set up, by code that runs once and is fetched cold while the K/V
+// stream loads the memory system). The split therefore charges every segment start
+// kSegPenaltyTiles extra tiles, when the batch is small enough to keep the count of
+// sequences with tokens in shared memory and every CTA gets well over that many tiles.
+constexpr int kSegPenaltyTiles = 3;
+constexpr int kPenaltyMaxB = 2048;
 constexpr int kDotBias = 0x4B400000;    // bit pattern of 1.5 * 2^23
 constexpr float kDotBiasF = 12582912.0f; // 1.5 * 2^23
 
@@ -78,7 +93,10 @@ struct SmemLayout {
     uint32_t off_k, off_v, off_ks, off_vs; // within a slot
     uint32_t off_full, off_empty, off_mbar, off_mask, off_misc, off_slots, off_ptab, off_cstart,
         off_prefix, off_scratch;
-    uint32_t total; // bytes from the 1024-aligned base
+    uint32_t off_nseq;  // prefix count of sequences with tokens (B <= kPenaltyMaxB), else 0
+    uint32_t off_qbuf;  // quantised query of a CTA's second segment (0 bytes when it did not fit)
+    uint32_t qbuf_rows; // query rows per (KV head, slice) pair kept there; 0 = no buffer
+    uint32_t total;     // bytes from the 1024-aligned base
 };
 
 __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages, int B,
@@ -86,12 +104,11 @@ __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages,
 {
     SmemLayout L;
     const uint32_t kv = (uint32_t)(TT * HPC * kD);
-    const uint32_t sc = align_up((uint32_t)(TT * HPC * 4), 128);
     L.off_k = 0;
     L.off_v = kv;
     L.off_ks = 2 * kv;
-    L.off_vs = 2 * kv + sc;
-    L.stage_bytes = align_up(2 * kv + 2 * sc, 1024);
+    L.off_vs = 2 * kv + kScaleGap;
+    L.stage_bytes = align_up(2 * kv + 2 * kScaleGap, 1024);
     uint32_t o = (uint32_t)n_stages * L.stage_bytes;
     L.off_full = o;
     o += 8 * kMaxStages;
@@ -101,8 +118,8 @@ __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages,
     o += 8;
     L.off_mask = o;
     o += 4 * kMaxStages;
-    L.off_misc = o;
-    o += 64;
+    L.off_misc = o; // 8-byte aligned: the prefix scan's per-warp 64-bit sums
+    o += 128;
     L.off_slots = o;
     o += 4 * 32;
     L.off_ptab = o; // producer: physical slot of every box of the next 32 tiles
@@ -113,9 +130,20 @@ __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages,
     o = align_up(o + 4u * (uint32_t)(B + 1), 16);
     L.off_scratch = o;
     o += 4u * (uint32_t)scratch_floats;
+    L.off_nseq = 0;
+    if (B <= kPenaltyMaxB) {
+        L.off_nseq = align_up(o, 16);
+        o = L.off_nseq + 4u * (uint32_t)(B + 1);
+    }
+    L.off_qbuf = align_up(o, 16);
+    L.qbuf_rows = 0;
     L.total = o;
     return L;
 }
+
+// Bytes per query row in the second-segment buffer: 32 code words (lane-fragment order) and
+// the 4 block scales.
+constexpr uint32_t kQRowBytes = 32 * 4 + kNB * 4;
 
 struct DecodeParams {
     float *out;
@@ -159,6 +187,7 @@ __device__ __forceinline__ float4 ldcg_f4(const float *p)
 __device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
 {
     int lo = 0, hi = g - 1;
+#pragma unroll 1
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (cstart[mid] <= x)
@@ -170,45 +199,90 @@ __device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
 }
 
 // Per-sequence tile prefix: prefix[b + 1] = sum over b' <= b of nhc * ceil(L_b' / TT).
-__device__ void build_prefix(const DecodeParams &p, int *prefix, volatile int *wsum, int tid,
-                             int warp, int lane)
+// Per-sequence prefixes, one block-wide scan of (tiles, has tokens) packed in 64 bits:
+// prefix[b + 1] = sum over b' <= b of nhc * ceil(L_b' / TT); nseq[b + 1] (when nseq is
+// given) = number of sequences b' <= b with L_b' > 0.
+__device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
+                             volatile unsigned long long *wsum, int tid, int warp, int lane)
 {
     const int cap = p.mbps * p.bs;
-    int carry = 0;
+    unsigned long long carry = 0;
+#pragma unroll 1
     for (int base = 0; base < p.B; base += kThreads) {
         const int b = base + tid;
-        int v = 0;
+        unsigned long long v = 0;
         if (b < p.B) {
             int L = p.seq_lens[b];
             if (L < 0 || L > cap) {
                 atomicOr(p.errors, kErrSeqLen);
                 L = L < 0 ? 0 : cap;
             }
-            v = ((L + p.TT - 1) / p.TT) * p.nhc;
+            v = ((unsigned long long)(((L + p.TT - 1) / p.TT) * p.nhc) << 32) | (L > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(kFullMask, v, o);
+            const unsigned long long t = __shfl_up_sync(kFullMask, v, o);
             if (lane >= o)
                 v += t;
         }
         if (lane == 31)
             wsum[warp] = v;
         __syncthreads();
-        int off = carry, total = 0;
+        unsigned long long off = carry, total = 0;
+#pragma unroll 1
         for (int w = 0; w < kThreads / 32; ++w) {
-            const int ws = wsum[w];
+            const unsigned long long ws = wsum[w];
             if (w < warp)
                 off += ws;
             total += ws;
         }
-        if (b < p.B)
-            prefix[b + 1] = off + v;
+        if (b < p.B) {
+            prefix[b + 1] = (int)((off + v) >> 32);
+            if (nseq)
+                nseq[b + 1] = (int)((off + v) & 0xffffffffu);
+        }
         carry += total;
         __syncthreads();
     }
-    if (tid == 0)
+    if (tid == 0) {
         prefix[0] = 0;
+        if (nseq)
+            nseq[0] = 0;
+    }
+}
+
+// First tile of CTA i (of g) when segment starts are charged P extra tiles: the virtual
+// list puts P units before the tiles of every segment; CTA i starts at virtual unit
+// floor(i * V / g) and takes the tile it lands on (or the segment's first tile when it
+// lands in the segment's penalty).
+__device__ int penalised_start(const DecodeParams &p, const int *prefix, const int *nseq, int P,
+                               long long V, int g, int i)
+{
+    const int N = prefix[p.B];
+    if (i >= g)
+        return N;
+    const long long vi = (long long)i * V / g;
+    const long long pseg = (long long)P * p.nhc; // penalty units of one sequence's segments
+    auto vpre = [&](int b) { return (long long)prefix[b] + pseg * nseq[b]; };
+    int lo = 0, hi = p.B - 1; // largest b with vpre(b) <= vi
+#pragma unroll 1
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (vpre(mid) <= vi)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const int ntb = (prefix[lo + 1] - prefix[lo]) / p.nhc;
+    if (ntb == 0)
+        return prefix[lo];
+    const long long off = vi - vpre(lo);
+    const long long len = ntb + P;
+    const int hc = (int)(off / len);
+    const int r = (int)(off - hc * len);
+    const int j = r > P ? r - P : 0;
+    const int x = prefix[lo] + (hc < p.nhc ? hc * ntb + j : p.nhc * ntb);
+    return x < N ? x : N;
 }
 
 __device__ __forceinline__ int clamp_len(int L, int cap)
@@ -222,6 +296,8 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                         const CUtensorMap *tmKs, const CUtensorMap *tmVs, uint8_t *smem,
                         const int *prefix, int t0, int t1, int lane)
 {
+    // Every loop here stays rolled: the producer issues a handful of instructions per stage,
+    // and its code must not crowd the consumers' out of the instruction cache.
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
     int *mask = reinterpret_cast<int *>(smem + p.lay.off_mask);
@@ -234,12 +310,14 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     bool aborted = false;
 
     int *ptab = reinterpret_cast<int *>(smem + p.lay.off_ptab);
+#pragma unroll 1
     for (int xb = t0; xb < t1 && !aborted; xb += 32) {
         // lane l resolves tile xb + l: its head chunk and the physical slot of every box
         const int x = xb + lane;
         int hc = 0;
         if (x < t1) {
             int lo = 0, hi = p.B - 1; // largest b with prefix[b] <= x
+#pragma unroll 1
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
                 if (prefix[mid] <= x)
@@ -255,6 +333,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
             const int lt = local - hc * ntb;
             const int tok0 = lt * p.TT;
             const int L = clamp_len(__ldg(p.seq_lens + b), cap);
+#pragma unroll 1
             for (int bx = 0; bx < p.n_boxes; ++bx) {
                 const int tk = tok0 + bx * p.box_tok;
                 int sl = -1;
@@ -270,6 +349,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
         }
         __syncwarp();
         const int n = (t1 - xb) < 32 ? (t1 - xb) : 32;
+#pragma unroll 1
         for (int i = 0; i < n; ++i) {
             const int hci = __shfl_sync(kFullMask, hc, i);
             int ok = 1;
@@ -281,6 +361,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                     const int *sl = ptab + i * kMaxBoxes;
                     uint32_t bytes = 0;
                     int loaded = 0;
+#pragma unroll 1
                     for (int bx = 0; bx < p.n_boxes; ++bx)
                         if (sl[bx] >= 0) {
                             bytes += 2 * (kv_box + sc_box);
@@ -290,6 +371,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                     mask[stage] = loaded;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     uint8_t *sb = smem + (size_t)stage * p.lay.stage_bytes;
+#pragma unroll 1
                     for (int bx = 0; bx < p.n_boxes; ++bx) {
                         const int slot = sl[bx];
                         if (slot < 0)
@@ -329,6 +411,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     }
     // Every copy this warp issued must have landed before the CTA may exit.
     if (lane == 0) {
+#pragma unroll 1
         for (int s = 0; s < p.n_stages; ++s)
             if ((issued >> s) & 1u)
                 mbar_wait(&full[s], (issued_par >> s) & 1u, kWaitLimitNs);
@@ -406,6 +489,53 @@ __device__ __forceinline__ QueryFrag<NT> load_query(const DecodeParams &p, int b
     return st;
 }
 
+// The second-segment query buffer holds, per (KV head, slice) pair, the quantised rows of
+// this warp's query tile in lane-fragment order: row r, word (j * 4 + c) * 2 + half is the
+// code word that lane (g = row, c) puts into qa[j][half ? 2 : 0] (or [3] / [1] for the rows
+// 8-15 of a two-tile warp), followed by the row's 4 block scales.
+template <int NT, bool kPack>
+__device__ __forceinline__ void store_query(uint32_t buf, const QueryFrag<NT> &qf, int g, int c)
+{
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        if (kPack && g >= 4)
+            continue; // rows 4-7 repeat rows 0-3
+        const uint32_t row = buf + (uint32_t)(r * 8 + g) * kQRowBytes;
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            sts64(row + ((j * 4 + c) * 2) * 4, qf.qa[j][r == 0 ? 0 : 1], qf.qa[j][r == 0 ? 2 : 3]);
+            if (c == 0)
+                sts_f32(row + 128 + 4 * j, qf.qs[r][j]);
+        }
+    }
+}
+
+template <int NT, bool kPack>
+__device__ __forceinline__ QueryFrag<NT> load_query_smem(uint32_t buf, int g, int c)
+{
+    QueryFrag<NT> qf;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (r >= NT) {
+#pragma unroll
+            for (int j = 0; j < kNB; ++j) {
+                qf.qa[j][1] = 0u;
+                qf.qa[j][3] = 0u;
+            }
+            continue;
+        }
+        const uint32_t row = buf + (uint32_t)(r * 8 + (kPack ? (g & 3) : g)) * kQRowBytes;
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            const uint2 w = lds64(row + ((j * 4 + c) * 2) * 4);
+            qf.qa[j][r == 0 ? 0 : 1] = w.x;
+            qf.qa[j][r == 0 ? 2 : 3] = w.y;
+            qf.qs[r][j] = lds_f32(row + 128 + 4 * j);
+        }
+    }
+    return qf;
+}
+
 template <int NT>
 __device__ __forceinline__ void reset_state(WarpState<NT> &st)
 {
@@ -422,13 +552,15 @@ __device__ __forceinline__ void reset_state(WarpState<NT> &st)
     }
 }
 
-// Per-thread shared-memory offsets that are the same for every stage. Subtile u of a
-// warp covers stage tokens ts * 16 * kSub + 16 * u + [0, 16).
+// Per-thread shared-memory byte offsets within a stage (the stage's shared address is added
+// once per stage; every fragment load then uses one register plus an immediate). Subtile u
+// of a warp covers stage tokens ts * 16 * kSub + 16 * u + [0, 16), which lie in one TMA box
+// (boxes hold at least 16 tokens), so the second 8-token half of a subtile is 8 rows
+// (1024 bytes) further on and has the same 128-byte swizzle phase.
 struct ThreadOffsets {
-    uint32_t k[kSub][2][kNB]; // K fragment loads (subtile, QK n-tile, quant block)
-    uint32_t v[kSub][4];      // V rows 2c, 2c+1, 2c+8, 2c+9 (channel chunk g)
-    uint32_t s[kSub][2][2];   // scale of tokens nt*8 + 2c + e
-    int tok[kSub][2][2];      // stage-local token index of (u, nt, e)
+    uint32_t k[kSub][kNB]; // K fragment (subtile u, quant block j) of tokens 0-7; 8-15: +1024
+    uint32_t v[kSub][2];   // V row of token 2c + e (e = 0, 1); token 2c + e + 8: +1024
+    uint32_t s[kSub][2][2]; // K scale of token (u, nt, e); its V scale is kScaleGap further
 };
 
 __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int kl, int ts, int g,
@@ -437,30 +569,25 @@ __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int
     ThreadOffsets o;
     const int lb = p.log2_box, bt = p.box_tok, H = p.HPC;
     auto row_kv = [&](int tok) { return ((tok >> lb) * H + kl) * bt + (tok & (bt - 1)); };
-    auto row_sc = [&](int tok) { return ((tok >> lb) * bt + (tok & (bt - 1))) * H + kl; };
 #pragma unroll
     for (int u = 0; u < kSub; ++u) {
         const int t0 = (ts * kSub + u) * 16;
+        const int rk = row_kv(t0 + g); // row & 7 == g
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int r = row_kv(t0 + nt * 8 + g);
+        for (int j = 0; j < kNB; ++j)
+            o.k[u][j] = p.lay.off_k + rk * 128 + ((((2 * j) | (c >> 1)) ^ g) << 4) +
+                        ((c & 1) << 3);
 #pragma unroll
-            for (int j = 0; j < kNB; ++j)
-                o.k[u][nt][j] = p.lay.off_k + r * 128 + ((((2 * j) | (c >> 1)) ^ (r & 7)) << 4) +
-                                ((c & 1) << 3);
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int tok = t0 + nt * 8 + 2 * c + e;
-                o.tok[u][nt][e] = tok;
-                o.s[u][nt][e] = 4 * row_sc(tok);
-            }
+        for (int e = 0; e < 2; ++e) {
+            const int rv = row_kv(t0 + 2 * c + e); // row & 7 == 2c + e
+            o.v[u][e] = p.lay.off_v + rv * 128 + ((g ^ (2 * c + e)) << 4);
         }
+        // scales sit token-major ([token][head]) in stage token order
 #pragma unroll
-        for (int qv = 0; qv < 4; ++qv) {
-            const int t = 2 * c + (qv & 1) + (qv >> 1) * 8;
-            const int r = row_kv(t0 + t);
-            o.v[u][qv] = p.lay.off_v + r * 128 + ((g ^ (r & 7)) << 4);
-        }
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                o.s[u][nt][e] = p.lay.off_ks + 4 * ((t0 + nt * 8 + 2 * c + e) * H + kl);
     }
     return o;
 }
@@ -471,13 +598,14 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 }
 
 // One stage: kSub 16-token subtiles of one KV head for this warp, folded into the online
-// softmax as one block. kMasked: some tokens of the stage are past the sequence end or in a
-// block that was not loaded.
-template <int NT, bool kPack, bool kDump, bool kMasked>
+// softmax as one block. sb: shared address of the stage; tl0: stage-local index of this
+// thread's first token; vmask: bit k set when token k of the warp's 32-token window holds
+// data (clear past the sequence end and in blocks that were not loaded).
+template <int NT, bool kPack, bool kDump>
 __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<NT> &st,
-                                              const ThreadOffsets &o, const uint8_t *sb,
-                                              int nvalid, int loaded, int b, int hc, int kl,
-                                              int slice, int tok0, int g, int c)
+                                              const ThreadOffsets &o, uint32_t sb, int tl0,
+                                              uint32_t vmask, float scale_log2, int b, int hc,
+                                              int kl, int slice, int tok0, int g, int c)
 {
     // ---- V rows first: their int8 -> f16 conversion overlaps the softmax chain below
     uint4 R[kSub][4];
@@ -485,10 +613,12 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
     for (int u = 0; u < kSub; ++u)
 #pragma unroll
         for (int qv = 0; qv < 4; ++qv)
-            R[u][qv] = *reinterpret_cast<const uint4 *>(sb + o.v[u][qv]);
-    // ---- scores: int8 MMA per quant block, exact int32 block dots. The accumulator
-    // starts at the bit pattern of 1.5 * 2^23, so each result read as fp32 is
-    // 1.5 * 2^23 + dot exactly (|dot| <= 32 * 127 * 127 < 2^22).
+            R[u][qv] = lds128(sb + o.v[u][qv & 1] + (qv >> 1) * 1024);
+    // ---- scores: int8 MMA per quant block, exact int32 block dots. The four block MMAs of
+    // an 8-token group accumulate into one int32 register set that starts at the bit
+    // pattern of 1.5 * 2^23, so after block j it holds 1.5 * 2^23 + dot_0 + ... + dot_j
+    // (|sum| <= 4 * 32 * 127 * 127 < 2^22): read as fp32 every partial sum is exact, and
+    // dot_j is the exact difference of two consecutive ones.
     float s[NT][kSub][2][2];
 #pragma unroll
     for (int r = 0; r < NT; ++r)
@@ -501,111 +631,130 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
     for (int u = 0; u < kSub; ++u) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
+            int prev[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
 #pragma unroll
             for (int j = 0; j < kNB; ++j) {
-                const uint2 kk = *reinterpret_cast<const uint2 *>(sb + o.k[u][nt][j]);
+                const uint2 kk = lds64(sb + o.k[u][j] + nt * 1024);
                 int d[4];
-                mma_s8_16832_biased(d, st.qa[j][0], NT == 2 ? st.qa[j][1] : 0u, st.qa[j][2],
-                                    NT == 2 ? st.qa[j][3] : 0u, kk.x, kk.y);
+                mma_s8_16832_acc(d, st.qa[j][0], NT == 2 ? st.qa[j][1] : 0u, st.qa[j][2],
+                                 NT == 2 ? st.qa[j][3] : 0u, kk.x, kk.y, prev);
                 if constexpr (kDump) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int r = q >> 1, e = q & 1;
                         const int hg = kPack ? g : slice * 16 + r * 8 + g;
                         const bool row_ok = kPack ? (r == 0 && g < 4) : (r < NT);
-                        const int tl = o.tok[u][nt][e];
-                        if (row_ok && hg < p.G && tl < nvalid &&
-                            ((loaded >> (tl >> p.log2_box)) & 1)) {
+                        const int tl = tl0 + u * 16 + nt * 8 + e;
+                        if (row_ok && hg < p.G && ((vmask >> (tl - tl0 + 2 * c)) & 1u)) {
                             const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
                             p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) *
                                            kNB +
-                                       j] = d[q] - kDotBias;
+                                       j] = d[q] - prev[q];
                         }
                     }
                 }
-                s[0][u][nt][0] += (__int_as_float(d[0]) - kDotBiasF) * st.qs[0][j];
-                s[0][u][nt][1] += (__int_as_float(d[1]) - kDotBiasF) * st.qs[0][j];
+                s[0][u][nt][0] += (__int_as_float(d[0]) - __int_as_float(prev[0])) * st.qs[0][j];
+                s[0][u][nt][1] += (__int_as_float(d[1]) - __int_as_float(prev[1])) * st.qs[0][j];
                 if constexpr (NT == 2) {
-                    s[NT - 1][u][nt][0] += (__int_as_float(d[2]) - kDotBiasF) * st.qs[NT - 1][j];
-                    s[NT - 1][u][nt][1] += (__int_as_float(d[3]) - kDotBiasF) * st.qs[NT - 1][j];
+                    s[NT - 1][u][nt][0] +=
+                        (__int_as_float(d[2]) - __int_as_float(prev[2])) * st.qs[NT - 1][j];
+                    s[NT - 1][u][nt][1] +=
+                        (__int_as_float(d[3]) - __int_as_float(prev[3])) * st.qs[NT - 1][j];
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    prev[q] = d[q];
             }
         }
     }
-    // ---- per-token K and V scales; masking of tokens past the sequence end
-    float kss[kSub][2][2], vsv[kSub][2][2], vex[kSub][2][2];
-    bool val[kSub][2][2];
+    // ---- per-token K and V scales (the K scale carries the softmax scale and log2 e)
+    float kss[kSub][2][2], vsv[kSub][2][2];
 #pragma unroll
     for (int u = 0; u < kSub; ++u)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int tl = o.tok[u][nt][e];
-                val[u][nt][e] = !kMasked || (tl < nvalid && ((loaded >> (tl >> p.log2_box)) & 1));
-                kss[u][nt][e] =
-                    *reinterpret_cast<const float *>(sb + p.lay.off_ks + o.s[u][nt][e]) *
-                    p.scale_log2;
-                const float vv =
-                    *reinterpret_cast<const float *>(sb + p.lay.off_vs + o.s[u][nt][e]);
-                vsv[u][nt][e] = val[u][nt][e] ? vv : 0.f;
-                // floor(log2 |vs|) from the exponent field, clamped to [-100, 100]
-                vex[u][nt][e] = fminf(fmaxf(exponent_as_float(vv), -kVExpLimit), kVExpLimit);
+                kss[u][nt][e] = lds_f32(sb + o.s[u][nt][e]) * scale_log2;
+                vsv[u][nt][e] = lds_f32(sb + o.s[u][nt][e] + kScaleGap);
             }
+    // masked tokens (rare: a segment's last tile, bad block-table entries) get score -inf
+    // and V scale 0, whatever stale data their slots hold
+    if (vmask != 0xffffffffu) {
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    if (!((vmask >> (u * 16 + nt * 8 + 2 * c + e)) & 1u)) {
+#pragma unroll
+                        for (int r = 0; r < NT; ++r)
+                            s[r][u][nt][e] = -INFINITY;
+                        kss[u][nt][e] = 1.f;
+                        vsv[u][nt][e] = 0.f;
+                    }
+    }
     // ---- online softmax (base 2), blockwise over the stage's tokens. M: running max of the
-    // scores (denominator). A: running max of score + log2(vs) - 14 (numerator), so that
-    // every weight * vs * 2^(M - A) entering the f16 MMA is below 2^15.
+    // scores (denominator). A: running max of log2 of the numerator terms w * vs (relative to
+    // 2^M) minus 14, so that every w * vs * 2^(M - A) entering the f16 MMA is below 2^15 and
+    // the largest one is at least 2^14; A >= M - 114 keeps 2^(M - A) finite.
     float alpha_a[NT];
     uint32_t bh[NT][kSub][2], bl[NT][kSub][2];
 #pragma unroll
     for (int r = 0; r < NT; ++r) {
-        float m = -INFINITY, a = -INFINITY;
+        float m = -INFINITY;
 #pragma unroll
         for (int u = 0; u < kSub; ++u)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float v = val[u][nt][e] ? s[r][u][nt][e] * kss[u][nt][e] : -INFINITY;
+                    const float v = s[r][u][nt][e] * kss[u][nt][e];
                     s[r][u][nt][e] = v;
                     m = fmaxf(m, v);
-                    a = fmaxf(a, v + vex[u][nt][e]);
                 }
         m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
-        a = fmaxf(a, __shfl_xor_sync(kFullMask, a, 1));
         m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
-        a = fmaxf(a, __shfl_xor_sync(kFullMask, a, 2));
         const float mn = fmaxf(st.M[r], m);
-        const float an = fmaxf(st.A[r], a - 14.f);
         const float ms = (mn == -INFINITY) ? 0.f : mn;
-        const float as = (an == -INFINITY) ? 0.f : an;
-        const float alpha_s = exp2f(st.M[r] - ms);
-        alpha_a[r] = exp2f(st.A[r] - as);
+        const float alpha_s = fast_exp2(st.M[r] - ms);
         st.M[r] = mn;
-        st.A[r] = an;
-        const float cvs = exp2f(ms - as); // 2^(M - A), within [2^-86, 2^114]
-        float ws = 0.f;
+        float ws = 0.f, pmax = 0.f;
+        float w[kSub][2][2];
 #pragma unroll
-        for (int u = 0; u < kSub; ++u) {
-            float pw[2][2];
+        for (int u = 0; u < kSub; ++u)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float w = exp2f(s[r][u][nt][e] - ms);
-                    ws += w;
-                    pw[nt][e] = w * (vsv[u][nt][e] * cvs);
+                    const float x = fast_exp2(s[r][u][nt][e] - ms);
+                    ws += x;
+                    w[u][nt][e] = x * vsv[u][nt][e];
+                    pmax = fmaxf(pmax, w[u][nt][e]);
                 }
-            // weights as split f16 B operands (column n = head g, k = token)
+        st.S[r] = st.S[r] * alpha_s + ws;
+        pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 1));
+        pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 2));
+        // floor(log2 pmax) from the exponent field (pmax = 0 gives -127)
+        const float an_stage = ms + exponent_as_float(pmax) - 14.f;
+        const float an =
+            (mn == -INFINITY) ? -INFINITY : fmaxf(fmaxf(st.A[r], an_stage), mn - 114.f);
+        const float as = (an == -INFINITY) ? 0.f : an;
+        alpha_a[r] = fast_exp2(st.A[r] - as);
+        st.A[r] = an;
+        const float cvs = fast_exp2(ms - as); // 2^(M - A), at most 2^114
+        // weights as split f16 B operands (column n = head g, k = token)
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                const __half2 h = __floats2half2_rn(pw[nt][0], pw[nt][1]);
-                const float r0 = pw[nt][0] - __low2float(h), r1 = pw[nt][1] - __high2float(h);
+                const float p0 = w[u][nt][0] * cvs, p1 = w[u][nt][1] * cvs;
+                const __half2 h = __floats2half2_rn(p0, p1);
+                const float r0 = p0 - __low2float(h), r1 = p1 - __high2float(h);
                 bh[r][u][nt] = *reinterpret_cast<const uint32_t *>(&h);
                 bl[r][u][nt] = pack_f16x2(r0, r1);
             }
-        }
-        st.S[r] = st.S[r] * alpha_s + ws;
     }
     // ---- rescale factors of the accumulator columns (in packed mode rows 4-7 repeat rows
     // 0-3, so the source lane of column col carries head col & 3 either way)
@@ -656,6 +805,260 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
     }
 }
 
+// ------------------------------------------------------------------ packed path (group <= 4)
+//
+// With at most 4 query heads per KV head, rows 4-7 of the QK tile repeat rows 0-3. The
+// packed path uses the repeat to halve the softmax work: lanes of rows 0-3 ("lower" lanes)
+// take the first 16 tokens of the warp's 32, lanes of rows 4-7 the last 16, and the row
+// reductions add one xor-16 step. PV then runs on the int8 tensor cores:
+//  * A = V^T straight from the TMA-swizzled tile through ldmatrix .trans (no conversion),
+//    rows = channels 16m + g (and + 8), k = tokens in the order tau(k) below;
+//  * B = the exact integer P = round(w * vs * 2^(M - A) * 2^8) < 2^23 (an FFMA against
+//    2^23 leaves it in the low mantissa bits) split into its three bytes: n-tile 0 holds
+//    byte 0 of heads 0-3 in columns 0-3 and byte 1 in columns 4-7, n-tile 1 byte 2;
+//  * the int32 accumulators run over up to 4 stages (128 tokens: |sum| < 2^22, so the
+//    biased fp32 view stays exact) and are folded into the fp32 accumulator when that limit
+//    is reached, when A rises, and at the end of a segment.
+// k -> token within a 16-token subtile: k = 4c + i holds token 2c + (i & 1) + 8 (i >> 1),
+// i.e. the tokens whose scores lane (g, c) holds after the QK MMAs.
+constexpr int kPackFoldEvery = 4;
+constexpr float kTwo23 = 8388608.0f;
+
+struct PackedOffsets {
+    uint32_t k[kSub][kNB]; // K fragments, as ThreadOffsets::k
+    uint32_t s[2][2];      // K scale of this lane's kept token (nt, e); V scale kScaleGap on
+    uint32_t v;            // ldmatrix row address of this lane; XOR (16 m) selects chunk m
+};
+
+__device__ __forceinline__ PackedOffsets make_packed_offsets(const DecodeParams &p, int kl,
+                                                             int ts, int g, int c, int lane)
+{
+    PackedOffsets o;
+    const int lb = p.log2_box, bt = p.box_tok, H = p.HPC;
+    auto row_kv = [&](int tok) { return ((tok >> lb) * H + kl) * bt + (tok & (bt - 1)); };
+#pragma unroll
+    for (int u = 0; u < kSub; ++u) {
+        const int rk = row_kv((ts * kSub + u) * 16 + g);
+#pragma unroll
+        for (int j = 0; j < kNB; ++j)
+            o.k[u][j] = p.lay.off_k + rk * 128 + ((((2 * j) | (c >> 1)) ^ g) << 4) +
+                        ((c & 1) << 3);
+    }
+    const int uk = g >> 2; // subtile whose tokens this lane keeps
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            o.s[nt][e] =
+                p.lay.off_ks + 4 * (((ts * kSub + uk) * 16 + nt * 8 + 2 * c + e) * H + kl);
+    // ldmatrix: lanes 0-15 give the rows of matrix 0 (subtile 0), lanes 16-31 of matrix 1
+    const int kk = lane & 15;
+    const int tau = 2 * (kk >> 2) + (kk & 1) + 8 * ((kk >> 1) & 1);
+    const int tok = (ts * kSub + (lane >> 4)) * 16 + tau;
+    o.v = p.lay.off_v + row_kv(tok) * 128 + ((tok & 7) << 4);
+    return o;
+}
+
+struct PackedAcc {
+    int D[8][2][4]; // int32 PV accumulators (m-tile, n-tile), biased by 1.5 * 2^23
+    int n;          // stages accumulated since the last fold
+};
+
+// acc = (acc + D) * f per column: D's digits recombined (k0, k1: weights of n-tiles 0 and 1
+// in this lane's columns), f = 2^(A_old - A_new) of the column's head.
+template <int NT>
+__device__ __forceinline__ void packed_fold(WarpState<NT> &st, const PackedAcc &pa, float k0,
+                                            float k1, float f0, float f1)
+{
+    const float kb = -kDotBiasF * (k0 + k1);
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float v = fmaf(__int_as_float(pa.D[m][0][k]), k0,
+                                 fmaf(__int_as_float(pa.D[m][1][k]), k1, kb));
+            st.acc[0][m][k] = (st.acc[0][m][k] + v) * ((k & 1) ? f1 : f0);
+        }
+}
+
+template <int NT>
+__device__ __forceinline__ void packed_rescale(WarpState<NT> &st, float f0, float f1)
+{
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            st.acc[0][m][k] *= (k & 1) ? f1 : f0;
+}
+
+template <int NT, bool kDump>
+__device__ __forceinline__ void process_stage_packed(const DecodeParams &p, WarpState<NT> &st,
+                                                     PackedAcc &pa, const PackedOffsets &o,
+                                                     uint32_t sb, int tl0, uint32_t vmask,
+                                                     float scale_log2, int b, int hc, int kl,
+                                                     int tok0, int g, int c, float k0, float k1)
+{
+    const bool lower = g < 4;
+    const int uk = lower ? 0 : 1;
+    // ---- scores of this lane's 16-token half (see process_stage for the exact chain)
+    float s[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        int p0[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
+        int p1[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
+        float prev[2] = {kDotBiasF, kDotBiasF};
+        s[nt][0] = s[nt][1] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            const uint2 kk0 = lds64(sb + o.k[0][j] + nt * 1024);
+            const uint2 kk1 = lds64(sb + o.k[1][j] + nt * 1024);
+            int d0[4], d1[4];
+            mma_s8_16832_acc(d0, st.qa[j][0], 0u, st.qa[j][2], 0u, kk0.x, kk0.y, p0);
+            mma_s8_16832_acc(d1, st.qa[j][0], 0u, st.qa[j][2], 0u, kk1.x, kk1.y, p1);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float cur = __int_as_float(lower ? d0[e] : d1[e]);
+                if constexpr (kDump) {
+                    const int tl = tl0 + uk * 16 + nt * 8 + e;
+                    const int hg = g & 3;
+                    if (hg < p.G && ((vmask >> (uk * 16 + nt * 8 + 2 * c + e)) & 1u)) {
+                        const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
+                        p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) *
+                                       kNB +
+                                   j] = __float_as_int(cur) - __float_as_int(prev[e]);
+                    }
+                }
+                s[nt][e] += (cur - prev[e]) * st.qs[0][j];
+                prev[e] = cur;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                p0[q] = d0[q];
+                p1[q] = d1[q];
+            }
+        }
+    }
+    // ---- scales of the kept tokens; masked tokens get score -inf and V scale 0
+    float kss[2][2], vsv[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            kss[nt][e] = lds_f32(sb + o.s[nt][e]) * scale_log2;
+            vsv[nt][e] = lds_f32(sb + o.s[nt][e] + kScaleGap);
+        }
+    if (vmask != 0xffffffffu) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                if (!((vmask >> (uk * 16 + nt * 8 + 2 * c + e)) & 1u)) {
+                    s[nt][e] = -INFINITY;
+                    kss[nt][e] = 1.f;
+                    vsv[nt][e] = 0.f;
+                }
+    }
+    // ---- online softmax (base 2) over the stage's 32 tokens (M, S, A as in process_stage)
+    float m = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float v = s[nt][e] * kss[nt][e];
+            s[nt][e] = v;
+            m = fmaxf(m, v);
+        }
+    m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 16));
+    const float mn = fmaxf(st.M[0], m);
+    const float ms = (mn == -INFINITY) ? 0.f : mn;
+    const float alpha_s = fast_exp2(st.M[0] - ms);
+    st.M[0] = mn;
+    float ws = 0.f, pmax = 0.f, w[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float x = fast_exp2(s[nt][e] - ms);
+            ws += x;
+            w[nt][e] = x * vsv[nt][e];
+            pmax = fmaxf(pmax, w[nt][e]);
+        }
+    st.S[0] = st.S[0] * alpha_s + ws;
+    pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 1));
+    pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 2));
+    pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 16));
+    const float an_stage = ms + exponent_as_float(pmax) - 14.f;
+    const float an = (mn == -INFINITY) ? -INFINITY : fmaxf(fmaxf(st.A[0], an_stage), mn - 114.f);
+    const float as = (an == -INFINITY) ? 0.f : an;
+    const bool rose = an != st.A[0];
+    const float alpha_a = rose ? fast_exp2(st.A[0] - as) : 1.f;
+    st.A[0] = an;
+    // ---- fold the int32 accumulators (scale of the old A) before this stage's products
+    if (__any_sync(kFullMask, rose) || pa.n == kPackFoldEvery) {
+        // columns 2c, 2c + 1 hold heads (2c) & 3, (2c + 1) & 3: rows 2c, 2c + 1 (or the
+        // repeats 2c + 4, 2c + 5), i.e. lanes 8c and 8c + 4
+        const float f0 = __shfl_sync(kFullMask, alpha_a, 8 * c);
+        const float f1 = __shfl_sync(kFullMask, alpha_a, 8 * c + 4);
+        if (pa.n > 0)
+            packed_fold(st, pa, k0, k1, f0, f1);
+        else
+            packed_rescale(st, f0, f1);
+        pa.n = 0;
+    }
+    // ---- P as exact integers, split into byte planes for the B operands
+    const float cvs8 = fast_exp2(ms - as + 8.f); // 2^(M - A + 8)
+    uint32_t X[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            X[nt][e] = __float_as_uint(fmaf(w[nt][e], cvs8, kTwo23));
+    const uint32_t x01 = prmt(X[0][0], X[0][1], 0x5140u), x23 = prmt(X[1][0], X[1][1], 0x5140u);
+    const uint32_t y01 = prmt(X[0][0], X[0][1], 0x7362u), y23 = prmt(X[1][0], X[1][1], 0x7362u);
+    const uint32_t pl0 = prmt(x01, x23, 0x5410u), pl1 = prmt(x01, x23, 0x7632u);
+    const uint32_t pl2 = prmt(y01, y23, 0x5410u);
+    // partner lane (row g ^ 4) holds the other 16 tokens of the same head
+    const uint32_t r1 = __shfl_xor_sync(kFullMask, lower ? pl1 : pl0, 16);
+    const uint32_t r2 = __shfl_xor_sync(kFullMask, pl2, 16);
+    const uint32_t bA0 = lower ? pl0 : r1, bA1 = lower ? r1 : pl1; // n-tile 0: bytes 0 | 1
+    const uint32_t bB0 = pl2, bB1 = r2;                            // n-tile 1: byte 2
+    // ---- PV: V^T fragments by ldmatrix .trans, two u8 n-tiles per 16-channel m-tile
+    const uint32_t vrow = sb + o.v;
+    if (pa.n == 0) {
+        const int z[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x2_trans_b8(a0, a1, a2, a3, vrow ^ (uint32_t)(mt << 4));
+            mma_s8u8_16832_acc(pa.D[mt][0], a0, a1, a2, a3, bA0, bA1, z);
+            mma_s8u8_16832_acc(pa.D[mt][1], a0, a1, a2, a3, bB0, bB1, z);
+        }
+    } else {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x2_trans_b8(a0, a1, a2, a3, vrow ^ (uint32_t)(mt << 4));
+            mma_s8u8_16832_acc(pa.D[mt][0], a0, a1, a2, a3, bA0, bA1, pa.D[mt][0]);
+            mma_s8u8_16832_acc(pa.D[mt][1], a0, a1, a2, a3, bB0, bB1, pa.D[mt][1]);
+        }
+    }
+    ++pa.n;
+}
+
+// Packed layout: lane (g, c) holds channels 16 m + g (k = 0, 1) and 16 m + g + 8 (k = 2, 3)
+// of columns 2c + (k & 1).
+template <int NT>
+__device__ __forceinline__ void store_packed(float *dst, const WarpState<NT> &st, int q, float f)
+{
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        dst[16 * m] = st.acc[0][m][q] * f;
+        dst[16 * m + 8] = st.acc[0][m][q + 2] * f;
+    }
+}
+
 // Write the 16 channels 16g..16g+15 of column head (pv, col) scaled by f.
 template <int NT>
 __device__ __forceinline__ void store_row16(float *dst, const WarpState<NT> &st, int pv, int q,
@@ -682,6 +1085,8 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
     for (int r = 0; r < NT; ++r) {
         st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 1);
         st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 2);
+        if constexpr (kPack) // rows g and g ^ 4 summed different tokens of one head
+            st.S[r] += __shfl_xor_sync(kFullMask, st.S[r], 16);
     }
 
     // merge the token subtiles of each (KV head, slice) pair inside the CTA (the scratch
@@ -709,6 +1114,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
         }
         consumer_bar();
         if (ts == 0) {
+#pragma unroll 1
             for (int k = 1; k < p.subtiles; ++k) {
                 const float *reg = scr + (size_t)((k - 1) * p.pairs + pair) * p.scratch_stride;
 #pragma unroll
@@ -774,8 +1180,12 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
                     const int hg = slice * 16 + pv * 8 + col;
                     if (col_lane && hg < p.G) {
                         const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
-                        float *dst = p.out + ((long long)b * p.Hq + h) * kD + 16 * g;
-                        store_row16(dst, st, pv, q, sc > 0.f ? exp2f(ac - mc) / sc : 0.f);
+                        const float f = sc > 0.f ? exp2f(ac - mc) / sc : 0.f;
+                        float *dst = p.out + ((long long)b * p.Hq + h) * kD;
+                        if constexpr (kPack)
+                            store_packed(dst + g, st, q, f);
+                        else
+                            store_row16(dst + 16 * g, st, pv, q, f);
                     }
                 }
         }
@@ -794,9 +1204,13 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int hg = slice * 16 + pv * 8 + 2 * c + q;
-                if (col_lane && hg < p.G)
-                    store_row16(slotp + (size_t)(kl * p.G + hg) * kSlotRow + 16 * g, st, pv, q,
-                                1.0f);
+                if (col_lane && hg < p.G) {
+                    float *dst = slotp + (size_t)(kl * p.G + hg) * kSlotRow;
+                    if constexpr (kPack)
+                        store_packed(dst + g, st, q, 1.0f);
+                    else
+                        store_row16(dst + 16 * g, st, pv, q, 1.0f);
+                }
             }
         if (c == 0) {
 #pragma unroll
@@ -826,6 +1240,7 @@ __device__ __forceinline__ SegCursor cursor_at(const DecodeParams &p, const int 
 {
     SegCursor cu;
     int lo = 0, hi = p.B - 1;
+#pragma unroll 1
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (prefix[mid] <= x)
@@ -853,6 +1268,11 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
     const int kl = pair / p.slices, slice = pair % p.slices;
     const int g = lane >> 2, c = lane & 3;
     const ThreadOffsets o = make_offsets(p, kl, ts, g, c);
+    const PackedOffsets po = make_packed_offsets(p, kl, ts, g, c, lane);
+    PackedAcc pa;
+    pa.n = 0;
+    // weights of this lane's two n-tile columns in the packed PV (bytes 0 | 2, or byte 1)
+    const float k0 = c < 2 ? 0.00390625f : 1.f, k1 = c < 2 ? 256.f : 0.f;
     WarpState<NT> st;
     reset_state(st);
 #pragma unroll
@@ -869,14 +1289,37 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
     bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
     int stage = 0;
     uint32_t phase = 0;
+    const uint32_t smem_base = smem_addr(smem);
+    const uint32_t stage_bytes = p.lay.stage_bytes;
+    const float scale_log2 = p.scale_log2;
+    const int tl0 = ts * kSub * 16 + 2 * c;
+    const int all_boxes = (1 << p.n_boxes) - 1;
+    const uint32_t qbuf = smem_base + p.lay.off_qbuf +
+                          (uint32_t)pair * p.lay.qbuf_rows * kQRowBytes;
+    // The quantised query of the CTA's second segment is prepared before the first stage
+    // (while the first loads are in flight) and kept in shared memory, so that switching
+    // segments in the middle of the stream costs neither a global round trip nor the
+    // quantisation code. Warps of one (KV head, slice) pair hold the same rows; the ts == 0
+    // warp writes them.
+    const SegCursor first = cursor_at(p, prefix, t0);
+    const bool prefetch_q = p.lay.qbuf_rows != 0 && first.seg1 < t1;
+    if (prefetch_q) {
+        const SegCursor c1 = cursor_at(p, prefix, first.seg1);
+        const QueryFrag<NT> qf = load_query<NT, kPack>(p, c1.b, c1.hc, kl, slice, g, c);
+        if (ts == 0)
+            store_query<NT, kPack>(qbuf, qf, g, c);
+        consumer_bar();
+    }
+    int seg_index = 0;
     // Outer loop: one segment (this CTA's tiles of one sequence and head chunk) per pass.
-    // The inner loop over the segment's tiles holds only wait / compute / release, so the
-    // hot code stays small enough for the instruction cache.
     for (int x = t0; x < t1;) {
         const SegCursor cu = cursor_at(p, prefix, x);
         const int x_end = cu.seg1 < t1 ? cu.seg1 : t1;
         {
-            const QueryFrag<NT> qf = load_query<NT, kPack>(p, cu.b, cu.hc, kl, slice, g, c);
+            const QueryFrag<NT> qf = (prefetch_q && seg_index == 1)
+                                         ? load_query_smem<NT, kPack>(qbuf, g, c)
+                                         : load_query<NT, kPack>(p, cu.b, cu.hc, kl, slice, g, c);
+            ++seg_index;
 #pragma unroll
             for (int j = 0; j < kNB; ++j) {
 #pragma unroll
@@ -887,6 +1330,7 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                     st.qs[r][j] = qf.qs[r][j];
             }
             reset_state(st);
+            pa.n = 0;
         }
         for (; x < x_end; ++x) {
             const int tok0 = (x - cu.seg0) * p.TT;
@@ -896,10 +1340,21 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                 atomicOr(p.errors, kErrTimeout);
             }
             if (!dead) {
-                const int loaded = reinterpret_cast<volatile int *>(smem + p.lay.off_mask)[stage];
-                const uint8_t *sb = smem + (size_t)stage * p.lay.stage_bytes;
-                process_stage<NT, kPack, kDump, true>(p, st, o, sb, nvalid, loaded, cu.b, cu.hc,
-                                                      kl, slice, tok0, g, c);
+                const int loaded = (int)lds_u32(smem_base + p.lay.off_mask + 4u * stage);
+                const uint32_t sb = smem_base + (uint32_t)stage * stage_bytes;
+                // bit k: token k of this warp's 32-token window holds data
+                uint32_t vmask = 0xffffffffu;
+                if (nvalid != p.TT || loaded != all_boxes) {
+                    const int tk = ts * kSub * 16 + lane;
+                    vmask = __ballot_sync(kFullMask,
+                                          tk < nvalid && ((loaded >> (tk >> p.log2_box)) & 1));
+                }
+                if constexpr (kPack)
+                    process_stage_packed<NT, kDump>(p, st, pa, po, sb, tl0, vmask, scale_log2,
+                                                    cu.b, cu.hc, kl, tok0, g, c, k0, k1);
+                else
+                    process_stage<NT, kPack, kDump>(p, st, o, sb, tl0, vmask, scale_log2, cu.b,
+                                                    cu.hc, kl, slice, tok0, g, c);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[stage]);
@@ -908,6 +1363,10 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                 stage = 0;
                 phase ^= 1u;
             }
+        }
+        if constexpr (kPack) {
+            if (pa.n > 0)
+                packed_fold(st, pa, k0, k1, 1.f, 1.f);
         }
         finalize_segment<NT, kPack>(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c,
                                     warp * 32 + lane, prefix, cstart, gcta, t0, t1);
@@ -927,7 +1386,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
     int *prefix = reinterpret_cast<int *>(smem + p.lay.off_prefix);
-    volatile int *misc = reinterpret_cast<volatile int *>(smem + p.lay.off_misc);
 
     if (tid == 0) {
         for (int s = 0; s < p.n_stages; ++s) {
@@ -954,24 +1412,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.split_desc[2 * blockIdx.x] = make_int4(0, 0, 0, 0);
         p.split_desc[2 * blockIdx.x + 1] = make_int4(0, 0, 0, 0);
     }
-    build_prefix(p, prefix, misc + 2, tid, warp, lane);
+    int *nseq = p.lay.off_nseq ? reinterpret_cast<int *>(smem + p.lay.off_nseq) : nullptr;
+    build_prefix(p, prefix, nseq,
+                 reinterpret_cast<volatile unsigned long long *>(smem + p.lay.off_misc), tid,
+                 warp, lane);
     __syncthreads();
 
     const int N = prefix[p.B];
     int *cstart = reinterpret_cast<int *>(smem + p.lay.off_cstart);
     // rows of empty sequences are zero
+#pragma unroll 1
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
         if (prefix[b + 1] != prefix[b])
             continue;
         float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
+#pragma unroll 1
         for (int i = tid; i < p.Hq * kD / 4; i += kThreads)
             row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const int gcta = N < (int)gridDim.x ? N : (int)gridDim.x;
     {
+        // plain split: floor(i * N / gcta); penalised split (see kSegPenaltyTiles) when the
+        // sequence counts are at hand and every CTA's share is at least 4 penalties, so that
+        // no CTA's share can fall inside one segment's penalty (an empty CTA in the middle
+        // of a split segment would break the contributor numbering)
+        const long long V = nseq ? (long long)N + (long long)kSegPenaltyTiles * p.nhc * nseq[p.B]
+                                 : (long long)N;
+        const bool pen = nseq && gcta > 0 && V / gcta >= 4 * kSegPenaltyTiles;
         const int qn = N / (gcta > 0 ? gcta : 1), rn = N - qn * (gcta > 0 ? gcta : 1);
+#pragma unroll 1
         for (int i = tid; i <= gcta; i += kThreads)
-            cstart[i] = i * qn + (i * rn) / gcta; // == floor(i * N / gcta)
+            cstart[i] = pen ? penalised_start(p, prefix, nseq, kSegPenaltyTiles, V, gcta, i)
+                            : i * qn + (i * rn) / gcta;
     }
     __syncthreads();
     if ((int)blockIdx.x >= gcta)
@@ -980,11 +1452,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warp specialisation: the producer warpgroup hands most of its registers to the two
     // consumer warpgroups (the sums match the launch allocation, checked by static_assert).
     if (warp >= kConsumerWarps) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::producer));
         if (warp == kProducerWarp)
             produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::consumer));
         consume<NT, kPack, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
     }
 }

@@ -182,6 +182,23 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
     return v;
 }
 
+__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b)
+{
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ float lds_f32(uint32_t addr)
 {
     float v;
@@ -212,6 +229,43 @@ __device__ __forceinline__ void mma_s8_16832_biased(int (&d)[4], uint32_t a0, ui
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0x4B400000));
 }
 
+// D(16x8 s32) = C + A(16x32 s8, row) * B(32x8 s8, col).
+__device__ __forceinline__ void mma_s8_16832_acc(int (&d)[4], uint32_t a0, uint32_t a1,
+                                                 uint32_t a2, uint32_t a3, uint32_t b0,
+                                                 uint32_t b1, const int (&c)[4])
+{
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]),
+          "r"(c[2]), "r"(c[3]));
+}
+
+// D(16x8 s32) = C + A(16x32 s8, row) * B(32x8 u8, col).
+__device__ __forceinline__ void mma_s8u8_16832_acc(int (&d)[4], uint32_t a0, uint32_t a1,
+                                                   uint32_t a2, uint32_t a3, uint32_t b0,
+                                                   uint32_t b1, const int (&c)[4])
+{
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]),
+          "r"(c[2]), "r"(c[3]));
+}
+
+// Two transposed 16x16 byte matrices from shared memory: lanes 0-15 give the row addresses
+// of matrix 0, lanes 16-31 those of matrix 1 (16-byte aligned). Lane (g, c) receives
+// {r0, r1} = bytes [4c..4c+3][g] and [4c..4c+3][g + 8] of matrix 0 (row index first) and
+// {r2, r3} the same of matrix 1: the A fragment of an m16n8k32 8-bit MMA whose rows are
+// the matrices' columns.
+__device__ __forceinline__ void ldsm_x2_trans_b8(uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                                 uint32_t &r3, uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
 // C(16x8 f32) += A(16x16 f16, row) * B(16x8 f16, col).
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
                                               uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1)
@@ -231,6 +285,15 @@ __device__ __forceinline__ void mma_f16_16816_zero_c(float (&d)[4], uint32_t a0,
         "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz: about 2 ulp; results below 2^-126
+// flush to zero, 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // ---------------------------------------------------------------- bit tricks
