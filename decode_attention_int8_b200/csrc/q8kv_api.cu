@@ -172,8 +172,8 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
         return Q8KV_ERR_UNSUPPORTED;
     const long long tiles_per_seq = ((long long)s.mbps * s.bs + pl.TT - 1) / pl.TT;
     const long long tiles_max = (long long)s.B * pl.nhc * tiles_per_seq;
-    if (tiles_max >= (1LL << 31))
-        return Q8KV_ERR_UNSUPPORTED; // tile indices are 32-bit
+    if (tiles_max >= (1LL << 30))
+        return Q8KV_ERR_UNSUPPORTED; // tile indices (and the penalised split) are 32-bit
     pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
     if (2 * pl.grid > kCombineMaxDesc)
         return Q8KV_ERR_UNSUPPORTED;

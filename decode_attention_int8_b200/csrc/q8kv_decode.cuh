@@ -206,19 +206,41 @@ __device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
                              volatile unsigned long long *wsum, int tid, int warp, int lane)
 {
     const int cap = p.mbps * p.bs;
+    auto item = [&](int b) -> unsigned long long {
+        int L = p.seq_lens[b];
+        if (L < 0 || L > cap) {
+            atomicOr(p.errors, kErrSeqLen);
+            L = L < 0 ? 0 : cap;
+        }
+        return ((unsigned long long)(((L + p.TT - 1) / p.TT) * p.nhc) << 32) | (L > 0 ? 1u : 0u);
+    };
+    if (p.B <= 32) { // one warp: no block-wide pass (the caller synchronises once)
+        if (warp == 0) {
+            unsigned long long v = lane < p.B ? item(lane) : 0ull;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long t = __shfl_up_sync(kFullMask, v, o);
+                if (lane >= o)
+                    v += t;
+            }
+            if (lane < p.B) {
+                prefix[lane + 1] = (int)(v >> 32);
+                if (nseq)
+                    nseq[lane + 1] = (int)(v & 0xffffffffu);
+            }
+            if (lane == 0) {
+                prefix[0] = 0;
+                if (nseq)
+                    nseq[0] = 0;
+            }
+        }
+        return;
+    }
     unsigned long long carry = 0;
 #pragma unroll 1
     for (int base = 0; base < p.B; base += kThreads) {
         const int b = base + tid;
-        unsigned long long v = 0;
-        if (b < p.B) {
-            int L = p.seq_lens[b];
-            if (L < 0 || L > cap) {
-                atomicOr(p.errors, kErrSeqLen);
-                L = L < 0 ? 0 : cap;
-            }
-            v = ((unsigned long long)(((L + p.TT - 1) / p.TT) * p.nhc) << 32) | (L > 0 ? 1u : 0u);
-        }
+        unsigned long long v = b < p.B ? item(b) : 0ull;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const unsigned long long t = __shfl_up_sync(kFullMask, v, o);
@@ -229,7 +251,7 @@ __device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
             wsum[warp] = v;
         __syncthreads();
         unsigned long long off = carry, total = 0;
-#pragma unroll 1
+#pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) {
             const unsigned long long ws = wsum[w];
             if (w < warp)
@@ -251,24 +273,28 @@ __device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
     }
 }
 
-// First tile of CTA i (of g) when segment starts are charged P extra tiles: the virtual
-// list puts P units before the tiles of every segment; CTA i starts at virtual unit
-// floor(i * V / g) and takes the tile it lands on (or the segment's first tile when it
-// lands in the segment's penalty).
-__device__ int penalised_start(const DecodeParams &p, const int *prefix, const int *nseq, int P,
-                               long long V, int g, int i)
+// First tile of CTA i (of g) in the work split. Plain split: floor(i * N / g). Penalised
+// split (pseg > 0): the virtual list puts pseg = P * nhc units before every sequence with
+// tokens (P before each of its nhc segments); CTA i starts at virtual unit
+// floor(i * V / g) and takes the tile it lands on, or the segment's first tile when it
+// lands in the segment's penalty. All quantities fit 32 bits (V < 2^31 is checked on the
+// host side through the tile count).
+__device__ int cta_start(const DecodeParams &p, const int *prefix, const int *nseq, int pseg,
+                         int V, int g, int i)
 {
     const int N = prefix[p.B];
     if (i >= g)
         return N;
-    const long long vi = (long long)i * V / g;
-    const long long pseg = (long long)P * p.nhc; // penalty units of one sequence's segments
-    auto vpre = [&](int b) { return (long long)prefix[b] + pseg * nseq[b]; };
-    int lo = 0, hi = p.B - 1; // largest b with vpre(b) <= vi
+    const int qv = V / g, rv = V - qv * g;
+    const int vi = i * qv + (i * rv) / g; // floor(i * V / g) without 64-bit division
+    if (pseg == 0)
+        return vi;
+    const int P = pseg / p.nhc;
+    int lo = 0, hi = p.B - 1; // largest b with vprefix(b) <= vi
 #pragma unroll 1
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (vpre(mid) <= vi)
+        if (prefix[mid] + pseg * nseq[mid] <= vi)
             lo = mid;
         else
             hi = mid - 1;
@@ -276,12 +302,10 @@ __device__ int penalised_start(const DecodeParams &p, const int *prefix, const i
     const int ntb = (prefix[lo + 1] - prefix[lo]) / p.nhc;
     if (ntb == 0)
         return prefix[lo];
-    const long long off = vi - vpre(lo);
-    const long long len = ntb + P;
-    const int hc = (int)(off / len);
-    const int r = (int)(off - hc * len);
-    const int j = r > P ? r - P : 0;
-    const int x = prefix[lo] + (hc < p.nhc ? hc * ntb + j : p.nhc * ntb);
+    const int off = vi - (prefix[lo] + pseg * nseq[lo]);
+    const int hc = off / (ntb + P);
+    const int r = off - hc * (ntb + P);
+    const int x = prefix[lo] + (hc < p.nhc ? hc * ntb + (r > P ? r - P : 0) : p.nhc * ntb);
     return x < N ? x : N;
 }
 
@@ -1420,45 +1444,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int N = prefix[p.B];
     int *cstart = reinterpret_cast<int *>(smem + p.lay.off_cstart);
-    // rows of empty sequences are zero
-#pragma unroll 1
-    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-        if (prefix[b + 1] != prefix[b])
-            continue;
-        float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
-#pragma unroll 1
-        for (int i = tid; i < p.Hq * kD / 4; i += kThreads)
-            row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
     const int gcta = N < (int)gridDim.x ? N : (int)gridDim.x;
-    {
-        // plain split: floor(i * N / gcta); penalised split (see kSegPenaltyTiles) when the
-        // sequence counts are at hand and every CTA's share is at least 4 penalties, so that
-        // no CTA's share can fall inside one segment's penalty (an empty CTA in the middle
-        // of a split segment would break the contributor numbering)
-        const long long V = nseq ? (long long)N + (long long)kSegPenaltyTiles * p.nhc * nseq[p.B]
-                                 : (long long)N;
-        const bool pen = nseq && gcta > 0 && V / gcta >= 4 * kSegPenaltyTiles;
-        const int qn = N / (gcta > 0 ? gcta : 1), rn = N - qn * (gcta > 0 ? gcta : 1);
+    // Work split (see kSegPenaltyTiles): penalised when the sequence counts are at hand and
+    // every CTA's share is at least 4 penalties, so that no CTA's share can fall inside one
+    // segment's penalty (an empty CTA in the middle of a split segment would break the
+    // contributor numbering). Only this CTA's own range is computed before the producer
+    // starts; the consumers fill in the rest of the table (needed at segment ends).
+    const int nseg_units = nseq ? kSegPenaltyTiles * p.nhc * nseq[p.B] : 0;
+    const bool pen = nseq && gcta > 0 && (N + nseg_units) / gcta >= 4 * kSegPenaltyTiles;
+    const int pseg = pen ? kSegPenaltyTiles * p.nhc : 0;
+    const int V = N + (pen ? nseg_units : 0);
+    if (gcta == 0) { // no sequence has tokens: every row is zero
 #pragma unroll 1
-        for (int i = tid; i <= gcta; i += kThreads)
-            cstart[i] = pen ? penalised_start(p, prefix, nseq, kSegPenaltyTiles, V, gcta, i)
-                            : i * qn + (i * rn) / gcta;
+        for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+            float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
+#pragma unroll 1
+            for (int i = tid; i < p.Hq * kD / 4; i += kThreads)
+                row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
     }
+    if (tid < 2 && (int)blockIdx.x + tid <= gcta)
+        cstart[blockIdx.x + tid] = cta_start(p, prefix, nseq, pseg, V, gcta, blockIdx.x + tid);
     __syncthreads();
     if ((int)blockIdx.x >= gcta)
         return;
     const int t0 = cstart[blockIdx.x], t1 = cstart[blockIdx.x + 1];
+    // (the rest of the table and the zero rows of empty sequences: consumers, below)
     // Warp specialisation: the producer warpgroup hands most of its registers to the two
     // consumer warpgroups (the sums match the launch allocation, checked by static_assert).
     if (warp >= kConsumerWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::producer));
         if (warp == kProducerWarp)
             produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
-    } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::consumer));
-        consume<NT, kPack, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
+        return;
     }
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::consumer));
+    const int ctid = warp * 32 + lane;
+#pragma unroll 1
+    for (int i = ctid; i <= gcta; i += kConsumerThreads)
+        if (i != (int)blockIdx.x && i != (int)blockIdx.x + 1)
+            cstart[i] = cta_start(p, prefix, nseq, pseg, V, gcta, i);
+    // rows of empty sequences are zero (spread over the CTAs that have tiles)
+#pragma unroll 1
+    for (int b = blockIdx.x; b < p.B; b += gcta) {
+        if (prefix[b + 1] != prefix[b])
+            continue;
+        float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
+#pragma unroll 1
+        for (int i = ctid; i < p.Hq * kD / 4; i += kConsumerThreads)
+            row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    consumer_bar();
+    consume<NT, kPack, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
 }
 
 } // namespace q8kv
