@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-accuracy", action="store_true",
+                    help="skip the q8-vs-fp32 information report")
     return ap.parse_args()
 
 
@@ -161,6 +163,46 @@ def workload_config(w, n_copies, extra):
                f" > {L2_BYTES / 1e6:.0f} MB L2)"}
     d.update(extra)
     return d
+
+
+def q8_vs_fp32(w, got, n_rows=64, seed=0):
+    """Information only: how far the q8 path's output is from attention over the unquantised
+    fp32 q, K, V (plain fp64 numpy softmax(q K^T * scale) V on a sample of (sequence, head)
+    rows). This measures the int8 quantisation itself, not the kernel's arithmetic."""
+    import numpy as np
+
+    from decode_attention_int8_b200 import inputs
+
+    c = w.cfg
+    fp32_pool_bytes = 2 * 4 * w.k.size
+    if fp32_pool_bytes > (2 << 30):
+        return {"skipped": f"the unquantised fp32 pools would take {fp32_pool_bytes / 1e9:.1f} GB "
+                           "of host memory"}
+    w32 = inputs.make(c, keep_fp32=True)
+    P, bs, Hk, D = w32.k.shape
+    k32 = w32.k32.reshape(P * bs, Hk, D)
+    v32 = w32.v32.reshape(P * bs, Hk, D)
+    rng = np.random.default_rng(seed)
+    G = c.n_q_heads // c.n_kv_heads
+    diffs, refs = [], []
+    for _ in range(n_rows):
+        b = int(rng.integers(0, c.B))
+        h = int(rng.integers(0, c.n_q_heads))
+        L = int(w32.seq_lens[b])
+        if L == 0:
+            continue
+        t = np.arange(L)
+        slot = w32.block_table[b, t // bs].astype(np.int64) * bs + t % bs
+        kf = k32[slot, h // G].astype(np.float64)
+        vf = v32[slot, h // G].astype(np.float64)
+        sc = kf @ w32.q[b, h].astype(np.float64) * w32.scale
+        pr = np.exp(sc - sc.max())
+        ref = pr @ vf / pr.sum()
+        refs.append(ref)
+        diffs.append(np.asarray(got[b, h], np.float64) - ref)
+    d, r = np.array(diffs), np.array(refs)
+    return {"max_abs": float(np.abs(d).max()), "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(r)),
+            "rows": len(refs), "reference": "fp64 attention over the unquantised fp32 q, K, V"}
 
 
 def cpu_baseline(w, min_seconds=10.0):
@@ -401,6 +443,9 @@ def main():
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0 and world == 1 and not args.no_accuracy:
+        torch.cuda.synchronize(dev)
+        line["q8_vs_fp32"] = q8_vs_fp32(w, out.cpu().numpy())
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
