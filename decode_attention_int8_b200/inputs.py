@@ -7,10 +7,10 @@ Recipe (the five named workloads below, plus ``make_custom`` for test grids):
   - q: fp32, iid N(0, 1), shape [B][n_q_heads][head_dim].
   - K, V: fp32 drawn iid per element (N(0, 1), or Student-t with 3 degrees of freedom),
     K optionally plus a per-(KV head, channel) bias held constant over tokens, then
-    quantised per (token, KV head) row: scale = max|x| / 127 (fp32), code =
-    clamp(round-half-even(x / scale), -127, 127); an all-zero row gets scale 1/127 and
-    codes 0. The pools are int8 [num_blocks][block_size][n_kv_heads][head_dim] with fp32
-    scales [num_blocks][block_size][n_kv_heads].
+    quantised per (token, KV head) row with the cache-write rule (``quantize_rows``:
+    scale = max|x| * fl(1/127), code = clamp(round-half-even(x * fl(127 / max|x|)),
+    -127, 127), fp32). The pools are int8 [num_blocks][block_size][n_kv_heads][head_dim]
+    with fp32 scales [num_blocks][block_size][n_kv_heads].
   - block_table: int32 [B][max_blocks_per_seq]; sequence b owns ceil(L_b / block_size)
     physical blocks, assigned in order ("identity") or from a random permutation of the
     pool ("permutation"); unused entries are -1.
@@ -125,17 +125,17 @@ def _draw(rng: np.random.Generator, dist: str, shape) -> np.ndarray:
 
 
 def quantize_rows(x: np.ndarray):
-    """Per-row int8 quantisation of the input data (the cache-writer's recipe):
-    scale = max|x| / 127, code = clamp(rne(x / scale), -127, 127); zero rows get
-    scale 1/127 and codes 0. All arithmetic in fp32."""
+    """Per-row int8 quantisation that turns the drawn fp32 K/V into cache contents, with
+    the same rule as the library's cache write: amax = max|x| (1 when below 1e-6),
+    scale = amax * fl(1/127), code = clamp(rne(x * fl(127 / amax)), -127, 127), every
+    operation rounded to fp32. Finite inputs only (the draws always are)."""
     x = np.asarray(x, np.float32)
     amax = np.max(np.abs(x), axis=-1)
-    zero = amax == 0
-    scale = np.where(zero, np.float32(1.0) / np.float32(127.0), amax / np.float32(127.0))
-    scale = scale.astype(np.float32)
-    codes = np.rint(x / scale[..., None])
+    amax = np.where(amax < np.float32(1e-6), np.float32(1.0), amax).astype(np.float32)
+    scale = (amax * (np.float32(1.0) / np.float32(127.0))).astype(np.float32)
+    inv = (np.float32(127.0) / amax).astype(np.float32)
+    codes = np.rint((x * inv[..., None]).astype(np.float32))
     codes = np.clip(codes, -127, 127).astype(np.int8)
-    codes[zero] = 0
     return codes, scale
 
 

@@ -83,6 +83,8 @@ def _load():
                 "q8kvo_decode_all": [cp, P, P],
                 "q8kvo_decode_pairs": [cp, P, P, l, P],
                 "q8kvo_attn_fp32": [cp, P, P, P, i, i, P],
+                "q8kvo_quantize_kv_row": [P, i, P, P, P],
+                "q8kvo_cache_write": [P, P, P, P, P, P, P, l, i, i, i, i, l, P],
             }
             for name, args in sigs.items():
                 fn = getattr(lib, name)
@@ -94,6 +96,10 @@ def _load():
 
 class OracleError(RuntimeError):
     pass
+
+
+FLAG_SLOT = 0x8
+FLAG_NONFINITE = 0x10
 
 
 def _ptr(a: np.ndarray | None):
@@ -217,3 +223,39 @@ def attn_fp32(cache: PagedCache, q: np.ndarray, k32: np.ndarray, v32: np.ndarray
     _check(_load().q8kvo_attn_fp32(cache.ref(), _ptr(q), _ptr(k32), _ptr(v32), b, h, _ptr(out)),
            "attn_fp32")
     return out
+
+
+def quantize_kv_row(x: np.ndarray):
+    """Cache quantisation of one K or V row: (int8 codes, fp32 scale, flags)."""
+    x = _c(x, np.float32).reshape(-1)
+    codes = np.empty(x.shape, np.int8)
+    scale = np.zeros(1, np.float32)
+    flags = ctypes.c_uint(0)
+    _check(_load().q8kvo_quantize_kv_row(_ptr(x), x.shape[0], _ptr(codes), _ptr(scale),
+                                         ctypes.byref(flags)), "quantize_kv_row")
+    return codes, np.float32(scale[0]), int(flags.value)
+
+
+def cache_write(k, v, ks, vs, k_new, v_new, slot_mapping, token_stride=None) -> int:
+    """KV-cache write into the host pools k, v [P][bs][Hk][D] (int8) and ks, vs
+    [P][bs][Hk] (fp32), modified in place, from k_new, v_new: fp32 arrays whose first axis
+    is the token and whose rows (token i, head h) start at i * token_stride + h * D in the
+    flattened array (token_stride defaults to Hk * D). Returns the flags."""
+    for a, dt in ((k, np.int8), (v, np.int8), (ks, np.float32), (vs, np.float32)):
+        if a.dtype != dt or not a.flags.c_contiguous:
+            raise ValueError("pools must be C-contiguous int8 / fp32 arrays")
+    P, bs, Hk, D = k.shape
+    if v.shape != k.shape or ks.shape != (P, bs, Hk) or vs.shape != (P, bs, Hk):
+        raise ValueError("pool shapes disagree")
+    slots = _c(slot_mapping, np.int64).reshape(-1)
+    n = slots.shape[0]
+    stride = Hk * D if token_stride is None else int(token_stride)
+    k_new = _c(k_new, np.float32).reshape(-1)
+    v_new = _c(v_new, np.float32).reshape(-1)
+    if n and (k_new.shape[0] < (n - 1) * stride + Hk * D or v_new.shape != k_new.shape):
+        raise ValueError("k_new / v_new too small for the token count and stride")
+    flags = ctypes.c_uint(0)
+    _check(_load().q8kvo_cache_write(_ptr(k), _ptr(v), _ptr(ks), _ptr(vs), _ptr(k_new),
+                                     _ptr(v_new), _ptr(slots), n, Hk, D, bs, P, stride,
+                                     ctypes.byref(flags)), "cache_write")
+    return int(flags.value)

@@ -86,6 +86,107 @@ int q8kvo_quantize_q(const float *q, long n, int8_t *qi, float *qsc)
     return Q8KVO_OK;
 }
 
+/* ---------------------------------------------------------------- KV-cache write */
+
+/* One K or V row of n values for the cache. The walk-through keeps one scale per
+ * (token, KV head) (trdm.cn/news/511694, the kernel signature's "per-token per-head"
+ * kscale comment) and turns it into the dequantisation multiplier by one multiply with
+ * 1/127 at use (section 2 part 2, kscale * KVQ_INV); the quantiser is the one section 2
+ * part 1 gives for Q ("Q8_0 isomorphic"), applied to the whole row as one block:
+ *   amax  = max |x_i|                       (fp32)
+ *   if amax < 1e-6: amax = 1                (all-zero row -> codes 0, scale 1/127)
+ *   scale = amax * (1/127)                  (fp32: the multiplier stored in the cache)
+ *   inv   = 127 / amax                      (fp32, correctly rounded)
+ *   code  = clamp(rne(x_i * inv), -127, 127) (product rounded to fp32 first)
+ * A row holding an infinity or a NaN has no meaningful scale: its codes are 0, its scale
+ * is a quiet NaN and *flags gets Q8KVO_FLAG_NONFINITE. */
+static void quantize_kv_row(const float *x, int n, int8_t *codes, float *scale,
+                            unsigned *flags)
+{
+    float amax = 0.0f;
+    int finite = 1;
+    for (int i = 0; i < n && !MUT(15); ++i) {
+        if (!isfinite(x[i]))
+            finite = 0;
+        float a = fabsf(x[i]);
+        if (a > amax)
+            amax = a;
+    }
+    for (int i = 0; i < n && i < 32 && MUT(15); ++i) { /* planted: first 32 channels */
+        if (!isfinite(x[i]))
+            finite = 0;
+        if (fabsf(x[i]) > amax)
+            amax = fabsf(x[i]);
+    }
+    if (!finite) {
+        for (int i = 0; i < n; ++i)
+            codes[i] = 0;
+        *scale = NAN;
+        *flags |= Q8KVO_FLAG_NONFINITE;
+        return;
+    }
+    if (amax < 1e-6f)
+        amax = 1.0f;
+    *scale = MUT(17) ? amax : amax * (1.0f / 127.0f);
+    float inv = 127.0f / amax;
+    for (int i = 0; i < n; ++i) {
+        float prod = x[i] * inv;
+        double r = MUT(16) ? trunc((double)prod) : round_half_even((double)prod);
+        if (r > 127.0)
+            r = 127.0;
+        if (r < -127.0)
+            r = -127.0;
+        codes[i] = (int8_t)r;
+    }
+}
+
+int q8kvo_quantize_kv_row(const float *x, int n, int8_t *codes, float *scale, unsigned *flags)
+{
+    if (!x || !codes || !scale || !flags || n <= 0)
+        return Q8KVO_EINVAL;
+    quantize_kv_row(x, n, codes, scale, flags);
+    return Q8KVO_OK;
+}
+
+/* Write n_tokens new (token, KV head) rows of K and of V into the paged pools.
+ * Token i goes to physical slot slot_mapping[i] = block * block_size + offset (the
+ * block-table mapping of beaiera.top "deepseek-attention-div64", section "Top-K index
+ * global mapping"); a negative slot marks a padding entry and is skipped, as the same
+ * section prescribes for its -1 entries. A slot at or past num_blocks * block_size is
+ * skipped too and sets Q8KVO_FLAG_SLOT. Row (i, h) of k_new starts at
+ * k_new[i * token_stride + h * head_dim]; it lands at k[(slot * n_kv_heads + h) * head_dim]
+ * and its scale at ks[slot * n_kv_heads + h] (same for V). Slots are taken in token order,
+ * so when two tokens name one slot the later one wins. */
+int q8kvo_cache_write(int8_t *k, int8_t *v, float *ks, float *vs, const float *k_new,
+                      const float *v_new, const int64_t *slot_mapping, long n_tokens,
+                      int n_kv_heads, int head_dim, int block_size, int num_blocks,
+                      long token_stride, unsigned *flags)
+{
+    if (!k || !v || !ks || !vs || !k_new || !v_new || !slot_mapping || !flags)
+        return Q8KVO_EINVAL;
+    if (n_tokens < 0 || n_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
+        token_stride < (long)n_kv_heads * head_dim)
+        return Q8KVO_EINVAL;
+    const int64_t n_slots = (int64_t)num_blocks * block_size;
+    for (long i = 0; i < n_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        if (slot >= n_slots) {
+            *flags |= Q8KVO_FLAG_SLOT;
+            continue;
+        }
+        for (int h = 0; h < n_kv_heads; ++h) {
+            int hd = MUT(18) ? (h + 1) % n_kv_heads : h;
+            long src = i * token_stride + (long)h * head_dim;
+            long row = (long)slot * n_kv_heads + hd;
+            quantize_kv_row(k_new + src, head_dim, k + row * head_dim, ks + row, flags);
+            quantize_kv_row(v_new + src, head_dim, v + row * head_dim, vs + row, flags);
+        }
+    }
+    return Q8KVO_OK;
+}
+
 /* ---------------------------------------------------------------- cache access */
 
 static int check_cache(const q8kvo_cache *c)

@@ -17,7 +17,10 @@
  *     (softmax weight x per-(token, head) V scale);
  *   - section 2, part 3 ("normalise the output"): one division by S at the end;
  *   - section 3 ("consequences of the change"): the naive variant that stores every
- *     score first is functionally equivalent (used here as a cross-check).
+ *     score first is functionally equivalent (used here as a cross-check);
+ *   - the opening and the kernel signature (KV compressed to q8 with one scale per
+ *     (token, KV head), applied as scale * 1/127 at use): the KV-cache write that fills
+ *     the pools, with the section 2 part 1 quantiser applied to whole rows.
  * GQA head mapping kv_head = q_head / (n_q_heads / n_kv_heads) follows the llama2.c
  * attention loop (aicoding.csdn.net, "attention core logic").
  * The block-table -> slot mapping follows beaiera.top "deepseek-attention-div64",
@@ -72,6 +75,25 @@ typedef struct {
 /* Quantise n fp32 values (n a multiple of 32) block by block.
  * qi[n] receives the int8 codes, qsc[n/32] the per-block fp32 scales. */
 int q8kvo_quantize_q(const float *q, long n, int8_t *qi, float *qsc);
+
+/* Flags of the KV-cache write (the same bits as the CUDA library's device error word). */
+#define Q8KVO_FLAG_SLOT 0x8u       /* a slot at or past num_blocks * block_size (skipped) */
+#define Q8KVO_FLAG_NONFINITE 0x10u /* a row held an infinity or a NaN (codes 0, scale NaN) */
+
+/* Quantise one K or V row of n fp32 values for the cache: one fp32 dequantisation
+ * multiplier for the row and n int8 codes (rule in q8kv_oracle.c). Non-finite rows set
+ * Q8KVO_FLAG_NONFINITE in *flags. */
+int q8kvo_quantize_kv_row(const float *x, int n, int8_t *codes, float *scale, unsigned *flags);
+
+/* KV-cache write: quantise the n_tokens x n_kv_heads rows of k_new and v_new (fp32, row
+ * (i, h) at [i * token_stride + h * head_dim]) and store codes and scales at physical slot
+ * slot_mapping[i] of the pools k, v [num_blocks][block_size][n_kv_heads][head_dim] and
+ * ks, vs [num_blocks][block_size][n_kv_heads]. Negative slots are skipped; slots past the
+ * pool are skipped and set Q8KVO_FLAG_SLOT. */
+int q8kvo_cache_write(int8_t *k, int8_t *v, float *ks, float *vs, const float *k_new,
+                      const float *v_new, const int64_t *slot_mapping, long n_tokens,
+                      int n_kv_heads, int head_dim, int block_size, int num_blocks,
+                      long token_stride, unsigned *flags);
 
 /* int32 dot product of each 32-element block of the quantised query of (b, h) with
  * the K row of every token of sequence b: dots[t][j], t < seq_lens[b], j < head_dim/32. */

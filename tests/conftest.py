@@ -54,3 +54,31 @@ def load_golden_qquant():
     for c in cases:
         assert c["q"].shape == (32,) and c["codes"].shape == (32,), c["name"]
     return cases
+
+
+def load_golden_kvquant():
+    """Parse tests/golden/kvquant_cases.txt into dicts: name, x, codes, scale_bits
+    (int, "approx" or "nan") and flags."""
+    import numpy as np
+
+    path = os.path.join(ROOT, "tests", "golden", "kvquant_cases.txt")
+    cases, cur = [], None
+    for raw in open(path):
+        line = raw.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, *vals = line.split()
+        if key == "case":
+            cur = {"name": vals[0]}
+            cases.append(cur)
+        elif key == "x":
+            cur["x"] = np.array([float(v) for v in vals], np.float32)
+        elif key == "codes":
+            cur["codes"] = np.array([int(v) for v in vals], np.int8)
+        elif key == "scale_bits":
+            cur["scale_bits"] = vals[0] if vals[0] in ("approx", "nan") else int(vals[0], 16)
+        elif key == "flags":
+            cur["flags"] = int(vals[0])
+    for c in cases:
+        assert c["x"].shape == c["codes"].shape == (64,), c["name"]
+    return cases

@@ -25,6 +25,10 @@ MUTANTS = {
     10: "running sum S not rescaled when M rises",
     13: "softmax scale applied twice",
     14: "K channel index shifted by one inside a block",
+    15: "cache row scale taken from the first 32 channels only",
+    16: "cache codes truncated instead of rounded half-to-even",
+    17: "cache stores max|x| instead of the dequantisation multiplier",
+    18: "cache row written under the next KV head",
 }
 
 
@@ -34,7 +38,8 @@ def test_planted_mistake_is_caught(mutant, tmp_path):
     env = dict(os.environ, Q8KV_ORACLE_LIB=lib)
     r = subprocess.run(
         [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-         "tests/test_oracle_qquant.py", "tests/test_oracle_attention.py"],
+         "tests/test_oracle_qquant.py", "tests/test_oracle_attention.py",
+         "tests/test_oracle_cache_write.py"],
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {mutant} ({MUTANTS[mutant]}) passed every pin"
     assert "failed" in r.stdout, r.stdout[-2000:]
