@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-accuracy", action="store_true",
                     help="skip the q8-vs-fp32 information report")
+    ap.add_argument("--no-cache-write", action="store_true",
+                    help="skip the KV-cache write information report")
     return ap.parse_args()
 
 
@@ -413,16 +415,7 @@ def main():
 
     peak, peak_kind = measured_peak()
     achieved = algo / (kernel_ms * 1e-3) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.txt")
-    if os.path.exists(tpath):
-        h = source_hash()
-        with open(tpath) as f:
-            for ln in f:
-                parts = ln.split()
-                if len(parts) == 3 and not ln.startswith("#") and parts[0] == c.name \
-                        and parts[1] == h:
-                    traffic = int(parts[2])
+    traffic = recorded_traffic(c.name, "decode")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
@@ -443,6 +436,11 @@ def main():
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+    if not args.no_cache_write:
+        # information, after the timed region: the write path that fills the cache
+        del pools, argsets
+        torch.cuda.empty_cache()
+        line["cache_write"] = bench_cache_write(dev, stream)
     if rank == 0 and world == 1 and not args.no_accuracy:
         torch.cuda.synchronize(dev)
         line["q8_vs_fp32"] = q8_vs_fp32(w, out.cpu().numpy())
@@ -454,17 +452,108 @@ def main():
     return 0
 
 
-def source_hash() -> str:
-    """Hash of the kernel sources (traffic figures are valid only for the exact kernel)."""
+CACHE_WRITE_SOURCES = ("q8kv_cache_write.cuh", "q8kv_ptx.cuh")
+
+
+def source_hash(kernel: str = "decode") -> str:
+    """Hash of the sources a kernel is built from (traffic figures are valid only for the
+    exact kernel): the cache write's own header and the PTX helpers, or, for the decode
+    call, every other source of the library (its kernels, helpers and launch plan)."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_attention_int8_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        mine = name in CACHE_WRITE_SOURCES if kernel == "cache_write" else \
+            name != "q8kv_cache_write.cuh"
+        if not mine:
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def recorded_traffic(name: str, kernel: str = "decode"):
+    """DRAM bytes per launch recorded under profiles/ for this workload and exact source."""
+    tpath = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(tpath):
+        return None
+    h = source_hash(kernel)
+    with open(tpath) as f:
+        for ln in f:
+            parts = ln.split()
+            if len(parts) == 3 and not ln.startswith("#") and parts[0] == name and parts[1] == h:
+                return int(parts[2])
+    return None
+
+
+def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):
+    """Information: the KV-cache write (q8kv_cache_write), timed like the decode call.
+
+    prompt_fill: fresh fp32 K/V rows for all 65536 tokens of the 16 x 4096-token GQA
+    workload (8 KV heads, head_dim 128) written to the slots of its permuted block table;
+    537 MB of fp32 rows in and 138 MB of codes and scales out per call, more than the L2.
+    decode_step: one new token per sequence (16 x 8 rows), the append of a decode step,
+    bound by launch latency rather than by bandwidth."""
+    import numpy as np
+    import torch
+
+    import decode_attention_int8_b200 as q8
+    from decode_attention_int8_b200 import inputs
+
+    cfg = inputs.CONFIGS[1]
+    rows = inputs.make_prompt_fill(cfg)
+    n, Hk, D, bs = rows.n_tokens, cfg.n_kv_heads, cfg.head_dim, cfg.block_size
+    P = int(rows.slots.max()) // bs + 1
+    k = torch.zeros((P, bs, Hk, D), dtype=torch.int8, device=dev)
+    v = torch.zeros_like(k)
+    ks = torch.zeros((P, bs, Hk), dtype=torch.float32, device=dev)
+    vs = torch.zeros_like(ks)
+    kn = torch.from_numpy(rows.k_new).to(dev).view(n, Hk, D)
+    vn = torch.from_numpy(rows.v_new).to(dev).view(n, Hk, D)
+    slots = torch.from_numpy(rows.slots).to(dev)
+    step_idx = torch.arange(step_B, device=dev) * (n // step_B) + (n // step_B - 1)
+    s_kn, s_vn, s_slots = kn[step_idx].contiguous(), vn[step_idx].contiguous(), slots[step_idx]
+
+    def timed(args_):
+        for _ in range(warmup):
+            q8.q8kv_cache_write(*args_, stream=stream)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            q8.q8kv_cache_write(*args_, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps
+
+    q8.q8kv_device_errors(clear=True)
+    ms_fill = timed((k, v, ks, vs, kn, vn, slots))
+    ms_step = timed((k, v, ks, vs, s_kn, s_vn, s_slots))
+    errs = q8.q8kv_device_errors(clear=True)
+    algo = rows.algorithmic_bytes()
+    peak, peak_kind = measured_peak()
+    achieved = algo / (ms_fill * 1e-3) / 1e9
+    step_bytes = step_B * Hk * 2 * (5 * D + 4) + 8 * step_B
+    return {
+        "prompt_fill": {
+            "workload": f"gqa_batch prompt fill: {n} tokens x {Hk} KV heads x {D}, block {bs}, "
+                        f"permuted {P}-block table",
+            "us_per_call": round(ms_fill * 1e3, 3), "calls": steps,
+            "algorithmic_bytes": algo,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": recorded_traffic("gqa_prompt_fill", "cache_write"),
+                         "kernel": "q8kv::cache_write_kernel<128>"},
+            "l2": "inputs (537 MB of fp32 rows) and outputs (138 MB) larger than L2"},
+        "decode_step": {"workload": f"one new token per sequence: {step_B} x {Hk} rows",
+                        "us_per_call": round(ms_step * 1e3, 3), "calls": steps,
+                        "algorithmic_bytes": step_bytes,
+                        "note": "launch-latency bound (bytes fit in L2)"},
+        "device_errors": errs,
+    }
 
 
 if __name__ == "__main__":

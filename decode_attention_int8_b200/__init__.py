@@ -5,12 +5,15 @@ this package is its ctypes binding plus the seeded synthetic workload generators
 """
 from ._lib import (  # noqa: F401
     DEVERR_BLOCK_TABLE,
+    DEVERR_NONFINITE,
     DEVERR_SEQ_LEN,
+    DEVERR_SLOT,
     DEVERR_TIMEOUT,
     EXPORTS,
     Q8KVError,
     lib,
     lib_path,
+    q8kv_cache_write,
     q8kv_debug_block_dots,
     q8kv_debug_quantize_q,
     q8kv_decode_attn,

@@ -21,6 +21,8 @@ Q8KV_OK = 0
 DEVERR_SEQ_LEN = 0x1
 DEVERR_BLOCK_TABLE = 0x2
 DEVERR_TIMEOUT = 0x4
+DEVERR_SLOT = 0x8
+DEVERR_NONFINITE = 0x10
 
 EXPORTS = (
     "q8kv_decode_attn",
@@ -28,6 +30,7 @@ EXPORTS = (
     "q8kv_workspace_init",
     "q8kv_decode_attn_ws",
     "q8kv_decode_attn_static",
+    "q8kv_cache_write",
     "q8kv_debug_quantize_q",
     "q8kv_debug_block_dots",
     "q8kv_device_errors",
@@ -66,6 +69,7 @@ def lib():
                 "q8kv_workspace_init": ([P, Z, P], I),
                 "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
                 "q8kv_decode_attn_static": ([P] * 8 + [I] * 7 + [F, P], I),
+                "q8kv_cache_write": ([P] * 7 + [I] * 5 + [ctypes.c_longlong, P], I),
                 "q8kv_debug_quantize_q": ([P, P, P, I, I, P], I),
                 "q8kv_debug_block_dots": ([P, I] + [P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
@@ -170,6 +174,35 @@ def q8kv_decode_attn_static(out, q, k_blocks, v_blocks, kscale, vscale, block_ta
                                          _ptr(seq_lens), *geo, float(scale), _stream(stream)),
            "q8kv_decode_attn_static")
     return out
+
+
+def q8kv_cache_write(k_blocks, v_blocks, kscale, vscale, k_new, v_new, slot_mapping,
+                     stream=None):
+    """Quantise the new rows k_new, v_new [n_tokens][n_kv_heads][head_dim] (fp32; the
+    token dimension may be strided, e.g. a slice of a fused QKV projection) and store them
+    at the physical slots slot_mapping [n_tokens] (int64; negative = padding) of the pools."""
+    _need(k_blocks, "k_blocks", torch.int8, 4)
+    _need(v_blocks, "v_blocks", torch.int8, 4)
+    _need(kscale, "kscale", torch.float32, 3)
+    _need(vscale, "vscale", torch.float32, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    P, bs, Hk, D = k_blocks.shape
+    if tuple(v_blocks.shape) != (P, bs, Hk, D) or tuple(kscale.shape) != (P, bs, Hk) or \
+            tuple(vscale.shape) != (P, bs, Hk):
+        raise ValueError("pool shapes disagree")
+    n = int(slot_mapping.shape[0])
+    for t, name in ((k_new, "k_new"), (v_new, "v_new")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA float32 tensor")
+        if tuple(t.shape) != (n, Hk, D) or t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name}: expected shape {(n, Hk, D)} with contiguous rows, got "
+                             f"{tuple(t.shape)} strides {t.stride()}")
+    if n > 1 and k_new.stride(0) != v_new.stride(0):
+        raise ValueError("k_new and v_new must have the same token stride")
+    stride = int(k_new.stride(0)) if n > 1 else Hk * D
+    _check(lib().q8kv_cache_write(_ptr(k_blocks), _ptr(v_blocks), _ptr(kscale), _ptr(vscale),
+                                  _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), n, Hk, D, bs, P,
+                                  stride, _stream(stream)), "q8kv_cache_write")
 
 
 def q8kv_debug_quantize_q(qi, qsc, q, stream=None):

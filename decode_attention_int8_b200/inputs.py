@@ -28,7 +28,7 @@ from dataclasses import dataclass, field, replace
 import numpy as np
 
 # Stream identifiers of the PCG64 seed sequences.
-_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS = range(6)
+_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS, _S_NEWK, _S_NEWV, _S_SLOTS, _S_MAG = range(10)
 _CHUNK_SLOTS = 4096  # pool slots generated per independent random stream
 
 
@@ -236,3 +236,112 @@ def _make(cfg: Config, seq_lens, max_blocks_per_seq, extra_blocks, keep_fp32, th
 
 def with_config(cfg: Config, **kw) -> Config:
     return replace(cfg, **kw)
+
+
+# ---------------------------------------------------------------- KV-cache write inputs
+
+
+@dataclass
+class CacheRows:
+    """New K/V rows for the KV-cache write and where they go."""
+    k_new: np.ndarray  # fp32 [n_tokens][token_stride] (row (i, h) at [i][h * D:(h + 1) * D])
+    v_new: np.ndarray
+    slots: np.ndarray  # int64 [n_tokens]; -1 = padding
+    n_kv_heads: int
+    head_dim: int
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.slots.shape[0])
+
+    def algorithmic_bytes(self) -> int:
+        """Bytes one write must move: every non-padding (token, KV head) K and V row read
+        (fp32) and written (int8 codes + fp32 scale), and the slot mapping read."""
+        n = int(np.count_nonzero(self.slots >= 0))
+        rows = n * self.n_kv_heads
+        return rows * 2 * (4 * self.head_dim + self.head_dim + 4) + 8 * self.n_tokens
+
+
+def _mixed_rows(seed, stream, n, Hk, D, threads):
+    """Rows of N(0, 1) or Student-t(3) draws times a per-row magnitude in {1e-3, 1, 30},
+    with about 1 row in 64 all zero and 1 in 64 below 1e-6 everywhere."""
+    out = np.empty((n, Hk, D), np.float32)
+    chunk = _CHUNK_SLOTS
+    n_chunks = -(-n // chunk)
+
+    def work(i):
+        lo, hi = i * chunk, min(n, (i + 1) * chunk)
+        rng = _rng(seed, stream, i)
+        x = rng.standard_normal((hi - lo, Hk, D), dtype=np.float32)
+        heavy = rng.random((hi - lo, Hk)) < 0.25
+        if heavy.any():
+            x[heavy] = rng.standard_t(3.0, (int(heavy.sum()), D)).astype(np.float32)
+        kind = rng.integers(0, 64, size=(hi - lo, Hk))
+        mag = np.choose(kind % 3, [np.float32(1e-3), np.float32(1.0), np.float32(30.0)])
+        mag = np.where(kind == 0, np.float32(0.0), mag)
+        mag = np.where(kind == 1, np.float32(1e-7), mag)
+        out[lo:hi] = x * mag[..., None].astype(np.float32)
+
+    if threads > 1 and n_chunks > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(work, range(n_chunks)))
+    else:
+        for i in range(n_chunks):
+            work(i)
+    return out
+
+
+def _strided(rows: np.ndarray, token_stride: int | None, fill: float) -> np.ndarray:
+    n, Hk, D = rows.shape
+    stride = token_stride or Hk * D
+    buf = np.full((n, stride), fill, np.float32)
+    buf[:, :Hk * D] = rows.reshape(n, Hk * D)
+    return buf
+
+
+def make_cache_rows(n_tokens, n_kv_heads, head_dim, num_blocks, block_size, *, seed=0,
+                    pad_every=0, token_stride=None, threads=None) -> CacheRows:
+    """Rows for a scattered write: n_tokens distinct slots drawn from a random permutation
+    of the pool, every pad_every-th token (if > 0) marked as padding (-1). With a
+    token_stride above n_kv_heads * head_dim the unused tail of every token is NaN (it
+    stands for the other heads of a fused projection and must never be read)."""
+    threads = threads or min(32, os.cpu_count() or 1)
+    n_slots = num_blocks * block_size
+    if n_tokens > n_slots:
+        raise ValueError("more tokens than slots")
+    slots = _rng(seed, _S_SLOTS).permutation(n_slots)[:n_tokens].astype(np.int64)
+    if pad_every > 0:
+        slots[pad_every - 1::pad_every] = -1
+    k = _mixed_rows(seed, _S_NEWK, n_tokens, n_kv_heads, head_dim, threads)
+    v = _mixed_rows(seed, _S_NEWV, n_tokens, n_kv_heads, head_dim, threads)
+    return CacheRows(_strided(k, token_stride, np.nan), _strided(v, token_stride, np.nan), slots,
+                     n_kv_heads, head_dim)
+
+
+def prompt_slots(block_table: np.ndarray, seq_lens, block_size: int) -> np.ndarray:
+    """Slot of every token of every sequence, sequence after sequence (a prompt fill):
+    block_table[b][t // block_size] * block_size + t % block_size."""
+    parts = []
+    for b, L in enumerate(np.asarray(seq_lens, np.int64)):
+        t = np.arange(L, dtype=np.int64)
+        parts.append(block_table[b, t // block_size].astype(np.int64) * block_size + t % block_size)
+    return np.concatenate(parts) if parts else np.zeros(0, np.int64)
+
+
+def make_prompt_fill(cfg: Config | int, *, threads: int | None = None) -> CacheRows:
+    """Fresh fp32 K/V rows for every token of a named workload, with the slots its block
+    table gives them: the write that fills that workload's whole cache."""
+    if isinstance(cfg, int):
+        cfg = CONFIGS[cfg]
+    threads = threads or min(32, os.cpu_count() or 1)
+    lens = _seq_lens(cfg)
+    bs = cfg.block_size
+    need = int(((lens.astype(np.int64) + bs - 1) // bs).sum())
+    mbps = max(1, -(-int(lens.max(initial=0)) // bs))
+    bt = build_block_table(lens, bs, mbps, cfg.table, max(1, need), _rng(cfg.seed, _S_TABLE))
+    slots = prompt_slots(bt, lens, bs)
+    n = int(slots.shape[0])
+    Hk, D = cfg.n_kv_heads, cfg.head_dim
+    k = _mixed_rows(cfg.seed, _S_NEWK, n, Hk, D, threads)
+    v = _mixed_rows(cfg.seed, _S_NEWV, n, Hk, D, threads)
+    return CacheRows(k.reshape(n, Hk * D), v.reshape(n, Hk * D), slots, Hk, D)

@@ -80,6 +80,8 @@ typedef enum {
 #define Q8KV_DEVERR_SEQ_LEN 0x1u     /* a seq_len was negative or too long (clamped)     */
 #define Q8KV_DEVERR_BLOCK_TABLE 0x2u /* a block-table entry was outside the pool (skipped) */
 #define Q8KV_DEVERR_TIMEOUT 0x4u     /* a pipeline wait ran past its limit (kernel gave up) */
+#define Q8KV_DEVERR_SLOT 0x8u        /* cache write: a slot past the pool (row skipped)     */
+#define Q8KV_DEVERR_NONFINITE 0x10u  /* cache write: a row held inf or NaN (codes 0, NaN scale) */
 
 /*
  * Decode attention with a library-managed workspace (one per device, grown on demand
@@ -169,6 +171,46 @@ q8kv_status q8kv_decode_attn_static(float *out, const float *q, const int8_t *k_
                                     int n_kv_heads, int head_dim, int kv_block_size,
                                     int max_blocks_per_seq, int num_kv_blocks, float scale,
                                     cudaStream_t stream);
+
+/*
+ * KV-cache write: quantise n_tokens new K rows and V rows per KV head and store them, with
+ * their scales, at the given physical slots of the pools the decode entry points read.
+ *
+ * Quantisation of each (token, KV head) row of head_dim values, for K and V alike (the
+ * walk-through's cache keeps one scale per (token, KV head), kernel signature comment, and
+ * forms the dequantisation multiplier as scale * 1/127, section 2 part 2; the quantiser is
+ * step 1's, taken over the whole row), in IEEE fp32:
+ *   amax = max|x| (1 when below 1e-6), scale = amax * fl(1/127),
+ *   code = clamp(round-half-to-even(x * fl(127 / amax)), -127, 127)
+ * kscale / vscale receive `scale` (the multiplier value = code * scale of the layouts
+ * above). A row holding an infinity or a NaN is stored as codes 0 with a NaN scale and
+ * sets Q8KV_DEVERR_NONFINITE.
+ *
+ * Placement (beaiera.top "deepseek-attention-div64", "Top-K index global mapping"):
+ * token i goes to slot s = slot_mapping[i] = block * kv_block_size + offset; row h lands at
+ * k_blocks[s][h][:] with its scale at kscale[s][h] (the same for V). A negative slot marks
+ * padding: the token is skipped. A slot >= num_kv_blocks * kv_block_size is skipped and
+ * sets Q8KV_DEVERR_SLOT. Slots must be distinct within one call (two tokens naming one
+ * slot race; which one lands is unspecified).
+ *
+ *   k_blocks, v_blocks, kscale, vscale: the pools (layouts above), written in place
+ *   k_new, v_new  fp32; row (i, h) starts at element i * token_stride + h * head_dim
+ *                 (16-byte aligned)
+ *   slot_mapping  int64 [n_tokens]
+ *   n_tokens      >= 0 (0: nothing is enqueued, and k_new, v_new, slot_mapping may be null)
+ *   head_dim      64, 128 or 256 (other multiples of 32: Q8KV_ERR_UNSUPPORTED)
+ *   token_stride  floats between consecutive tokens' rows (0 = n_kv_heads * head_dim;
+ *                 otherwise >= that and a multiple of 4, e.g. the row stride of a fused
+ *                 QKV projection)
+ * One kernel launch, asynchronous on `stream`; it may be scheduled while the previous
+ * kernel on the stream drains and waits for it before reading anything (programmatic
+ * dependent launch), and a decode call enqueued after it sees the written rows.
+ */
+q8kv_status q8kv_cache_write(int8_t *k_blocks, int8_t *v_blocks, float *kscale, float *vscale,
+                             const float *k_new, const float *v_new,
+                             const int64_t *slot_mapping, int n_tokens, int n_kv_heads,
+                             int head_dim, int kv_block_size, int num_kv_blocks,
+                             long long token_stride, cudaStream_t stream);
 
 /* Debug: the Q quantisation alone (step 1) on n_rows rows of head_dim fp32 values
  * (head_dim a multiple of 32). qi int8 [n_rows][head_dim], qsc fp32

@@ -46,7 +46,7 @@ def test_status_strings_and_version():
     assert L.q8kv_status_string(0) == b"ok"
     assert L.q8kv_status_string(2) == b"unsupported shape"
     assert L.q8kv_status_string(99) == b"unknown status"
-    assert L.q8kv_version() == 100
+    assert L.q8kv_version() == 101
 
 
 def _call(**over):
@@ -94,3 +94,40 @@ def test_debug_entry_points_reject_bad_arguments():
     assert L.q8kv_debug_block_dots(P(0x1000), 63, *args) == INVALID  # < max_blocks * block_size
     assert L.q8kv_workspace_init(None, 16, None) == INVALID
     assert L.q8kv_device_errors(None, 0) == INVALID
+
+
+def _write(**over):
+    """q8kv_cache_write with fake (aligned, never dereferenced) pointers."""
+    a = dict(k=0x10000, v=0x20000, ks=0x30000, vs=0x40000, kn=0x50000, vn=0x60000, sl=0x70000,
+             n=4, Hk=2, D=128, bs=16, P=8, stride=0)
+    a.update(over)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return q8.lib().q8kv_cache_write(P(a["k"]), P(a["v"]), P(a["ks"]), P(a["vs"]), P(a["kn"]),
+                                     P(a["vn"]), P(a["sl"]), a["n"], a["Hk"], a["D"], a["bs"],
+                                     a["P"], a["stride"], None)
+
+
+@pytest.mark.parametrize("field", ["k", "v", "ks", "vs", "kn", "vn", "sl"])
+def test_cache_write_null_pointer_rejected(field):
+    assert _write(**{field: None}) == INVALID
+
+
+@pytest.mark.parametrize("over", [dict(n=-1), dict(Hk=0), dict(D=0), dict(D=100), dict(bs=0),
+                                  dict(P=0), dict(stride=255), dict(stride=258), dict(kn=0x50004),
+                                  dict(vn=0x60008), dict(k=0x10001), dict(ks=0x30002),
+                                  dict(sl=0x70004)])
+def test_cache_write_bad_arguments_rejected(over):
+    assert _write(**over) == INVALID
+
+
+@pytest.mark.parametrize("D", [32, 96, 160, 512])
+def test_cache_write_unsupported_head_dim(D):
+    assert _write(D=D) == UNSUPPORTED
+
+
+def test_cache_write_of_no_tokens_enqueues_nothing():
+    # returns before any CUDA call, so it succeeds even without a GPU; the row pointers of
+    # an empty call may be null (an empty torch tensor has none)
+    assert _write(n=0) == OK
+    assert _write(n=0, kn=None, vn=None, sl=None) == OK
+    assert _write(n=0, k=None) == INVALID
