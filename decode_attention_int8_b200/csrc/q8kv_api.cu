@@ -10,7 +10,6 @@
 #include <mutex>
 
 #include "q8kv.h"
-#include "q8kv_cache_write.cuh"
 #include "q8kv_combine.cuh"
 #include "q8kv_decode.cuh"
 #include "q8kv_qquant.cuh"
@@ -21,8 +20,7 @@ using namespace q8kv;
 
 static_assert(kCombineSlotRow == kSlotRow, "partial row layout differs between the kernels");
 static_assert(kErrSeqLen == Q8KV_DEVERR_SEQ_LEN && kErrBlockTable == Q8KV_DEVERR_BLOCK_TABLE &&
-                  kErrTimeout == Q8KV_DEVERR_TIMEOUT && kErrSlot == Q8KV_DEVERR_SLOT &&
-                  kErrNonFinite == Q8KV_DEVERR_NONFINITE,
+                  kErrTimeout == Q8KV_DEVERR_TIMEOUT,
               "device error bits differ from the header");
 
 __device__ unsigned g_device_errors = 0;
@@ -475,25 +473,6 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
                 : launch_kernel<2, false, false>(*dev, p, pl, mk, mv, mks, mvs, stream);
 }
 
-template <int D>
-q8kv_status launch_cache_write(const CacheWriteParams &p, int sms, cudaStream_t stream)
-{
-    // one full wave of resident blocks, striding over the rows
-    const long long want = (p.n_rows + kWriteWarps - 1) / kWriteWarps;
-    const long long cap = (long long)write_blocks_per_sm(D) * sms;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(want < cap ? want : cap));
-    cfg.blockDim = dim3(kWriteThreads);
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    Q8KV_CUDA(cudaLaunchKernelEx(&cfg, cache_write_kernel<D>, p));
-    return Q8KV_OK;
-}
-
 } // namespace
 
 // Scratch of q8kv_decode_attn_static: split-KV counters and partial results at the same
@@ -635,61 +614,6 @@ q8kv_status q8kv_decode_attn_static(float *out, const float *q, const int8_t *k_
     return run(c, scratch, Q8KV_STATIC_SCRATCH_BYTES, false, stream);
 }
 
-q8kv_status q8kv_cache_write(int8_t *k_blocks, int8_t *v_blocks, float *kscale, float *vscale,
-                             const float *k_new, const float *v_new,
-                             const int64_t *slot_mapping, int n_tokens, int n_kv_heads,
-                             int head_dim, int kv_block_size, int num_kv_blocks,
-                             long long token_stride, cudaStream_t stream)
-{
-    if (!k_blocks || !v_blocks || !kscale || !vscale)
-        return Q8KV_ERR_INVALID_ARG;
-    if (n_tokens < 0 || n_kv_heads <= 0 || head_dim <= 0 || head_dim % 32 != 0 ||
-        kv_block_size <= 0 || num_kv_blocks <= 0)
-        return Q8KV_ERR_INVALID_ARG;
-    const long long row = (long long)n_kv_heads * head_dim;
-    if (token_stride == 0)
-        token_stride = row;
-    if (token_stride < row || token_stride % 4 != 0)
-        return Q8KV_ERR_INVALID_ARG;
-    if (!aligned16(k_blocks) || !aligned16(v_blocks) ||
-        (reinterpret_cast<uintptr_t>(kscale) & 3u) != 0 ||
-        (reinterpret_cast<uintptr_t>(vscale) & 3u) != 0)
-        return Q8KV_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
-        return Q8KV_ERR_UNSUPPORTED;
-    if (n_tokens == 0) // nothing to write (the row pointers may be null)
-        return Q8KV_OK;
-    if (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new) ||
-        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) != 0)
-        return Q8KV_ERR_INVALID_ARG;
-    DeviceInfo *dev = nullptr;
-    q8kv_status st;
-    {
-        std::lock_guard<std::mutex> lock(g_mutex);
-        st = device_info(&dev);
-    }
-    if (st != Q8KV_OK)
-        return st;
-    CacheWriteParams p;
-    p.k = k_blocks;
-    p.v = v_blocks;
-    p.ks = kscale;
-    p.vs = vscale;
-    p.k_new = k_new;
-    p.v_new = v_new;
-    p.slots = slot_mapping;
-    p.n_rows = (long long)n_tokens * n_kv_heads;
-    p.token_stride = token_stride;
-    p.n_slots = (long long)num_kv_blocks * kv_block_size;
-    p.Hk = n_kv_heads;
-    p.errors = dev->errors;
-    if (head_dim == 64)
-        return launch_cache_write<64>(p, dev->sms, stream);
-    if (head_dim == 128)
-        return launch_cache_write<128>(p, dev->sms, stream);
-    return launch_cache_write<256>(p, dev->sms, stream);
-}
-
 q8kv_status q8kv_debug_quantize_q(int8_t *qi, float *qsc, const float *q, int n_rows,
                                   int head_dim, cudaStream_t stream)
 {
@@ -774,3 +698,6 @@ int q8kv_version(void)
 }
 
 } // extern "C"
+
+// The KV-cache write entry point (uses the device bookkeeping above).
+#include "q8kv_cache_write_api.cuh"

@@ -16,15 +16,19 @@
 // section prescribes; a slot past the pool is skipped and sets a device error bit.
 //
 // How: the same page describes vLLM's fused cache-write kernel as one warp per (token,
-// head) with 16-byte vector accesses; that shape suits B200 too. Here one warp owns one
-// (token, KV head) pair and quantises its K and its V row together: each lane loads D/32
-// consecutive floats of each row with 8- or 16-byte streaming loads (the rows are read
-// once), the maximum is a 5-step butterfly over the warp, and each lane stores its D/32
-// codes as one 2- or 4-byte word, so a warp writes each int8 row as one contiguous
-// segment. Consecutive warps take consecutive KV heads of a token, so the scales of one
-// slot (adjacent floats) are written by neighbouring warps. The grid is a whole number of
-// resident blocks per SM and strides over the (token, head) pairs. The loads of a pair do
-// not depend on its slot, so they are issued together with the slot load.
+// head) with 16-byte vector accesses. On B200 that layout spends more issue slots on the
+// per-row scalar work (index arithmetic, the correctly rounded division, a 5-step
+// reduction, all replicated over 32 lanes) than on the 128 elements, so here a row gets
+// LPR = 8 lanes (16 for head_dim 256) and a warp takes 32 / LPR (token, KV head) pairs at
+// once, with their K and V rows: each lane loads head_dim / LPR floats of each row as
+// 16-byte streaming loads in which the row's LPR lanes cover 16 * LPR contiguous bytes
+// (the rows are read once), the row maximum is a 3- or 4-step butterfly inside the lane
+// group, and each lane stores 4 codes per 16-byte chunk, so every store instruction
+// writes 4 * LPR contiguous bytes of each row. The pairs are taken in (token, head) order,
+// so the scales of one slot (adjacent floats) come from neighbouring lanes. The grid is
+// one wave of resident blocks striding over the pairs, with the (token, head) position
+// advanced incrementally (no 64-bit division in the loop). The loads of a pair do not
+// depend on its slot, so they are issued together with the slot load.
 #pragma once
 
 #include <cstdint>
@@ -37,11 +41,23 @@ constexpr unsigned kErrSlot = 0x8u;       // a slot past the pool (row skipped)
 constexpr unsigned kErrNonFinite = 0x10u; // a row held an infinity or a NaN
 constexpr int kWriteThreads = 256;
 constexpr int kWriteWarps = kWriteThreads / 32;
-// Resident blocks per SM: 8 (2048 threads, 32 registers each) where the row fits in that,
-// 6 for head_dim 256 (its two 16-byte loads per row need more registers).
-__host__ __device__ constexpr int write_blocks_per_sm(int D)
+
+// Lanes per row: 8 for head_dim 64 and 128, 16 for 256, so that a lane holds at most 16
+// floats of each of its K and V rows.
+__host__ __device__ constexpr int write_lanes_per_row(int D)
 {
-    return D == 256 ? 6 : 8;
+    return D == 256 ? 16 : 8;
+}
+// (token, KV head) pairs per warp and iteration.
+__host__ __device__ constexpr int write_pairs_per_warp(int D)
+{
+    return 32 / write_lanes_per_row(D);
+}
+// Resident blocks per SM: 4 (1024 threads of up to 64 registers; a lane holds up to 32
+// floats of K and V). Each warp has 4 KB of loads in flight, 128 KB per SM.
+__host__ __device__ constexpr int write_blocks_per_sm(int)
+{
+    return 4;
 }
 
 struct CacheWriteParams {
@@ -49,57 +65,54 @@ struct CacheWriteParams {
     float *ks, *vs;
     const float *k_new, *v_new;
     const int64_t *slots;
-    long long n_rows;       // n_tokens * Hk
+    long long n_tokens;
     long long token_stride; // floats from one token's rows to the next token's
     long long n_slots;      // num_blocks * block_size
     int Hk;
     unsigned *errors;
 };
 
-// D/32 consecutive floats of one row per lane.
+// One lane's share of a row: C chunks of 4 floats; chunk c covers elements
+// 4 * (sub + LPR * c) .. + 3, where sub is the lane's index inside the row's lane group.
 template <int D>
 struct RowFrag {
-    static constexpr int E = D / 32;
-    float x[E];
+    static constexpr int LPR = write_lanes_per_row(D);
+    static constexpr int C = D / (4 * LPR);
+    float4 x[C];
 };
 
 template <int D>
-__device__ __forceinline__ RowFrag<D> load_frag(const float *row, int lane)
+__device__ __forceinline__ RowFrag<D> load_frag(const float *row, int sub)
 {
     RowFrag<D> f;
-    if constexpr (D == 64) {
-        const float2 a = __ldcs(reinterpret_cast<const float2 *>(row) + lane);
-        f.x[0] = a.x;
-        f.x[1] = a.y;
-    } else {
 #pragma unroll
-        for (int c = 0; c < D / 128; ++c) {
-            const float4 a = __ldcs(reinterpret_cast<const float4 *>(row + 128 * c) + lane);
-            f.x[4 * c + 0] = a.x;
-            f.x[4 * c + 1] = a.y;
-            f.x[4 * c + 2] = a.z;
-            f.x[4 * c + 3] = a.w;
-        }
-    }
+    for (int c = 0; c < RowFrag<D>::C; ++c)
+        f.x[c] = __ldcs(reinterpret_cast<const float4 *>(row) + sub + RowFrag<D>::LPR * c);
     return f;
 }
 
-// Row maximum of |x| over the warp, and whether every element of the row is finite.
+// Maximum of |x| over the row (the lane group), and whether every element is finite.
 template <int D>
 __device__ __forceinline__ float row_amax(const RowFrag<D> &f, bool &finite)
 {
     float m = 0.f;
     bool fin = true;
 #pragma unroll
-    for (int i = 0; i < RowFrag<D>::E; ++i) {
-        const float a = fabsf(f.x[i]);
-        fin = fin && (a <= 3.402823466e38f); // false for inf and NaN
-        m = fmaxf(m, a);
-    }
+    for (int c = 0; c < RowFrag<D>::C; ++c) {
+        const float a[4] = {fabsf(f.x[c].x), fabsf(f.x[c].y), fabsf(f.x[c].z), fabsf(f.x[c].w)};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+        for (int i = 0; i < 4; ++i) {
+            fin = fin && (a[i] <= 3.402823466e38f); // false for inf and NaN
+            m = fmaxf(m, a[i]);
+        }
+    }
+    unsigned bad = fin ? 0u : 1u;
+#pragma unroll
+    for (int o = RowFrag<D>::LPR / 2; o > 0; o >>= 1) {
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    finite = __all_sync(0xffffffffu, fin);
+        bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+    }
+    finite = bad == 0u;
     return m;
 }
 
@@ -110,10 +123,11 @@ __device__ __forceinline__ uint32_t code_byte(float x, float inv)
     return static_cast<uint32_t>(c) & 0xffu;
 }
 
-// Quantise the lane's fragment of one row and store its codes; returns the row's scale.
+// Quantise one row (every lane of the warp takes part in the reductions) and, if `store`,
+// write the lane's codes; returns the row's scale and sets `bad` for a non-finite row.
 template <int D>
-__device__ __forceinline__ float quantise_store(const RowFrag<D> &f, int8_t *dst, int lane,
-                                                bool &bad)
+__device__ __forceinline__ float quantise_row(const RowFrag<D> &f, int8_t *dst, bool store,
+                                              int sub, bool &bad)
 {
     bool finite;
     float amax = row_amax<D>(f, finite);
@@ -122,20 +136,18 @@ __device__ __forceinline__ float quantise_store(const RowFrag<D> &f, int8_t *dst
     if (finite) {
         if (amax < 1e-6f)
             amax = 1.0f;
-        scale = __fmul_rn(amax, __fdiv_rn(1.0f, 127.0f));
+        scale = __fmul_rn(amax, 0x1.020408p-7f); // fl(1/127)
         inv = __fdiv_rn(127.0f, amax);
     }
-    uint32_t w[RowFrag<D>::E];
+    if (store) {
 #pragma unroll
-    for (int i = 0; i < RowFrag<D>::E; ++i)
-        w[i] = finite ? code_byte(f.x[i], inv) : 0u;
-    if constexpr (D == 64) {
-        reinterpret_cast<uint16_t *>(dst)[lane] = static_cast<uint16_t>(w[0] | (w[1] << 8));
-    } else {
-#pragma unroll
-        for (int c = 0; c < D / 128; ++c)
-            reinterpret_cast<uint32_t *>(dst + 128 * c)[lane] =
-                w[4 * c] | (w[4 * c + 1] << 8) | (w[4 * c + 2] << 16) | (w[4 * c + 3] << 24);
+        for (int c = 0; c < RowFrag<D>::C; ++c) {
+            uint32_t w = 0u;
+            if (finite)
+                w = code_byte(f.x[c].x, inv) | (code_byte(f.x[c].y, inv) << 8) |
+                    (code_byte(f.x[c].z, inv) << 16) | (code_byte(f.x[c].w, inv) << 24);
+            reinterpret_cast<uint32_t *>(dst)[sub + RowFrag<D>::LPR * c] = w;
+        }
     }
     return scale;
 }
@@ -144,39 +156,62 @@ template <int D>
 __global__ void __launch_bounds__(kWriteThreads, write_blocks_per_sm(D))
     cache_write_kernel(const __grid_constant__ CacheWriteParams p)
 {
+    constexpr int LPR = write_lanes_per_row(D);
+    constexpr int PPW = write_pairs_per_warp(D);
     // the new rows may come from the kernel before this one on the stream
     grid_dep_wait();
     grid_dep_launch();
-    const int lane = threadIdx.x & 31;
-    const long long nw = (long long)gridDim.x * kWriteWarps;
+    const int lane = threadIdx.x & 31, sub = lane % LPR;
+    // this lane's (token, head) pair, advanced by `step` pairs per iteration
+    const long long n_pairs = p.n_tokens * p.Hk;
+    const long long step = (long long)gridDim.x * kWriteWarps * PPW;
+    const long long wbase = ((long long)blockIdx.x * kWriteWarps + (threadIdx.x >> 5)) * PPW;
+    const long long first = wbase + lane / LPR;
+    long long tok = first / p.Hk;
+    int h = (int)(first - tok * p.Hk);
+    const long long dtok = step / p.Hk;
+    const int dh = (int)(step - dtok * p.Hk);
     unsigned err = 0;
+    // warp-uniform loop: the row reductions shuffle across the whole warp
 #pragma unroll 1
-    for (long long r = (long long)blockIdx.x * kWriteWarps + (threadIdx.x >> 5); r < p.n_rows;
-         r += nw) {
-        const long long tok = r / p.Hk;
-        const int h = (int)(r - tok * p.Hk);
-        const long long src = tok * p.token_stride + (long long)h * D;
-        const long long slot = __ldg(p.slots + tok);
-        const RowFrag<D> fk = load_frag<D>(p.k_new + src, lane);
-        const RowFrag<D> fv = load_frag<D>(p.v_new + src, lane);
-        if (slot < 0)
-            continue; // padding entry
+    for (long long base = wbase; base < n_pairs; base += step) {
+        long long slot = -1;
+        RowFrag<D> fk, fv;
+        if (tok < p.n_tokens) {
+            const long long src = tok * p.token_stride + (long long)h * D;
+            slot = __ldg(p.slots + tok);
+            fk = load_frag<D>(p.k_new + src, sub);
+            fv = load_frag<D>(p.v_new + src, sub);
+        } else {
+#pragma unroll
+            for (int c = 0; c < RowFrag<D>::C; ++c)
+                fk.x[c] = fv.x[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         if (slot >= p.n_slots) {
             err |= kErrSlot;
-            continue;
+            slot = -1;
         }
-        const long long row = slot * p.Hk + h;
+        const bool store = slot >= 0; // negative: padding entry (or no pair)
+        const long long row = store ? slot * p.Hk + h : 0;
         bool bad_k, bad_v;
-        const float sk = quantise_store<D>(fk, p.k + row * D, lane, bad_k);
-        const float sv = quantise_store<D>(fv, p.v + row * D, lane, bad_v);
-        if (lane == 0)
-            p.ks[row] = sk;
-        else if (lane == 1)
-            p.vs[row] = sv;
-        if (bad_k || bad_v)
-            err |= kErrNonFinite;
+        const float sk = quantise_row<D>(fk, p.k + row * D, store, sub, bad_k);
+        const float sv = quantise_row<D>(fv, p.v + row * D, store, sub, bad_v);
+        if (store) {
+            if (sub == 0)
+                p.ks[row] = sk;
+            else if (sub == 1)
+                p.vs[row] = sv;
+            if (bad_k || bad_v)
+                err |= kErrNonFinite;
+        }
+        tok += dtok;
+        h += dh;
+        if (h >= p.Hk) {
+            h -= p.Hk;
+            ++tok;
+        }
     }
-    if (err && lane == 0)
+    if (err)
         atomicOr(p.errors, err);
 }
 

@@ -28,7 +28,7 @@ from dataclasses import dataclass, field, replace
 import numpy as np
 
 # Stream identifiers of the PCG64 seed sequences.
-_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS, _S_NEWK, _S_NEWV, _S_SLOTS, _S_MAG = range(10)
+_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS, _S_NEWK, _S_NEWV, _S_SLOTS, _S_MAG, _S_MQ = range(11)
 _CHUNK_SLOTS = 4096  # pool slots generated per independent random stream
 
 
@@ -345,3 +345,13 @@ def make_prompt_fill(cfg: Config | int, *, threads: int | None = None) -> CacheR
     k = _mixed_rows(cfg.seed, _S_NEWK, n, Hk, D, threads)
     v = _mixed_rows(cfg.seed, _S_NEWV, n, Hk, D, threads)
     return CacheRows(k.reshape(n, Hk * D), v.reshape(n, Hk * D), slots, Hk, D)
+
+
+# ---------------------------------------------------------------- several queries per sequence
+
+
+def multi_queries(B: int, n_queries: int, n_q_heads: int, head_dim: int, *, seed: int = 0):
+    """fp32 queries [B][n_queries][n_q_heads][head_dim], iid N(0, 1): the new tokens of a
+    multi-token (speculative) decode step, one row per (sequence, new token, head)."""
+    return _rng(seed, _S_MQ).standard_normal((B, n_queries, n_q_heads, head_dim),
+                                             dtype=np.float32)

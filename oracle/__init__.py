@@ -84,6 +84,8 @@ def _load():
                 "q8kvo_decode_pairs": [cp, P, P, l, P],
                 "q8kvo_attn_fp32": [cp, P, P, P, i, i, P],
                 "q8kvo_quantize_kv_row": [P, i, P, P, P],
+                "q8kvo_decode_multi": [cp, P, i, P],
+                "q8kvo_decode_multi_rows": [cp, P, i, P, l, P],
                 "q8kvo_cache_write": [P, P, P, P, P, P, P, l, i, i, i, i, l, P],
             }
             for name, args in sigs.items():
@@ -210,6 +212,27 @@ def decode_pairs(cache: PagedCache, q: np.ndarray, pairs) -> np.ndarray:
     out = np.zeros((pairs.shape[0], cache.head_dim), np.float64)
     _check(_load().q8kvo_decode_pairs(cache.ref(), _ptr(q), _ptr(pairs), pairs.shape[0],
                                       _ptr(out)), "decode_pairs")
+    return out
+
+
+def decode_multi(cache: PagedCache, q: np.ndarray, n_queries: int) -> np.ndarray:
+    """fp64 output [B][n_queries][n_q_heads][head_dim] of a causal multi-query decode:
+    q is [B][n_queries][n_q_heads][head_dim], query i sees seq_lens[b] - (n_queries - 1 - i)
+    tokens."""
+    q = _c(q, np.float32)
+    out = np.zeros((cache.B, n_queries, cache.n_q_heads, cache.head_dim), np.float64)
+    _check(_load().q8kvo_decode_multi(cache.ref(), _ptr(q), int(n_queries), _ptr(out)),
+           "decode_multi")
+    return out
+
+
+def decode_multi_rows(cache: PagedCache, q: np.ndarray, n_queries: int, rows) -> np.ndarray:
+    """fp64 outputs [n][head_dim] of chosen (b, query index, head) rows."""
+    q = _c(q, np.float32)
+    rows = _c(rows, np.int32).reshape(-1, 3)
+    out = np.zeros((rows.shape[0], cache.head_dim), np.float64)
+    _check(_load().q8kvo_decode_multi_rows(cache.ref(), _ptr(q), int(n_queries), _ptr(rows),
+                                           rows.shape[0], _ptr(out)), "decode_multi_rows")
     return out
 
 

@@ -324,11 +324,11 @@ int q8kvo_scores(const q8kvo_cache *c, const float *q, int b, int h, double *s)
  *   else:      w = exp(s - M)
  *   S += w;  acc[d] += w * vs * V[d]
  * and finally out = acc / S. */
-static int decode_online_one(const q8kvo_cache *c, const float *q, int b, int h, double *out,
-                             double *m_trace, long *n_iter, int8_t *qi, float *qsc, double *acc)
+static int decode_row(const q8kvo_cache *c, const float *qh, int b, int h, int L, double *out,
+                      double *m_trace, long *n_iter, int8_t *qi, float *qsc, double *acc)
 {
-    int D = c->head_dim, kvh = kv_head_of(c, h), L = c->seq_lens[b];
-    int rc = quantized_query(c, q, b, h, qi, qsc);
+    int D = c->head_dim, kvh = kv_head_of(c, h);
+    int rc = q8kvo_quantize_q(qh, D, qi, qsc);
     if (rc)
         return rc;
     double M = -INFINITY, S = 0.0;
@@ -364,6 +364,14 @@ static int decode_online_one(const q8kvo_cache *c, const float *q, int b, int h,
     if (n_iter)
         *n_iter = iters;
     return Q8KVO_OK;
+}
+
+/* The single-query decode of (b, h): query row q[b][h], every cached token. */
+static int decode_online_one(const q8kvo_cache *c, const float *q, int b, int h, double *out,
+                             double *m_trace, long *n_iter, int8_t *qi, float *qsc, double *acc)
+{
+    const float *qh = q + ((long)b * c->n_q_heads + h) * c->head_dim;
+    return decode_row(c, qh, b, h, c->seq_lens[b], out, m_trace, n_iter, qi, qsc, acc);
 }
 
 static int scratch_alloc(int D, int8_t **qi, float **qsc, double **acc)
@@ -450,6 +458,80 @@ int q8kvo_decode_pairs(const q8kvo_cache *c, const float *q, const int32_t *pair
     for (long i = 0; i < n && rc == Q8KVO_OK; ++i)
         rc = decode_online_one(c, q, pairs[2 * i], pairs[2 * i + 1], out + i * c->head_dim, NULL,
                                NULL, qi, qsc, acc);
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
+/* ---------------------------------------------------------------- several queries */
+
+/* Tokens visible to query i of n_queries of sequence b: the new queries are the last
+ * n_queries tokens of the sequence (already in the cache), and each attends to itself and
+ * everything before it (causal), so query i sees seq_lens[b] - (n_queries - 1 - i)
+ * tokens; fewer than none means none. */
+static int visible_len(const q8kvo_cache *c, int b, int n_queries, int i)
+{
+    int L = c->seq_lens[b] - (n_queries - 1 - (MUT(19) ? 0 : i)) - (MUT(20) ? 1 : 0);
+    return L > 0 ? L : 0;
+}
+
+int q8kvo_decode_multi(const q8kvo_cache *c, const float *q, int n_queries, double *out)
+{
+    int rc = check_q8(c, q, out);
+    if (rc)
+        return rc;
+    if (n_queries <= 0)
+        return Q8KVO_EINVAL;
+    for (int b = 0; b < c->B; ++b)
+        if ((rc = check_seq(c, b, 0)))
+            return rc;
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    const long D = c->head_dim;
+    for (int b = 0; b < c->B && rc == Q8KVO_OK; ++b)
+        for (int i = 0; i < n_queries && rc == Q8KVO_OK; ++i)
+            for (int h = 0; h < c->n_q_heads && rc == Q8KVO_OK; ++h) {
+                long row = ((long)b * n_queries + i) * c->n_q_heads + h;
+                rc = decode_row(c, q + row * D, b, h, visible_len(c, b, n_queries, i),
+                                out + row * D, NULL, NULL, qi, qsc, acc);
+            }
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
+int q8kvo_decode_multi_rows(const q8kvo_cache *c, const float *q, int n_queries,
+                            const int32_t *rows, long n, double *out)
+{
+    int rc = check_q8(c, q, out);
+    if (rc)
+        return rc;
+    if (n_queries <= 0 || !rows || n < 0)
+        return Q8KVO_EINVAL;
+    for (long r = 0; r < n; ++r) {
+        int b = rows[3 * r], i = rows[3 * r + 1], h = rows[3 * r + 2];
+        if (i < 0 || i >= n_queries)
+            return Q8KVO_EINVAL;
+        if ((rc = check_seq(c, b, h)))
+            return rc;
+    }
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    const long D = c->head_dim;
+    for (long r = 0; r < n && rc == Q8KVO_OK; ++r) {
+        int b = rows[3 * r], i = rows[3 * r + 1], h = rows[3 * r + 2];
+        long qrow = ((long)b * n_queries + i) * c->n_q_heads + h;
+        rc = decode_row(c, q + qrow * D, b, h, visible_len(c, b, n_queries, i), out + r * D,
+                        NULL, NULL, qi, qsc, acc);
+    }
     free(qi);
     free(qsc);
     free(acc);

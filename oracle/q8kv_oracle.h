@@ -21,6 +21,9 @@
  *   - the opening and the kernel signature (KV compressed to q8 with one scale per
  *     (token, KV head), applied as scale * 1/127 at use): the KV-cache write that fills
  *     the pools, with the section 2 part 1 quantiser applied to whole rows.
+ * Several query tokens per sequence (the multi-query "TILE" decode of the llama.cpp
+ * change on baguaai.com's FlashAttention page) are the same single pass per (sequence,
+ * query, head), each query seeing the cache up to its own position (causal).
  * GQA head mapping kv_head = q_head / (n_q_heads / n_kv_heads) follows the llama2.c
  * attention loop (aicoding.csdn.net, "attention core logic").
  * The block-table -> slot mapping follows beaiera.top "deepseek-attention-div64",
@@ -107,6 +110,18 @@ int q8kvo_scores(const q8kvo_cache *c, const float *q, int b, int h, double *s);
  * n_iter (optional) receives the number of token iterations executed. */
 int q8kvo_decode_online(const q8kvo_cache *c, const float *q, int b, int h,
                         double *out, double *m_trace, long *n_iter);
+
+/* Decode with several new query tokens per sequence (speculative or multi-token decode):
+ * q and out are [B][n_queries][n_q_heads][head_dim] (out in fp64); seq_lens[b] counts every
+ * cached token including the n_queries new ones, and query i attends causally to tokens
+ * t < seq_lens[b] - (n_queries - 1 - i); a query that sees no token gets a zero row.
+ * n_queries = 1 is q8kvo_decode_all. */
+int q8kvo_decode_multi(const q8kvo_cache *c, const float *q, int n_queries, double *out);
+
+/* The same for n chosen rows: rows[3*r .. 3*r+2] = (b, query index i, head h);
+ * out[n][head_dim] (fp64). */
+int q8kvo_decode_multi_rows(const q8kvo_cache *c, const float *q, int n_queries,
+                            const int32_t *rows, long n, double *out);
 
 /* Naive three-pass variant (all scores, then max, then exp/sum, then weighted V). */
 int q8kvo_decode_threepass(const q8kvo_cache *c, const float *q, int b, int h, double *out);

@@ -29,6 +29,8 @@ MUTANTS = {
     16: "cache codes truncated instead of rounded half-to-even",
     17: "cache stores max|x| instead of the dequantisation multiplier",
     18: "cache row written under the next KV head",
+    19: "every query of a multi-query step sees only the first query's tokens",
+    20: "multi-query visible length one token short",
 }
 
 
@@ -39,7 +41,7 @@ def test_planted_mistake_is_caught(mutant, tmp_path):
     r = subprocess.run(
         [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
          "tests/test_oracle_qquant.py", "tests/test_oracle_attention.py",
-         "tests/test_oracle_cache_write.py"],
+         "tests/test_oracle_cache_write.py", "tests/test_oracle_multi_query.py"],
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {mutant} ({MUTANTS[mutant]}) passed every pin"
     assert "failed" in r.stdout, r.stdout[-2000:]
