@@ -53,6 +53,11 @@ def parse():
                     help="skip the q8-vs-fp32 information report")
     ap.add_argument("--no-cache-write", action="store_true",
                     help="skip the KV-cache write information report")
+    ap.add_argument("--no-multi-query", action="store_true",
+                    help="skip the multi-query decode information report")
+    ap.add_argument("--accuracy-study", action="store_true",
+                    help="instead of timing: the q8-vs-fp32 output error study over the "
+                         "workloads and K/V distributions (one JSON line)")
     return ap.parse_args()
 
 
@@ -226,6 +231,105 @@ def cpu_baseline(w, min_seconds=10.0):
                       f"{reps} passes, {dt:.1f} s, single-threaded C oracle"}
 
 
+def _err_stats(got, ref):
+    import numpy as np
+
+    d = np.asarray(got, np.float64) - np.asarray(ref, np.float64)
+    r = np.asarray(ref, np.float64)
+    return {"max_abs": float(np.abs(d).max()), "mean_abs": float(np.abs(d).mean()),
+            "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(r)),
+            "row_rel_l2_p99": float(np.percentile(np.linalg.norm(d, axis=1) /
+                                                  np.maximum(np.linalg.norm(r, axis=1), 1e-300),
+                                                  99))}
+
+
+def accuracy_rows(w, out_gpu, n_rows, seed):
+    """Error of the q8 path against attention over the unquantised fp32 q, K, V on sampled
+    (sequence, head) rows: the CUDA output and the oracle's q8 decode, each against the
+    oracle's fp64 attention of the fp32 data (the fp32 rows of the sampled sequences are
+    regenerated from their random streams)."""
+    import numpy as np
+
+    import oracle
+    from decode_attention_int8_b200 import inputs
+
+    c = w.cfg
+    bs, Hk, D = c.block_size, c.n_kv_heads, c.head_dim
+    rng = np.random.default_rng(seed)
+    live = [b for b in range(c.B) if w.seq_lens[b] > 0]
+    pairs = sorted({(int(rng.choice(live)), int(rng.integers(0, c.n_q_heads)))
+                    for _ in range(n_rows)})
+    cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens, c.n_q_heads,
+                              w.scale)
+    q8_oracle = oracle.decode_pairs(cache, w.q, pairs)
+    fp32, gpu = [], []
+    for b in sorted({b for b, _ in pairs}):
+        L = int(w.seq_lens[b])
+        nblk = -(-L // bs)
+        blocks = w.block_table[b, :nblk].astype(np.int64)
+        slots = (blocks[:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+        k32 = inputs.fp32_rows(w, "k", slots).reshape(nblk, bs, Hk, D)
+        v32 = inputs.fp32_rows(w, "v", slots).reshape(nblk, bs, Hk, D)
+        compact = oracle.PagedCache(w.k[blocks], w.v[blocks], w.ks[blocks], w.vs[blocks],
+                                    np.arange(nblk, dtype=np.int32)[None, :],
+                                    np.array([L], np.int32), c.n_q_heads, w.scale)
+        for bb, h in pairs:
+            if bb == b:
+                fp32.append(oracle.attn_fp32(compact, w.q[b:b + 1], k32, v32, 0, h))
+                gpu.append(out_gpu[b, h])
+    fp32, gpu = np.array(fp32), np.array(gpu)
+    return {"rows": len(pairs), "cuda_q8_vs_fp32": _err_stats(gpu, fp32),
+            "oracle_q8_vs_fp32": _err_stats(q8_oracle, fp32),
+            "cuda_vs_oracle_q8_max_abs": float(np.abs(gpu - q8_oracle).max())}
+
+
+def run_accuracy_study(args):
+    """Survey row f2 (the walk-through's announced q8-vs-fp32 comparison): how far the q8
+    path's attention output is from attention over the unquantised fp32 data, per workload
+    and per K/V distribution, for the CUDA kernel and for the oracle's q8 arithmetic."""
+    import numpy as np
+    import torch
+
+    import decode_attention_int8_b200 as q8
+    from decode_attention_int8_b200 import inputs
+
+    _, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    def gpu_out(w):
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        out = torch.empty(w.q.shape, dtype=torch.float32, device=dev)
+        q8.q8kv_decode_attn(out, t(w.q), t(w.k), t(w.v), t(w.ks), t(w.vs), t(w.block_table),
+                            t(w.seq_lens), w.scale)
+        torch.cuda.synchronize(dev)
+        return out.cpu().numpy()
+
+    results = []
+    sample = {0: 64, 1: 256, 2: 32, 3: 96, 4: 96}
+    for i, cfg in enumerate(inputs.CONFIGS):
+        w = inputs.make(cfg)
+        r = accuracy_rows(w, gpu_out(w), sample[i], seed=i)
+        r.update({"workload": cfg.name, "k_dist": cfg.k_dist, "v_dist": cfg.v_dist,
+                  "k_bias_std": cfg.k_bias_std})
+        results.append(r)
+        del w
+    # distributions at one shape: 4 sequences of 4096 tokens, 32/8 heads, block 64
+    for name, kw in [("normal", {}), ("student_t3 K and V", dict(k_dist="student_t3",
+                                                                 v_dist="student_t3")),
+                     ("K bias std 2", dict(k_bias_std=2.0)), ("K bias std 6", dict(k_bias_std=6.0)),
+                     ("student_t3 K + bias 6", dict(k_dist="student_t3", k_bias_std=6.0))]:
+        w = inputs.make_custom(4, 32, 8, 128, [4096] * 4, 64, seed=50, **kw)
+        r = accuracy_rows(w, gpu_out(w), 128, seed=50)
+        r.update({"workload": f"4 x 4096 tokens, 32/8 heads: {name}"})
+        results.append(r)
+    print(json.dumps({"study": "q8 KV + q8 Q attention output vs fp64 attention over the "
+                               "unquantised fp32 q, K, V", "results": results}), flush=True)
+    return 0
+
+
 def run_reference(args):
     """--impl reference: the oracle on the host cores, on this arm's workload and metric."""
     world, rank, _ = dist_env()
@@ -284,6 +388,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.accuracy_study:
+        return run_accuracy_study(args)
     world, rank, local = dist_env()
     import numpy as np
     import torch
@@ -436,6 +542,11 @@ def main():
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+    if not args.no_multi_query:
+        # information, after the timed region: the same workload with n_queries new tokens
+        # per sequence (speculative decode), through q8kv_decode_attn_multi
+        line["multi_query"] = bench_multi_query(w, pools, bt, lens, dev, stream,
+                                                steps=max(10, min(args.steps, 2000)))
     if not args.no_cache_write:
         # information, after the timed region: the write path that fills the cache
         del pools, argsets
@@ -486,6 +597,57 @@ def recorded_traffic(name: str, kernel: str = "decode"):
             if len(parts) == 3 and not ln.startswith("#") and parts[0] == name and parts[1] == h:
                 return int(parts[2])
     return None
+
+
+def bench_multi_query(w, pools, bt, lens, dev, stream, steps, warmup=20, nqs=(2, 4, 8)):
+    """Information: q8kv_decode_attn_multi on the benchmark workload with nq new query
+    tokens per sequence (causal), timed like the single-query call (back-to-back calls
+    between two events, the same rotated KV pools). Algorithmic bytes: the KV bytes of one
+    single-query call plus nq times its q and out bytes."""
+    import numpy as np
+    import torch
+
+    import decode_attention_int8_b200 as q8
+    from decode_attention_int8_b200 import inputs
+
+    c = w.cfg
+    fn = q8.lib().q8kv_decode_attn_multi
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    P_ = lambda x: ctypes.c_void_p(x.data_ptr())
+    peak, _ = measured_peak()
+    res = {}
+    for nq in nqs:
+        if nq * c.group > 128:
+            continue
+        q = torch.from_numpy(inputs.multi_queries(c.B, nq, c.n_q_heads, c.head_dim,
+                                                  seed=c.seed)).to(dev)
+        out = torch.empty_like(q)
+        q8.q8kv_decode_attn_multi(out, q, *pools[0], bt, lens, w.scale, stream=stream)
+        argsets = [(P_(out), P_(q), P_(k), P_(v), P_(ks), P_(vs), P_(bt), P_(lens), c.B, nq,
+                    c.n_q_heads, c.n_kv_heads, c.head_dim, c.block_size, w.max_blocks_per_seq,
+                    w.num_blocks, ctypes.c_float(w.scale), sp) for (k, v, ks, vs) in pools]
+        for i in range(warmup):
+            fn(*argsets[i % len(argsets)])
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            st = fn(*argsets[i % len(argsets)])
+            if st != 0:
+                raise q8.Q8KVError(st, "q8kv_decode_attn_multi")
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / steps
+        algo = w.algorithmic_bytes() + (nq - 1) * 2 * int(w.q.nbytes)
+        gbs = algo / (ms * 1e-3) / 1e9
+        res[f"nq{nq}"] = {"us_per_call": round(ms * 1e3, 3), "GB/s": round(gbs, 2),
+                          "frac_of_measured_hbm": round(gbs / peak, 4),
+                          "query_rows_per_kv_head": nq * c.group,
+                          "algorithmic_bytes": algo}
+    res["workload"] = (f"{c.name} with nq new query tokens per sequence (causal), "
+                       f"q/out [{c.B}][nq][{c.n_q_heads}][{c.head_dim}]")
+    return res
 
 
 def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):

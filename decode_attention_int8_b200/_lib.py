@@ -26,6 +26,7 @@ DEVERR_NONFINITE = 0x10
 
 EXPORTS = (
     "q8kv_decode_attn",
+    "q8kv_decode_attn_multi",
     "q8kv_workspace_bytes",
     "q8kv_workspace_init",
     "q8kv_decode_attn_ws",
@@ -65,6 +66,7 @@ def lib():
             P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
             sig = {
                 "q8kv_decode_attn": ([P] * 8 + [I] * 7 + [F, P], I),
+                "q8kv_decode_attn_multi": ([P] * 8 + [I] * 8 + [F, P], I),
                 "q8kv_workspace_bytes": ([I, I, I, I], Z),
                 "q8kv_workspace_init": ([P, Z, P], I),
                 "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
@@ -105,9 +107,11 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}")
 
 
-def _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens):
-    _need(out, "out", torch.float32, 3)
-    _need(q, "q", torch.float32, 3)
+def _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+              contiguous=True):
+    if contiguous:  # (a multi-query caller passes views of its checked 4-D tensors)
+        _need(out, "out", torch.float32, 3)
+        _need(q, "q", torch.float32, 3)
     _need(k_blocks, "k_blocks", torch.int8, 4)
     _need(v_blocks, "v_blocks", torch.int8, 4)
     _need(kscale, "kscale", torch.float32, 3)
@@ -137,6 +141,24 @@ def q8kv_decode_attn(out, q, k_blocks, v_blocks, kscale, vscale, block_table, se
     _check(lib().q8kv_decode_attn(_ptr(out), _ptr(q), _ptr(k_blocks), _ptr(v_blocks),
                                   _ptr(kscale), _ptr(vscale), _ptr(block_table), _ptr(seq_lens),
                                   *geo, float(scale), _stream(stream)), "q8kv_decode_attn")
+    return out
+
+
+def q8kv_decode_attn_multi(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+                           scale, stream=None):
+    """Causal decode of n_queries new tokens per sequence: q, out [B][n_queries][Hq][D];
+    query i of sequence b sees seq_lens[b] - (n_queries - 1 - i) tokens."""
+    _need(out, "out", torch.float32, 4)
+    _need(q, "q", torch.float32, 4)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out and q must have the same shape [B][n_queries][Hq][D]")
+    B, nq, Hq, D = q.shape
+    geo = _geometry(out[:, 0], q[:, 0], k_blocks, v_blocks, kscale, vscale, block_table,
+                    seq_lens, contiguous=False)
+    _check(lib().q8kv_decode_attn_multi(_ptr(out), _ptr(q), _ptr(k_blocks), _ptr(v_blocks),
+                                        _ptr(kscale), _ptr(vscale), _ptr(block_table),
+                                        _ptr(seq_lens), geo[0], nq, *geo[1:], float(scale),
+                                        _stream(stream)), "q8kv_decode_attn_multi")
     return out
 
 

@@ -92,6 +92,7 @@ q8kv_status encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn)
 
 struct Shape {
     int B, Hq, Hk, D, bs, mbps, P;
+    int nq = 1; // query tokens per sequence
 };
 
 // How the work is tiled for one shape on one device.
@@ -163,9 +164,12 @@ void plan_workspace(int grid, Plan &pl)
 
 q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
 {
-    if (s.B <= 0 || s.bs <= 0 || s.mbps <= 0 || s.P <= 0)
+    if (s.B <= 0 || s.bs <= 0 || s.mbps <= 0 || s.P <= 0 || s.nq <= 0)
         return Q8KV_ERR_INVALID_ARG;
-    q8kv_status st = plan_heads(s.Hq, s.Hk, s.D, pl);
+    // the nq query tokens of a sequence share its KV tiles: the tiling sees nq * Hq rows
+    if ((long long)s.nq * s.Hq > (1LL << 20))
+        return Q8KV_ERR_UNSUPPORTED;
+    q8kv_status st = plan_heads(s.nq * s.Hq, s.Hk, s.D, pl);
     if (st != Q8KV_OK)
         return st;
     if (!is_pow2(s.bs) || s.bs < 16 || s.bs > 256)
@@ -329,7 +333,7 @@ q8kv_status check_call(const Call &c)
     if (!c.out || !c.q || !c.k || !c.v || !c.ks || !c.vs || !c.bt || !c.lens)
         return Q8KV_ERR_INVALID_ARG;
     if (c.s.B <= 0 || c.s.Hq <= 0 || c.s.Hk <= 0 || c.s.D <= 0 || c.s.bs <= 0 || c.s.mbps <= 0 ||
-        c.s.P <= 0 || c.s.Hq % c.s.Hk != 0 || c.s.D % 32 != 0)
+        c.s.P <= 0 || c.s.Hq % c.s.Hk != 0 || c.s.D % 32 != 0 || c.s.nq <= 0)
         return Q8KV_ERR_INVALID_ARG;
     if (!std::isfinite(c.scale))
         return Q8KV_ERR_INVALID_ARG;
@@ -379,6 +383,10 @@ q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl
     cp.n_desc = 2 * pl.grid;
     cp.Hq = p.Hq;
     cp.heads_seg = p.heads_seg;
+    cp.G = p.G;
+    cp.Gq = p.Gq;
+    cp.nq = p.nq;
+    cp.HPC = p.HPC;
     cudaLaunchConfig_t cc = cfg;
     cc.gridDim = dim3((unsigned)dev.sms);
     cc.blockDim = dim3(kCombineThreads);
@@ -443,6 +451,8 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.Hq = c.s.Hq;
     p.Hk = c.s.Hk;
     p.G = pl.G;
+    p.nq = c.s.nq;
+    p.Gq = c.s.Hq / c.s.Hk;
     p.bs = c.s.bs;
     p.mbps = c.s.mbps;
     p.num_blocks = c.s.P;
@@ -532,6 +542,24 @@ q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
            Shape{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
                  num_kv_blocks},
            scale, nullptr, 0};
+    return run(c, nullptr, 0, true, stream);
+}
+
+q8kv_status q8kv_decode_attn_multi(float *out, const float *q, const int8_t *k_blocks,
+                                   const int8_t *v_blocks, const float *kscale,
+                                   const float *vscale, const int32_t *block_table,
+                                   const int32_t *seq_lens, int B, int n_queries, int n_q_heads,
+                                   int n_kv_heads, int head_dim, int kv_block_size,
+                                   int max_blocks_per_seq, int num_kv_blocks, float scale,
+                                   cudaStream_t stream)
+{
+    if (n_queries <= 0)
+        return Q8KV_ERR_INVALID_ARG;
+    Shape sh{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
+             num_kv_blocks};
+    sh.nq = n_queries;
+    Call c{out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens, sh, scale, nullptr,
+           0};
     return run(c, nullptr, 0, true, stream);
 }
 
@@ -694,7 +722,7 @@ int q8kv_last_cuda_error(void)
 
 int q8kv_version(void)
 {
-    return 101;
+    return 102;
 }
 
 } // extern "C"

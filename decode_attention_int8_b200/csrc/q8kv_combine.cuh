@@ -41,6 +41,8 @@ struct CombineParams {
     const int4 *desc;      // [n_desc] {b, hc, n (0: none), first slot}
     int n_desc;
     int Hq, heads_seg;
+    int G, Gq, nq, HPC;    // query rows per KV head (nq tokens x Gq heads), tokens, KV heads
+                           // per segment
 };
 
 constexpr int kCombineBatchIn = 8; // inputs a thread loads at once
@@ -189,8 +191,13 @@ __global__ void __launch_bounds__(kCombineThreads)
                 st += part_s[r0 + k];
             }
             const float f = st > 0.f ? exp2f(ua - um) / st : 0.f;
-            float *dst = p.out + ((long long)b * p.Hq + (long long)hc * H + hl) * 128 +
-                         q * kCombineQuarter + 4 * fl;
+            // segment row hl is query row hl % G of KV head hc * HPC + hl / G; that row is
+            // query token hg / Gq, head kvh * Gq + hg % Gq of the [B][nq][Hq] output
+            const int kvh = hc * p.HPC + hl / p.G, hg = hl % p.G;
+            const int ti = hg / p.Gq;
+            const long long orow =
+                ((long long)b * p.nq + ti) * p.Hq + (long long)kvh * p.Gq + (hg - ti * p.Gq);
+            float *dst = p.out + orow * 128 + q * kCombineQuarter + 4 * fl;
             *reinterpret_cast<float4 *>(dst) = make_float4(t.x * f, t.y * f, t.z * f, t.w * f);
         }
         __syncthreads(); // part_* are reused by the next batch

@@ -157,7 +157,8 @@ struct DecodeParams {
     unsigned *errors;    // device error word
     int32_t *dbg_dots;   // [B][Hq][dbg_max_len][kNB] (debug instantiation only)
     int dbg_max_len;
-    int B, Hq, Hk, G;
+    int B, Hq, Hk, G;    // G: query rows per KV head = nq * Gq (the tiling's group)
+    int nq, Gq;          // query tokens per sequence; query heads per KV head
     int bs, mbps, num_blocks;
     int HPC, nhc, slices, pairs, subtiles, TT, box_tok, log2_box, n_boxes, n_stages;
     int scale_bulk;      // 1: scales by contiguous bulk copy (HPC == Hk); 0: 2-D tensor map
@@ -180,6 +181,16 @@ __device__ __forceinline__ float ldcg_f(const float *p)
 __device__ __forceinline__ float4 ldcg_f4(const float *p)
 {
     return __ldcg(reinterpret_cast<const float4 *>(p));
+}
+
+// Row of q / out that query row hg of KV head kvh of sequence b maps to. The nq query
+// tokens of a sequence share its KV tiles, so a KV head's rows are its Gq query heads for
+// each of the nq tokens: row hg is token hg / Gq, head kvh * Gq + hg % Gq, and q, out are
+// [B][nq][Hq][128]. With one token per sequence this is b * Hq + kvh * Gq + hg.
+__device__ __forceinline__ long long q_row(const DecodeParams &p, int b, int kvh, int hg)
+{
+    const int i = hg / p.Gq, gq = hg - i * p.Gq;
+    return ((long long)b * p.nq + i) * p.Hq + (long long)kvh * p.Gq + gq;
 }
 
 // CTA owning flat tile x: the largest i with cstart[i] <= x, where cstart[i] = i * N / g
@@ -481,8 +492,7 @@ __device__ __forceinline__ QueryFrag<NT> load_query(const DecodeParams &p, int b
         }
         const int hg = kPack ? (g & 3) : slice * 16 + r * 8 + g;
         const bool valid = hg < p.G;
-        const float *qrow =
-            p.q + ((long long)b * p.Hq + (long long)(hc * p.HPC + kl) * p.G + hg) * kD;
+        const float *qrow = p.q + (valid ? q_row(p, b, hc * p.HPC + kl, hg) : 0) * kD;
         float v[kNB][8];
 #pragma unroll
         for (int j = 0; j < kNB; ++j) {
@@ -628,8 +638,9 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 template <int NT, bool kPack, bool kDump>
 __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<NT> &st,
                                               const ThreadOffsets &o, uint32_t sb, int tl0,
-                                              uint32_t vmask, float scale_log2, int b, int hc,
-                                              int kl, int slice, int tok0, int g, int c)
+                                              uint32_t vmask, bool causal, const int (&lim)[NT],
+                                              float scale_log2, int b, int hc, int kl,
+                                              int slice, int tok0, int g, int c)
 {
     // ---- V rows first: their int8 -> f16 conversion overlaps the softmax chain below
     uint4 R[kSub][4];
@@ -703,21 +714,29 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
                 vsv[u][nt][e] = lds_f32(sb + o.s[u][nt][e] + kScaleGap);
             }
     // masked tokens (rare: a segment's last tile, bad block-table entries) get score -inf
-    // and V scale 0, whatever stale data their slots hold
-    if (vmask != 0xffffffffu) {
+    // and V scale 0, whatever stale data their slots hold; with several queries per
+    // sequence, a token after a row's own position gets score -inf in that row only
+    if (vmask != 0xffffffffu || causal) {
 #pragma unroll
         for (int u = 0; u < kSub; ++u)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    if (!((vmask >> (u * 16 + nt * 8 + 2 * c + e)) & 1u)) {
+                for (int e = 0; e < 2; ++e) {
+                    const int j = u * 16 + nt * 8 + 2 * c + e;
+                    if (!((vmask >> j) & 1u)) {
 #pragma unroll
                         for (int r = 0; r < NT; ++r)
                             s[r][u][nt][e] = -INFINITY;
                         kss[u][nt][e] = 1.f;
                         vsv[u][nt][e] = 0.f;
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < NT; ++r)
+                            if (j >= lim[r])
+                                s[r][u][nt][e] = -INFINITY;
                     }
+                }
     }
     // ---- online softmax (base 2), blockwise over the stage's tokens. M: running max of the
     // scores (denominator). A: running max of log2 of the numerator terms w * vs (relative to
@@ -919,8 +938,9 @@ template <int NT, bool kDump>
 __device__ __forceinline__ void process_stage_packed(const DecodeParams &p, WarpState<NT> &st,
                                                      PackedAcc &pa, const PackedOffsets &o,
                                                      uint32_t sb, int tl0, uint32_t vmask,
-                                                     float scale_log2, int b, int hc, int kl,
-                                                     int tok0, int g, int c, float k0, float k1)
+                                                     bool causal, int lim, float scale_log2,
+                                                     int b, int hc, int kl, int tok0, int g,
+                                                     int c, float k0, float k1)
 {
     const bool lower = g < 4;
     const int uk = lower ? 0 : 1;
@@ -971,16 +991,20 @@ __device__ __forceinline__ void process_stage_packed(const DecodeParams &p, Warp
             kss[nt][e] = lds_f32(sb + o.s[nt][e]) * scale_log2;
             vsv[nt][e] = lds_f32(sb + o.s[nt][e] + kScaleGap);
         }
-    if (vmask != 0xffffffffu) {
+    if (vmask != 0xffffffffu || causal) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-                if (!((vmask >> (uk * 16 + nt * 8 + 2 * c + e)) & 1u)) {
+            for (int e = 0; e < 2; ++e) {
+                const int j = uk * 16 + nt * 8 + 2 * c + e;
+                if (!((vmask >> j) & 1u)) {
                     s[nt][e] = -INFINITY;
                     kss[nt][e] = 1.f;
                     vsv[nt][e] = 0.f;
+                } else if (j >= lim) {
+                    s[nt][e] = -INFINITY; // after this row's own position
                 }
+            }
     }
     // ---- online softmax (base 2) over the stage's 32 tokens (M, S, A as in process_stage)
     float m = -INFINITY;
@@ -1203,9 +1227,8 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
                     const float ac = __shfl_sync(kFullMask, st.A[pv], 4 * col);
                     const int hg = slice * 16 + pv * 8 + col;
                     if (col_lane && hg < p.G) {
-                        const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
                         const float f = sc > 0.f ? exp2f(ac - mc) / sc : 0.f;
-                        float *dst = p.out + ((long long)b * p.Hq + h) * kD;
+                        float *dst = p.out + q_row(p, b, hc * p.HPC + kl, hg) * kD;
                         if constexpr (kPack)
                             store_packed(dst + g, st, q, f);
                         else
@@ -1310,6 +1333,14 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         for (int j = 0; j < kNB; ++j)
             st.qs[r][j] = 0.f;
 
+    // With nq query tokens per sequence, query row hg (token hg / Gq) may not see the last
+    // fut = nq - 1 - hg / Gq tokens of the sequence (they come after its own position).
+    int fut[NT];
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        const int hg = kPack ? (g & 3) : slice * 16 + r * 8 + g;
+        fut[r] = hg < p.G ? p.nq - 1 - hg / p.Gq : 0;
+    }
     bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
     int stage = 0;
     uint32_t phase = 0;
@@ -1373,12 +1404,22 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                     vmask = __ballot_sync(kFullMask,
                                           tk < nvalid && ((loaded >> (tk >> p.log2_box)) & 1));
                 }
+                // rows may see window tokens [0, lim): only in the last nq - 1 tokens of a
+                // sequence does that differ between rows (never with one query per sequence)
+                const int win0 = tok0 + ts * kSub * 16;
+                const bool causal = p.nq > 1 && cu.L - (p.nq - 1) - win0 < 32;
+                int lim[NT];
+#pragma unroll
+                for (int r = 0; r < NT; ++r)
+                    lim[r] = cu.L - fut[r] - win0;
                 if constexpr (kPack)
-                    process_stage_packed<NT, kDump>(p, st, pa, po, sb, tl0, vmask, scale_log2,
-                                                    cu.b, cu.hc, kl, tok0, g, c, k0, k1);
+                    process_stage_packed<NT, kDump>(p, st, pa, po, sb, tl0, vmask, causal, lim[0],
+                                                    scale_log2, cu.b, cu.hc, kl, tok0, g, c, k0,
+                                                    k1);
                 else
-                    process_stage<NT, kPack, kDump>(p, st, o, sb, tl0, vmask, scale_log2, cu.b,
-                                                    cu.hc, kl, slice, tok0, g, c);
+                    process_stage<NT, kPack, kDump>(p, st, o, sb, tl0, vmask, causal, lim,
+                                                    scale_log2, cu.b, cu.hc, kl, slice, tok0, g,
+                                                    c);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[stage]);
@@ -1457,9 +1498,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (gcta == 0) { // no sequence has tokens: every row is zero
 #pragma unroll 1
         for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-            float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
+            float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.nq * p.Hq * kD);
 #pragma unroll 1
-            for (int i = tid; i < p.Hq * kD / 4; i += kThreads)
+            for (int i = tid; i < p.nq * p.Hq * kD / 4; i += kThreads)
                 row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
@@ -1490,9 +1531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = blockIdx.x; b < p.B; b += gcta) {
         if (prefix[b + 1] != prefix[b])
             continue;
-        float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.Hq * kD);
+        float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.nq * p.Hq * kD);
 #pragma unroll 1
-        for (int i = ctid; i < p.Hq * kD / 4; i += kConsumerThreads)
+        for (int i = ctid; i < p.nq * p.Hq * kD / 4; i += kConsumerThreads)
             row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     consumer_bar();

@@ -355,3 +355,28 @@ def multi_queries(B: int, n_queries: int, n_q_heads: int, head_dim: int, *, seed
     multi-token (speculative) decode step, one row per (sequence, new token, head)."""
     return _rng(seed, _S_MQ).standard_normal((B, n_queries, n_q_heads, head_dim),
                                              dtype=np.float32)
+
+
+def fp32_rows(w: Workload, which: str, slots) -> np.ndarray:
+    """The unquantised fp32 K ("k") or V ("v") rows [len(slots)][n_kv_heads][head_dim] that
+    the workload's pool slots were quantised from, regenerated from the random streams of
+    only the chunks that hold them (a sample of a large workload needs no full fp32 pool)."""
+    c = w.cfg
+    bs, Hk, D = c.block_size, c.n_kv_heads, c.head_dim
+    n_slots = w.num_blocks * bs
+    slots = np.asarray(slots, np.int64).reshape(-1)
+    stream, dist = (_S_K, c.k_dist) if which == "k" else (_S_V, c.v_dist)
+    bias = None
+    if which == "k" and c.k_bias_std:
+        bias = (_rng(c.seed, _S_BIAS).standard_normal((Hk, D), dtype=np.float32)
+                * np.float32(c.k_bias_std))
+    out = np.empty((slots.shape[0], Hk, D), np.float32)
+    chunk_of = slots // _CHUNK_SLOTS
+    for ch in np.unique(chunk_of):
+        lo, hi = int(ch) * _CHUNK_SLOTS, min(n_slots, (int(ch) + 1) * _CHUNK_SLOTS)
+        x = _draw(_rng(c.seed, stream, int(ch)), dist, (hi - lo, Hk, D))
+        if bias is not None:
+            x += bias[None, :, :]
+        sel = chunk_of == ch
+        out[sel] = x[slots[sel] - lo]
+    return out

@@ -51,10 +51,14 @@
  * entry outside [0, num_kv_blocks) makes the kernel skip that block's tokens; each of
  * these sets a bit in a device-side error word that q8kv_device_errors() reads.
  *
- * Supported shapes of the decode kernel: head_dim 128; kv_block_size a multiple of 16 in
- * [16, 256]; n_q_heads a multiple of n_kv_heads with group n_q_heads / n_kv_heads <= 128;
- * n_kv_heads <= 8, or a multiple of 4; B <= 16384; num_kv_blocks * kv_block_size < 2^31.
- * Other shapes return Q8KV_ERR_UNSUPPORTED.
+ * Supported shapes of the decode kernel: head_dim 128; kv_block_size a power of two in
+ * [16, 256]; n_q_heads a multiple of n_kv_heads; query rows per KV head R (the group
+ * n_q_heads / n_kv_heads, times n_queries for q8kv_decode_attn_multi) at most 128, with
+ * n_kv_heads a power of two <= 8 or a multiple of 4 when R <= 32, n_kv_heads <= 2 when
+ * R <= 64, and n_kv_heads = 1 above (a tile holds 8 / ceil_pow2(R / 16) KV heads, and a
+ * tile with fewer KV heads than the cache needs at least 4 of them for its scale copies);
+ * B <= 16384; num_kv_blocks * kv_block_size < 2^31. Other shapes return
+ * Q8KV_ERR_UNSUPPORTED.
  */
 #ifndef Q8KV_H
 #define Q8KV_H
@@ -108,6 +112,31 @@ q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
                              int n_q_heads, int n_kv_heads, int head_dim, int kv_block_size,
                              int max_blocks_per_seq, int num_kv_blocks, float scale,
                              cudaStream_t stream);
+
+/*
+ * Decode attention with several new query tokens per sequence (speculative or multi-token
+ * decode), library-managed workspace. The llama.cpp change on baguaai.com's FlashAttention
+ * page moves quantised-KV decode from a per-query (VEC) kernel to a tiled (TILE) one; here
+ * the n_queries tokens of a sequence share every K/V tile it streams, as extra rows of the
+ * same tensor-core tiles, so the cache is read once for all of them.
+ *
+ *   q, out     fp32 [B][n_queries][n_q_heads][head_dim]
+ *   seq_lens   tokens in the cache per sequence, the n_queries new ones included (they are
+ *              its last n_queries tokens, written beforehand, e.g. by q8kv_cache_write)
+ * Query i of sequence b attends causally to tokens t < seq_lens[b] - (n_queries - 1 - i),
+ * with the single-query arithmetic of q8kv_decode_attn per (b, i, head); a query that sees
+ * no token (seq_lens[b] < n_queries - i) gets a zero row. n_queries = 1 is
+ * q8kv_decode_attn. Supported shapes: as above with R = n_queries * n_q_heads /
+ * n_kv_heads rows per KV head. Other arguments, errors and asynchrony as
+ * q8kv_decode_attn.
+ */
+q8kv_status q8kv_decode_attn_multi(float *out, const float *q, const int8_t *k_blocks,
+                                   const int8_t *v_blocks, const float *kscale,
+                                   const float *vscale, const int32_t *block_table,
+                                   const int32_t *seq_lens, int B, int n_queries, int n_q_heads,
+                                   int n_kv_heads, int head_dim, int kv_block_size,
+                                   int max_blocks_per_seq, int num_kv_blocks, float scale,
+                                   cudaStream_t stream);
 
 /* Bytes of workspace q8kv_decode_attn_ws needs for these sizes on the current device
  * (0 if the sizes are invalid or unsupported). */

@@ -46,7 +46,7 @@ def test_status_strings_and_version():
     assert L.q8kv_status_string(0) == b"ok"
     assert L.q8kv_status_string(2) == b"unsupported shape"
     assert L.q8kv_status_string(99) == b"unknown status"
-    assert L.q8kv_version() == 101
+    assert L.q8kv_version() == 102
 
 
 def _call(**over):

@@ -1,0 +1,103 @@
+"""Multi-query decode (q8kv_decode_attn_multi) against the fp64 oracle: n_queries new
+tokens per sequence share the K/V tiles, each query attending causally up to its own
+position. Tolerance as for the single-query decode: max-abs <= 1e-4, rel-L2 <= 1e-5.
+
+Covers every tiling the query rows can take (n_queries x group = 2 to 128 rows per KV
+head: the packed path, one and two 8-row tiles, several 16-row slices), ragged lengths
+around the causal window (shorter than n_queries, equal, tile and block boundaries), one
+query (bit-equal to q8kv_decode_attn), the full-size 16 x 4096-token GQA workload with
+4 queries per sequence on sampled rows, and the shape limit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_int8_b200 as q8
+import oracle
+from decode_attention_int8_b200 import inputs
+from gpu_util import assert_close, oracle_cache, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def run_multi(w, q):
+    d = to_device(w)
+    qd = torch.from_numpy(np.ascontiguousarray(q)).cuda()
+    out = torch.full(qd.shape, float("nan"), dtype=torch.float32, device="cuda")
+    q8.q8kv_decode_attn_multi(out, qd, d["k"], d["v"], d["ks"], d["vs"], d["bt"], d["lens"],
+                              w.scale)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("nq,Hq,Hk", [
+    (2, 4, 2),    # 4 rows per KV head: packed path
+    (3, 8, 8),    # 3 rows (one padding row): packed path
+    (2, 32, 8),   # 8 rows: one 8-row tile
+    (4, 32, 8),   # 16 rows: two 8-row tiles
+    (3, 32, 8),   # 12 rows
+    (8, 32, 8),   # 32 rows: two 16-row slices, 4 KV heads per tile
+    (8, 16, 2),   # 64 rows: four 16-row slices
+    (16, 8, 1),   # 128 rows: the largest tiling (one KV head per tile)
+    (5, 20, 4),   # 25 rows, 2 slices
+])
+@pytest.mark.parametrize("bs", [16, 64])
+def test_tilings_and_causal_edges(nq, Hq, Hk, bs):
+    lens = [1, nq - 1 if nq > 1 else 1, nq, nq + 1, 31, 32, 33, bs + nq - 1, 3 * bs + 5, 700]
+    w = inputs.make_custom(len(lens), Hq, Hk, 128, lens, bs, seed=nq * 100 + Hq + bs)
+    q = inputs.multi_queries(len(lens), nq, Hq, 128, seed=nq + bs)
+    got = run_multi(w, q)
+    ref = oracle.decode_multi(oracle_cache(w), q, nq)
+    for b, L in enumerate(lens):
+        for i in range(nq):
+            if L - (nq - 1 - i) <= 0:
+                assert np.all(got[b, i] == 0.0), f"b={b} i={i}: no visible token, not zero"
+    assert_close(got, ref, f"nq={nq} Hq={Hq} Hk={Hk} bs={bs}")
+
+
+def test_one_query_equals_the_single_query_call():
+    w = inputs.make_custom(3, 32, 8, 128, [1000, 17, 4096], 64, seed=5)
+    got = run_multi(w, w.q[:, None])
+    d = to_device(w)
+    out = torch.empty(d["q"].shape, dtype=torch.float32, device="cuda")
+    q8.q8kv_decode_attn(out, d["q"], d["k"], d["v"], d["ks"], d["vs"], d["bt"], d["lens"],
+                        w.scale)
+    torch.cuda.synchronize()
+    assert np.array_equal(got[:, 0], out.cpu().numpy())
+
+
+def test_long_split_sequence_with_many_queries():
+    # one long sequence split over every SM: the causal window sits in the last CTA's share
+    nq, Hq, Hk = 8, 16, 4  # 32 rows per KV head
+    w = inputs.make_custom(1, Hq, Hk, 128, [60001], 128, seed=11, k_bias_std=2.0)
+    q = inputs.multi_queries(1, nq, Hq, 128, seed=11)
+    assert_close(run_multi(w, q), oracle.decode_multi(oracle_cache(w), q, nq), "long, nq=8")
+
+
+def test_gqa_batch_workload_with_four_queries():
+    # the benchmark's 16 x 4096-token workload with 3 draft tokens + 1 (nq = 4), as timed
+    # by bench.py; 160 sampled (sequence, query, head) rows against the oracle
+    cfg = inputs.CONFIGS[1]
+    nq = 4
+    w = inputs.make(cfg)
+    q = inputs.multi_queries(cfg.B, nq, cfg.n_q_heads, cfg.head_dim, seed=cfg.seed)
+    got = run_multi(w, q)
+    rng = np.random.default_rng(0)
+    rows = np.stack([rng.integers(0, cfg.B, 160), rng.integers(0, nq, 160),
+                     rng.integers(0, cfg.n_q_heads, 160)], axis=1)
+    ref = oracle.decode_multi_rows(oracle_cache(w), q, nq, rows)
+    assert_close(got[rows[:, 0], rows[:, 1], rows[:, 2]], ref, "gqa_batch nq=4 sampled rows")
+
+
+@pytest.mark.parametrize("nq,Hq,Hk", [
+    (17, 64, 8),  # 136 rows per KV head: above the 128-row tiling
+    (16, 32, 8),  # 64 rows per KV head with 8 KV heads: a tile would hold 2 of the 8 KV
+                  # heads, whose scale slices (8 bytes) are below the 16-byte TMA minimum,
+                  # the same limit as a single query with group 64 over 8 KV heads
+])
+def test_unsupported_row_counts(nq, Hq, Hk):
+    w = inputs.make_custom(1, Hq, Hk, 128, [40], 16, seed=1)
+    q = inputs.multi_queries(1, nq, Hq, 128)
+    with pytest.raises(q8.Q8KVError) as e:
+        run_multi(w, q)
+    assert e.value.status == 2
