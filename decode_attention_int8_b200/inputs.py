@@ -28,7 +28,8 @@ from dataclasses import dataclass, field, replace
 import numpy as np
 
 # Stream identifiers of the PCG64 seed sequences.
-_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS, _S_NEWK, _S_NEWV, _S_SLOTS, _S_MAG, _S_MQ = range(11)
+(_S_Q, _S_K, _S_V, _S_TABLE, _S_BIAS, _S_LENS, _S_NEWK, _S_NEWV, _S_SLOTS, _S_MAG, _S_MQ,
+ _S_META) = range(12)
 _CHUNK_SLOTS = 4096  # pool slots generated per independent random stream
 
 
@@ -380,3 +381,25 @@ def fp32_rows(w: Workload, which: str, slots) -> np.ndarray:
         sel = chunk_of == ch
         out[sel] = x[slots[sel] - lo]
     return out
+
+
+# ---------------------------------------------------------------- QUEST metadata tables
+
+
+def quest_meta_table(seq_lens, block_size: int, *, seed: int = 0, extra_blocks: int = 0):
+    """Metadata block table for per-block K metadata: request r needs
+    ceil(ceil(L_r / block_size) / block_size) metadata blocks of block_size rows each; they
+    are drawn from a random permutation of the pool (as the block table is). Returns
+    (meta_table int32 [B][max_meta_per_seq] with -1 in unused entries, num_meta_blocks)."""
+    L = np.asarray(seq_lens, np.int64)
+    nkv = (L + block_size - 1) // block_size
+    nmeta = (nkv + block_size - 1) // block_size
+    mm = max(1, int(nmeta.max(initial=0)))
+    total = max(1, int(nmeta.sum()) + int(extra_blocks))
+    order = _rng(seed, _S_META).permutation(total)
+    table = np.full((len(L), mm), -1, np.int32)
+    off = 0
+    for r, n in enumerate(nmeta):
+        table[r, :n] = order[off:off + n]
+        off += int(n)
+    return table, total

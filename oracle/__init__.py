@@ -86,6 +86,7 @@ def _load():
                 "q8kvo_quantize_kv_row": [P, i, P, P, P],
                 "q8kvo_decode_multi": [cp, P, i, P],
                 "q8kvo_decode_multi_rows": [cp, P, i, P, l, P],
+                "q8kvo_quest_metadata": [cp, P, i, i, P, P],
                 "q8kvo_cache_write": [P, P, P, P, P, P, P, l, i, i, i, i, l, P],
             }
             for name, args in sigs.items():
@@ -234,6 +235,20 @@ def decode_multi_rows(cache: PagedCache, q: np.ndarray, n_queries: int, rows) ->
     _check(_load().q8kvo_decode_multi_rows(cache.ref(), _ptr(q), int(n_queries), _ptr(rows),
                                            rows.shape[0], _ptr(out)), "decode_multi_rows")
     return out
+
+
+def quest_metadata(cache: PagedCache, meta_table: np.ndarray, num_meta_blocks: int,
+                   fill: float = np.nan):
+    """(maxb, minb) fp32 [num_meta_blocks][block_size][n_kv_heads][head_dim] of the q8
+    cache's K (rows no request owns keep ``fill``)."""
+    meta_table = _c(meta_table, np.int32)
+    bs, Hk, D = cache.struct.block_size, cache.struct.n_kv_heads, cache.head_dim
+    maxb = np.full((num_meta_blocks, bs, Hk, D), fill, np.float32)
+    minb = np.full((num_meta_blocks, bs, Hk, D), fill, np.float32)
+    _check(_load().q8kvo_quest_metadata(cache.ref(), _ptr(meta_table), int(meta_table.shape[1]),
+                                        int(num_meta_blocks), _ptr(maxb), _ptr(minb)),
+           "quest_metadata")
+    return maxb, minb
 
 
 def attn_fp32(cache: PagedCache, q: np.ndarray, k32: np.ndarray, v32: np.ndarray, b: int,

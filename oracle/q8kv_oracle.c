@@ -538,6 +538,73 @@ int q8kvo_decode_multi_rows(const q8kvo_cache *c, const float *q, int n_queries,
     return rc;
 }
 
+/* ---------------------------------------------------------------- QUEST metadata */
+
+/* Per-block K metadata for QUEST-style block selection, following the CANN
+ * quest_prefill_metadata guide (xdnf.cn/news/235188, "reference implementation" and
+ * "source-level principles"): for request r with L = seq_lens[r] tokens, KV block j
+ * (j < ceil(L / bs)) holds tokens [j * bs, min((j + 1) * bs, L)); its row of metadata block
+ * m = j / bs (rows = bs per metadata block) is row j % bs of physical metadata block
+ * meta_table[r][m], and for every KV head h and channel d
+ *   maxb[.][j % bs][h][d] = max over the block's tokens of K[slot][h][d]
+ *   minb[.][j % bs][h][d] = min over the same tokens
+ * where K is the dequantised cache value code * kscale[slot][h] (fp32 product). Rows of the
+ * request's last metadata block after its last KV block are zero in both. */
+int q8kvo_quest_metadata(const q8kvo_cache *c, const int32_t *meta_table, int max_meta_per_seq,
+                         int num_meta_blocks, float *maxb, float *minb)
+{
+    int rc = check_cache(c);
+    if (rc)
+        return rc;
+    if (!c->k || !c->ks || !meta_table || !maxb || !minb || max_meta_per_seq <= 0 ||
+        num_meta_blocks <= 0)
+        return Q8KVO_EINVAL;
+    const int bs = c->block_size, Hk = c->n_kv_heads, D = c->head_dim;
+    const long row_floats = (long)Hk * D; /* one metadata row: every head's D channels */
+    for (int r = 0; r < c->B; ++r) {
+        if ((rc = check_seq(c, r, 0)))
+            return rc;
+        const int L = c->seq_lens[r];
+        const int nkv = (L + bs - 1) / bs;
+        const int nmeta = (nkv + bs - 1) / bs;
+        if (nmeta > max_meta_per_seq)
+            return Q8KVO_ERANGE;
+        for (int m = 0; m < nmeta; ++m) {
+            const int mb = meta_table[(long)r * max_meta_per_seq + m];
+            if (mb < 0 || mb >= num_meta_blocks)
+                return Q8KVO_ERANGE;
+            for (int row = 0; row < bs; ++row) {
+                const int j = m * bs + row;
+                float *mx = maxb + ((long)mb * bs + row) * row_floats;
+                float *mn = minb + ((long)mb * bs + row) * row_floats;
+                if (j >= nkv) { /* after the request's last KV block */
+                    for (long e = 0; e < row_floats; ++e)
+                        mx[e] = mn[e] = MUT(22) ? 1.0f : 0.0f;
+                    continue;
+                }
+                const int t0 = j * bs;
+                const int t1 = MUT(21) ? t0 + bs : (t0 + bs < L ? t0 + bs : L);
+                for (int h = 0; h < Hk; ++h)
+                    for (int d = 0; d < D; ++d) {
+                        float hi = -INFINITY, lo = INFINITY;
+                        for (int t = t0; t < t1; ++t) {
+                            const long slot = slot_of(c, r, t);
+                            const float code = (float)c->k[(slot * Hk + h) * (long)D + d];
+                            const float v = MUT(23) ? code : code * c->ks[slot * Hk + h];
+                            if (v > hi)
+                                hi = v;
+                            if (v < lo)
+                                lo = v;
+                        }
+                        mx[(long)h * D + d] = hi;
+                        mn[(long)h * D + d] = lo;
+                    }
+            }
+        }
+    }
+    return Q8KVO_OK;
+}
+
 /* ---------------------------------------------------------------- three pass */
 
 /* The naive form the walk-through (section 3) contrasts with, laid out like the

@@ -21,6 +21,8 @@
  *   - the opening and the kernel signature (KV compressed to q8 with one scale per
  *     (token, KV head), applied as scale * 1/127 at use): the KV-cache write that fills
  *     the pools, with the section 2 part 1 quantiser applied to whole rows.
+ * The QUEST block metadata (per-channel max / min of K over each KV block) follows the
+ * CANN quest_prefill_metadata guide (xdnf.cn/news/235188) on the q8 pool.
  * Several query tokens per sequence (the multi-query "TILE" decode of the llama.cpp
  * change on baguaai.com's FlashAttention page) are the same single pass per (sequence,
  * query, head), each query seeing the cache up to its own position (causal).
@@ -122,6 +124,15 @@ int q8kvo_decode_multi(const q8kvo_cache *c, const float *q, int n_queries, doub
  * out[n][head_dim] (fp64). */
 int q8kvo_decode_multi_rows(const q8kvo_cache *c, const float *q, int n_queries,
                             const int32_t *rows, long n, double *out);
+
+/* QUEST-style per-block K metadata (CANN quest_prefill_metadata guide, xdnf.cn/news/235188):
+ * maxb, minb fp32 [num_meta_blocks][block_size][n_kv_heads][head_dim]; row j % bs of
+ * metadata block meta_table[r][j / bs] holds the per-channel max / min of the dequantised
+ * K over the tokens of request r's KV block j; unused rows of a request's last metadata
+ * block are zero. meta_table int32 [B][max_meta_per_seq]. Other fields of c as above
+ * (v, vs, n_q_heads and scale are not used). */
+int q8kvo_quest_metadata(const q8kvo_cache *c, const int32_t *meta_table, int max_meta_per_seq,
+                         int num_meta_blocks, float *maxb, float *minb);
 
 /* Naive three-pass variant (all scores, then max, then exp/sum, then weighted V). */
 int q8kvo_decode_threepass(const q8kvo_cache *c, const float *q, int b, int h, double *out);

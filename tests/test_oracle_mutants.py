@@ -31,6 +31,9 @@ MUTANTS = {
     18: "cache row written under the next KV head",
     19: "every query of a multi-query step sees only the first query's tokens",
     20: "multi-query visible length one token short",
+    21: "QUEST tail block reduced over the whole block",
+    22: "QUEST unused metadata rows not zeroed",
+    23: "QUEST metadata of the raw codes (scale dropped)",
 }
 
 
@@ -41,7 +44,8 @@ def test_planted_mistake_is_caught(mutant, tmp_path):
     r = subprocess.run(
         [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
          "tests/test_oracle_qquant.py", "tests/test_oracle_attention.py",
-         "tests/test_oracle_cache_write.py", "tests/test_oracle_multi_query.py"],
+         "tests/test_oracle_cache_write.py", "tests/test_oracle_multi_query.py",
+         "tests/test_oracle_quest.py"],
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {mutant} ({MUTANTS[mutant]}) passed every pin"
     assert "failed" in r.stdout, r.stdout[-2000:]
