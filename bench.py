@@ -55,6 +55,8 @@ def parse():
                     help="skip the KV-cache write information report")
     ap.add_argument("--no-multi-query", action="store_true",
                     help="skip the multi-query decode information report")
+    ap.add_argument("--no-quest", action="store_true",
+                    help="skip the QUEST block-metadata information report")
     ap.add_argument("--accuracy-study", action="store_true",
                     help="instead of timing: the q8-vs-fp32 output error study over the "
                          "workloads and K/V distributions (one JSON line)")
@@ -243,11 +245,12 @@ def _err_stats(got, ref):
                                                   99))}
 
 
-def accuracy_rows(w, out_gpu, n_rows, seed):
+def accuracy_rows(w, out_gpu, n_rows, seed, max_seqs=8):
     """Error of the q8 path against attention over the unquantised fp32 q, K, V on sampled
     (sequence, head) rows: the CUDA output and the oracle's q8 decode, each against the
     oracle's fp64 attention of the fp32 data (the fp32 rows of the sampled sequences are
-    regenerated from their random streams)."""
+    regenerated from their random streams, so at most max_seqs sequences are sampled and
+    the rows are spread over their heads)."""
     import numpy as np
 
     import oracle
@@ -257,8 +260,11 @@ def accuracy_rows(w, out_gpu, n_rows, seed):
     bs, Hk, D = c.block_size, c.n_kv_heads, c.head_dim
     rng = np.random.default_rng(seed)
     live = [b for b in range(c.B) if w.seq_lens[b] > 0]
-    pairs = sorted({(int(rng.choice(live)), int(rng.integers(0, c.n_q_heads)))
-                    for _ in range(n_rows)})
+    seqs = rng.choice(live, size=min(max_seqs, len(live), n_rows), replace=False)
+    per = max(1, n_rows // len(seqs))
+    pairs = sorted({(int(b), int(h)) for b in seqs
+                    for h in rng.choice(c.n_q_heads, size=min(per, c.n_q_heads),
+                                        replace=False)})
     cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens, c.n_q_heads,
                               w.scale)
     q8_oracle = oracle.decode_pairs(cache, w.q, pairs)
@@ -268,8 +274,12 @@ def accuracy_rows(w, out_gpu, n_rows, seed):
         nblk = -(-L // bs)
         blocks = w.block_table[b, :nblk].astype(np.int64)
         slots = (blocks[:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
-        k32 = inputs.fp32_rows(w, "k", slots).reshape(nblk, bs, Hk, D)
-        v32 = inputs.fp32_rows(w, "v", slots).reshape(nblk, bs, Hk, D)
+        if w.k32 is not None:  # the workload kept its unquantised draws
+            k32 = w.k32.reshape(-1, Hk, D)[slots].reshape(nblk, bs, Hk, D)
+            v32 = w.v32.reshape(-1, Hk, D)[slots].reshape(nblk, bs, Hk, D)
+        else:
+            k32 = inputs.fp32_rows(w, "k", slots).reshape(nblk, bs, Hk, D)
+            v32 = inputs.fp32_rows(w, "v", slots).reshape(nblk, bs, Hk, D)
         compact = oracle.PagedCache(w.k[blocks], w.v[blocks], w.ks[blocks], w.vs[blocks],
                                     np.arange(nblk, dtype=np.int32)[None, :],
                                     np.array([L], np.int32), c.n_q_heads, w.scale)
@@ -308,23 +318,36 @@ def run_accuracy_study(args):
         return out.cpu().numpy()
 
     results = []
-    sample = {0: 64, 1: 256, 2: 32, 3: 96, 4: 96}
-    for i, cfg in enumerate(inputs.CONFIGS):
-        w = inputs.make(cfg)
-        r = accuracy_rows(w, gpu_out(w), sample[i], seed=i)
-        r.update({"workload": cfg.name, "k_dist": cfg.k_dist, "v_dist": cfg.v_dist,
+    # the first three workloads whole (their unquantised draws kept); the two multi-GB ones
+    # with their recipe on 8 sequences (the fp32 copies of 4 GB pools would not fit the
+    # host budget of this study)
+    C = inputs.CONFIGS
+    lens3 = inputs._seq_lens(C[3])[:8]
+    study = [(C[0], inputs.make(C[0], keep_fp32=True), 64),
+             (C[1], inputs.make(C[1], keep_fp32=True), 256),
+             (C[2], inputs.make(C[2], keep_fp32=True), 32),
+             (C[3], inputs.make_custom(8, 64, 8, 128, lens3, 128, k_dist="student_t3",
+                                       v_dist="student_t3", seed=3, keep_fp32=True,
+                                       name="ragged_outliers (8 of its 64 sequences)"), 96),
+             (C[4], inputs.make_custom(8, 32, 8, 128, [8192] * 8, 64, seed=4, keep_fp32=True,
+                                       name="bandwidth (8 of its 256 sequences)"), 96)]
+    for i, (cfg, w, n) in enumerate(study):
+        r = accuracy_rows(w, gpu_out(w), n, seed=i)
+        r.update({"workload": w.cfg.name, "k_dist": cfg.k_dist, "v_dist": cfg.v_dist,
                   "k_bias_std": cfg.k_bias_std})
         results.append(r)
-        del w
+        print(json.dumps({"partial": r}), flush=True)
+    del study
     # distributions at one shape: 4 sequences of 4096 tokens, 32/8 heads, block 64
     for name, kw in [("normal", {}), ("student_t3 K and V", dict(k_dist="student_t3",
                                                                  v_dist="student_t3")),
                      ("K bias std 2", dict(k_bias_std=2.0)), ("K bias std 6", dict(k_bias_std=6.0)),
                      ("student_t3 K + bias 6", dict(k_dist="student_t3", k_bias_std=6.0))]:
-        w = inputs.make_custom(4, 32, 8, 128, [4096] * 4, 64, seed=50, **kw)
+        w = inputs.make_custom(4, 32, 8, 128, [4096] * 4, 64, seed=50, keep_fp32=True, **kw)
         r = accuracy_rows(w, gpu_out(w), 128, seed=50)
         r.update({"workload": f"4 x 4096 tokens, 32/8 heads: {name}"})
         results.append(r)
+        print(json.dumps({"partial": r}), flush=True)
     print(json.dumps({"study": "q8 KV + q8 Q attention output vs fp64 attention over the "
                                "unquantised fp32 q, K, V", "results": results}), flush=True)
     return 0
@@ -547,11 +570,14 @@ def main():
         # per sequence (speculative decode), through q8kv_decode_attn_multi
         line["multi_query"] = bench_multi_query(w, pools, bt, lens, dev, stream,
                                                 steps=max(10, min(args.steps, 2000)))
-    if not args.no_cache_write:
-        # information, after the timed region: the write path that fills the cache
+    if not args.no_cache_write or not args.no_quest:
         del pools, argsets
         torch.cuda.empty_cache()
+    if not args.no_cache_write:
+        # information, after the timed region: the write path that fills the cache
         line["cache_write"] = bench_cache_write(dev, stream)
+    if not args.no_quest:
+        line["quest_metadata"] = bench_quest(dev, stream)
     if rank == 0 and world == 1 and not args.no_accuracy:
         torch.cuda.synchronize(dev)
         line["q8_vs_fp32"] = q8_vs_fp32(w, out.cpu().numpy())
@@ -564,19 +590,25 @@ def main():
 
 
 CACHE_WRITE_SOURCES = ("q8kv_cache_write.cuh", "q8kv_cache_write_api.cuh", "q8kv_ptx.cuh")
+QUEST_SOURCES = ("q8kv_quest.cuh", "q8kv_quest_api.cuh", "q8kv_ptx.cuh")
 
 
 def source_hash(kernel: str = "decode") -> str:
     """Hash of the sources a kernel is built from (traffic figures are valid only for the
-    exact kernel): the cache write's own kernel and host files and the PTX helpers, or, for
-    the decode call, every other source of the library (its kernels, helpers and plan)."""
+    exact kernel): the cache write's or the QUEST metadata's own kernel and host files and
+    the PTX helpers, or, for the decode call, every other source of the library (its
+    kernels, helpers and plan)."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_attention_int8_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        mine = name in CACHE_WRITE_SOURCES if kernel == "cache_write" else \
-            not name.startswith("q8kv_cache_write")
+        if kernel == "cache_write":
+            mine = name in CACHE_WRITE_SOURCES
+        elif kernel == "quest":
+            mine = name in QUEST_SOURCES
+        else:
+            mine = not name.startswith(("q8kv_cache_write", "q8kv_quest"))
         if not mine:
             continue
         with open(os.path.join(csrc, name), "rb") as f:
@@ -648,6 +680,58 @@ def bench_multi_query(w, pools, bt, lens, dev, stream, steps, warmup=20, nqs=(2,
     res["workload"] = (f"{c.name} with nq new query tokens per sequence (causal), "
                        f"q/out [{c.B}][nq][{c.n_q_heads}][{c.head_dim}]")
     return res
+
+
+def bench_quest(dev, stream, steps=20, warmup=3, B=20, L=32768, Hk=8, bs=128):
+    """Information: QUEST block metadata (q8kv_quest_metadata) on the CANN guide's benchmark
+    shape (N = 8 KV heads, D = 128, block 128, B = 20 requests of 32768 tokens), over the q8
+    K pool. Algorithmic bytes: the K codes and scales of every token, the used block-table
+    and metadata-table entries, and both metadata arrays' used rows written."""
+    import numpy as np
+    import torch
+
+    import decode_attention_int8_b200 as q8
+    from decode_attention_int8_b200 import inputs
+
+    w = inputs.make_custom(B, Hk, Hk, 128, [L] * B, bs, seed=42)
+    meta, n_meta = inputs.quest_meta_table(w.seq_lens, bs, seed=42)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    k, ks, bt, lens, mt = t(w.k), t(w.ks), t(w.block_table), t(w.seq_lens), t(meta)
+    mx = torch.empty((n_meta, bs, Hk, 128), dtype=torch.float32, device=dev)
+    mn = torch.empty_like(mx)
+    q8.q8kv_quest_metadata(mx, mn, k, ks, bt, lens, mt, stream=stream)
+    fn = q8.lib().q8kv_quest_metadata
+    P_ = lambda x: ctypes.c_void_p(x.data_ptr())
+    a = (P_(mx), P_(mn), P_(k), P_(ks), P_(bt), P_(lens), P_(mt), B, Hk, 128, bs,
+         int(bt.shape[1]), int(mt.shape[1]), w.num_blocks, n_meta,
+         ctypes.c_void_p(stream.cuda_stream))
+    for _ in range(warmup):
+        fn(*a)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        st = fn(*a)
+        if st != 0:
+            raise q8.Q8KVError(st, "q8kv_quest_metadata")
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    nkv = -(-L // bs)
+    nmeta = -(-nkv // bs)
+    algo = (B * L * Hk * (128 + 4) + 4 * B * nkv + 4 * B * nmeta + 4 * B
+            + 2 * B * nmeta * bs * Hk * 128 * 4)
+    peak, peak_kind = measured_peak()
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"workload": f"{B} requests x {L} tokens, {Hk} KV heads, D 128, block {bs} "
+                        f"(the CANN guide's benchmark shape), q8 K pool {w.k.nbytes / 1e6:.0f} MB",
+            "us_per_call": round(ms * 1e3, 3), "calls": steps, "algorithmic_bytes": algo,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                         "traffic": recorded_traffic("quest_b20_l32768", "quest"),
+                         "kernel": "q8kv::quest_metadata_kernel"},
+            "device_errors": q8.q8kv_device_errors(clear=True)}
 
 
 def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):

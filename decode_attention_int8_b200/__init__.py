@@ -5,6 +5,7 @@ this package is its ctypes binding plus the seeded synthetic workload generators
 """
 from ._lib import (  # noqa: F401
     DEVERR_BLOCK_TABLE,
+    DEVERR_META,
     DEVERR_NONFINITE,
     DEVERR_SEQ_LEN,
     DEVERR_SLOT,
@@ -20,6 +21,7 @@ from ._lib import (  # noqa: F401
     q8kv_decode_attn_multi,
     q8kv_decode_attn_static,
     q8kv_decode_attn_ws,
+    q8kv_quest_metadata,
     q8kv_device_errors,
     q8kv_version,
     q8kv_workspace_bytes,

@@ -23,6 +23,7 @@ DEVERR_BLOCK_TABLE = 0x2
 DEVERR_TIMEOUT = 0x4
 DEVERR_SLOT = 0x8
 DEVERR_NONFINITE = 0x10
+DEVERR_META = 0x20
 
 EXPORTS = (
     "q8kv_decode_attn",
@@ -32,6 +33,7 @@ EXPORTS = (
     "q8kv_decode_attn_ws",
     "q8kv_decode_attn_static",
     "q8kv_cache_write",
+    "q8kv_quest_metadata",
     "q8kv_debug_quantize_q",
     "q8kv_debug_block_dots",
     "q8kv_device_errors",
@@ -72,6 +74,7 @@ def lib():
                 "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
                 "q8kv_decode_attn_static": ([P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_cache_write": ([P] * 7 + [I] * 5 + [ctypes.c_longlong, P], I),
+                "q8kv_quest_metadata": ([P] * 7 + [I] * 8 + [P], I),
                 "q8kv_debug_quantize_q": ([P, P, P, I, I, P], I),
                 "q8kv_debug_block_dots": ([P, I] + [P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
@@ -225,6 +228,34 @@ def q8kv_cache_write(k_blocks, v_blocks, kscale, vscale, k_new, v_new, slot_mapp
     _check(lib().q8kv_cache_write(_ptr(k_blocks), _ptr(v_blocks), _ptr(kscale), _ptr(vscale),
                                   _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), n, Hk, D, bs, P,
                                   stride, _stream(stream)), "q8kv_cache_write")
+
+
+def q8kv_quest_metadata(maxblocks, minblocks, k_blocks, kscale, block_table, seq_lens,
+                        meta_block_table, stream=None):
+    """Per-block K metadata: maxblocks, minblocks fp32 [num_meta][block_size][Hk][D] get the
+    per-channel max / min of the dequantised K of each KV block (row j % block_size of
+    metadata block meta_block_table[r][j // block_size])."""
+    _need(maxblocks, "maxblocks", torch.float32, 4)
+    _need(minblocks, "minblocks", torch.float32, 4)
+    _need(k_blocks, "k_blocks", torch.int8, 4)
+    _need(kscale, "kscale", torch.float32, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    _need(meta_block_table, "meta_block_table", torch.int32, 2)
+    P, bs, Hk, D = k_blocks.shape
+    nm = int(maxblocks.shape[0])
+    if tuple(maxblocks.shape) != (nm, bs, Hk, D) or tuple(minblocks.shape) != (nm, bs, Hk, D):
+        raise ValueError("maxblocks/minblocks must be [num_meta_blocks][block_size][Hk][D]")
+    if tuple(kscale.shape) != (P, bs, Hk):
+        raise ValueError("kscale must be [num_blocks][block_size][Hk]")
+    B = int(seq_lens.shape[0])
+    if block_table.shape[0] != B or meta_block_table.shape[0] != B:
+        raise ValueError("block tables and seq_lens disagree on the batch size")
+    _check(lib().q8kv_quest_metadata(_ptr(maxblocks), _ptr(minblocks), _ptr(k_blocks),
+                                     _ptr(kscale), _ptr(block_table), _ptr(seq_lens),
+                                     _ptr(meta_block_table), B, Hk, D, bs,
+                                     int(block_table.shape[1]), int(meta_block_table.shape[1]),
+                                     P, nm, _stream(stream)), "q8kv_quest_metadata")
 
 
 def q8kv_debug_quantize_q(qi, qsc, q, stream=None):

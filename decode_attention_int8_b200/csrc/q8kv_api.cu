@@ -98,7 +98,7 @@ struct Shape {
 // How the work is tiled for one shape on one device.
 struct Plan {
     int G, slices, NT, HPC, nhc, pairs, subtiles, TT, box_tok, log2_box, n_boxes, n_stages;
-    int scale_bulk, heads_seg, scratch_stride, grid;
+    int scale_bulk, sc_heads, heads_seg, scratch_stride, grid;
     SmemLayout lay;
     size_t smem_bytes;
     size_t ws_desc_off, ws_part_off, ws_bytes;
@@ -141,8 +141,12 @@ q8kv_status plan_heads(int Hq, int Hk, int D, Plan &pl)
     while (pl.HPC * 2 <= max_hpc && Hk % (pl.HPC * 2) == 0)
         pl.HPC *= 2;
     pl.scale_bulk = (pl.HPC == Hk) ? 1 : 0;
-    if (!pl.scale_bulk && (pl.HPC < 4 || Hk % 4 != 0))
+    // A tile with fewer heads than the cache loads its scales through a 2-D tensor map
+    // whose rows (Hk * 4 bytes) and boxes (at least 4 heads: 16 bytes) must be 16-byte
+    // multiples; a tile of 1 or 2 heads loads the aligned 4-head box around them.
+    if (!pl.scale_bulk && Hk % 4 != 0)
         return Q8KV_ERR_UNSUPPORTED;
+    pl.sc_heads = pl.scale_bulk ? pl.HPC : (pl.HPC < 4 ? 4 : pl.HPC);
     pl.nhc = Hk / pl.HPC;
     pl.pairs = pl.HPC * pl.slices;
     pl.subtiles = kConsumerWarps / pl.pairs;
@@ -190,7 +194,7 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     const int scratch_floats = (pl.subtiles - 1) * pl.pairs * pl.scratch_stride;
     pl.n_stages = 0;
     for (int n = kMaxStages; n >= 2; --n) {
-        SmemLayout L = make_layout(pl.TT, pl.HPC, n, s.B, scratch_floats, pl.grid);
+        SmemLayout L = make_layout(pl.TT, pl.HPC, pl.sc_heads, n, s.B, scratch_floats, pl.grid);
         if ((size_t)L.total + 1024 <= (size_t)dev.smem_optin) {
             pl.n_stages = n;
             pl.lay = L;
@@ -249,7 +253,7 @@ q8kv_status encode_maps_uncached(const Shape &s, const Plan &pl, const int8_t *k
     if (!pl.scale_bulk) {
         cuuint64_t sd[2] = {(cuuint64_t)s.Hk, slots};
         cuuint64_t ss[1] = {(cuuint64_t)s.Hk * 4};
-        cuuint32_t sb[2] = {(cuuint32_t)pl.HPC, (cuuint32_t)pl.box_tok};
+        cuuint32_t sb[2] = {(cuuint32_t)pl.sc_heads, (cuuint32_t)pl.box_tok};
         cuuint32_t se[2] = {1, 1};
         r = enc(mks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(ks), sd, ss, sb, se,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -269,11 +273,12 @@ q8kv_status encode_maps_uncached(const Shape &s, const Plan &pl, const int8_t *k
 // cache reuse them (a small round-robin cache, guarded by g_mutex).
 struct MapKey {
     const void *k, *v, *ks, *vs;
-    int Hk, bs, P, HPC, box_tok, scale_bulk;
+    int Hk, bs, P, HPC, box_tok, scale_bulk, sc_heads;
     bool operator==(const MapKey &o) const
     {
         return k == o.k && v == o.v && ks == o.ks && vs == o.vs && Hk == o.Hk && bs == o.bs &&
-               P == o.P && HPC == o.HPC && box_tok == o.box_tok && scale_bulk == o.scale_bulk;
+               P == o.P && HPC == o.HPC && box_tok == o.box_tok && scale_bulk == o.scale_bulk &&
+               sc_heads == o.sc_heads;
     }
 };
 
@@ -291,7 +296,8 @@ q8kv_status encode_maps(const Shape &s, const Plan &pl, const int8_t *k, const i
                         const float *ks, const float *vs, CUtensorMap *mk, CUtensorMap *mv,
                         CUtensorMap *mks, CUtensorMap *mvs)
 {
-    const MapKey key{k, v, ks, vs, s.Hk, s.bs, s.P, pl.HPC, pl.box_tok, pl.scale_bulk};
+    const MapKey key{k, v, ks, vs, s.Hk, s.bs, s.P, pl.HPC, pl.box_tok, pl.scale_bulk,
+                     pl.sc_heads};
     std::lock_guard<std::mutex> lock(g_mutex);
     for (auto &e : g_maps) {
         if (e.used && e.key == key) {
@@ -467,6 +473,7 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.n_boxes = pl.n_boxes;
     p.n_stages = pl.n_stages;
     p.scale_bulk = pl.scale_bulk;
+    p.sc_heads = pl.sc_heads;
     p.heads_seg = pl.heads_seg;
     p.scratch_stride = pl.scratch_stride;
     p.scale_log2 = (float)((double)c.scale * 1.4426950408889634);
@@ -729,3 +736,6 @@ int q8kv_version(void)
 
 // The KV-cache write entry point (uses the device bookkeeping above).
 #include "q8kv_cache_write_api.cuh"
+
+// The QUEST block-metadata entry point.
+#include "q8kv_quest_api.cuh"

@@ -65,7 +65,6 @@ constexpr int kMaxBoxes = 16;       // TMA boxes per stage
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
 constexpr int kSlotRow = kD + 4;    // per-head partial: kD accumulator floats, M, S, A, pad
-constexpr uint32_t kScaleGap = 1024; // bytes from a stage's K scales to its V scales (>= TT*HPC*4)
 // Work split: a segment that starts in the middle of a CTA's range costs that CTA about
 // three tiles' time (the finished segment's accumulators are folded, reduced and written
 // and the next query is set up, by code that runs once and is fetched cold while the K/V
@@ -91,6 +90,7 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a)
 struct SmemLayout {
     uint32_t stage_bytes; // one ring slot: K | V | kscale | vscale
     uint32_t off_k, off_v, off_ks, off_vs; // within a slot
+    uint32_t sc_gap;      // bytes from a stage's K scales to its V scales (TT * sc_heads * 4)
     uint32_t off_full, off_empty, off_mbar, off_mask, off_misc, off_slots, off_ptab, off_cstart,
         off_prefix, off_scratch;
     uint32_t off_nseq;  // prefix count of sequences with tokens (B <= kPenaltyMaxB), else 0
@@ -99,16 +99,17 @@ struct SmemLayout {
     uint32_t total;     // bytes from the 1024-aligned base
 };
 
-__host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int n_stages, int B,
-                                                  int scratch_floats, int grid)
+__host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int sc_heads, int n_stages,
+                                                  int B, int scratch_floats, int grid)
 {
     SmemLayout L;
     const uint32_t kv = (uint32_t)(TT * HPC * kD);
+    L.sc_gap = align_up((uint32_t)(TT * sc_heads * 4), 128);
     L.off_k = 0;
     L.off_v = kv;
     L.off_ks = 2 * kv;
-    L.off_vs = 2 * kv + kScaleGap;
-    L.stage_bytes = align_up(2 * kv + 2 * kScaleGap, 1024);
+    L.off_vs = 2 * kv + L.sc_gap;
+    L.stage_bytes = align_up(2 * kv + 2 * L.sc_gap, 1024);
     uint32_t o = (uint32_t)n_stages * L.stage_bytes;
     L.off_full = o;
     o += 8 * kMaxStages;
@@ -162,6 +163,9 @@ struct DecodeParams {
     int bs, mbps, num_blocks;
     int HPC, nhc, slices, pairs, subtiles, TT, box_tok, log2_box, n_boxes, n_stages;
     int scale_bulk;      // 1: scales by contiguous bulk copy (HPC == Hk); 0: 2-D tensor map
+    int sc_heads;        // KV heads per scale box: HPC, or 4 when a tile holds fewer heads
+                         // (a box row must be 16 bytes); the tile's heads sit at column
+                         // (hc * HPC) % sc_heads of it
     int heads_seg;       // query heads per segment (HPC * G)
     int scratch_stride;  // floats per (subtile, pair) merge region
     float scale_log2;    // softmax scale * log2(e)
@@ -339,7 +343,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     const uint64_t pol = l2_policy_evict_first();
     const int cap = p.mbps * p.bs;
     const uint32_t kv_box = (uint32_t)(p.box_tok * p.HPC * kD);
-    const uint32_t sc_box = (uint32_t)(p.box_tok * p.HPC * 4);
+    const uint32_t sc_box = (uint32_t)(p.box_tok * p.sc_heads * 4);
     int stage = 0;
     uint32_t phase = 0, issued = 0, issued_par = 0;
     bool aborted = false;
@@ -367,13 +371,17 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
             hc = local / ntb;
             const int lt = local - hc * ntb;
             const int tok0 = lt * p.TT;
+            const int32_t *bt_row = p.block_table + (long long)b * p.mbps;
+            // the tile's first block-table entry is loaded together with the sequence length
+            // (one round trip instead of two: tok0 < L <= mbps * bs, so it is in the row)
+            const int ph0 = __ldg(bt_row + tok0 / p.bs);
             const int L = clamp_len(__ldg(p.seq_lens + b), cap);
 #pragma unroll 1
             for (int bx = 0; bx < p.n_boxes; ++bx) {
                 const int tk = tok0 + bx * p.box_tok;
                 int sl = -1;
                 if (tk < L) {
-                    const int ph = __ldg(p.block_table + (long long)b * p.mbps + tk / p.bs);
+                    const int ph = bx == 0 ? ph0 : __ldg(bt_row + tk / p.bs);
                     if (ph >= 0 && ph < p.num_blocks)
                         sl = ph * p.bs + (tk % p.bs);
                     else
@@ -422,10 +430,11 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
                             bulk_load(sb + p.lay.off_vs + bx * sc_box, p.vscale + e0, sc_box,
                                       &full[stage], pol);
                         } else {
-                            tma_load_2d(sb + p.lay.off_ks + bx * sc_box, tmKs, &full[stage],
-                                        hci * p.HPC, slot, pol);
-                            tma_load_2d(sb + p.lay.off_vs + bx * sc_box, tmVs, &full[stage],
-                                        hci * p.HPC, slot, pol);
+                            const int h0 = (hci * p.HPC / p.sc_heads) * p.sc_heads;
+                            tma_load_2d(sb + p.lay.off_ks + bx * sc_box, tmKs, &full[stage], h0,
+                                        slot, pol);
+                            tma_load_2d(sb + p.lay.off_vs + bx * sc_box, tmVs, &full[stage], h0,
+                                        slot, pol);
                         }
                     }
                     issued |= 1u << stage;
@@ -594,7 +603,8 @@ __device__ __forceinline__ void reset_state(WarpState<NT> &st)
 struct ThreadOffsets {
     uint32_t k[kSub][kNB]; // K fragment (subtile u, quant block j) of tokens 0-7; 8-15: +1024
     uint32_t v[kSub][2];   // V row of token 2c + e (e = 0, 1); token 2c + e + 8: +1024
-    uint32_t s[kSub][2][2]; // K scale of token (u, nt, e); its V scale is kScaleGap further
+    uint32_t s[kSub][2][2]; // K scale of token (u, nt, e) at column kl (add the segment's
+                            // column offset); its V scale is sc_gap further
 };
 
 __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int kl, int ts, int g,
@@ -621,7 +631,7 @@ __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e)
-                o.s[u][nt][e] = p.lay.off_ks + 4 * ((t0 + nt * 8 + 2 * c + e) * H + kl);
+                o.s[u][nt][e] = p.lay.off_ks + 4 * ((t0 + nt * 8 + 2 * c + e) * p.sc_heads + kl);
     }
     return o;
 }
@@ -637,7 +647,8 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 // data (clear past the sequence end and in blocks that were not loaded).
 template <int NT, bool kPack, bool kDump>
 __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<NT> &st,
-                                              const ThreadOffsets &o, uint32_t sb, int tl0,
+                                              const ThreadOffsets &o, uint32_t sb,
+                                              uint32_t sbs, int tl0,
                                               uint32_t vmask, bool causal, const int (&lim)[NT],
                                               float scale_log2, int b, int hc, int kl,
                                               int slice, int tok0, int g, int c)
@@ -710,8 +721,8 @@ __device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<N
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                kss[u][nt][e] = lds_f32(sb + o.s[u][nt][e]) * scale_log2;
-                vsv[u][nt][e] = lds_f32(sb + o.s[u][nt][e] + kScaleGap);
+                kss[u][nt][e] = lds_f32(sbs + o.s[u][nt][e]) * scale_log2;
+                vsv[u][nt][e] = lds_f32(sbs + o.s[u][nt][e] + p.lay.sc_gap);
             }
     // masked tokens (rare: a segment's last tile, bad block-table entries) get score -inf
     // and V scale 0, whatever stale data their slots hold; with several queries per
@@ -869,7 +880,7 @@ constexpr float kTwo23 = 8388608.0f;
 
 struct PackedOffsets {
     uint32_t k[kSub][kNB]; // K fragments, as ThreadOffsets::k
-    uint32_t s[2][2];      // K scale of this lane's kept token (nt, e); V scale kScaleGap on
+    uint32_t s[2][2];      // K scale of this lane's kept token (nt, e); V scale sc_gap on
     uint32_t v;            // ldmatrix row address of this lane; XOR (16 m) selects chunk m
 };
 
@@ -893,7 +904,8 @@ __device__ __forceinline__ PackedOffsets make_packed_offsets(const DecodeParams 
 #pragma unroll
         for (int e = 0; e < 2; ++e)
             o.s[nt][e] =
-                p.lay.off_ks + 4 * (((ts * kSub + uk) * 16 + nt * 8 + 2 * c + e) * H + kl);
+                p.lay.off_ks +
+                4 * (((ts * kSub + uk) * 16 + nt * 8 + 2 * c + e) * p.sc_heads + kl);
     // ldmatrix: lanes 0-15 give the rows of matrix 0 (subtile 0), lanes 16-31 of matrix 1
     const int kk = lane & 15;
     const int tau = 2 * (kk >> 2) + (kk & 1) + 8 * ((kk >> 1) & 1);
@@ -937,8 +949,9 @@ __device__ __forceinline__ void packed_rescale(WarpState<NT> &st, float f0, floa
 template <int NT, bool kDump>
 __device__ __forceinline__ void process_stage_packed(const DecodeParams &p, WarpState<NT> &st,
                                                      PackedAcc &pa, const PackedOffsets &o,
-                                                     uint32_t sb, int tl0, uint32_t vmask,
-                                                     bool causal, int lim, float scale_log2,
+                                                     uint32_t sb, uint32_t sbs, int tl0,
+                                                     uint32_t vmask, bool causal, int lim,
+                                                     float scale_log2,
                                                      int b, int hc, int kl, int tok0, int g,
                                                      int c, float k0, float k1)
 {
@@ -988,8 +1001,8 @@ __device__ __forceinline__ void process_stage_packed(const DecodeParams &p, Warp
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            kss[nt][e] = lds_f32(sb + o.s[nt][e]) * scale_log2;
-            vsv[nt][e] = lds_f32(sb + o.s[nt][e] + kScaleGap);
+            kss[nt][e] = lds_f32(sbs + o.s[nt][e]) * scale_log2;
+            vsv[nt][e] = lds_f32(sbs + o.s[nt][e] + p.lay.sc_gap);
         }
     if (vmask != 0xffffffffu || causal) {
 #pragma unroll
@@ -1370,6 +1383,7 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
     for (int x = t0; x < t1;) {
         const SegCursor cu = cursor_at(p, prefix, x);
         const int x_end = cu.seg1 < t1 ? cu.seg1 : t1;
+        const uint32_t scol4 = 4u * (uint32_t)((cu.hc * p.HPC) % p.sc_heads);
         {
             const QueryFrag<NT> qf = (prefetch_q && seg_index == 1)
                                          ? load_query_smem<NT, kPack>(qbuf, g, c)
@@ -1412,12 +1426,13 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
 #pragma unroll
                 for (int r = 0; r < NT; ++r)
                     lim[r] = cu.L - fut[r] - win0;
+                const uint32_t sbs = sb + scol4; // this segment's scale column
                 if constexpr (kPack)
-                    process_stage_packed<NT, kDump>(p, st, pa, po, sb, tl0, vmask, causal, lim[0],
-                                                    scale_log2, cu.b, cu.hc, kl, tok0, g, c, k0,
-                                                    k1);
+                    process_stage_packed<NT, kDump>(p, st, pa, po, sb, sbs, tl0, vmask, causal,
+                                                    lim[0], scale_log2, cu.b, cu.hc, kl, tok0, g,
+                                                    c, k0, k1);
                 else
-                    process_stage<NT, kPack, kDump>(p, st, o, sb, tl0, vmask, causal, lim,
+                    process_stage<NT, kPack, kDump>(p, st, o, sb, sbs, tl0, vmask, causal, lim,
                                                     scale_log2, cu.b, cu.hc, kl, slice, tok0, g,
                                                     c);
                 __syncwarp();

@@ -53,12 +53,11 @@
  *
  * Supported shapes of the decode kernel: head_dim 128; kv_block_size a power of two in
  * [16, 256]; n_q_heads a multiple of n_kv_heads; query rows per KV head R (the group
- * n_q_heads / n_kv_heads, times n_queries for q8kv_decode_attn_multi) at most 128, with
- * n_kv_heads a power of two <= 8 or a multiple of 4 when R <= 32, n_kv_heads <= 2 when
- * R <= 64, and n_kv_heads = 1 above (a tile holds 8 / ceil_pow2(R / 16) KV heads, and a
- * tile with fewer KV heads than the cache needs at least 4 of them for its scale copies);
- * B <= 16384; num_kv_blocks * kv_block_size < 2^31. Other shapes return
- * Q8KV_ERR_UNSUPPORTED.
+ * n_q_heads / n_kv_heads, times n_queries for q8kv_decode_attn_multi) at most 128; a tile
+ * holds up to 8 / ceil_pow2(R / 16) KV heads, and when it holds fewer than n_kv_heads (its
+ * scales then come through a 2-D copy whose rows must be 16-byte multiples) n_kv_heads
+ * must be a multiple of 4; B <= 16384; num_kv_blocks * kv_block_size < 2^31. Other shapes
+ * return Q8KV_ERR_UNSUPPORTED.
  */
 #ifndef Q8KV_H
 #define Q8KV_H
@@ -86,6 +85,8 @@ typedef enum {
 #define Q8KV_DEVERR_TIMEOUT 0x4u     /* a pipeline wait ran past its limit (kernel gave up) */
 #define Q8KV_DEVERR_SLOT 0x8u        /* cache write: a slot past the pool (row skipped)     */
 #define Q8KV_DEVERR_NONFINITE 0x10u  /* cache write: a row held inf or NaN (codes 0, NaN scale) */
+#define Q8KV_DEVERR_META 0x20u       /* QUEST metadata: a metadata-table entry outside its pool
+                                        (row skipped), or a table too short for a request */
 
 /*
  * Decode attention with a library-managed workspace (one per device, grown on demand
@@ -240,6 +241,37 @@ q8kv_status q8kv_cache_write(int8_t *k_blocks, int8_t *v_blocks, float *kscale, 
                              const int64_t *slot_mapping, int n_tokens, int n_kv_heads,
                              int head_dim, int kv_block_size, int num_kv_blocks,
                              long long token_stride, cudaStream_t stream);
+
+/*
+ * QUEST-style per-block K metadata (CANN quest_prefill_metadata guide, xdnf.cn/news/235188):
+ * for every request r, KV block j < ceil(seq_lens[r] / kv_block_size) and KV head h, the
+ * per-channel maximum and minimum of the dequantised K (code * kscale, one fp32 product)
+ * over the block's tokens (the last block: only its tokens < seq_lens[r]). A metadata block
+ * holds kv_block_size rows, one per KV block: KV block j of request r is row
+ * j % kv_block_size of physical metadata block meta_block_table[r][j / kv_block_size].
+ * The rows of a request's last metadata block after its last KV block are set to zero in
+ * both arrays; metadata blocks no request uses are not touched. QUEST bounds q . k over a
+ * block from these two vectors to choose the blocks a decode step reads.
+ *
+ *   maxblocks, minblocks  fp32 [num_meta_blocks][kv_block_size][n_kv_heads][head_dim],
+ *                         16-byte aligned, written
+ *   k_blocks, kscale      the K pool and its scales (layouts above); v is not read
+ *   block_table, seq_lens as for decode
+ *   meta_block_table      int32 [B][max_meta_blocks_per_seq]
+ *   head_dim              128
+ * Device-side checks: a seq_len outside [0, max_blocks_per_seq * kv_block_size] is clamped
+ * (Q8KV_DEVERR_SEQ_LEN); a block-table entry outside the pool skips its row
+ * (Q8KV_DEVERR_BLOCK_TABLE); a metadata-table entry outside [0, num_meta_blocks), or a
+ * request needing more than max_meta_blocks_per_seq metadata blocks, sets
+ * Q8KV_DEVERR_META (the rows it cannot place are skipped). One kernel launch, asynchronous
+ * on `stream`, programmatic dependent launch as the other kernels.
+ */
+q8kv_status q8kv_quest_metadata(float *maxblocks, float *minblocks, const int8_t *k_blocks,
+                                const float *kscale, const int32_t *block_table,
+                                const int32_t *seq_lens, const int32_t *meta_block_table, int B,
+                                int n_kv_heads, int head_dim, int kv_block_size,
+                                int max_blocks_per_seq, int max_meta_blocks_per_seq,
+                                int num_kv_blocks, int num_meta_blocks, cudaStream_t stream);
 
 /* Debug: the Q quantisation alone (step 1) on n_rows rows of head_dim fp32 values
  * (head_dim a multiple of 32). qi int8 [n_rows][head_dim], qsc fp32

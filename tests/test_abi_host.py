@@ -131,3 +131,22 @@ def test_cache_write_of_no_tokens_enqueues_nothing():
     assert _write(n=0) == OK
     assert _write(n=0, kn=None, vn=None, sl=None) == OK
     assert _write(n=0, k=None) == INVALID
+
+
+def test_quest_metadata_bad_arguments_rejected():
+    L = q8.lib()
+    P = ctypes.c_void_p
+    ptrs = [P(0x10000 * i) for i in range(1, 8)]
+    sizes = [2, 8, 128, 16, 4, 1, 8, 2]  # B, Hk, D, bs, mbps, mmbpr, num_blocks, num_meta
+    for i in range(7):
+        bad = list(ptrs)
+        bad[i] = None
+        assert L.q8kv_quest_metadata(*bad, *sizes, None) == INVALID
+    for i in range(8):
+        bad = list(sizes)
+        bad[i] = 0
+        assert L.q8kv_quest_metadata(*ptrs, *bad, None) == INVALID
+    assert L.q8kv_quest_metadata(P(0x10004), *ptrs[1:], *sizes, None) == INVALID  # alignment
+    odd = list(sizes)
+    odd[2] = 64
+    assert L.q8kv_quest_metadata(*ptrs, *odd, None) == UNSUPPORTED

@@ -49,6 +49,29 @@ def test_large_groups(G):
     check_full(w, f"G={G}")
 
 
+@pytest.mark.parametrize("G,Hk", [(64, 8), (48, 4), (128, 4), (40, 12)])
+def test_tiles_narrower_than_the_scale_box(G, Hk):
+    # tiles of 1 or 2 KV heads out of 4+: the scales come in the aligned 4-head box around
+    # the tile's heads, and the tile's column in it changes from one head chunk to the next
+    lens = [77, 300, 1]
+    w = inputs.make_custom(3, Hk * G, Hk, 128, lens, 32, seed=G + Hk)
+    check_full(w, f"G={G} Hk={Hk}")
+
+
+@pytest.mark.parametrize("B,Hq,Hk,ragged", [
+    (16, 32, 8, False),  # the benchmark's head layout with shorter sequences
+    (16, 32, 8, True),
+    (30, 16, 4, False),  # about one sequence per SM
+    (37, 8, 4, True),
+    (9, 144, 16, False), # group 9 (two 8-row query tiles), 16 KV heads
+])
+def test_batches_near_the_sm_count(B, Hq, Hk, ragged):
+    rng = np.random.default_rng(B + Hk)
+    lens = (rng.integers(1, 3000, B) if ragged else np.full(B, 1500)).tolist()
+    w = inputs.make_custom(B, Hq, Hk, 128, lens, 64, seed=B * Hk)
+    check_full(w, f"B={B} Hq={Hq} Hk={Hk} ragged={ragged}")
+
+
 def test_zero_query_blocks_and_identity_table():
     w = inputs.make_custom(3, 16, 4, 128, [40, 64, 9], 16, table="identity", seed=5)
     w.q[0, :, :32] = 0.0  # whole quant block zero

@@ -39,6 +39,7 @@ def run_multi(w, q):
     (8, 32, 8),   # 32 rows: two 16-row slices, 4 KV heads per tile
     (8, 16, 2),   # 64 rows: four 16-row slices
     (16, 8, 1),   # 128 rows: the largest tiling (one KV head per tile)
+    (16, 32, 8),  # 64 rows over 8 KV heads: 2-head tiles with 4-head scale boxes
     (5, 20, 4),   # 25 rows, 2 slices
 ])
 @pytest.mark.parametrize("bs", [16, 64])
@@ -91,9 +92,8 @@ def test_gqa_batch_workload_with_four_queries():
 
 @pytest.mark.parametrize("nq,Hq,Hk", [
     (17, 64, 8),  # 136 rows per KV head: above the 128-row tiling
-    (16, 32, 8),  # 64 rows per KV head with 8 KV heads: a tile would hold 2 of the 8 KV
-                  # heads, whose scale slices (8 bytes) are below the 16-byte TMA minimum,
-                  # the same limit as a single query with group 64 over 8 KV heads
+    (16, 24, 6),  # 64 rows per KV head with 6 KV heads: a tile holds 2 of them, and the
+                  # scale rows of 6 heads (24 bytes) are no 16-byte multiple
 ])
 def test_unsupported_row_counts(nq, Hq, Hk):
     w = inputs.make_custom(1, Hq, Hk, 128, [40], 16, seed=1)
