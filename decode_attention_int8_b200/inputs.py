@@ -140,11 +140,36 @@ def quantize_rows(x: np.ndarray):
     return codes, scale
 
 
-def _fill_pool(seed, stream, dist, P, bs, Hk, D, bias, keep_fp32, threads):
-    """Generate one int8 pool and its scales chunk by chunk (deterministic per chunk)."""
+def quantize_q4_0_rows(x: np.ndarray):
+    """q4_0 blocks of 32 channels (llama.cpp's rule, this library's packing) of fp32 rows
+    [..., D]: m = the value of largest magnitude with its sign, d = m / -8,
+    code = min(15, trunc(x * (1 / d) + 8.5)) in fp32, d stored as binary16; codes packed
+    two per byte (channel 2i low nibble, 2i + 1 high). Returns (packed uint8 [..., D/2],
+    d uint16 binary16 bits [..., D/32])."""
+    x = np.asarray(x, np.float32)
+    blk = x.reshape(x.shape[:-1] + (x.shape[-1] // 32, 32))
+    idx = np.argmax(np.abs(blk), axis=-1)
+    m = np.take_along_axis(blk, idx[..., None], axis=-1)[..., 0]
+    d = (m / np.float32(-8.0)).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(d != 0, np.float32(1.0) / d, np.float32(0.0)).astype(np.float32)
+    t = (blk * inv[..., None]).astype(np.float32) + np.float32(8.5)
+    q = np.minimum(15, np.trunc(t.astype(np.float32)).astype(np.int32))
+    q = q.reshape(x.shape)
+    packed = (q[..., 0::2] | (q[..., 1::2] << 4)).astype(np.uint8)
+    return packed, d.astype(np.float16).view(np.uint16)
+
+
+def _fill_pool(seed, stream, dist, P, bs, Hk, D, bias, keep_fp32, threads, q4=False):
+    """Generate one pool and its scales chunk by chunk (deterministic per chunk): int8 codes
+    and fp32 row scales, or (q4) packed 4-bit codes and binary16 block scales."""
     slots = P * bs
-    codes = np.empty((slots, Hk, D), np.int8)
-    scales = np.empty((slots, Hk), np.float32)
+    if q4:
+        codes = np.empty((slots, Hk, D // 2), np.uint8)
+        scales = np.empty((slots, Hk, D // 32), np.uint16)
+    else:
+        codes = np.empty((slots, Hk, D), np.int8)
+        scales = np.empty((slots, Hk), np.float32)
     raw = np.empty((slots, Hk, D), np.float32) if keep_fp32 else None
     n_chunks = -(-slots // _CHUNK_SLOTS)
 
@@ -153,7 +178,7 @@ def _fill_pool(seed, stream, dist, P, bs, Hk, D, bias, keep_fp32, threads):
         x = _draw(_rng(seed, stream, i), dist, (hi - lo, Hk, D))
         if bias is not None:
             x += bias[None, :, :]
-        c, s = quantize_rows(x)
+        c, s = quantize_q4_0_rows(x) if q4 else quantize_rows(x)
         codes[lo:hi] = c
         scales[lo:hi] = s
         if raw is not None:
@@ -166,7 +191,7 @@ def _fill_pool(seed, stream, dist, P, bs, Hk, D, bias, keep_fp32, threads):
         for i in range(n_chunks):
             work(i)
     shape = (P, bs, Hk, D)
-    return (codes.reshape(shape), scales.reshape(P, bs, Hk),
+    return (codes.reshape((P, bs) + codes.shape[1:]), scales.reshape((P, bs) + scales.shape[1:]),
             None if raw is None else raw.reshape(shape))
 
 
@@ -403,3 +428,75 @@ def quest_meta_table(seq_lens, block_size: int, *, seed: int = 0, extra_blocks: 
         table[r, :n] = order[off:off + n]
         off += int(n)
     return table, total
+
+
+# ---------------------------------------------------------------- q4_0 caches
+
+
+@dataclass
+class WorkloadQ4:
+    """A workload whose cache is in the q4_0 format, drawn from the same random streams as
+    the q8 workload of the same Config (so the two hold the same unquantised values)."""
+    cfg: Config
+    q: np.ndarray  # fp32 [B][Hq][D]
+    k4: np.ndarray  # uint8 [P][bs][Hk][D/2]
+    v4: np.ndarray
+    kd: np.ndarray  # uint16 binary16 bits [P][bs][Hk][D/32]
+    vd: np.ndarray
+    block_table: np.ndarray
+    seq_lens: np.ndarray
+    scale: float
+    k32: np.ndarray | None = field(default=None, repr=False)
+    v32: np.ndarray | None = field(default=None, repr=False)
+
+    @property
+    def num_blocks(self) -> int:
+        return int(self.k4.shape[0])
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_table.shape[1])
+
+    def algorithmic_bytes(self) -> int:
+        """Every valid (token, KV head) K and V row (D/2 code bytes + 2 * D/32 scale bytes
+        each) once, q read and out written (fp32), the used block-table entries, seq_lens."""
+        c = self.cfg
+        L = self.seq_lens.astype(np.int64)
+        units = int(L.sum()) * c.n_kv_heads
+        nblk = int(((L + c.block_size - 1) // c.block_size).sum())
+        row = c.head_dim // 2 + 2 * (c.head_dim // 32)
+        return (units * 2 * row + c.B * c.n_q_heads * c.head_dim * 4 * 2 + 4 * nblk + 4 * c.B)
+
+
+def make_q4(cfg: Config | int, *, seq_lens=None, keep_fp32: bool = False,
+            threads: int | None = None) -> WorkloadQ4:
+    """The named (or given) workload with a q4_0 cache."""
+    if isinstance(cfg, int):
+        cfg = CONFIGS[cfg]
+    threads = threads or min(32, os.cpu_count() or 1)
+    seq_lens = _seq_lens(cfg) if seq_lens is None else np.asarray(seq_lens, np.int32)
+    bs, Hk, D = cfg.block_size, cfg.n_kv_heads, cfg.head_dim
+    need = int(((seq_lens.astype(np.int64) + bs - 1) // bs).sum())
+    P = max(1, need)
+    mbps = max(1, -(-int(seq_lens.max(initial=0)) // bs))
+    q = _rng(cfg.seed, _S_Q).standard_normal((cfg.B, cfg.n_q_heads, D), dtype=np.float32)
+    bias = None
+    if cfg.k_bias_std:
+        bias = (_rng(cfg.seed, _S_BIAS).standard_normal((Hk, D), dtype=np.float32)
+                * np.float32(cfg.k_bias_std))
+    k4, kd, k32 = _fill_pool(cfg.seed, _S_K, cfg.k_dist, P, bs, Hk, D, bias, keep_fp32,
+                             threads, q4=True)
+    v4, vd, v32 = _fill_pool(cfg.seed, _S_V, cfg.v_dist, P, bs, Hk, D, None, keep_fp32,
+                             threads, q4=True)
+    bt = build_block_table(seq_lens, bs, mbps, cfg.table, P, _rng(cfg.seed, _S_TABLE))
+    scale = float(np.float32(1.0) / np.float32(math.sqrt(D)))
+    return WorkloadQ4(cfg, q, k4, v4, kd, vd, bt, seq_lens.astype(np.int32), scale, k32, v32)
+
+
+def make_q4_custom(B, n_q_heads, n_kv_heads, head_dim, seq_lens, block_size, *,
+                   table="permutation", k_dist="normal", v_dist="normal", k_bias_std=0.0, seed=0,
+                   keep_fp32=False, name="custom_q4") -> WorkloadQ4:
+    seq_lens = np.asarray(seq_lens, np.int32).reshape(B)
+    cfg = Config(name, B, n_q_heads, n_kv_heads, head_dim, int(seq_lens.max(initial=0)),
+                 block_size, table, k_dist, v_dist, k_bias_std, seed)
+    return make_q4(cfg, seq_lens=seq_lens, keep_fp32=keep_fp32)

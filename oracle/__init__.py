@@ -58,6 +58,27 @@ class Cache(ctypes.Structure):
     ]
 
 
+class CacheQ4(ctypes.Structure):
+    """Mirror of ``q8kvo_cache_q4``."""
+
+    _fields_ = [
+        ("k4", ctypes.c_void_p),
+        ("v4", ctypes.c_void_p),
+        ("kd", ctypes.c_void_p),
+        ("vd", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+        ("B", ctypes.c_int),
+        ("n_q_heads", ctypes.c_int),
+        ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("block_size", ctypes.c_int),
+        ("max_blocks_per_seq", ctypes.c_int),
+        ("num_blocks", ctypes.c_int),
+        ("scale", ctypes.c_float),
+    ]
+
+
 def build_variant(mutant: int, out_path: str) -> str:
     """Compile the oracle with planted mistake ``mutant`` switched on (pin-strength test)."""
     subprocess.check_call(["gcc", *CFLAGS, f"-DQ8KVO_MUTANT={int(mutant)}", _SRC, "-o", out_path,
@@ -87,6 +108,10 @@ def _load():
                 "q8kvo_decode_multi": [cp, P, i, P],
                 "q8kvo_decode_multi_rows": [cp, P, i, P, l, P],
                 "q8kvo_quest_metadata": [cp, P, i, i, P, P],
+                "q8kvo_f32_to_f16": [P, l, P],
+                "q8kvo_quantize_q4_0": [P, l, P, P],
+                "q8kvo_decode_q4_all": [ctypes.POINTER(CacheQ4), P, P],
+                "q8kvo_decode_q4_pairs": [ctypes.POINTER(CacheQ4), P, P, l, P],
                 "q8kvo_cache_write": [P, P, P, P, P, P, P, l, i, i, i, i, l, P],
             }
             for name, args in sigs.items():
@@ -297,3 +322,58 @@ def cache_write(k, v, ks, vs, k_new, v_new, slot_mapping, token_stride=None) -> 
                                      _ptr(v_new), _ptr(slots), n, Hk, D, bs, P, stride,
                                      ctypes.byref(flags)), "cache_write")
     return int(flags.value)
+
+
+def f32_to_f16(x: np.ndarray) -> np.ndarray:
+    """binary16 bits (uint16) of fp32 values, round to nearest even."""
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _check(_load().q8kvo_f32_to_f16(_ptr(x), x.size, _ptr(out)), "f32_to_f16")
+    return out
+
+
+def quantize_q4_0(x: np.ndarray):
+    """q4_0 codes packed two per byte [..., n/2] and binary16 scales [..., n/32] of fp32
+    rows [..., n] (n a multiple of 32)."""
+    x = _c(x, np.float32)
+    n = x.shape[-1]
+    packed = np.empty(x.shape[:-1] + (n // 2,), np.uint8)
+    d16 = np.empty(x.shape[:-1] + (n // 32,), np.uint16)
+    _check(_load().q8kvo_quantize_q4_0(_ptr(x), x.size, _ptr(packed), _ptr(d16)), "quantize_q4_0")
+    return packed, d16
+
+
+class PagedCacheQ4:
+    """Host-side paged q4_0 KV cache handed to the oracle (keeps the arrays alive)."""
+
+    def __init__(self, k4, v4, kd, vd, block_table, seq_lens, n_q_heads, scale):
+        self.k4, self.v4 = _c(k4, np.uint8), _c(v4, np.uint8)
+        self.kd, self.vd = _c(kd, np.uint16), _c(vd, np.uint16)
+        self.block_table = _c(block_table, np.int32)
+        self.seq_lens = _c(seq_lens, np.int32)
+        P, bs, Hk, half = self.k4.shape
+        self.struct = CacheQ4(_ptr(self.k4), _ptr(self.v4), _ptr(self.kd), _ptr(self.vd),
+                              _ptr(self.block_table), _ptr(self.seq_lens),
+                              int(self.seq_lens.shape[0]), int(n_q_heads), int(Hk), 2 * int(half),
+                              int(bs), int(self.block_table.shape[1]), int(P),
+                              float(np.float32(scale)))
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def decode_q4_all(cache: PagedCacheQ4, q: np.ndarray) -> np.ndarray:
+    q = _c(q, np.float32)
+    s = cache.struct
+    out = np.zeros((s.B, s.n_q_heads, s.head_dim), np.float64)
+    _check(_load().q8kvo_decode_q4_all(cache.ref(), _ptr(q), _ptr(out)), "decode_q4_all")
+    return out
+
+
+def decode_q4_pairs(cache: PagedCacheQ4, q: np.ndarray, pairs) -> np.ndarray:
+    q = _c(q, np.float32)
+    pairs = _c(pairs, np.int32).reshape(-1, 2)
+    out = np.zeros((pairs.shape[0], cache.struct.head_dim), np.float64)
+    _check(_load().q8kvo_decode_q4_pairs(cache.ref(), _ptr(q), _ptr(pairs), pairs.shape[0],
+                                         _ptr(out)), "decode_q4_pairs")
+    return out

@@ -605,6 +605,233 @@ int q8kvo_quest_metadata(const q8kvo_cache *c, const int32_t *meta_table, int ma
     return Q8KVO_OK;
 }
 
+/* ---------------------------------------------------------------- q4_0 KV cache */
+
+/* IEEE binary16 from binary32, round to nearest even (written from the format definition:
+ * 1 sign bit, 5 exponent bits with bias 15, 10 fraction bits; subnormals below 2^-14). */
+static uint16_t f32_to_f16(float f)
+{
+    uint32_t x;
+    memcpy(&x, &f, 4);
+    uint32_t sign = (x >> 16) & 0x8000u;
+    uint32_t ax = x & 0x7fffffffu;
+    if (ax >= 0x7f800000u) /* inf or NaN */
+        return (uint16_t)(sign | 0x7c00u | (ax > 0x7f800000u ? 0x200u : 0u));
+    double a;
+    float af;
+    memcpy(&af, &ax, 4);
+    a = (double)af;
+    if (a >= 65520.0) /* rounds to infinity */
+        return (uint16_t)(sign | 0x7c00u);
+    int e;
+    frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+    int q = e - 1; /* a in [2^q, 2^(q+1)) */
+    if (q < -14)
+        q = -14; /* subnormal range: fixed spacing 2^-24 */
+    double step = ldexp(1.0, q - 10);
+    double n = a / step; /* exact: a power-of-two division */
+    double r = floor(n);
+    double frac = n - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))
+        r += 1.0;
+    double v = r * step; /* the rounded magnitude */
+    if (v >= 65520.0)
+        return (uint16_t)(sign | 0x7c00u);
+    uint32_t bits;
+    if (v < ldexp(1.0, -14)) {
+        bits = (uint32_t)(v / ldexp(1.0, -24)); /* subnormal fraction */
+    } else {
+        int ee;
+        double mm = frexp(v, &ee); /* v = mm * 2^ee, mm in [0.5, 1) */
+        bits = ((uint32_t)(ee - 1 + 15) << 10) | ((uint32_t)((mm * 2.0 - 1.0) * 1024.0) & 0x3ffu);
+    }
+    return (uint16_t)(sign | bits);
+}
+
+static double f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1, e = (h >> 10) & 0x1f, f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp(1.0 + f / 1024.0, e - 15);
+    return sign ? -v : v;
+}
+
+int q8kvo_f32_to_f16(const float *x, long n, uint16_t *out)
+{
+    if (!x || !out || n < 0)
+        return Q8KVO_EINVAL;
+    for (long i = 0; i < n; ++i)
+        out[i] = f32_to_f16(x[i]);
+    return Q8KVO_OK;
+}
+
+/* One 32-value block in the llama.cpp q4_0 format (baguaai.com FlashAttention page: the
+ * q4_0 / q8_0 quantised KV caches of llama.cpp; the format is llama.cpp's):
+ *   m    = the value of largest magnitude, sign kept (the first one on ties)
+ *   d    = m / -8                          (fp32)
+ *   id   = d != 0 ? 1 / d : 0              (fp32)
+ *   q_i  = min(15, trunc(x_i * id + 8.5))  (fp32 products and sums; 0 <= q_i <= 15)
+ *   stored: the 4-bit codes and d rounded to binary16; value = (q - 8) * d16.
+ * Codes are packed two per byte: channel 2i in the low nibble of byte i, 2i + 1 in the high
+ * nibble (this library's layout). */
+static void quantize_q4_block(const float *x, uint8_t *packed, uint16_t *d16)
+{
+    float amax = 0.0f, m = 0.0f;
+    for (int i = 0; i < 32; ++i)
+        if (fabsf(x[i]) > amax) {
+            amax = fabsf(x[i]);
+            m = x[i];
+        }
+    const float d = m / -8.0f;
+    const float id = d != 0.0f ? 1.0f / d : 0.0f;
+    for (int i = 0; i < 32; i += 2) {
+        int q[2];
+        for (int k = 0; k < 2; ++k) {
+            const float t = x[i + k] * id + 8.5f;
+            int qi = (int)t; /* trunc; t >= 0 */
+            q[k] = (qi > 15 && !MUT(27)) ? 15 : qi;
+        }
+        packed[i / 2] = (uint8_t)(MUT(24) ? (q[1] | (q[0] << 4)) : (q[0] | (q[1] << 4)));
+    }
+    *d16 = f32_to_f16(d);
+}
+
+int q8kvo_quantize_q4_0(const float *x, long n, uint8_t *packed, uint16_t *d16)
+{
+    if (!x || !packed || !d16 || n < 0 || (n % 32) != 0)
+        return Q8KVO_EINVAL;
+    for (long i = 0; i < n; ++i)
+        if (!isfinite(x[i]))
+            return Q8KVO_EINVAL;
+    for (long b = 0; b < n / 32; ++b)
+        quantize_q4_block(x + 32 * b, packed + 16 * b, d16 + b);
+    return Q8KVO_OK;
+}
+
+static int q4_code(const uint8_t *row, int i)
+{
+    const uint8_t byte = row[i / 2];
+    return (int)((i & 1) ? (byte >> 4) : (byte & 0x0f)) - (MUT(25) ? 0 : 8);
+}
+
+static int check_q4(const q8kvo_cache_q4 *c)
+{
+    if (!c || !c->k4 || !c->v4 || !c->kd || !c->vd || !c->block_table || !c->seq_lens)
+        return Q8KVO_EINVAL;
+    if (c->B <= 0 || c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+        (c->head_dim % 32) != 0 || c->block_size <= 0 || c->max_blocks_per_seq <= 0 ||
+        c->num_blocks <= 0 || (c->n_q_heads % c->n_kv_heads) != 0 || !isfinite(c->scale))
+        return Q8KVO_EINVAL;
+    return Q8KVO_OK;
+}
+
+/* Decode of one (b, h) over a q4_0 cache, walk-through section 2 with the q4_0 blocks:
+ *   dot_j = sum_{i in block j} qi_i * (code_i - 8)               (int32, exact)
+ *   s_t   = (sum_j dot_j * qsc_j * dk_j) * scale                 (fp64)
+ *   online softmax as for the q8 cache, acc[d] += w * dv_{j(d)} * (code_d - 8). */
+static int decode_q4_row(const q8kvo_cache_q4 *c, const float *q, int b, int h, double *out,
+                         int8_t *qi, float *qsc, double *acc)
+{
+    const int D = c->head_dim, nb = D / 32, Hk = c->n_kv_heads;
+    const int kvh = h / (c->n_q_heads / Hk);
+    int L = c->seq_lens[b];
+    if (L < 0 || (long)L > (long)c->max_blocks_per_seq * c->block_size)
+        return Q8KVO_ERANGE;
+    int rc = q8kvo_quantize_q(q + ((long)b * c->n_q_heads + h) * D, D, qi, qsc);
+    if (rc)
+        return rc;
+    double M = -INFINITY, S = 0.0;
+    for (int d = 0; d < D; ++d)
+        acc[d] = 0.0;
+    for (int t = 0; t < L; ++t) {
+        const int blk = c->block_table[(long)b * c->max_blocks_per_seq + t / c->block_size];
+        if (blk < 0 || blk >= c->num_blocks)
+            return Q8KVO_ERANGE;
+        const long row = ((long)blk * c->block_size + t % c->block_size) * Hk + kvh;
+        const uint8_t *krow = c->k4 + row * (D / 2);
+        const uint8_t *vrow = c->v4 + row * (D / 2);
+        const uint16_t *kd = c->kd + row * nb, *vd = c->vd + row * nb;
+        double s = 0.0;
+        for (int j = 0; j < nb; ++j) {
+            int32_t dot = 0;
+            for (int i = 32 * j; i < 32 * j + 32; ++i)
+                dot += (int32_t)qi[i] * q4_code(krow, i);
+            s += (double)dot * (double)qsc[j] * f16_to_f64(kd[MUT(26) ? 0 : j]);
+        }
+        s *= (double)c->scale;
+        double w;
+        if (s > M) {
+            const double f = exp(M - s);
+            S *= f;
+            for (int d = 0; d < D; ++d)
+                acc[d] *= f;
+            M = s;
+            w = 1.0;
+        } else {
+            w = exp(s - M);
+        }
+        S += w;
+        for (int d = 0; d < D; ++d)
+            acc[d] += w * f16_to_f64(vd[d / 32]) * (double)q4_code(vrow, d);
+    }
+    for (int d = 0; d < D; ++d)
+        out[d] = L > 0 ? acc[d] / S : 0.0;
+    return Q8KVO_OK;
+}
+
+int q8kvo_decode_q4_pairs(const q8kvo_cache_q4 *c, const float *q, const int32_t *pairs, long n,
+                          double *out)
+{
+    int rc = check_q4(c);
+    if (rc)
+        return rc;
+    if (!q || !pairs || !out || n < 0)
+        return Q8KVO_EINVAL;
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    for (long r = 0; r < n && rc == Q8KVO_OK; ++r) {
+        const int b = pairs[2 * r], h = pairs[2 * r + 1];
+        if (b < 0 || b >= c->B || h < 0 || h >= c->n_q_heads)
+            rc = Q8KVO_EINVAL;
+        else
+            rc = decode_q4_row(c, q, b, h, out + r * c->head_dim, qi, qsc, acc);
+    }
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
+int q8kvo_decode_q4_all(const q8kvo_cache_q4 *c, const float *q, double *out)
+{
+    int rc = check_q4(c);
+    if (rc)
+        return rc;
+    if (!q || !out)
+        return Q8KVO_EINVAL;
+    int8_t *qi;
+    float *qsc;
+    double *acc;
+    if ((rc = scratch_alloc(c->head_dim, &qi, &qsc, &acc)))
+        return rc;
+    for (int b = 0; b < c->B && rc == Q8KVO_OK; ++b)
+        for (int h = 0; h < c->n_q_heads && rc == Q8KVO_OK; ++h)
+            rc = decode_q4_row(c, q, b, h, out + ((long)b * c->n_q_heads + h) * c->head_dim, qi,
+                               qsc, acc);
+    free(qi);
+    free(qsc);
+    free(acc);
+    return rc;
+}
+
 /* ---------------------------------------------------------------- three pass */
 
 /* The naive form the walk-through (section 3) contrasts with, laid out like the

@@ -134,6 +134,43 @@ int q8kvo_decode_multi_rows(const q8kvo_cache *c, const float *q, int n_queries,
 int q8kvo_quest_metadata(const q8kvo_cache *c, const int32_t *meta_table, int max_meta_per_seq,
                          int num_meta_blocks, float *maxb, float *minb);
 
+/* A paged q4_0 KV cache (llama.cpp's q4_0 blocks, this library's packing):
+ *   k4, v4   uint8  [num_blocks][block_size][n_kv_heads][head_dim / 2]  two 4-bit codes per
+ *            byte: channel 2i in the low nibble of byte i, 2i + 1 in the high nibble
+ *   kd, vd   binary16 bits [num_blocks][block_size][n_kv_heads][head_dim / 32]: the scale d
+ *            of each 32-channel block; value = (code - 8) * d
+ * Other fields as q8kvo_cache. */
+typedef struct {
+    const uint8_t *k4;
+    const uint8_t *v4;
+    const uint16_t *kd;
+    const uint16_t *vd;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    int B;
+    int n_q_heads;
+    int n_kv_heads;
+    int head_dim;
+    int block_size;
+    int max_blocks_per_seq;
+    int num_blocks;
+    float scale;
+} q8kvo_cache_q4;
+
+/* binary16 bits of n fp32 values, round to nearest even. */
+int q8kvo_f32_to_f16(const float *x, long n, uint16_t *out);
+
+/* q4_0 quantisation of n fp32 values (n a multiple of 32): packed [n / 2] codes and
+ * d16 [n / 32] binary16 scales (rule in q8kv_oracle.c). */
+int q8kvo_quantize_q4_0(const float *x, long n, uint8_t *packed, uint16_t *d16);
+
+/* Single-query decode over a q4_0 cache (fp64 out [B][n_q_heads][head_dim], or the chosen
+ * (b, h) pairs): the query quantisation and the online softmax of the q8 decode, with
+ * the K and V values (code - 8) * d of their 32-channel blocks. */
+int q8kvo_decode_q4_all(const q8kvo_cache_q4 *c, const float *q, double *out);
+int q8kvo_decode_q4_pairs(const q8kvo_cache_q4 *c, const float *q, const int32_t *pairs, long n,
+                          double *out);
+
 /* Naive three-pass variant (all scores, then max, then exp/sum, then weighted V). */
 int q8kvo_decode_threepass(const q8kvo_cache *c, const float *q, int b, int h, double *out);
 
