@@ -57,6 +57,8 @@ def parse():
                     help="skip the multi-query decode information report")
     ap.add_argument("--no-quest", action="store_true",
                     help="skip the QUEST block-metadata information report")
+    ap.add_argument("--no-q4", action="store_true",
+                    help="skip the q4_0-cache decode information report")
     ap.add_argument("--accuracy-study", action="store_true",
                     help="instead of timing: the q8-vs-fp32 output error study over the "
                          "workloads and K/V distributions (one JSON line)")
@@ -570,6 +572,8 @@ def main():
         # per sequence (speculative decode), through q8kv_decode_attn_multi
         line["multi_query"] = bench_multi_query(w, pools, bt, lens, dev, stream,
                                                 steps=max(10, min(args.steps, 2000)))
+    if not args.no_q4:
+        line["q4_0_decode"] = bench_q4(dev, stream, steps=max(10, min(args.steps, 2000)))
     if not args.no_cache_write or not args.no_quest:
         del pools, argsets
         torch.cuda.empty_cache()
@@ -732,6 +736,56 @@ def bench_quest(dev, stream, steps=20, warmup=3, B=20, L=32768, Hk=8, bs=128):
                          "traffic": recorded_traffic("quest_b20_l32768", "quest"),
                          "kernel": "q8kv::quest_metadata_kernel"},
             "device_errors": q8.q8kv_device_errors(clear=True)}
+
+
+def bench_q4(dev, stream, steps=2000, warmup=20):
+    """Information: q8kv_decode_attn_q4 on the benchmark's 16 x 4096-token GQA workload with
+    a q4_0 cache drawn from the same random streams (pool rotated over copies larger than
+    the L2, back-to-back calls between two events)."""
+    import numpy as np
+    import torch
+
+    import decode_attention_int8_b200 as q8
+    from decode_attention_int8_b200 import inputs
+
+    w = inputs.make_q4(1)
+    c = w.cfg
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    pool_bytes = w.k4.nbytes + w.v4.nbytes + w.kd.nbytes + w.vd.nbytes
+    n_copies = max(2, math.ceil(4 * L2_BYTES / pool_bytes) + 1)
+    pools = [(t(w.k4), t(w.v4), t(w.kd.view(np.float16)), t(w.vd.view(np.float16)))
+             for _ in range(n_copies)]
+    q, bt, lens = t(w.q), t(w.block_table), t(w.seq_lens)
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    q8.q8kv_decode_attn_q4(out, q, *pools[0], bt, lens, w.scale, stream=stream)
+    fn = q8.lib().q8kv_decode_attn_q4
+    P_ = lambda x: ctypes.c_void_p(x.data_ptr())
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    args = [(P_(out), P_(q), P_(k), P_(v), P_(kd), P_(vd), P_(bt), P_(lens), c.B, c.n_q_heads,
+             c.n_kv_heads, c.head_dim, c.block_size, w.max_blocks_per_seq, w.num_blocks,
+             ctypes.c_float(w.scale), sp) for (k, v, kd, vd) in pools]
+    for i in range(warmup):
+        fn(*args[i % n_copies])
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        st = fn(*args[i % n_copies])
+        if st != 0:
+            raise q8.Q8KVError(st, "q8kv_decode_attn_q4")
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    algo = w.algorithmic_bytes()
+    peak, peak_kind = measured_peak()
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"workload": f"{c.name} with a q4_0 cache ({algo / 1e6:.1f} MB per call)",
+            "us_per_call": round(ms * 1e3, 3), "calls": steps, "algorithmic_bytes": algo,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                         "kernel": "q8kv::q4_decode_kernel + q8kv::q4_combine_kernel"},
+            "l2": f"pool rotated over {n_copies} copies"}
 
 
 def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):

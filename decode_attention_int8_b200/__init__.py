@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     q8kv_debug_quantize_q,
     q8kv_decode_attn,
     q8kv_decode_attn_multi,
+    q8kv_decode_attn_q4,
     q8kv_decode_attn_static,
     q8kv_decode_attn_ws,
     q8kv_quest_metadata,

@@ -28,6 +28,7 @@ DEVERR_META = 0x20
 EXPORTS = (
     "q8kv_decode_attn",
     "q8kv_decode_attn_multi",
+    "q8kv_decode_attn_q4",
     "q8kv_workspace_bytes",
     "q8kv_workspace_init",
     "q8kv_decode_attn_ws",
@@ -69,6 +70,7 @@ def lib():
             sig = {
                 "q8kv_decode_attn": ([P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_decode_attn_multi": ([P] * 8 + [I] * 8 + [F, P], I),
+                "q8kv_decode_attn_q4": ([P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_workspace_bytes": ([I, I, I, I], Z),
                 "q8kv_workspace_init": ([P, Z, P], I),
                 "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
@@ -162,6 +164,34 @@ def q8kv_decode_attn_multi(out, q, k_blocks, v_blocks, kscale, vscale, block_tab
                                         _ptr(kscale), _ptr(vscale), _ptr(block_table),
                                         _ptr(seq_lens), geo[0], nq, *geo[1:], float(scale),
                                         _stream(stream)), "q8kv_decode_attn_multi")
+    return out
+
+
+def q8kv_decode_attn_q4(out, q, k4_blocks, v4_blocks, kd, vd, block_table, seq_lens, scale,
+                        stream=None):
+    """Decode attention over a q4_0 cache: k4/v4 uint8 [P][bs][Hk][D/2] (two codes per byte,
+    channel 2i in the low nibble), kd/vd binary16 [P][bs][Hk][D/32] (torch.float16, or
+    16-bit integers holding the bits); q, out fp32 [B][Hq][D]."""
+    _need(out, "out", torch.float32, 3)
+    _need(q, "q", torch.float32, 3)
+    _need(k4_blocks, "k4_blocks", torch.uint8, 4)
+    _need(v4_blocks, "v4_blocks", torch.uint8, 4)
+    for t, name in ((kd, "kd"), (vd, "vd")):
+        if t.dtype not in (torch.float16, torch.int16, torch.uint16) or t.dim() != 4 or \
+                not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous CUDA 16-bit tensor with 4 dims")
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    P, bs, Hk, half = k4_blocks.shape
+    if tuple(out.shape) != (B, Hq, D) or 2 * half != D or tuple(v4_blocks.shape) != (P, bs, Hk, half):
+        raise ValueError("q/out/k4/v4 shapes disagree")
+    if tuple(kd.shape) != (P, bs, Hk, D // 32) or tuple(vd.shape) != (P, bs, Hk, D // 32):
+        raise ValueError("kd/vd must be [num_blocks][block_size][n_kv_heads][head_dim/32]")
+    _check(lib().q8kv_decode_attn_q4(_ptr(out), _ptr(q), _ptr(k4_blocks), _ptr(v4_blocks),
+                                     _ptr(kd), _ptr(vd), _ptr(block_table), _ptr(seq_lens), B,
+                                     Hq, Hk, D, bs, int(block_table.shape[1]), P, float(scale),
+                                     _stream(stream)), "q8kv_decode_attn_q4")
     return out
 
 

@@ -739,3 +739,6 @@ int q8kv_version(void)
 
 // The QUEST block-metadata entry point.
 #include "q8kv_quest_api.cuh"
+
+// The q4_0-cache decode entry point.
+#include "q8kv_q4_api.cuh"

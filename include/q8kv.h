@@ -139,6 +139,30 @@ q8kv_status q8kv_decode_attn_multi(float *out, const float *q, const int8_t *k_b
                                    int max_blocks_per_seq, int num_kv_blocks, float scale,
                                    cudaStream_t stream);
 
+/*
+ * Decode attention over a q4_0 KV cache (llama.cpp's q4_0 blocks, one of the quantised
+ * KV-cache types of the llama.cpp change on baguaai.com's FlashAttention page),
+ * library-managed workspace:
+ *   k4_blocks, v4_blocks  uint8 [num_kv_blocks][kv_block_size][n_kv_heads][head_dim / 2]:
+ *                         4-bit codes, channel 2i in the low nibble of byte i, 2i + 1 in
+ *                         the high nibble
+ *   kd, vd                binary16 bits [num_kv_blocks][kv_block_size][n_kv_heads]
+ *                         [head_dim / 32]: the scale d of each 32-channel block
+ * The value of channel c of a row is (code_c - 8) * d_(c / 32). With the query quantised
+ * as in step 1 above, token t scores
+ *   s_t = (sum_j dot_j * qsc_j * dk_tj) * scale,  dot_j = sum over block j of qi * (code - 8)
+ * (exact int32), and out is the online-softmax average of the V values. Other arguments,
+ * layouts and asynchrony as q8kv_decode_attn; kd and vd must be 8-byte aligned. Supported:
+ * head_dim 128; group n_q_heads / n_kv_heads <= 16; B * n_kv_heads <= 65535. Two kernel
+ * launches (per chunk of 256 tokens, then a merge of the chunks).
+ */
+q8kv_status q8kv_decode_attn_q4(float *out, const float *q, const uint8_t *k4_blocks,
+                                const uint8_t *v4_blocks, const uint16_t *kd,
+                                const uint16_t *vd, const int32_t *block_table,
+                                const int32_t *seq_lens, int B, int n_q_heads, int n_kv_heads,
+                                int head_dim, int kv_block_size, int max_blocks_per_seq,
+                                int num_kv_blocks, float scale, cudaStream_t stream);
+
 /* Bytes of workspace q8kv_decode_attn_ws needs for these sizes on the current device
  * (0 if the sizes are invalid or unsupported). */
 size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim);

@@ -150,3 +150,25 @@ def test_quest_metadata_bad_arguments_rejected():
     odd = list(sizes)
     odd[2] = 64
     assert L.q8kv_quest_metadata(*ptrs, *odd, None) == UNSUPPORTED
+
+
+def test_q4_decode_bad_arguments_rejected():
+    L = q8.lib()
+    P = ctypes.c_void_p
+    ptrs = [P(0x10000 * i) for i in range(1, 9)]
+    sizes = [2, 8, 2, 128, 16, 4, 8]  # B, Hq, Hk, D, bs, mbps, P
+    for i in range(8):
+        bad = list(ptrs)
+        bad[i] = None
+        assert L.q8kv_decode_attn_q4(*bad, *sizes, 0.1, None) == INVALID
+    for i in range(7):
+        bad = list(sizes)
+        bad[i] = 0
+        assert L.q8kv_decode_attn_q4(*ptrs, *bad, 0.1, None) == INVALID
+    assert L.q8kv_decode_attn_q4(*ptrs, 2, 9, 2, 128, 16, 4, 8, 0.1, None) == INVALID
+    assert L.q8kv_decode_attn_q4(*ptrs, *sizes, float("nan"), None) == INVALID
+    odd = list(ptrs)
+    odd[4] = P(0x50004)  # kd not 8-byte aligned
+    assert L.q8kv_decode_attn_q4(*odd, *sizes, 0.1, None) == INVALID
+    assert L.q8kv_decode_attn_q4(*ptrs, 2, 8, 2, 64, 16, 4, 8, 0.1, None) == UNSUPPORTED
+    assert L.q8kv_decode_attn_q4(*ptrs, 2, 34, 2, 128, 16, 4, 8, 0.1, None) == UNSUPPORTED
