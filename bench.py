@@ -296,7 +296,7 @@ def accuracy_rows(w, out_gpu, n_rows, seed, max_seqs=8):
 
 
 def run_accuracy_study(args):
-    """Survey row f2 (the walk-through's announced q8-vs-fp32 comparison): how far the q8
+    """The q8-vs-fp32 comparison the walk-through announces as its next article: how far the q8
     path's attention output is from attention over the unquantised fp32 data, per workload
     and per K/V distribution, for the CUDA kernel and for the oracle's q8 arithmetic."""
     import numpy as np
