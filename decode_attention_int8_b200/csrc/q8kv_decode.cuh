@@ -66,12 +66,15 @@ constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull; // 1 s per pipeline wait
 constexpr int kSlotRow = kD + 4;    // per-head partial: kD accumulator floats, M, S, A, pad
 // Work split: a segment that starts in the middle of a CTA's range costs that CTA about
-// three tiles' time (the finished segment's accumulators are folded, reduced and written
-// and the next query is set up, by code that runs once and is fetched cold while the K/V
-// stream loads the memory system). The split therefore charges every segment start
-// kSegPenaltyTiles extra tiles, when the batch is small enough to keep the count of
-// sequences with tokens in shared memory and every CTA gets well over that many tiles.
-constexpr int kSegPenaltyTiles = 3;
+// four to five tiles' time (the finished segment's accumulators are folded, reduced and
+// written and the next query is set up, by code that runs once and is fetched cold while
+// the K/V stream loads the memory system; per-CTA timestamps on the 16 x 4096-token
+// workload put the CTAs that switch segments 2-3 us behind the others when charged three
+// tiles). The split therefore charges every segment start kSegPenaltyTiles extra tiles,
+// when the batch is small enough to keep the count of sequences with tokens in shared
+// memory and every CTA's share is at least twice that (so that no share fits inside one
+// segment's charge, which would leave a CTA without tiles in the middle of a segment).
+constexpr int kSegPenaltyTiles = 5;
 constexpr int kPenaltyMaxB = 2048;
 constexpr int kDotBias = 0x4B400000;    // bit pattern of 1.5 * 2^23
 constexpr float kDotBiasF = 12582912.0f; // 1.5 * 2^23
@@ -1502,12 +1505,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *cstart = reinterpret_cast<int *>(smem + p.lay.off_cstart);
     const int gcta = N < (int)gridDim.x ? N : (int)gridDim.x;
     // Work split (see kSegPenaltyTiles): penalised when the sequence counts are at hand and
-    // every CTA's share is at least 4 penalties, so that no CTA's share can fall inside one
+    // every CTA's share is at least 2 penalties, so that no CTA's share can fall inside one
     // segment's penalty (an empty CTA in the middle of a split segment would break the
     // contributor numbering). Only this CTA's own range is computed before the producer
     // starts; the consumers fill in the rest of the table (needed at segment ends).
     const int nseg_units = nseq ? kSegPenaltyTiles * p.nhc * nseq[p.B] : 0;
-    const bool pen = nseq && gcta > 0 && (N + nseg_units) / gcta >= 4 * kSegPenaltyTiles;
+    const bool pen = nseq && gcta > 0 && (N + nseg_units) / gcta >= 2 * kSegPenaltyTiles;
     const int pseg = pen ? kSegPenaltyTiles * p.nhc : 0;
     const int V = N + (pen ? nseg_units : 0);
     if (gcta == 0) { // no sequence has tokens: every row is zero
