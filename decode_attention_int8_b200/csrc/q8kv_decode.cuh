@@ -18,13 +18,13 @@
 //    policy) and the scales with bulk copies into an n-stage ring guarded by mbarriers.
 //  * Warps 0-7 consume: each owns (KV head, 16-head slice of its query group, 16-token
 //    subtile). QK is an int8 tensor-core MMA (m16n8k32, one MMA per 32-channel quant
-//    block, so each MMA result is exactly one int32 block dot). PV is an f16 MMA
-//    (m16n8k16) on exact f16 copies of the int8 V codes with the fp32 weights split into
-//    hi + lo f16 halves (about 22 significant bits).
-//  * The online softmax runs per 16-token subtile in base 2. The denominator S keeps the
-//    softmax running max M; the V accumulator keeps its own running max A of
-//    (score + log2 V scale), so the weight * V scale that enters the f16 halves is at
-//    most 2^15 and the largest one is at least 2^14 (full f16 precision whatever the
+//    block, so each MMA result is exactly one int32 block dot). PV is an int8 x u8
+//    tensor-core MMA too: V^T straight from the swizzled tile through ldmatrix .trans, and
+//    the weights as exact 23-bit integers split into byte planes (one n-tile each).
+//  * The online softmax runs per stage in base 2. The denominator S keeps the softmax
+//    running max M; the V accumulator keeps its own running max A of
+//    (score + log2 V scale), so the integer weight w * vs * 2^(M - A + 8) is below 2^23
+//    and the largest one of a stage is at least 2^22 (22 significant bits whatever the
 //    spread of the V scales). Both are ordinary online maxima: rescale when they rise.
 //  * Per-warp states are merged in shared memory. A segment that one CTA covers whole is
 //    normalised and written out here; a CTA that covers only part of one leaves its
@@ -605,7 +605,6 @@ __device__ __forceinline__ void reset_state(WarpState<NT> &st)
 // (1024 bytes) further on and has the same 128-byte swizzle phase.
 struct ThreadOffsets {
     uint32_t k[kSub][kNB]; // K fragment (subtile u, quant block j) of tokens 0-7; 8-15: +1024
-    uint32_t v[kSub][2];   // V row of token 2c + e (e = 0, 1); token 2c + e + 8: +1024
     uint32_t s[kSub][2][2]; // K scale of token (u, nt, e) at column kl (add the segment's
                             // column offset); its V scale is sc_gap further
 };
@@ -624,11 +623,6 @@ __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int
         for (int j = 0; j < kNB; ++j)
             o.k[u][j] = p.lay.off_k + rk * 128 + ((((2 * j) | (c >> 1)) ^ g) << 4) +
                         ((c & 1) << 3);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int rv = row_kv(t0 + 2 * c + e); // row & 7 == 2c + e
-            o.v[u][e] = p.lay.off_v + rv * 128 + ((g ^ (2 * c + e)) << 4);
-        }
         // scales sit token-major ([token][head]) in stage token order
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -637,229 +631,6 @@ __device__ __forceinline__ ThreadOffsets make_offsets(const DecodeParams &p, int
                 o.s[u][nt][e] = p.lay.off_ks + 4 * ((t0 + nt * 8 + 2 * c + e) * p.sc_heads + kl);
     }
     return o;
-}
-
-__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
-{
-    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
-
-// One stage: kSub 16-token subtiles of one KV head for this warp, folded into the online
-// softmax as one block. sb: shared address of the stage; tl0: stage-local index of this
-// thread's first token; vmask: bit k set when token k of the warp's 32-token window holds
-// data (clear past the sequence end and in blocks that were not loaded).
-template <int NT, bool kPack, bool kDump>
-__device__ __forceinline__ void process_stage(const DecodeParams &p, WarpState<NT> &st,
-                                              const ThreadOffsets &o, uint32_t sb,
-                                              uint32_t sbs, int tl0,
-                                              uint32_t vmask, bool causal, const int (&lim)[NT],
-                                              float scale_log2, int b, int hc, int kl,
-                                              int slice, int tok0, int g, int c)
-{
-    // ---- V rows first: their int8 -> f16 conversion overlaps the softmax chain below
-    uint4 R[kSub][4];
-#pragma unroll
-    for (int u = 0; u < kSub; ++u)
-#pragma unroll
-        for (int qv = 0; qv < 4; ++qv)
-            R[u][qv] = lds128(sb + o.v[u][qv & 1] + (qv >> 1) * 1024);
-    // ---- scores: int8 MMA per quant block, exact int32 block dots. The four block MMAs of
-    // an 8-token group accumulate into one int32 register set that starts at the bit
-    // pattern of 1.5 * 2^23, so after block j it holds 1.5 * 2^23 + dot_0 + ... + dot_j
-    // (|sum| <= 4 * 32 * 127 * 127 < 2^22): read as fp32 every partial sum is exact, and
-    // dot_j is the exact difference of two consecutive ones.
-    float s[NT][kSub][2][2];
-#pragma unroll
-    for (int r = 0; r < NT; ++r)
-#pragma unroll
-        for (int u = 0; u < kSub; ++u)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-                s[r][u][nt][0] = s[r][u][nt][1] = 0.f;
-#pragma unroll
-    for (int u = 0; u < kSub; ++u) {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            int prev[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
-#pragma unroll
-            for (int j = 0; j < kNB; ++j) {
-                const uint2 kk = lds64(sb + o.k[u][j] + nt * 1024);
-                int d[4];
-                mma_s8_16832_acc(d, st.qa[j][0], NT == 2 ? st.qa[j][1] : 0u, st.qa[j][2],
-                                 NT == 2 ? st.qa[j][3] : 0u, kk.x, kk.y, prev);
-                if constexpr (kDump) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int r = q >> 1, e = q & 1;
-                        const int hg = kPack ? g : slice * 16 + r * 8 + g;
-                        const bool row_ok = kPack ? (r == 0 && g < 4) : (r < NT);
-                        const int tl = tl0 + u * 16 + nt * 8 + e;
-                        if (row_ok && hg < p.G && ((vmask >> (tl - tl0 + 2 * c)) & 1u)) {
-                            const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
-                            p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) *
-                                           kNB +
-                                       j] = d[q] - prev[q];
-                        }
-                    }
-                }
-                s[0][u][nt][0] += (__int_as_float(d[0]) - __int_as_float(prev[0])) * st.qs[0][j];
-                s[0][u][nt][1] += (__int_as_float(d[1]) - __int_as_float(prev[1])) * st.qs[0][j];
-                if constexpr (NT == 2) {
-                    s[NT - 1][u][nt][0] +=
-                        (__int_as_float(d[2]) - __int_as_float(prev[2])) * st.qs[NT - 1][j];
-                    s[NT - 1][u][nt][1] +=
-                        (__int_as_float(d[3]) - __int_as_float(prev[3])) * st.qs[NT - 1][j];
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    prev[q] = d[q];
-            }
-        }
-    }
-    // ---- per-token K and V scales (the K scale carries the softmax scale and log2 e)
-    float kss[kSub][2][2], vsv[kSub][2][2];
-#pragma unroll
-    for (int u = 0; u < kSub; ++u)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                kss[u][nt][e] = lds_f32(sbs + o.s[u][nt][e]) * scale_log2;
-                vsv[u][nt][e] = lds_f32(sbs + o.s[u][nt][e] + p.lay.sc_gap);
-            }
-    // masked tokens (rare: a segment's last tile, bad block-table entries) get score -inf
-    // and V scale 0, whatever stale data their slots hold; with several queries per
-    // sequence, a token after a row's own position gets score -inf in that row only
-    if (vmask != 0xffffffffu || causal) {
-#pragma unroll
-        for (int u = 0; u < kSub; ++u)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int j = u * 16 + nt * 8 + 2 * c + e;
-                    if (!((vmask >> j) & 1u)) {
-#pragma unroll
-                        for (int r = 0; r < NT; ++r)
-                            s[r][u][nt][e] = -INFINITY;
-                        kss[u][nt][e] = 1.f;
-                        vsv[u][nt][e] = 0.f;
-                    } else {
-#pragma unroll
-                        for (int r = 0; r < NT; ++r)
-                            if (j >= lim[r])
-                                s[r][u][nt][e] = -INFINITY;
-                    }
-                }
-    }
-    // ---- online softmax (base 2), blockwise over the stage's tokens. M: running max of the
-    // scores (denominator). A: running max of log2 of the numerator terms w * vs (relative to
-    // 2^M) minus 14, so that every w * vs * 2^(M - A) entering the f16 MMA is below 2^15 and
-    // the largest one is at least 2^14; A >= M - 114 keeps 2^(M - A) finite.
-    float alpha_a[NT];
-    uint32_t bh[NT][kSub][2], bl[NT][kSub][2];
-#pragma unroll
-    for (int r = 0; r < NT; ++r) {
-        float m = -INFINITY;
-#pragma unroll
-        for (int u = 0; u < kSub; ++u)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float v = s[r][u][nt][e] * kss[u][nt][e];
-                    s[r][u][nt][e] = v;
-                    m = fmaxf(m, v);
-                }
-        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
-        const float mn = fmaxf(st.M[r], m);
-        const float ms = (mn == -INFINITY) ? 0.f : mn;
-        const float alpha_s = fast_exp2(st.M[r] - ms);
-        st.M[r] = mn;
-        float ws = 0.f, pmax = 0.f;
-        float w[kSub][2][2];
-#pragma unroll
-        for (int u = 0; u < kSub; ++u)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float x = fast_exp2(s[r][u][nt][e] - ms);
-                    ws += x;
-                    w[u][nt][e] = x * vsv[u][nt][e];
-                    pmax = fmaxf(pmax, w[u][nt][e]);
-                }
-        st.S[r] = st.S[r] * alpha_s + ws;
-        pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 1));
-        pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 2));
-        // floor(log2 pmax) from the exponent field (pmax = 0 gives -127)
-        const float an_stage = ms + exponent_as_float(pmax) - 14.f;
-        const float an =
-            (mn == -INFINITY) ? -INFINITY : fmaxf(fmaxf(st.A[r], an_stage), mn - 114.f);
-        const float as = (an == -INFINITY) ? 0.f : an;
-        alpha_a[r] = fast_exp2(st.A[r] - as);
-        st.A[r] = an;
-        const float cvs = fast_exp2(ms - as); // 2^(M - A), at most 2^114
-        // weights as split f16 B operands (column n = head g, k = token)
-#pragma unroll
-        for (int u = 0; u < kSub; ++u)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const float p0 = w[u][nt][0] * cvs, p1 = w[u][nt][1] * cvs;
-                const __half2 h = __floats2half2_rn(p0, p1);
-                const float r0 = p0 - __low2float(h), r1 = p1 - __high2float(h);
-                bh[r][u][nt] = *reinterpret_cast<const uint32_t *>(&h);
-                bl[r][u][nt] = pack_f16x2(r0, r1);
-            }
-    }
-    // ---- rescale factors of the accumulator columns (in packed mode rows 4-7 repeat rows
-    // 0-3, so the source lane of column col carries head col & 3 either way)
-    float f0[NT], f1[NT];
-#pragma unroll
-    for (int pv = 0; pv < NT; ++pv) {
-        f0[pv] = __shfl_sync(kFullMask, alpha_a[pv], 8 * c);
-        f1[pv] = __shfl_sync(kFullMask, alpha_a[pv], 8 * c + 4);
-    }
-    // ---- PV: rows = channels 16g + 2i (+1), k = tokens, columns = heads (packed mode:
-    // columns 0-3 high halves of heads 0-3, columns 4-7 their low halves). The stage's
-    // products are summed in a fresh tensor-core accumulator and folded into the running
-    // one with one round-to-nearest FFMA (which also applies the rescale factor): the
-    // tensor-core accumulation does not round to nearest, so chaining every stage of a
-    // long scan through it would let its error grow with the scan length.
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float d[NT][4];
-#pragma unroll
-        for (int u = 0; u < kSub; ++u) {
-            const uint32_t w0 = word_of(R[u][0], i >> 1), w1 = word_of(R[u][1], i >> 1);
-            const uint32_t w2 = word_of(R[u][2], i >> 1), w3 = word_of(R[u][3], i >> 1);
-            const uint32_t sl = (i & 1) ? 0x0602u : 0x0400u;
-            const uint32_t sh = (i & 1) ? 0x0703u : 0x0501u;
-            const uint32_t a0 = s8pair_to_f16x2(prmt(w0, w1, sl));
-            const uint32_t a1 = s8pair_to_f16x2(prmt(w0, w1, sh));
-            const uint32_t a2 = s8pair_to_f16x2(prmt(w2, w3, sl));
-            const uint32_t a3 = s8pair_to_f16x2(prmt(w2, w3, sh));
-#pragma unroll
-            for (int pv = 0; pv < NT; ++pv) {
-                const uint32_t b0 = (kPack && g >= 4) ? bl[pv][u][0] : bh[pv][u][0];
-                const uint32_t b1 = (kPack && g >= 4) ? bl[pv][u][1] : bh[pv][u][1];
-                if (u == 0)
-                    mma_f16_16816_zero_c(d[pv], a0, a1, a2, a3, b0, b1);
-                else
-                    mma_f16_16816(d[pv], a0, a1, a2, a3, b0, b1);
-                if constexpr (!kPack)
-                    mma_f16_16816(d[pv], a0, a1, a2, a3, bl[pv][u][0], bl[pv][u][1]);
-            }
-        }
-#pragma unroll
-        for (int pv = 0; pv < NT; ++pv) {
-            st.acc[pv][i][0] = fmaf(st.acc[pv][i][0], f0[pv], d[pv][0]);
-            st.acc[pv][i][1] = fmaf(st.acc[pv][i][1], f1[pv], d[pv][1]);
-            st.acc[pv][i][2] = fmaf(st.acc[pv][i][2], f0[pv], d[pv][2]);
-            st.acc[pv][i][3] = fmaf(st.acc[pv][i][3], f1[pv], d[pv][3]);
-        }
-    }
 }
 
 // ------------------------------------------------------------------ packed path (group <= 4)
@@ -1113,26 +884,207 @@ __device__ __forceinline__ void process_stage_packed(const DecodeParams &p, Warp
 
 // Packed layout: lane (g, c) holds channels 16 m + g (k = 0, 1) and 16 m + g + 8 (k = 2, 3)
 // of columns 2c + (k & 1).
-template <int NT>
-__device__ __forceinline__ void store_packed(float *dst, const WarpState<NT> &st, int q, float f)
+// ------------------------------------------------------------------ int8 PV, 5-16 rows
+//
+// One or two 8-row query tiles (5 to 16 query rows per KV head: a group of 5-16, or several
+// query tokens of a smaller group) take the packed path's int8 PV without its row repeat: lane
+// (g, c) keeps the scores of rows g (and g + 8) for tokens 2c, 2c + 1, 8 + 2c, 9 + 2c of
+// each 16-token subtile, which are exactly the k positions 4c..4c+3 (and 16 + 4c..) of the
+// B operand under the token order tau of the V^T ldmatrix load, so P needs no shuffle:
+// each of its three bytes is one n-tile of 8 head columns (three u8 MMAs per 16-channel
+// m-tile and row tile, no int8 -> f16 conversion of V). The stage's
+// int32 sums are folded into the fp32 accumulator at once (exact: |sum| < 2^22).
+template <int NT, bool kDump>
+__device__ __forceinline__ void process_stage_i8(const DecodeParams &p, WarpState<NT> &st,
+                                                 const ThreadOffsets &o, uint32_t vrow_off,
+                                                 uint32_t sb, uint32_t sbs, int tl0,
+                                                 uint32_t vmask, bool causal,
+                                                 const int (&lim)[NT], float scale_log2, int b,
+                                                 int hc, int kl, int slice, int tok0, int g,
+                                                 int c)
 {
+    // ---- scores: the exact int32 block dots of process_stage
+    float s[NT][kSub][2][2];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        dst[16 * m] = st.acc[0][m][q] * f;
-        dst[16 * m + 8] = st.acc[0][m][q + 2] * f;
+    for (int u = 0; u < kSub; ++u)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int r = 0; r < NT; ++r)
+                s[r][u][nt][0] = s[r][u][nt][1] = 0.f;
+            int prev[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
+#pragma unroll
+            for (int j = 0; j < kNB; ++j) {
+                const uint2 kk = lds64(sb + o.k[u][j] + nt * 1024);
+                int d[4];
+                mma_s8_16832_acc(d, st.qa[j][0], NT == 2 ? st.qa[j][1] : 0u, st.qa[j][2],
+                                 NT == 2 ? st.qa[j][3] : 0u, kk.x, kk.y, prev);
+                if constexpr (kDump) {
+#pragma unroll
+                    for (int q = 0; q < 2 * NT; ++q) {
+                        const int r = q >> 1, e = q & 1;
+                        const int hg = slice * 16 + r * 8 + g;
+                        const int tl = tl0 + u * 16 + nt * 8 + e;
+                        if (hg < p.G && ((vmask >> (tl - tl0 + 2 * c)) & 1u)) {
+                            const long long h = (long long)(hc * p.HPC + kl) * p.G + hg;
+                            p.dbg_dots[(((long long)b * p.Hq + h) * p.dbg_max_len + tok0 + tl) *
+                                           kNB +
+                                       j] = d[q] - prev[q];
+                        }
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < NT; ++r) {
+                    s[r][u][nt][0] +=
+                        (__int_as_float(d[2 * r]) - __int_as_float(prev[2 * r])) * st.qs[r][j];
+                    s[r][u][nt][1] += (__int_as_float(d[2 * r + 1]) -
+                                       __int_as_float(prev[2 * r + 1])) * st.qs[r][j];
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    prev[q] = d[q];
+            }
+        }
+    float kss[kSub][2][2], vsv[kSub][2][2];
+#pragma unroll
+    for (int u = 0; u < kSub; ++u)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                kss[u][nt][e] = lds_f32(sbs + o.s[u][nt][e]) * scale_log2;
+                vsv[u][nt][e] = lds_f32(sbs + o.s[u][nt][e] + p.lay.sc_gap);
+            }
+    if (vmask != 0xffffffffu || causal) {
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = u * 16 + nt * 8 + 2 * c + e;
+                    if (!((vmask >> j) & 1u)) {
+#pragma unroll
+                        for (int r = 0; r < NT; ++r)
+                            s[r][u][nt][e] = -INFINITY;
+                        kss[u][nt][e] = 1.f;
+                        vsv[u][nt][e] = 0.f;
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < NT; ++r)
+                            if (j >= lim[r])
+                                s[r][u][nt][e] = -INFINITY;
+                    }
+                }
+    }
+    // ---- online softmax of rows g (and g + 8) over the stage's 32 tokens; P as exact
+    // integers < 2^23, split in bytes (k order 4c + i <-> token 2c + (i & 1) + 8 (i >> 1))
+    float alpha_a[NT];
+    uint32_t pl[NT][3][kSub];
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float v = s[r][u][nt][e] * kss[u][nt][e];
+                    s[r][u][nt][e] = v;
+                    m = fmaxf(m, v);
+                }
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
+        const float mn = fmaxf(st.M[r], m);
+        const float ms = (mn == -INFINITY) ? 0.f : mn;
+        const float alpha_s = fast_exp2(st.M[r] - ms);
+        st.M[r] = mn;
+        float ws = 0.f, pmax = 0.f;
+#pragma unroll
+        for (int u = 0; u < kSub; ++u)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float x = fast_exp2(s[r][u][nt][e] - ms);
+                    ws += x;
+                    s[r][u][nt][e] = x * vsv[u][nt][e]; // the weight w * vs
+                    pmax = fmaxf(pmax, s[r][u][nt][e]);
+                }
+        st.S[r] = st.S[r] * alpha_s + ws;
+        pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 1));
+        pmax = fmaxf(pmax, __shfl_xor_sync(kFullMask, pmax, 2));
+        const float an_stage = ms + exponent_as_float(pmax) - 14.f;
+        const float an =
+            (mn == -INFINITY) ? -INFINITY : fmaxf(fmaxf(st.A[r], an_stage), mn - 114.f);
+        const float as = (an == -INFINITY) ? 0.f : an;
+        alpha_a[r] = fast_exp2(st.A[r] - as);
+        st.A[r] = an;
+        const float cvs8 = fast_exp2(ms - as + 8.f); // 2^(M - A + 8)
+#pragma unroll
+        for (int u = 0; u < kSub; ++u) {
+            uint32_t X[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    X[nt][e] = __float_as_uint(fmaf(s[r][u][nt][e], cvs8, kTwo23));
+            const uint32_t x01 = prmt(X[0][0], X[0][1], 0x5140u);
+            const uint32_t x23 = prmt(X[1][0], X[1][1], 0x5140u);
+            const uint32_t y01 = prmt(X[0][0], X[0][1], 0x7362u);
+            const uint32_t y23 = prmt(X[1][0], X[1][1], 0x7362u);
+            pl[r][0][u] = prmt(x01, x23, 0x5410u);
+            pl[r][1][u] = prmt(x01, x23, 0x7632u);
+            pl[r][2][u] = prmt(y01, y23, 0x5410u);
+        }
+    }
+    // ---- rescale factors of the accumulator columns (heads 2c, 2c + 1 of each row tile:
+    // the rows of lanes 8c, 8c + 4)
+    float f0[NT], f1[NT];
+#pragma unroll
+    for (int r = 0; r < NT; ++r) {
+        f0[r] = __shfl_sync(kFullMask, alpha_a[r], 8 * c);
+        f1[r] = __shfl_sync(kFullMask, alpha_a[r], 8 * c + 4);
+    }
+    // ---- PV: V^T by ldmatrix .trans (k = the 32 tokens in tau order), one u8 n-tile per
+    // byte of P and row tile; acc = acc * f + (S0 / 2^8 + S1 + S2 * 2^8), S_i the exact sums
+    const uint32_t vrow = sb + vrow_off;
+    const int z[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x2_trans_b8(a0, a1, a2, a3, vrow ^ (uint32_t)(mt << 4));
+#pragma unroll
+        for (int r = 0; r < NT; ++r) {
+            int d0[4], d1[4], d2[4];
+            mma_s8u8_16832_acc(d0, a0, a1, a2, a3, pl[r][0][0], pl[r][0][1], z);
+            mma_s8u8_16832_acc(d1, a0, a1, a2, a3, pl[r][1][0], pl[r][1][1], z);
+            mma_s8u8_16832_acc(d2, a0, a1, a2, a3, pl[r][2][0], pl[r][2][1], z);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                // the biased fp32 views minus the bias are the exact sums; recombine them
+                // with one rounding per step, smallest first
+                const float s0 = __int_as_float(d0[k]) - kDotBiasF;
+                const float s1 = __int_as_float(d1[k]) - kDotBiasF;
+                const float s2 = __int_as_float(d2[k]) - kDotBiasF;
+                const float v = fmaf(s2, 256.f, fmaf(s0, 0.00390625f, s1));
+                st.acc[r][mt][k] = fmaf(st.acc[r][mt][k], (k & 1) ? f1[r] : f0[r], v);
+            }
+        }
     }
 }
 
-// Write the 16 channels 16g..16g+15 of column head (pv, col) scaled by f.
+// Write channels 16m + g and 16m + g + 8 (m = 0..7) of column q's head scaled by f: the
+// channel order of the ldmatrix-fed int8 PV (the packed path and the one-tile int8 PV).
 template <int NT>
-__device__ __forceinline__ void store_row16(float *dst, const WarpState<NT> &st, int pv, int q,
-                                            float f)
+__device__ __forceinline__ void store_packed(float *dst, const WarpState<NT> &st, int pv, int q,
+                                             float f)
 {
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-        const float4 v = make_float4(st.acc[pv][i][q] * f, st.acc[pv][i][q + 2] * f,
-                                     st.acc[pv][i + 1][q] * f, st.acc[pv][i + 1][q + 2] * f);
-        *reinterpret_cast<float4 *>(dst + 2 * i) = v;
+    for (int m = 0; m < 8; ++m) {
+        dst[16 * m] = st.acc[pv][m][q] * f;
+        dst[16 * m + 8] = st.acc[pv][m][q + 2] * f;
     }
 }
 
@@ -1245,10 +1197,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
                     if (col_lane && hg < p.G) {
                         const float f = sc > 0.f ? exp2f(ac - mc) / sc : 0.f;
                         float *dst = p.out + q_row(p, b, hc * p.HPC + kl, hg) * kD;
-                        if constexpr (kPack)
-                            store_packed(dst + g, st, q, f);
-                        else
-                            store_row16(dst + 16 * g, st, pv, q, f);
+                        store_packed(dst + g, st, pv, q, f); // ldmatrix channel order
                     }
                 }
         }
@@ -1269,10 +1218,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
                 const int hg = slice * 16 + pv * 8 + 2 * c + q;
                 if (col_lane && hg < p.G) {
                     float *dst = slotp + (size_t)(kl * p.G + hg) * kSlotRow;
-                    if constexpr (kPack)
-                        store_packed(dst + g, st, q, 1.0f);
-                    else
-                        store_row16(dst + 16 * g, st, pv, q, 1.0f);
+                    store_packed(dst + g, st, pv, q, 1.0f);
                 }
             }
         if (c == 0) {
@@ -1435,9 +1381,8 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                                                     lim[0], scale_log2, cu.b, cu.hc, kl, tok0, g,
                                                     c, k0, k1);
                 else
-                    process_stage<NT, kPack, kDump>(p, st, o, sb, sbs, tl0, vmask, causal, lim,
-                                                    scale_log2, cu.b, cu.hc, kl, slice, tok0, g,
-                                                    c);
+                    process_stage_i8<NT, kDump>(p, st, o, po.v, sb, sbs, tl0, vmask, causal, lim,
+                                                scale_log2, cu.b, cu.hc, kl, slice, tok0, g, c);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[stage]);

@@ -3,7 +3,6 @@
 #pragma once
 
 #include <cstdint>
-#include <cuda_fp16.h>
 
 namespace q8kv {
 
@@ -266,27 +265,6 @@ __device__ __forceinline__ void ldsm_x2_trans_b8(uint32_t &r0, uint32_t &r1, uin
                  : "r"(addr));
 }
 
-// C(16x8 f32) += A(16x16 f16, row) * B(16x8 f16, col).
-__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
-                                              uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-                 "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// D(16x8 f32) = A(16x16 f16, row) * B(16x8 f16, col), accumulator input zero.
-__device__ __forceinline__ void mma_f16_16816_zero_c(float (&d)[4], uint32_t a0, uint32_t a1,
-                                                     uint32_t a2, uint32_t a3, uint32_t b0,
-                                                     uint32_t b1)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
-}
-
 // 2^x with the hardware approximation (ex2.approx.ftz: about 2 ulp; results below 2^-126
 // flush to zero, 2^-inf = 0).
 __device__ __forceinline__ float fast_exp2(float x)
@@ -303,32 +281,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
-}
-
-// Two int8 codes sitting in bytes 0 and 2 of `t` (bytes 1 and 3 ignored) -> f16x2 holding
-// the same integers exactly. The byte is biased by 128 and placed in the mantissa of
-// 1024.0 (0x6400, unit spacing), giving 1152 + code, and 1152 is subtracted.
-__device__ __forceinline__ uint32_t s8pair_to_f16x2(uint32_t t)
-{
-    uint32_t biased = (t & 0x00FF00FFu) ^ 0x64806480u;
-    __half2 h = *reinterpret_cast<__half2 *>(&biased);
-    const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
-    h = __hsub2(h, off);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// Pack two fp32 values into f16x2 (x in the low half).
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
-{
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// Exact int32 -> fp32 for |x| < 2^22 without the conversion unit: the integer is added
-// to the bit pattern of 1.5 * 2^23 (unit spacing) and 1.5 * 2^23 is subtracted.
-__device__ __forceinline__ float small_int_to_float(int x)
-{
-    return __int_as_float(x + 0x4B400000) - 12582912.0f;
 }
 
 // floor(log2 |v|) of a normal fp32 value, as fp32, from its exponent field (no conversion
