@@ -12,23 +12,30 @@
 //   out   = sum_t exp(s_t - M) * (code_t - 8) * dv_t,block / sum_t exp(s_t - M).
 // Codes are packed two per byte, channel 2i in the low nibble of byte i.
 //
-// How (B200): q4_0 halves the bytes per token again (72 B per row with its scales), and
-// the per-block scales make every 32 channels of V a separate weight, which does not map
-// onto the int8 tensor-core path of the q8 kernel; the work per byte is small enough for
-// the CUDA cores. The sequence is cut into chunks of kQ4Chunk tokens (flash-decoding);
+// How (B200): the sequence is cut into chunks of kQ4Chunk = 256 tokens (flash-decoding);
 // one 256-thread CTA takes one (sequence, KV head, chunk) and all G query heads of the KV
-// head:
-//   * scores, lanes = tokens: each lane loads its token's 64-byte K row and 8 bytes of
-//     scales, splits each 32-bit word of nibbles into the even and the odd channels with
-//     two masks (no per-element unpacking), and forms each block dot with dp4a
-//     (u8 codes x s8 query, the query stored in the same even / odd channel order in
-//     shared memory) minus 8 times the block's query sum;
-//   * softmax per chunk in shared memory (exp2, base-2 scores);
-//   * the same lane also loads its token's V row and scales (with the K row: one round
-//     trip after the block table) into shared memory;
-//   * PV, lanes = channels: each warp walks its share of the chunk's tokens out of shared
-//     memory, a lane reading the 2 bytes of its 4 channels, and the per-warp sums are
-//     added in shared memory;
+// head, and both contractions run on the int8 tensor cores (mma.sync m16n8k32):
+//   * loads: each warp copies its 32-token slice (K and V rows, 64 bytes each, and their
+//     scales) into shared memory with cp.async, one token per lane; a row's 16-byte
+//     chunks sit at XOR-swizzled positions so that both ldmatrix patterns below are free
+//     of bank conflicts;
+//   * a nibble becomes a tensor-core operand with one or two logic instructions: for a
+//     byte x = (odd << 4) | even, (x ^ 0x88) & 0xF0 is the signed byte 16 * (odd - 8) and
+//     ((x << 4) ^ 0x80) & 0xF0 is 16 * (even - 8); the factor 16 is taken out in fp32;
+//   * QK: the rows of the A operand are (block j, head h) pairs r = j * GT + h, and row r
+//     holds q's block j only (zeros elsewhere), so one chained accumulator per row gives
+//     exactly that block's dot; B = K^T by ldmatrix (8 tokens x 4 blocks per load). Each
+//     dot is scaled by its own qsc * dk and the blocks of a head are summed in fp32;
+//   * softmax: the chunk's maximum per head over the 8 warps (shared memory), base 2;
+//   * PV: the weight w * dv_tj differs per 32-channel block, so a PV column is again a
+//     (block, head) pair; each weight becomes an exact integer
+//     P = round(w * dv * 2^(36 - e_j)), |P| < 2^22 (e_j the binary16 exponent field of the
+//     chunk's largest |dv| in block j), whose three bytes are three B operands (two
+//     unsigned, the top one signed). Warp w owns the 16 channels of parity (w & 1) in block
+//     w / 2 and runs over all 8 slices: A = V^T by ldmatrix .trans (k = tokens in the
+//     order tau of the QK accumulator layout, so P needs no shuffle), three MMAs per slice,
+//     int32 sums over 4 slices at a time (|sum| < 2^22, so the fp32 view of
+//     1.5 * 2^23 + sum is exact), recombined in fp32 and scaled by 2^(e_j - 32);
 //   * the chunk's partial (acc, max, sum) goes to the workspace, and q4_combine_kernel
 //     merges the chunks of every (sequence, head) with the usual log-sum-exp rescaling.
 #pragma once
@@ -37,7 +44,7 @@
 
 #include <cstdint>
 
-#include "q8kv_decode.cuh" // device error bits, kD, kNB
+#include "q8kv_decode.cuh" // device error bits, kD, kNB, kDotBias
 #include "q8kv_ptx.cuh"
 #include "q8kv_qquant.cuh"
 
@@ -45,10 +52,12 @@ namespace q8kv {
 
 constexpr int kQ4Threads = 256;
 constexpr int kQ4Warps = kQ4Threads / 32;
-constexpr int kQ4Chunk = 256;   // tokens per CTA: one per lane of the 8 warps in the scores
-constexpr int kQ4MaxG = 16;     // query heads per KV head
-constexpr int kQ4Row = kD / 2;  // code bytes per (token, KV head) row
-constexpr int kQ4SlotRow = kD + 4; // partial row: acc[128], M, S, pad
+constexpr int kQ4Chunk = kQ4Warps * 32; // tokens per CTA: one 32-token slice per warp
+constexpr int kQ4MaxG = 16;             // query heads per KV head
+constexpr int kQ4Row = kD / 2;          // code bytes per (token, KV head) row
+constexpr int kQ4SlotRow = kD + 4;      // partial row: acc[128], M, S, pad
+constexpr int kQ4FoldEvery = 4;         // slices summed in int32 before an fp32 fold
+constexpr float kQ4Bias = 12582912.0f;  // 1.5 * 2^23, the fp32 value of kDotBias
 
 struct Q4Params {
     float *out;
@@ -63,33 +72,95 @@ struct Q4Params {
     float scale_log2;
 };
 
-// Shared memory of one CTA (dynamic): query words, block sums and scales, the chunk's
-// scores / weights, and the per-warp PV sums.
-struct Q4Smem {
-    uint32_t qw[kQ4MaxG][32]; // word 2m: channels 8m, 8m+2, 8m+4, 8m+6; word 2m+1: the odd
-    int qsum[kQ4MaxG][kNB];   // sum of the block's query codes
-    float qsc[kQ4MaxG][kNB];
-    float ms[kQ4MaxG][2];     // chunk max and sum per head
+// GT: the instantiated group (1, 2, 4, 8 or 16, at least G; heads G..GT-1 are padding).
+template <int GT>
+struct Q4Shape {
+    static constexpr int R = 4 * GT;                   // (block, head) rows: r = j * GT + h
+    static constexpr int MT = R <= 16 ? 1 : R / 16;    // QK m-tiles
+    static constexpr int NS = R <= 8 ? 1 : R / 8;      // PV n-tiles (column sets)
+    static constexpr int SPB = GT <= 8 ? 1 : GT / 8;   // PV n-tiles per 32-channel block
+    static constexpr int NSLOT = GT <= 8 ? 1 : GT / 8; // heads whose scores a lane holds
 };
 
-// Dynamic shared memory: Q4Smem, the chunk's V codes [chunk][64 B] and V block scales
-// [chunk][4] (fp32), the scores / weights [G][chunk], and the per-warp PV sums [8][G][128].
-__host__ __device__ inline size_t q4_smem_bytes(int G)
+template <int GT>
+struct Q4Smem {
+    uint8_t k[kQ4Chunk][kQ4Row]; // 16-byte chunks at position chunk ^ q4_swz(token)
+    uint8_t v[kQ4Chunk][kQ4Row];
+    uint2 kd[kQ4Chunk];          // the 4 binary16 block scales of the token's row
+    uint2 vd[kQ4Chunk];
+    uint2 pb[kQ4Warps][Q4Shape<GT>::NS][3][32]; // P byte planes as PV B fragments
+    uint32_t qw[GT][32]; // word 2m: channels 8m, 8m+2, 8m+4, 8m+6; word 2m+1: the odd ones
+    float qsc[GT][kNB];
+    float smax[kQ4Warps][GT];
+    float ssum[kQ4Warps][GT];
+    uint32_t dvmax[kQ4Warps][kNB]; // largest |dv| bit pattern of the warp's slice per block
+    uint32_t valid[kQ4Warps];      // tokens of the slice with data
+};
+
+template <int GT>
+__host__ __device__ constexpr size_t q4_smem_bytes()
 {
-    return sizeof(Q4Smem) + (size_t)kQ4Chunk * (kQ4Row + 4 * kNB) +
-           sizeof(float) * (size_t)G * kQ4Chunk + sizeof(float) * (size_t)kQ4Warps * G * kD;
+    return sizeof(Q4Smem<GT>);
 }
 
-__device__ __forceinline__ int dp4a_us(uint32_t a_u8, uint32_t b_s8, int c)
+// Chunk position of a row's 16-byte chunk: for 8 consecutive tokens (the QK ldmatrix) and
+// for the tokens tau(0..7), tau(8..15) (the PV ldmatrix) the pairs (token & 1, swizzle)
+// are all distinct, so each 8-row phase touches 8 different bank groups.
+__device__ __forceinline__ uint32_t q4_swz(int tok)
 {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_u8), "r"(b_s8), "r"(c));
-    return d;
+    return (uint32_t)(((tok >> 1) & 1) | ((((tok >> 2) ^ (tok >> 3)) & 1) << 1));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                        uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// 16 * (code - 8) as signed bytes, for the even (low-nibble) and odd channels of 4 bytes.
+__device__ __forceinline__ uint32_t nib_even_s8x16(uint32_t x)
+{
+    return ((x << 4) ^ 0x80808080u) & 0xF0F0F0F0u;
+}
+
+__device__ __forceinline__ uint32_t nib_odd_s8x16(uint32_t x)
+{
+    return (x ^ 0x88888888u) & 0xF0F0F0F0u;
 }
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t h)
 {
     return __half2float(__ushort_as_half(h));
+}
+
+// Binary16 scale of block j (0..3) out of a token's 4 packed scales.
+__device__ __forceinline__ float half_of(uint2 w, int j)
+{
+    const uint32_t x = (j & 2) ? w.y : w.x;
+    return half_bits_to_float((uint16_t)(x >> ((j & 1) * 16)));
+}
+
+// a[j & 3] without indexing a register array by a run-time value.
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&a)[4], int j)
+{
+    const uint32_t lo = (j & 1) ? a[1] : a[0], hi = (j & 1) ? a[3] : a[2];
+    return (j & 2) ? hi : lo;
 }
 
 // Physical slot of token t of sequence b, or -1 (and an error bit) for a bad table entry.
@@ -103,19 +174,32 @@ __device__ __forceinline__ long long q4_slot(const Q4Params &p, int b, int t, un
     return (long long)ph * p.bs + t % p.bs;
 }
 
-// GM: the largest group the instantiation serves (4, 8 or 16): the PV accumulators of the
-// G heads live in registers, so smaller groups get a smaller, more resident kernel.
-template <int GM>
-__global__ void __launch_bounds__(kQ4Threads, GM <= 4 ? 4 : (GM <= 8 ? 3 : 2))
+// Block of QK row r_base + g (r_base a multiple of 8, g < 8); compile-time for GT >= 8.
+template <int GT>
+__device__ __forceinline__ int q4_row_block(int r_base, int g)
+{
+    if constexpr (GT >= 8)
+        return r_base / GT;
+    else
+        return (r_base + g) / GT;
+}
+
+// Does QK m-tile mt hold a row of block j?
+template <int GT>
+__host__ __device__ constexpr bool q4_tile_has_block(int mt, int j)
+{
+    return 16 * mt < (j + 1) * GT && j * GT < 16 * mt + 16;
+}
+
+template <int GT>
+__global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
     q4_decode_kernel(const __grid_constant__ Q4Params p)
 {
-    extern __shared__ __align__(16) uint8_t q4_smem_raw[];
-    Q4Smem &sm = *reinterpret_cast<Q4Smem *>(q4_smem_raw);
-    uint4 *vbuf = reinterpret_cast<uint4 *>(q4_smem_raw + sizeof(Q4Smem));  // [chunk][4]
-    float4 *vdbuf = reinterpret_cast<float4 *>(vbuf + kQ4Chunk * 4);       // [chunk]
-    float *sc = reinterpret_cast<float *>(vdbuf + kQ4Chunk);                // [G][chunk]
-    float *part = sc + p.G * kQ4Chunk;                                      // [warps][G][128]
+    using S = Q4Shape<GT>;
+    extern __shared__ __align__(128) uint8_t q4_smem_raw[];
+    Q4Smem<GT> &sm = *reinterpret_cast<Q4Smem<GT> *>(q4_smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
     const int bk = blockIdx.y, b = bk / p.Hk, kvh = bk - b * p.Hk;
     const int G = p.G;
 
@@ -134,175 +218,309 @@ __global__ void __launch_bounds__(kQ4Threads, GM <= 4 ? 4 : (GM <= 8 ? 3 : 2))
         return; // the combine only reads the chunks that hold tokens
     const int nt = min(kQ4Chunk, L - t0);
 
-    // ---- quantise the G query rows (4 blocks each; one quad of lanes per block)
-    for (int blk = warp * 8 + (lane >> 2); blk - (lane >> 2) < 4 * G; blk += kQ4Warps * 8) {
-        const int g = blk >> 2, j = blk & 3, part4 = lane & 3;
-        const bool live = g < G;
+    // ---- loads: lane = token of this warp's slice; tokens without data are zero-filled
+    {
+        const int tl = warp * 32 + lane;
+        long long slot = -1;
+        if (tl < nt)
+            slot = q4_slot(p, b, t0 + tl, err);
+        const bool ok = slot >= 0;
+        const long long row = ok ? slot * p.Hk + kvh : 0;
+        const uint32_t n16 = ok ? 16u : 0u, n8 = ok ? 8u : 0u;
+        const uint8_t *kr = p.k4 + row * kQ4Row, *vr = p.v4 + row * kQ4Row;
+        const uint32_t sw = q4_swz(tl);
+        const uint32_t kdst = smem_addr(&sm.k[tl][0]), vdst = smem_addr(&sm.v[tl][0]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            cp_async16(kdst + 16u * ((uint32_t)i ^ sw), kr + 16 * i, n16);
+            cp_async16(vdst + 16u * ((uint32_t)i ^ sw), vr + 16 * i, n16);
+        }
+        cp_async8(smem_addr(&sm.kd[tl]), p.kd + row * kNB, n8);
+        cp_async8(smem_addr(&sm.vd[tl]), p.vd + row * kNB, n8);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const unsigned vm = __ballot_sync(kFullMask, ok);
+        if (lane == 0)
+            sm.valid[warp] = vm;
+    }
+
+    // ---- quantise the GT query rows (4 blocks each; one quad of lanes per block; rows
+    // G..GT-1 are zero)
+    for (int blk = warp * 8 + g; blk - g < 4 * GT; blk += kQ4Warps * 8) {
+        const int h = blk >> 2, j = blk & 3;
+        const bool live = blk < 4 * GT && h < G;
         float v[8];
-        const float *qr = p.q + ((long long)b * p.Hq + (long long)kvh * G + (live ? g : 0)) * kD +
-                          32 * j + 8 * part4;
+        const float *qr = p.q + ((long long)b * p.Hq + (long long)kvh * G + (live ? h : 0)) * kD +
+                          32 * j + 8 * c;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             v[i] = live ? __ldg(qr + i) : 0.f;
         uint32_t lo, hi;
         float qs;
         quantize_block_quad(v, lo, hi, qs);
-        int s8 = 0; // the block's code sum (the whole warp shuffles)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            s8 += (int)(int8_t)(lo >> (8 * i)) + (int)(int8_t)(hi >> (8 * i));
-        s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
-        s8 += __shfl_xor_sync(0xffffffffu, s8, 2);
-        if (live) {
-            // channels 8 * part4 + 0..7 of the block: even ones -> word 2m, odd -> 2m + 1
-            const int m = 4 * j + part4;
-            sm.qw[g][2 * m] = __byte_perm(lo, hi, 0x6420);
-            sm.qw[g][2 * m + 1] = __byte_perm(lo, hi, 0x7531);
-            if (part4 == 0) {
-                sm.qsum[g][j] = s8;
-                sm.qsc[g][j] = qs;
-            }
+        if (blk < 4 * GT) {
+            // channels 8c + 0..7 of the block: even ones -> word 2m, odd -> 2m + 1
+            const int m = 4 * j + c;
+            sm.qw[h][2 * m] = __byte_perm(lo, hi, 0x6420);
+            sm.qw[h][2 * m + 1] = __byte_perm(lo, hi, 0x7531);
+            if (c == 0)
+                sm.qsc[h][j] = live ? qs : 0.f;
         }
     }
-    __syncthreads();
 
-    // ---- scores: lane = token. The token's K and V rows are loaded together (one round
-    // trip after the block table); V goes to shared memory for the PV pass.
+    // the slice's largest |dv| per block (this lane's own copy: visible after the wait)
+    asm volatile("cp.async.wait_all;" ::: "memory");
     {
-        const int tl = warp * 32 + lane; // token within the chunk
-        const bool valid = tl < nt;
-        long long slot = -1;
-        if (valid)
-            slot = q4_slot(p, b, t0 + tl, err);
-        if (slot >= 0) {
-            const long long row = slot * p.Hk + kvh;
-            const uint4 *kr = reinterpret_cast<const uint4 *>(p.k4 + row * kQ4Row);
-            const uint4 *vr = reinterpret_cast<const uint4 *>(p.v4 + row * kQ4Row);
-            uint4 kw[4], vw[4];
+        const uint2 vd = sm.vd[warp * 32 + lane];
+        const uint32_t a[4] = {vd.x & 0x7fffu, (vd.x >> 16) & 0x7fffu, vd.y & 0x7fffu,
+                               (vd.y >> 16) & 0x7fffu};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                kw[i] = __ldcs(kr + i);
-                vw[i] = __ldcs(vr + i);
-            }
-            const uint2 kdw = __ldcs(reinterpret_cast<const uint2 *>(p.kd + row * kNB));
-            const uint2 vdw = __ldcs(reinterpret_cast<const uint2 *>(p.vd + row * kNB));
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                vbuf[tl * 4 + i] = vw[i];
-            vdbuf[tl] = make_float4(half_bits_to_float((uint16_t)(vdw.x & 0xffffu)),
-                                    half_bits_to_float((uint16_t)(vdw.x >> 16)),
-                                    half_bits_to_float((uint16_t)(vdw.y & 0xffffu)),
-                                    half_bits_to_float((uint16_t)(vdw.y >> 16)));
-            float dk[kNB];
-            dk[0] = half_bits_to_float((uint16_t)(kdw.x & 0xffffu));
-            dk[1] = half_bits_to_float((uint16_t)(kdw.x >> 16));
-            dk[2] = half_bits_to_float((uint16_t)(kdw.y & 0xffffu));
-            dk[3] = half_bits_to_float((uint16_t)(kdw.y >> 16));
-            // block j: 4 words (16 bytes, 32 channels); word k: channels 32j + 8k .. + 7
-            for (int g = 0; g < G; ++g) {
-                float s = 0.f;
-#pragma unroll
-                for (int j = 0; j < kNB; ++j) {
-                    const uint32_t w[4] = {kw[j].x, kw[j].y, kw[j].z, kw[j].w};
-                    int dot = 0;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t ev = w[k] & 0x0f0f0f0fu, od = (w[k] >> 4) & 0x0f0f0f0fu;
-                        const int m = 4 * j + k;
-                        dot = dp4a_us(ev, sm.qw[g][2 * m], dot);
-                        dot = dp4a_us(od, sm.qw[g][2 * m + 1], dot);
-                    }
-                    dot -= 8 * sm.qsum[g][j];
-                    s = fmaf((float)dot * sm.qsc[g][j], dk[j], s);
-                }
-                sc[g * kQ4Chunk + tl] = s * p.scale_log2;
-            }
-        } else {
-            // no data: weight 0 against zero codes and a zero scale
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                vbuf[tl * 4 + i] = make_uint4(0u, 0u, 0u, 0u);
-            vdbuf[tl] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int g = 0; g < G; ++g)
-                sc[g * kQ4Chunk + tl] = -INFINITY;
+        for (int j = 0; j < kNB; ++j) {
+            const uint32_t m = __reduce_max_sync(kFullMask, a[j]);
+            if (lane == 0)
+                sm.dvmax[warp][j] = m;
         }
     }
-    __syncthreads();
+    __syncthreads(); // query codes, every slice's K, V and scales
 
-    // ---- softmax over the chunk, per head (warp w takes heads w, w + 8)
-    for (int g = warp; g < G; g += kQ4Warps) {
+    // ---- QK on the tensor cores: this warp's 4 n-tiles of 8 tokens
+    uint32_t qa[S::MT][kNB][4]; // A fragments: q's block j in the rows of block j, else 0
+    float wq[S::MT][2];         // qsc * scale_log2 / 16 of rows g and g + 8 (0: padding)
+    int jr[S::MT][2];           // the blocks of those rows
+#pragma unroll
+    for (int mt = 0; mt < S::MT; ++mt) {
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+            const int r = 16 * mt + 8 * hlf + g;
+            const int j = q4_row_block<GT>(16 * mt + 8 * hlf, g);
+            const int h = r % GT;
+            jr[mt][hlf] = j & 3;
+            wq[mt][hlf] = (r < S::R) ? sm.qsc[h][j & 3] * (p.scale_log2 * 0.0625f) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < kNB; ++jj) {
+                const bool on = (j == jj) && r < S::R;
+                qa[mt][jj][hlf] = on ? sm.qw[h][8 * jj + 2 * c] : 0u;
+                qa[mt][jj][hlf + 2] = on ? sm.qw[h][8 * jj + 2 * c + 1] : 0u;
+            }
+        }
+    }
+    const unsigned vmask = sm.valid[warp];
+    float sc[S::NSLOT][4][2]; // base-2 scores: head slot, n-tile, token 2c + e
+#pragma unroll
+    for (int ntile = 0; ntile < 4; ++ntile) {
+        const int tk = warp * 32 + 8 * ntile + (lane & 7); // ldmatrix row; matrix = block
+        const uint32_t addr =
+            smem_addr(&sm.k[tk][0]) + 16u * ((uint32_t)(lane >> 3) ^ q4_swz(tk));
+        uint32_t kr[4];
+        ldsm_x4(kr[0], kr[1], kr[2], kr[3], addr);
+        uint32_t kb0[4], kb1[4];
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+            kb0[j] = nib_even_s8x16(kr[j]);
+            kb1[j] = nib_odd_s8x16(kr[j]);
+        }
+        const int ta = warp * 32 + 8 * ntile + 2 * c;
+        const uint2 kd0 = sm.kd[ta], kd1 = sm.kd[ta + 1];
+#pragma unroll
+        for (int s = 0; s < S::NSLOT; ++s) {
+            sc[s][ntile][0] = 0.f;
+            sc[s][ntile][1] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < S::MT; ++mt) {
+            int d[4] = {kDotBias, kDotBias, kDotBias, kDotBias};
+#pragma unroll
+            for (int j = 0; j < kNB; ++j)
+                if (q4_tile_has_block<GT>(mt, j))
+                    mma_s8_16832_acc(d, qa[mt][j][0], qa[mt][j][1], qa[mt][j][2], qa[mt][j][3],
+                                     kb0[j], kb1[j], d);
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                const int slot = (GT == 16) ? hlf : 0;
+                const float x0 = __int_as_float(d[2 * hlf]) - kQ4Bias;
+                const float x1 = __int_as_float(d[2 * hlf + 1]) - kQ4Bias;
+                const int j = jr[mt][hlf];
+                sc[slot][ntile][0] = fmaf(x0, wq[mt][hlf] * half_of(kd0, j), sc[slot][ntile][0]);
+                sc[slot][ntile][1] = fmaf(x1, wq[mt][hlf] * half_of(kd1, j), sc[slot][ntile][1]);
+            }
+        }
+    }
+    // the blocks of one head sit in lanes whose g differs in the bits >= log2(GT)
+#pragma unroll
+    for (int s = 0; s < S::NSLOT; ++s)
+#pragma unroll
+        for (int ntile = 0; ntile < 4; ++ntile)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float x = sc[s][ntile][e];
+                if constexpr (GT <= 1)
+                    x += __shfl_xor_sync(kFullMask, x, 4);
+                if constexpr (GT <= 2)
+                    x += __shfl_xor_sync(kFullMask, x, 8);
+                if constexpr (GT <= 4)
+                    x += __shfl_xor_sync(kFullMask, x, 16);
+                const int t = 8 * ntile + 2 * c + e;
+                sc[s][ntile][e] = ((vmask >> t) & 1u) ? x : -INFINITY;
+            }
+
+    // ---- softmax: the slice's maximum per head, then the chunk's
+    const int hs = g % GT; // head of slot 0 (slot 1: hs + 8)
+#pragma unroll
+    for (int s = 0; s < S::NSLOT; ++s) {
         float m = -INFINITY;
-        for (int i = lane; i < kQ4Chunk; i += 32)
-            m = fmaxf(m, sc[g * kQ4Chunk + i]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const float ms = m == -INFINITY ? 0.f : m;
-        float ssum = 0.f;
-        for (int i = lane; i < kQ4Chunk; i += 32) {
-            const float w = fast_exp2(sc[g * kQ4Chunk + i] - ms);
-            sc[g * kQ4Chunk + i] = w;
-            ssum += w;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
-        if (lane == 0) {
-            sm.ms[g][0] = m;
-            sm.ms[g][1] = ssum;
-        }
+        for (int ntile = 0; ntile < 4; ++ntile)
+            m = fmaxf(m, fmaxf(sc[s][ntile][0], sc[s][ntile][1]));
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
+        if (c == 0 && g < GT)
+            sm.smax[warp][hs + 8 * s] = m;
     }
     __syncthreads();
-
-    // ---- PV: lane = 4 channels (4 * lane .. + 3, block lane / 8); warp w takes tokens w,
-    // w + 8, ... of the chunk
-    {
-        float acc[GM][4];
+    uint32_t emax[kNB];
 #pragma unroll
-        for (int g = 0; g < GM; ++g)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                acc[g][c] = 0.f;
-        const int jb = lane >> 3;
-        const uint16_t *vb16 = reinterpret_cast<const uint16_t *>(vbuf);
-        const float *vd32 = reinterpret_cast<const float *>(vdbuf);
-        for (int tl = warp; tl < nt; tl += kQ4Warps) {
-            const uint32_t nib = vb16[tl * kQ4Row / 2 + lane];
-            const float dv = vd32[tl * 4 + jb];
-            const float x0 = (float)((int)(nib & 0xfu) - 8), x1 = (float)((int)((nib >> 4) & 0xfu) - 8);
-            const float x2 = (float)((int)((nib >> 8) & 0xfu) - 8), x3 = (float)((int)(nib >> 12) - 8);
-#pragma unroll
-            for (int g = 0; g < GM; ++g) {
-                if (g < G) {
-                    const float wv = sc[g * kQ4Chunk + tl] * dv;
-                    acc[g][0] = fmaf(wv, x0, acc[g][0]);
-                    acc[g][1] = fmaf(wv, x1, acc[g][1]);
-                    acc[g][2] = fmaf(wv, x2, acc[g][2]);
-                    acc[g][3] = fmaf(wv, x3, acc[g][3]);
-                }
-            }
-        }
-#pragma unroll
-        for (int g = 0; g < GM; ++g)
-            if (g < G)
-                *reinterpret_cast<float4 *>(part + ((size_t)warp * G + g) * kD + 4 * lane) =
-                    make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-    }
-    __syncthreads();
-
-    // ---- the chunk's partial: sum the warps' rows, then acc, M, S to the workspace
-    float *dst = p.partials + (((size_t)bk * p.n_chunks + blockIdx.x) * G) * kQ4SlotRow;
-    for (int e = tid; e < G * kD; e += kQ4Threads) {
-        const int g = e / kD, d = e - g * kD;
-        float s = 0.f;
+    for (int j = 0; j < kNB; ++j) {
+        uint32_t x = 0;
 #pragma unroll
         for (int w = 0; w < kQ4Warps; ++w)
-            s += part[((size_t)w * G + g) * kD + d];
-        dst[(size_t)g * kQ4SlotRow + d] = s;
+            x = max(x, sm.dvmax[w][j]);
+        emax[j] = x >> 10; // binary16 exponent field of the chunk's largest |dv|
     }
-    for (int g = tid; g < G; g += kQ4Threads) {
-        dst[(size_t)g * kQ4SlotRow + kD] = sm.ms[g][0];
-        dst[(size_t)g * kQ4SlotRow + kD + 1] = sm.ms[g][1];
+#pragma unroll
+    for (int s = 0; s < S::NSLOT; ++s) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kQ4Warps; ++w)
+            m = fmaxf(m, sm.smax[w][hs + 8 * s]);
+        const float mref = m == -INFINITY ? 0.f : m;
+        float sum = 0.f;
+#pragma unroll
+        for (int ntile = 0; ntile < 4; ++ntile)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float w = fast_exp2(sc[s][ntile][e] - mref);
+                sc[s][ntile][e] = w;
+                sum += w;
+            }
+        sum += __shfl_xor_sync(kFullMask, sum, 1);
+        sum += __shfl_xor_sync(kFullMask, sum, 2);
+        if (c == 0 && g < GT)
+            sm.ssum[warp][hs + 8 * s] = sum;
+    }
+
+    // ---- P = round(w * dv * 2^(36 - e_j)) as byte planes, in PV B-fragment order: lane
+    // (g, c) holds column g of n-tile ns, i.e. row 8 ns + g = (block, head), and the tokens
+    // tau(4c + i) = 2c + (i & 1) + 8 (i >> 1) (+ 16 in the second register)
+#pragma unroll
+    for (int ns = 0; ns < S::NS; ++ns) {
+        const int rr = 8 * ns + g;
+        const int j = (rr / GT) & 3;
+        const int slot = (GT == 16) ? (ns & 1) : 0;
+        const bool live = rr < S::R;
+        const float pscale = exp2i(36 - (int)pick4(emax, j));
+        uint32_t planes[3][2];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            int P[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int ntile = 2 * half + (i >> 1), e = i & 1;
+                const int t = warp * 32 + 8 * ntile + 2 * c + e;
+                const float dvs = half_of(sm.vd[t], j) * pscale;
+                const float x = fmaf(sc[slot][ntile][e], dvs, kQ4Bias);
+                P[i] = live ? __float_as_int(x) - kDotBias : 0;
+            }
+            const uint32_t x01 = prmt((uint32_t)P[0], (uint32_t)P[1], 0x5140);
+            const uint32_t x23 = prmt((uint32_t)P[2], (uint32_t)P[3], 0x5140);
+            const uint32_t z01 = prmt((uint32_t)P[0], (uint32_t)P[1], 0x7362);
+            const uint32_t z23 = prmt((uint32_t)P[2], (uint32_t)P[3], 0x7362);
+            planes[0][half] = prmt(x01, x23, 0x5410);
+            planes[1][half] = prmt(x01, x23, 0x7632);
+            planes[2][half] = prmt(z01, z23, 0x5410);
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            sm.pb[warp][ns][k][lane] = make_uint2(planes[k][0], planes[k][1]);
+    }
+    __syncthreads(); // every slice's P
+
+    // ---- PV: warp w owns channels 32 jb + 2 m + par (m = 0..15), jb = w / 2, par = w & 1
+    const int jb = warp >> 1, par = warp & 1;
+    constexpr int SPB = S::SPB;
+    const int ns0 = (jb * GT) / 8; // first n-tile holding block jb's columns
+    const int kk = lane & 15;
+    const int vtok = (lane >> 4) * 16 + 2 * (kk >> 2) + (kk & 1) + 8 * ((kk >> 1) & 1);
+    const uint32_t vrow = smem_addr(&sm.v[vtok][0]) + 16u * ((uint32_t)jb ^ q4_swz(vtok));
+    int acc[SPB][3][4];
+    float o[SPB][4];
+#pragma unroll
+    for (int si = 0; si < SPB; ++si)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            o[si][e] = 0.f;
+#pragma unroll
+            for (int k = 0; k < 3; ++k)
+                acc[si][k][e] = kDotBias;
+        }
+    // sum_t A P = D0 + 256 D1 + 65536 D2 = 256 x with A = 16 (code - 8) and
+    // P = w dv 2^(36 - e), so sum_t w dv (code - 8) = x 2^(e - 32)
+    const float oscale = exp2i((int)pick4(emax, jb) - 32);
+#pragma unroll
+    for (int sl = 0; sl < kQ4Warps; ++sl) {
+        if (sl * 32 < nt) {
+            uint32_t r[4];
+            ldsm_x2_trans_b8(r[0], r[1], r[2], r[3], vrow + (uint32_t)(sl * 32 * kQ4Row));
+            uint32_t a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                a[i] = par ? nib_odd_s8x16(r[i]) : nib_even_s8x16(r[i]);
+#pragma unroll
+            for (int si = 0; si < SPB; ++si) {
+                const uint2 b0 = sm.pb[sl][ns0 + si][0][lane];
+                const uint2 b1 = sm.pb[sl][ns0 + si][1][lane];
+                const uint2 b2 = sm.pb[sl][ns0 + si][2][lane];
+                mma_s8u8_16832_acc(acc[si][0], a[0], a[1], a[2], a[3], b0.x, b0.y, acc[si][0]);
+                mma_s8u8_16832_acc(acc[si][1], a[0], a[1], a[2], a[3], b1.x, b1.y, acc[si][1]);
+                mma_s8_16832_acc(acc[si][2], a[0], a[1], a[2], a[3], b2.x, b2.y, acc[si][2]);
+            }
+        }
+        if ((sl % kQ4FoldEvery) == kQ4FoldEvery - 1) {
+#pragma unroll
+            for (int si = 0; si < SPB; ++si)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float f0 = __int_as_float(acc[si][0][e]) - kQ4Bias;
+                    const float f1 = __int_as_float(acc[si][1][e]) - kQ4Bias;
+                    const float f2 = __int_as_float(acc[si][2][e]) - kQ4Bias;
+                    const float x = fmaf(f0, 1.0f / 256.0f, fmaf(f2, 256.0f, f1));
+                    o[si][e] = fmaf(x, oscale, o[si][e]);
+#pragma unroll
+                    for (int k = 0; k < 3; ++k)
+                        acc[si][k][e] = kDotBias;
+                }
+        }
+    }
+
+    // ---- the chunk's partial: acc of block jb's columns, then M and S per head
+    float *dst = p.partials + (((size_t)bk * p.n_chunks + blockIdx.x) * G) * kQ4SlotRow;
+#pragma unroll
+    for (int si = 0; si < SPB; ++si)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = 8 * (ns0 + si) + 2 * c + (e & 1);
+            const int h = rr % GT;
+            const int ch = 32 * jb + 2 * (g + 8 * (e >> 1)) + par;
+            if (rr / GT == jb && h < G)
+                dst[(size_t)h * kQ4SlotRow + ch] = o[si][e];
+        }
+    if (warp == 0 && lane < G) {
+        float m = -INFINITY, s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kQ4Warps; ++w) {
+            m = fmaxf(m, sm.smax[w][lane]);
+            s += sm.ssum[w][lane];
+        }
+        dst[(size_t)lane * kQ4SlotRow + kD] = m;
+        dst[(size_t)lane * kQ4SlotRow + kD + 1] = s;
     }
     if (err)
         atomicOr(p.errors, err);

@@ -17,6 +17,21 @@ struct Q4Workspace {
 
 Q4Workspace g_q4[kMaxDevices];
 
+template <int GT>
+cudaError_t q4_set_smem()
+{
+    return cudaFuncSetAttribute(q4_decode_kernel<GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)q4_smem_bytes<GT>());
+}
+
+// The instantiation for groups up to GT (a power of two): heads G..GT-1 are padding.
+template <int GT>
+cudaError_t q4_launch(cudaLaunchConfig_t cfg, const Q4Params &p)
+{
+    cfg.dynamicSmemBytes = q4_smem_bytes<GT>();
+    return cudaLaunchKernelEx(&cfg, q4_decode_kernel<GT>, p);
+}
+
 } // namespace
 
 extern "C" {
@@ -67,15 +82,11 @@ q8kv_status q8kv_decode_attn_q4(float *out, const float *q, const uint8_t *k4_bl
             ws->bytes = ws_need;
         }
         if (!ws->attr_set) {
-            Q8KV_CUDA(cudaFuncSetAttribute(q4_decode_kernel<4>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)q4_smem_bytes(4)));
-            Q8KV_CUDA(cudaFuncSetAttribute(q4_decode_kernel<8>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)q4_smem_bytes(8)));
-            Q8KV_CUDA(cudaFuncSetAttribute(q4_decode_kernel<16>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)q4_smem_bytes(16)));
+            Q8KV_CUDA(q4_set_smem<1>());
+            Q8KV_CUDA(q4_set_smem<2>());
+            Q8KV_CUDA(q4_set_smem<4>());
+            Q8KV_CUDA(q4_set_smem<8>());
+            Q8KV_CUDA(q4_set_smem<16>());
             ws->attr_set = true;
         }
     }
@@ -105,16 +116,19 @@ q8kv_status q8kv_decode_attn_q4(float *out, const float *q, const uint8_t *k4_bl
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)n_chunks, (unsigned)(B * n_kv_heads));
     cfg.blockDim = dim3(kQ4Threads);
-    cfg.dynamicSmemBytes = q4_smem_bytes(G);
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (G <= 4)
-        Q8KV_CUDA(cudaLaunchKernelEx(&cfg, q4_decode_kernel<4>, p));
+    if (G <= 1)
+        Q8KV_CUDA(q4_launch<1>(cfg, p));
+    else if (G <= 2)
+        Q8KV_CUDA(q4_launch<2>(cfg, p));
+    else if (G <= 4)
+        Q8KV_CUDA(q4_launch<4>(cfg, p));
     else if (G <= 8)
-        Q8KV_CUDA(cudaLaunchKernelEx(&cfg, q4_decode_kernel<8>, p));
+        Q8KV_CUDA(q4_launch<8>(cfg, p));
     else
-        Q8KV_CUDA(cudaLaunchKernelEx(&cfg, q4_decode_kernel<16>, p));
+        Q8KV_CUDA(q4_launch<16>(cfg, p));
     cudaLaunchConfig_t cc = cfg;
     cc.gridDim = dim3((unsigned)(((long long)B * n_q_heads + 7) / 8));
     cc.blockDim = dim3(256);
