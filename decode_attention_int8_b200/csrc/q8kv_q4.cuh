@@ -69,6 +69,7 @@ struct Q4Params {
     float *partials; // [B * Hk][n_chunks][G][kQ4SlotRow]
     unsigned *errors;
     int B, Hq, Hk, G, bs, mbps, num_blocks, n_chunks;
+    int log2_bs; // log2(bs) when bs is a power of two, else -1
     float scale_log2;
 };
 
@@ -144,6 +145,13 @@ __device__ __forceinline__ uint32_t nib_odd_s8x16(uint32_t x)
     return (x ^ 0x88888888u) & 0xF0F0F0F0u;
 }
 
+// Either of the two above: sh = 4 gives the even channels, sh = 0 the odd ones (the XOR
+// with 0x88 and the mask leave the other nibble out either way).
+__device__ __forceinline__ uint32_t nib_s8x16(uint32_t x, uint32_t sh)
+{
+    return ((x << sh) ^ 0x88888888u) & 0xF0F0F0F0u;
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint16_t h)
 {
     return __half2float(__ushort_as_half(h));
@@ -156,22 +164,17 @@ __device__ __forceinline__ float half_of(uint2 w, int j)
     return half_bits_to_float((uint16_t)(x >> ((j & 1) * 16)));
 }
 
-// a[j & 3] without indexing a register array by a run-time value.
-__device__ __forceinline__ uint32_t pick4(const uint32_t (&a)[4], int j)
-{
-    const uint32_t lo = (j & 1) ? a[1] : a[0], hi = (j & 1) ? a[3] : a[2];
-    return (j & 2) ? hi : lo;
-}
-
 // Physical slot of token t of sequence b, or -1 (and an error bit) for a bad table entry.
 __device__ __forceinline__ long long q4_slot(const Q4Params &p, int b, int t, unsigned &err)
 {
-    const int ph = __ldg(p.block_table + (long long)b * p.mbps + t / p.bs);
+    const int blk = p.log2_bs >= 0 ? t >> p.log2_bs : t / p.bs;
+    const int off = t - blk * p.bs;
+    const int ph = __ldg(p.block_table + (long long)b * p.mbps + blk);
     if (ph < 0 || ph >= p.num_blocks) {
         err |= kErrBlockTable;
         return -1;
     }
-    return (long long)ph * p.bs + t % p.bs;
+    return (long long)ph * p.bs + off;
 }
 
 // Block of QK row r_base + g (r_base a multiple of 8, g < 8); compile-time for GT >= 8.
@@ -192,7 +195,7 @@ __host__ __device__ constexpr bool q4_tile_has_block(int mt, int j)
 }
 
 template <int GT>
-__global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
+__global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
     q4_decode_kernel(const __grid_constant__ Q4Params p)
 {
     using S = Q4Shape<GT>;
@@ -376,21 +379,19 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
             sm.smax[warp][hs + 8 * s] = m;
     }
     __syncthreads();
-    uint32_t emax[kNB];
-#pragma unroll
-    for (int j = 0; j < kNB; ++j) {
-        uint32_t x = 0;
-#pragma unroll
-        for (int w = 0; w < kQ4Warps; ++w)
-            x = max(x, sm.dvmax[w][j]);
-        emax[j] = x >> 10; // binary16 exponent field of the chunk's largest |dv|
-    }
+    // binary16 exponent field of the chunk's largest |dv| in block j: lane (g, c) reads
+    // warp g's value of block c; after the reduction over g, lane j holds block j's
+    uint32_t emax_c = sm.dvmax[g][c];
+    emax_c = max(emax_c, __shfl_xor_sync(kFullMask, emax_c, 4));
+    emax_c = max(emax_c, __shfl_xor_sync(kFullMask, emax_c, 8));
+    emax_c = max(emax_c, __shfl_xor_sync(kFullMask, emax_c, 16));
+    emax_c >>= 10;
 #pragma unroll
     for (int s = 0; s < S::NSLOT; ++s) {
-        float m = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kQ4Warps; ++w)
-            m = fmaxf(m, sm.smax[w][hs + 8 * s]);
+        // the chunk's maximum: lane (g, c) reads warps c and c + 4, then the c lanes merge
+        float m = fmaxf(sm.smax[c][hs + 8 * s], sm.smax[c + 4][hs + 8 * s]);
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
         const float mref = m == -INFINITY ? 0.f : m;
         float sum = 0.f;
 #pragma unroll
@@ -416,7 +417,7 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
         const int j = (rr / GT) & 3;
         const int slot = (GT == 16) ? (ns & 1) : 0;
         const bool live = rr < S::R;
-        const float pscale = exp2i(36 - (int)pick4(emax, j));
+        const float pscale = exp2i(36 - (int)__shfl_sync(kFullMask, emax_c, j));
         uint32_t planes[3][2];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -445,6 +446,7 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
 
     // ---- PV: warp w owns channels 32 jb + 2 m + par (m = 0..15), jb = w / 2, par = w & 1
     const int jb = warp >> 1, par = warp & 1;
+    const uint32_t vsh = par ? 0u : 4u; // nibble of this warp's channels, moved to the top
     constexpr int SPB = S::SPB;
     const int ns0 = (jb * GT) / 8; // first n-tile holding block jb's columns
     const int kk = lane & 15;
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
         }
     // sum_t A P = D0 + 256 D1 + 65536 D2 = 256 x with A = 16 (code - 8) and
     // P = w dv 2^(36 - e), so sum_t w dv (code - 8) = x 2^(e - 32)
-    const float oscale = exp2i((int)pick4(emax, jb) - 32);
+    const float oscale = exp2i((int)__shfl_sync(kFullMask, emax_c, jb) - 32);
 #pragma unroll
     for (int sl = 0; sl < kQ4Warps; ++sl) {
         if (sl * 32 < nt) {
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 8 ? 3 : 2)
             uint32_t a[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                a[i] = par ? nib_odd_s8x16(r[i]) : nib_even_s8x16(r[i]);
+                a[i] = nib_s8x16(r[i], vsh);
 #pragma unroll
             for (int si = 0; si < SPB; ++si) {
                 const uint2 b0 = sm.pb[sl][ns0 + si][0][lane];

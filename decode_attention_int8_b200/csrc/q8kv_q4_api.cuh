@@ -106,6 +106,10 @@ q8kv_status q8kv_decode_attn_q4(float *out, const float *q, const uint8_t *k4_bl
     p.Hk = n_kv_heads;
     p.G = G;
     p.bs = kv_block_size;
+    p.log2_bs = -1;
+    if ((kv_block_size & (kv_block_size - 1)) == 0)
+        for (p.log2_bs = 0; (1 << p.log2_bs) < kv_block_size; ++p.log2_bs) {
+        }
     p.mbps = max_blocks_per_seq;
     p.num_blocks = num_kv_blocks;
     p.n_chunks = (int)n_chunks;

@@ -1,8 +1,9 @@
 """Decode over a q4_0 cache (q8kv_decode_attn_q4) against the fp64 oracle, with the same
-tolerance as the q8 decode (max-abs <= 1e-4, rel-L2 <= 1e-5): groups 1 to 16, block sizes
-16 to 128, lengths around the 256-token chunks, Student-t data, empty sequences, the
-benchmark's 16 x 4096-token shape on sampled rows, and agreement with the q8 kernel on a
-cache that holds the same values."""
+tolerance as the q8 decode (max-abs <= 1e-4, rel-L2 <= 1e-5): groups 1 to 16 (powers of two,
+and 3, 6, 12 with padding heads), block sizes 16 to 128 (48: not a power of two), lengths
+around the 256-token chunks, Student-t data, empty sequences, the benchmark's 16 x
+4096-token shape on sampled rows, agreement with the q8 kernel on a cache that holds the
+same values, and bad block-table entries (flagged, their tokens skipped)."""
 import numpy as np
 import pytest
 import torch
@@ -34,7 +35,7 @@ def oracle_q4(w):
 
 
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
-@pytest.mark.parametrize("bs", [16, 64, 128])
+@pytest.mark.parametrize("bs", [16, 48, 64, 128])
 def test_groups_blocks_and_chunk_edges(G, bs):
     Hk = 2
     lens = [1, 255, 256, 257, 511, 1000, 0, 33]
@@ -78,3 +79,30 @@ def test_agrees_with_the_q8_kernel_on_the_same_values():
                            dev(rep(vs)), dev(w.block_table), dev(w.seq_lens), w.scale)
     torch.cuda.synchronize()
     assert_close(out4.cpu().numpy(), out8.cpu().numpy().astype(np.float64), "q4 vs q8 kernel")
+
+
+@pytest.mark.parametrize("G", [3, 6, 12])
+def test_groups_that_are_not_powers_of_two(G):
+    # served by the next power-of-two instantiation, whose extra heads are padding
+    Hk = 2
+    lens = [300, 1, 600]
+    w = inputs.make_q4_custom(len(lens), G * Hk, Hk, 128, lens, 64, seed=G)
+    assert_close(run_q4(w), oracle.decode_q4_all(oracle_q4(w), w.q), f"G={G}")
+
+
+def test_bad_block_table_entries_are_flagged_and_skipped():
+    w = inputs.make_q4_custom(3, 8, 2, 128, [300, 520, 64], 16, seed=21)
+    q8.q8kv_device_errors(clear=True)
+    ref = run_q4(w)
+    assert q8.q8kv_device_errors(clear=True) == 0
+    # an entry past the pool: tokens 320-335 of sequence 1 are skipped, the flag is raised
+    w.block_table[1, 20] = w.num_blocks + 5
+    got = run_q4(w)
+    assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
+    np.testing.assert_array_equal(got[0], ref[0])
+    np.testing.assert_array_equal(got[2], ref[2])
+    assert np.all(np.isfinite(got[1]))
+    # a negative entry
+    w.block_table[1, 20] = -3
+    run_q4(w)
+    assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
