@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "q8-KV decode attention: µs/call and effective KV GB/s (% of B200 HBM peak)"
 UNIT = "GB/s"
-DEFAULT_CONFIG = 1  # the batched GQA decode workload the metric is quoted on
+DEFAULT_WORKLOAD = 1  # the batched GQA decode workload the metric is quoted on
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAK_GBS = 6650.0
 LAUNCHES_PER_CALL = 2  # decode kernel + split combine kernel
@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
+    ap.add_argument("--config", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -323,7 +323,7 @@ def run_accuracy_study(args):
     # the first three workloads whole (their unquantised draws kept); the two multi-GB ones
     # with their recipe on 8 sequences (the fp32 copies of 4 GB pools would not fit the
     # host budget of this study)
-    C = inputs.CONFIGS
+    C = inputs.WORKLOADS
     lens3 = inputs._seq_lens(C[3])[:8]
     study = [(C[0], inputs.make(C[0], keep_fp32=True), 64),
              (C[1], inputs.make(C[1], keep_fp32=True), 256),
@@ -802,7 +802,7 @@ def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):
     import decode_attention_int8_b200 as q8
     from decode_attention_int8_b200 import inputs
 
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.WORKLOADS[1]
     rows = inputs.make_prompt_fill(cfg)
     n, Hk, D, bs = rows.n_tokens, cfg.n_kv_heads, cfg.head_dim, cfg.block_size
     P = int(rows.slots.max()) // bs + 1

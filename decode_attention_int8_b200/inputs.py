@@ -64,7 +64,7 @@ class Config:
 
 # The five workloads: shapes and distributions of long-context GQA decode over paged
 # int8 caches (head_dim 128, contexts 256 to 128K).
-CONFIGS = [
+WORKLOADS = [
     Config("tiny_mha", 1, 8, 8, 128, 256, 16, "identity", seed=0,
            description="B=1, 8/8 heads, L=256, block 16, identity table"),
     Config("gqa_batch", 16, 32, 8, 128, 4096, 64, "permutation", seed=1,
@@ -236,9 +236,9 @@ def make_custom(B, n_q_heads, n_kv_heads, head_dim, seq_lens, block_size, *, tab
 
 
 def make(cfg: Config | int, *, keep_fp32: bool = False, threads: int | None = None) -> Workload:
-    """The named workload ``cfg`` (a Config or an index into CONFIGS)."""
+    """The named workload ``cfg`` (a Config or an index into WORKLOADS)."""
     if isinstance(cfg, int):
-        cfg = CONFIGS[cfg]
+        cfg = WORKLOADS[cfg]
     return _make(cfg, _seq_lens(cfg), None, 0, keep_fp32, threads)
 
 
@@ -358,7 +358,7 @@ def make_prompt_fill(cfg: Config | int, *, threads: int | None = None) -> CacheR
     """Fresh fp32 K/V rows for every token of a named workload, with the slots its block
     table gives them: the write that fills that workload's whole cache."""
     if isinstance(cfg, int):
-        cfg = CONFIGS[cfg]
+        cfg = WORKLOADS[cfg]
     threads = threads or min(32, os.cpu_count() or 1)
     lens = _seq_lens(cfg)
     bs = cfg.block_size
@@ -472,7 +472,7 @@ def make_q4(cfg: Config | int, *, seq_lens=None, keep_fp32: bool = False,
             threads: int | None = None) -> WorkloadQ4:
     """The named (or given) workload with a q4_0 cache."""
     if isinstance(cfg, int):
-        cfg = CONFIGS[cfg]
+        cfg = WORKLOADS[cfg]
     threads = threads or min(32, os.cpu_count() or 1)
     seq_lens = _seq_lens(cfg) if seq_lens is None else np.asarray(seq_lens, np.int32)
     bs, Hk, D = cfg.block_size, cfg.n_kv_heads, cfg.head_dim

@@ -166,7 +166,7 @@ def test_no_tokens_changes_nothing():
 def test_prompt_fill_of_the_gqa_batch_workload():
     # the full-size write that the benchmark times: 16 x 4096 tokens x 8 KV heads, D 128,
     # slots of the workload's permuted 1024-block table
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.WORKLOADS[1]
     rows = inputs.make_prompt_fill(cfg)
     P = int(rows.slots.max()) // cfg.block_size + 1
     pools = host_pools(P, cfg.block_size, cfg.n_kv_heads, cfg.head_dim)

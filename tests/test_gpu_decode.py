@@ -216,8 +216,8 @@ def test_device_side_checks_flag_bad_tables_without_faulting():
 @pytest.mark.parametrize("idx", [0, 1, 2])
 def test_workload_full_parity(idx):
     w = inputs.make(idx)
-    max_abs, rel = check_full(w, inputs.CONFIGS[idx].name)
-    print(f"\n{inputs.CONFIGS[idx].name}: max_abs={max_abs:.3e} rel_l2={rel:.3e}")
+    max_abs, rel = check_full(w, inputs.WORKLOADS[idx].name)
+    print(f"\n{inputs.WORKLOADS[idx].name}: max_abs={max_abs:.3e} rel_l2={rel:.3e}")
 
 
 @pytest.mark.slow
@@ -235,6 +235,6 @@ def test_workload_sampled_parity(idx):
         pairs += [(b, 0), (b, Hq - 1)]
     ref = oracle.decode_pairs(oracle_cache(w), w.q, pairs)
     sel = np.stack([got[b, h] for b, h in pairs])
-    max_abs, rel = assert_close(sel, ref, inputs.CONFIGS[idx].name)
-    print(f"\n{inputs.CONFIGS[idx].name}: sampled {len(pairs)} rows max_abs={max_abs:.3e} "
+    max_abs, rel = assert_close(sel, ref, inputs.WORKLOADS[idx].name)
+    print(f"\n{inputs.WORKLOADS[idx].name}: sampled {len(pairs)} rows max_abs={max_abs:.3e} "
           f"rel_l2={rel:.3e}")

@@ -78,7 +78,7 @@ def test_long_split_sequence_with_many_queries():
 def test_gqa_batch_workload_with_four_queries():
     # the benchmark's 16 x 4096-token workload with 3 draft tokens + 1 (nq = 4), as timed
     # by bench.py; 160 sampled (sequence, query, head) rows against the oracle
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.WORKLOADS[1]
     nq = 4
     w = inputs.make(cfg)
     q = inputs.multi_queries(cfg.B, nq, cfg.n_q_heads, cfg.head_dim, seed=cfg.seed)
