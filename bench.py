@@ -595,13 +595,14 @@ def main():
 
 CACHE_WRITE_SOURCES = ("q8kv_cache_write.cuh", "q8kv_cache_write_api.cuh", "q8kv_ptx.cuh")
 QUEST_SOURCES = ("q8kv_quest.cuh", "q8kv_quest_api.cuh", "q8kv_ptx.cuh")
+Q4_SOURCES = ("q8kv_q4.cuh", "q8kv_q4_api.cuh", "q8kv_ptx.cuh", "q8kv_qquant.cuh", "q8kv_decode.cuh")
 
 
 def source_hash(kernel: str = "decode") -> str:
     """Hash of the sources a kernel is built from (traffic figures are valid only for the
-    exact kernel): the cache write's or the QUEST metadata's own kernel and host files and
-    the PTX helpers, or, for the decode call, every other source of the library (its
-    kernels, helpers and plan)."""
+    exact kernel): the cache write's, the QUEST metadata's or the q4_0 decode's own kernel
+    and host files and the helpers they include, or, for the q8 decode call, every other
+    source of the library (its kernels, helpers and plan)."""
     import hashlib
 
     h = hashlib.sha256()
@@ -611,8 +612,10 @@ def source_hash(kernel: str = "decode") -> str:
             mine = name in CACHE_WRITE_SOURCES
         elif kernel == "quest":
             mine = name in QUEST_SOURCES
+        elif kernel == "q4":
+            mine = name in Q4_SOURCES
         else:
-            mine = not name.startswith(("q8kv_cache_write", "q8kv_quest"))
+            mine = not name.startswith(("q8kv_cache_write", "q8kv_quest", "q8kv_q4"))
         if not mine:
             continue
         with open(os.path.join(csrc, name), "rb") as f:
@@ -784,6 +787,7 @@ def bench_q4(dev, stream, steps=2000, warmup=20):
             "us_per_call": round(ms * 1e3, 3), "calls": steps, "algorithmic_bytes": algo,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                         "traffic": recorded_traffic("gqa_batch_q4", "q4"),
                          "kernel": "q8kv::q4_decode_kernel + q8kv::q4_combine_kernel"},
             "l2": f"pool rotated over {n_copies} copies"}
 

@@ -87,9 +87,15 @@ template <int GT>
 struct Q4Smem {
     uint8_t k[kQ4Chunk][kQ4Row]; // 16-byte chunks at position chunk ^ q4_swz(token)
     uint8_t v[kQ4Chunk][kQ4Row];
-    uint2 kd[kQ4Chunk];          // the 4 binary16 block scales of the token's row
-    uint2 vd[kQ4Chunk];
-    uint2 pb[kQ4Warps][Q4Shape<GT>::NS][3][32]; // P byte planes as PV B fragments
+    float kdf[kQ4Chunk][kNB];    // the token's 4 block scales, converted once to fp32
+    float vdf[kQ4Chunk][kNB];
+    union {
+        uint2 pb[kQ4Warps][Q4Shape<GT>::NS][3][32]; // P byte planes as PV B fragments
+        struct {
+            uint2 kd[kQ4Chunk]; // binary16 scales as copied; read only before the first
+            uint2 vd[kQ4Chunk]; // barrier, long before the planes are written
+        } raw;
+    } u;
     uint32_t qw[GT][32]; // word 2m: channels 8m, 8m+2, 8m+4, 8m+6; word 2m+1: the odd ones
     float qsc[GT][kNB];
     float smax[kQ4Warps][GT];
@@ -97,6 +103,9 @@ struct Q4Smem {
     uint32_t dvmax[kQ4Warps][kNB]; // largest |dv| bit pattern of the warp's slice per block
     uint32_t valid[kQ4Warps];      // tokens of the slice with data
 };
+
+static_assert(sizeof(uint2) * kQ4Warps * 3 * 32 >= sizeof(uint2) * 2 * kQ4Chunk,
+              "the raw scales must fit in the P planes of one n-tile");
 
 template <int GT>
 __host__ __device__ constexpr size_t q4_smem_bytes()
@@ -238,8 +247,8 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
             cp_async16(kdst + 16u * ((uint32_t)i ^ sw), kr + 16 * i, n16);
             cp_async16(vdst + 16u * ((uint32_t)i ^ sw), vr + 16 * i, n16);
         }
-        cp_async8(smem_addr(&sm.kd[tl]), p.kd + row * kNB, n8);
-        cp_async8(smem_addr(&sm.vd[tl]), p.vd + row * kNB, n8);
+        cp_async8(smem_addr(&sm.u.raw.kd[tl]), p.kd + row * kNB, n8);
+        cp_async8(smem_addr(&sm.u.raw.vd[tl]), p.vd + row * kNB, n8);
         asm volatile("cp.async.commit_group;" ::: "memory");
         const unsigned vm = __ballot_sync(kFullMask, ok);
         if (lane == 0)
@@ -270,10 +279,16 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
         }
     }
 
-    // the slice's largest |dv| per block (this lane's own copy: visible after the wait)
+    // this lane's token: scales to fp32, and the slice's largest |dv| per block (the
+    // lane's own copies are visible to it after the wait)
     asm volatile("cp.async.wait_all;" ::: "memory");
     {
-        const uint2 vd = sm.vd[warp * 32 + lane];
+        const int tl = warp * 32 + lane;
+        const uint2 kd = sm.u.raw.kd[tl], vd = sm.u.raw.vd[tl];
+        *reinterpret_cast<float4 *>(&sm.kdf[tl][0]) =
+            make_float4(half_of(kd, 0), half_of(kd, 1), half_of(kd, 2), half_of(kd, 3));
+        *reinterpret_cast<float4 *>(&sm.vdf[tl][0]) =
+            make_float4(half_of(vd, 0), half_of(vd, 1), half_of(vd, 2), half_of(vd, 3));
         const uint32_t a[4] = {vd.x & 0x7fffu, (vd.x >> 16) & 0x7fffu, vd.y & 0x7fffu,
                                (vd.y >> 16) & 0x7fffu};
 #pragma unroll
@@ -322,7 +337,6 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
             kb1[j] = nib_odd_s8x16(kr[j]);
         }
         const int ta = warp * 32 + 8 * ntile + 2 * c;
-        const uint2 kd0 = sm.kd[ta], kd1 = sm.kd[ta + 1];
 #pragma unroll
         for (int s = 0; s < S::NSLOT; ++s) {
             sc[s][ntile][0] = 0.f;
@@ -342,8 +356,9 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
                 const float x0 = __int_as_float(d[2 * hlf]) - kQ4Bias;
                 const float x1 = __int_as_float(d[2 * hlf + 1]) - kQ4Bias;
                 const int j = jr[mt][hlf];
-                sc[slot][ntile][0] = fmaf(x0, wq[mt][hlf] * half_of(kd0, j), sc[slot][ntile][0]);
-                sc[slot][ntile][1] = fmaf(x1, wq[mt][hlf] * half_of(kd1, j), sc[slot][ntile][1]);
+                sc[slot][ntile][0] = fmaf(x0, wq[mt][hlf] * sm.kdf[ta][j], sc[slot][ntile][0]);
+                sc[slot][ntile][1] =
+                    fmaf(x1, wq[mt][hlf] * sm.kdf[ta + 1][j], sc[slot][ntile][1]);
             }
         }
     }
@@ -426,7 +441,7 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
             for (int i = 0; i < 4; ++i) {
                 const int ntile = 2 * half + (i >> 1), e = i & 1;
                 const int t = warp * 32 + 8 * ntile + 2 * c + e;
-                const float dvs = half_of(sm.vd[t], j) * pscale;
+                const float dvs = sm.vdf[t][j] * pscale;
                 const float x = fmaf(sc[slot][ntile][e], dvs, kQ4Bias);
                 P[i] = live ? __float_as_int(x) - kDotBias : 0;
             }
@@ -440,7 +455,7 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
         }
 #pragma unroll
         for (int k = 0; k < 3; ++k)
-            sm.pb[warp][ns][k][lane] = make_uint2(planes[k][0], planes[k][1]);
+            sm.u.pb[warp][ns][k][lane] = make_uint2(planes[k][0], planes[k][1]);
     }
     __syncthreads(); // every slice's P
 
@@ -477,9 +492,9 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
                 a[i] = nib_s8x16(r[i], vsh);
 #pragma unroll
             for (int si = 0; si < SPB; ++si) {
-                const uint2 b0 = sm.pb[sl][ns0 + si][0][lane];
-                const uint2 b1 = sm.pb[sl][ns0 + si][1][lane];
-                const uint2 b2 = sm.pb[sl][ns0 + si][2][lane];
+                const uint2 b0 = sm.u.pb[sl][ns0 + si][0][lane];
+                const uint2 b1 = sm.u.pb[sl][ns0 + si][1][lane];
+                const uint2 b2 = sm.u.pb[sl][ns0 + si][2][lane];
                 mma_s8u8_16832_acc(acc[si][0], a[0], a[1], a[2], a[3], b0.x, b0.y, acc[si][0]);
                 mma_s8u8_16832_acc(acc[si][1], a[0], a[1], a[2], a[3], b1.x, b1.y, acc[si][1]);
                 mma_s8_16832_acc(acc[si][2], a[0], a[1], a[2], a[3], b2.x, b2.y, acc[si][2]);
