@@ -6,15 +6,23 @@ split combine), through the C ABI. Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl reference]
 
+Headline: the bandwidth-saturating workload (B = 256 sequences of 8192 tokens, 32 q heads
+over 8 KV heads, 4.44 GB of K/V read per call), the largest of the five workloads and the
+one that fits a single GPU with the most work; the metric is not quoted on any one
+workload, so the largest is timed. The other four workloads, and the group-8 reading of
+the 16 x 4096-token batch, follow as per-workload legs of the same line, each with its
+own time, bandwidth, clocks and sampled-row parity against the oracle.
+
 Metric: effective KV bandwidth = algorithmic bytes of one call / time per call, where the
 algorithmic bytes are every valid (token, KV head) K row, V row and both scales once, plus
 q read and out written in fp32, the used block-table entries and seq_lens.
 
-Timing: the KV pool is rotated over enough copies that their total exceeds 4x the L2 size,
-so every call streams from HBM; W untimed calls, then K calls bracketed by a barrier and a
-device synchronisation, timed with CUDA events on the launching stream; the maximum over
-ranks is reported. Under torchrun every rank runs its own copy of the workload on its own
-GPU (independent sequences, no collective on the data path): weak scaling.
+Timing: inputs larger than L2 (the headline's 4.4 GB pool; smaller pools rotated over
+copies whose total exceeds 4x the L2 size; the tiny workload flushes L2 before each call);
+W untimed calls, then K calls bracketed by a barrier and a device synchronisation, timed
+with CUDA events on the launching stream; the maximum over ranks is reported. Under
+torchrun every rank runs its own copy of the workload on its own GPU (independent
+sequences, no collective on the data path): weak scaling.
 """
 from __future__ import annotations
 
@@ -24,7 +32,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -34,21 +41,25 @@ sys.path.insert(0, ROOT)
 
 METRIC = "q8-KV decode attention: µs/call and effective KV GB/s (% of B200 HBM peak)"
 UNIT = "GB/s"
-DEFAULT_WORKLOAD = 1  # the batched GQA decode workload the metric is quoted on
+DEFAULT_WORKLOAD = 4  # bandwidth: the largest single-GPU workload (4.44 GB per call)
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAK_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
 LAUNCHES_PER_CALL = 2  # decode kernel + split combine kernel
+PARITY_MAX_ABS, PARITY_REL_L2 = 1e-4, 1e-5  # output tolerance against the fp64 oracle
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the per-workload legs (the other workloads, group 8)")
     ap.add_argument("--no-accuracy", action="store_true",
                     help="skip the q8-vs-fp32 information report")
     ap.add_argument("--no-cache-write", action="store_true",
@@ -98,141 +109,430 @@ def measured_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples of one GPU while the timed region runs."""
+    """SM clock and clock-event reasons of one GPU, polled through NVML every 2 ms in a
+    background thread, so that even a timed region of a few milliseconds holds samples."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
-        self.window = None
+    def __init__(self, device):
+        self.samples = []  # (host monotonic time, sm MHz, reason bits)
+        self.h = None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            idx = torch.cuda._get_nvml_device_index(device)
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.h = None
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except Exception:
-            self.proc = None
+        if self.h is None:
+            return self
+        nv = self.nvml
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.monotonic(), line.strip()))
+        def run():
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((time.monotonic(), float(sm), int(rs)))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
 
-    def mark(self, t0: float, t1: float):
-        """Keep only the samples taken between host times t0 and t1 (the timed region)."""
-        self.window = (t0, t1)
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        return self
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = self.lines
-        if self.window is not None:
-            inside = [(t, ln) for t, ln in lines if self.window[0] <= t <= self.window[1]]
-            lines = inside if inside else lines
-        for _, ln in lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        """Median SM clock and the union of reasons over the samples taken between host
+        times t0 and t1 (the timed region); when none falls inside, the nearest sample
+        on either side."""
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"],
+                    "samples": 0}
+        s = list(self.samples)
+        inside = [x for x in s if t0 <= x[0] <= t1]
+        if not inside and s:
+            before = [x for x in s if x[0] < t0][-1:]
+            after = [x for x in s if x[0] > t1][:1]
+            inside = before + after
+        bits = 0
+        for x in inside:
+            bits |= x[2]
+        return {"sm_mhz": statistics.median([x[1] for x in inside]) if inside else None,
+                "sm_max_mhz": self.max_mhz,
+                "reasons": [n for n, b in self.REASONS if bits & b],
+                "samples": len(inside)}
 
 
-def workload_config(w, n_copies, extra):
+# ------------------------------------------------------------------ workloads on the device
+
+
+def n_pool_copies(pool_bytes: int) -> int:
+    """Device copies of the KV pool that the timed calls rotate over: enough for the copies
+    to exceed 4x the L2 size, 1 when the pool alone is that large, 0 (flush L2 before every
+    call instead) when even 64 copies would not be."""
+    if pool_bytes >= 4 * L2_BYTES:
+        return 1
+    n = math.ceil(4 * L2_BYTES / pool_bytes) + 1
+    return n if n <= 64 else 0
+
+
+def pool_bytes_of(w) -> int:
+    return int(w.k.nbytes + w.v.nbytes + w.ks.nbytes + w.vs.nbytes)
+
+
+def l2_note(w) -> str:
+    pb = pool_bytes_of(w)
+    n = n_pool_copies(pb)
+    if n == 1:
+        return f"inputs larger than L2: {pb / 1e9:.2f} GB KV pool > {L2_BYTES / 1e6:.0f} MB L2"
+    if n == 0:
+        return (f"L2 flushed before every call (a {2 * L2_BYTES / 1e6:.0f} MB buffer written); "
+                f"calls timed one at a time")
+    return (f"inputs larger than L2: KV pool rotated over {n} copies "
+            f"({n * pb / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)")
+
+
+def workload_config(w, world: int) -> dict:
+    """The `config` of a JSON line; both arms print the same dict for the same workload."""
     c = w.cfg
     lens = w.seq_lens
-    d = {"workload": c.name, "B": c.B, "n_q_heads": c.n_q_heads, "n_kv_heads": c.n_kv_heads,
-         "head_dim": c.head_dim, "kv_block_size": c.block_size,
-         "seq_len": int(lens.max()) if lens.min() == lens.max() else
-         f"ragged {int(lens.min())}..{int(lens.max())} (sum {int(lens.sum())})",
-         "num_kv_blocks": w.num_blocks, "algorithmic_bytes": w.algorithmic_bytes(),
-         "l2": f"inputs larger than L2: KV pool rotated over {n_copies} copies "
-               f"({n_copies * (w.k.nbytes + w.v.nbytes + w.ks.nbytes + w.vs.nbytes) / 1e6:.0f} MB"
-               f" > {L2_BYTES / 1e6:.0f} MB L2)"}
-    d.update(extra)
-    return d
+    return {"workload": c.name, "B": c.B, "n_q_heads": c.n_q_heads, "n_kv_heads": c.n_kv_heads,
+            "head_dim": c.head_dim, "kv_block_size": c.block_size,
+            "seq_len": int(lens.max()) if lens.min() == lens.max() else
+            f"ragged {int(lens.min())}..{int(lens.max())} (sum {int(lens.sum())})",
+            "num_kv_blocks": w.num_blocks, "algorithmic_bytes": w.algorithmic_bytes(),
+            "k_dist": c.k_dist, "v_dist": c.v_dist, "k_bias_std": c.k_bias_std, "seed": c.seed,
+            "l2": l2_note(w), "parallelism": f"replicas{world}"}
 
 
-def q8_vs_fp32(w, got, n_rows=64, seed=0):
+def sample_pairs(w, n_rows: int, seed: int):
+    """Random (sequence, head) rows of sequences with tokens, plus the first and last head of
+    the longest and the shortest sequence."""
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    live = np.flatnonzero(w.seq_lens > 0)
+    Hq = w.cfg.n_q_heads
+    pairs = {(int(live[i]), int(h)) for i, h in zip(rng.integers(0, len(live), n_rows),
+                                                    rng.integers(0, Hq, n_rows))}
+    for b in (int(live[np.argmax(w.seq_lens[live])]), int(live[np.argmin(w.seq_lens[live])])):
+        pairs |= {(b, 0), (b, Hq - 1)}
+    return sorted(pairs)
+
+
+def parity_rows(w, got, n_rows: int, seed: int) -> dict:
+    """The CUDA output against the fp64 oracle on sampled rows (every row when the workload
+    has at most n_rows): max |gpu - oracle| and relative L2, the outputs-equal column."""
+    import numpy as np
+
+    import oracle
+
+    cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
+                              w.cfg.n_q_heads, w.scale)
+    B, Hq = w.cfg.B, w.cfg.n_q_heads
+    t = time.perf_counter()
+    if B * Hq <= n_rows:
+        ref = oracle.decode_all(cache, w.q).reshape(B * Hq, -1)
+        sel = np.asarray(got, np.float64).reshape(B * Hq, -1)
+        rows = B * Hq
+    else:
+        pairs = sample_pairs(w, n_rows, seed)
+        ref = oracle.decode_pairs(cache, w.q, pairs)
+        sel = np.stack([np.asarray(got[b, h], np.float64) for b, h in pairs])
+        rows = len(pairs)
+    d = sel - ref
+    max_abs = float(np.abs(d).max())
+    rel = float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
+    return {"rows": rows, "of_rows": B * Hq, "max_abs": max_abs, "rel_l2": rel,
+            "within_tolerance": bool(np.all(np.isfinite(sel)) and max_abs <= PARITY_MAX_ABS
+                                     and rel <= PARITY_REL_L2),
+            "tolerance": {"max_abs": PARITY_MAX_ABS, "rel_l2": PARITY_REL_L2},
+            "oracle_s": round(time.perf_counter() - t, 2)}
+
+
+class DeviceWorkload:
+    """A workload on the device with its KV pool copies and prepared C-ABI argument sets
+    (one per pool copy), so that a timed call costs one foreign call and no marshalling."""
+
+    def __init__(self, w, dev, stream):
+        import numpy as np
+        import torch
+
+        import decode_attention_int8_b200 as q8
+
+        self.w, self.dev, self.stream = w, dev, stream
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        self.n_copies = n_pool_copies(pool_bytes_of(w))
+        self.q = t(w.q)
+        self.bt = t(w.block_table)
+        self.lens = t(w.seq_lens)
+        self.pools = [(t(w.k), t(w.v), t(w.ks), t(w.vs)) for _ in range(max(1, self.n_copies))]
+        self.out = torch.empty(self.q.shape, dtype=torch.float32, device=dev)
+        self.flush = (torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+                      if self.n_copies == 0 else None)
+        c = w.cfg
+        self.geo = (c.B, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block_size,
+                    w.max_blocks_per_seq, w.num_blocks)
+        self.sp = ctypes.c_void_p(stream.cuda_stream)
+        self.fn = q8.lib().q8kv_decode_attn
+        self.q8 = q8
+        self.argsets = [self.args(self.out, self.q, self.bt, self.lens, pool)
+                        for pool in self.pools]
+
+    def args(self, out, q, bt, lens, pool=None, stream=None):
+        P = lambda x: ctypes.c_void_p(x.data_ptr())
+        k, v, ks, vs = pool or self.pools[0]
+        sp = self.sp if stream is None else ctypes.c_void_p(stream.cuda_stream)
+        return (P(out), P(q), P(k), P(v), P(ks), P(vs), P(bt), P(lens), *self.geo,
+                ctypes.c_float(self.w.scale), sp)
+
+    def call(self, i: int):
+        st = self.fn(*self.argsets[i % len(self.argsets)])
+        if st != 0:
+            raise self.q8.Q8KVError(st, "q8kv_decode_attn")
+
+    def time_calls(self, n: int) -> float:
+        """ms per call of n calls: back to back between two events on the launching stream
+        (no event between calls, which would break the programmatic-dependent-launch overlap
+        of consecutive calls), or, for a flushed workload, the median of calls timed one at
+        a time after an L2 flush each."""
+        import torch
+
+        if self.flush is None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            for i in range(n):
+                self.call(i)
+            e1.record(self.stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / n
+        times = []
+        for i in range(n):
+            self.flush.fill_(i & 0xff)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            self.call(i)
+            e1.record(self.stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    def isolated_us(self, n: int) -> float:
+        """Median of single calls between their own events (information)."""
+        import torch
+
+        iso = []
+        for i in range(n):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            self.call(i)
+            e1.record(self.stream)
+            e1.synchronize()
+            iso.append(e0.elapsed_time(e1))
+        return statistics.median(iso) * 1e3
+
+    def result(self):
+        import torch
+
+        self.call(0)
+        torch.cuda.synchronize(self.dev)
+        return self.out.cpu().numpy()
+
+
+def e2e_pipelined(dw, steps: int, pg):
+    """End to end through the C ABI with host buffers, as a serving loop runs it: every step
+    copies that step's q, block table and seq_lens from pinned host memory to the device,
+    runs the call, and copies `out` back to pinned host memory. The copies run on their own
+    streams into double buffers, so step i + 1's inputs move while step i computes; the
+    events between the streams keep every buffer's reads after its writes. Timed with two
+    events on the compute stream around all steps."""
+    import torch
+
+    w, dev, comp = dw.w, dw.dev, dw.stream
+    hq = torch.from_numpy(w.q).pin_memory()
+    hbt = torch.from_numpy(w.block_table).pin_memory()
+    hlens = torch.from_numpy(w.seq_lens).pin_memory()
+    hout = [torch.empty(dw.out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    dq = [torch.empty_like(dw.q) for _ in range(2)]
+    dbt = [torch.empty_like(dw.bt) for _ in range(2)]
+    dlens = [torch.empty_like(dw.lens) for _ in range(2)]
+    dout = [torch.empty_like(dw.out) for _ in range(2)]
+    args = [dw.args(dout[j], dq[j], dbt[j], dlens[j], stream=comp) for j in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_comp, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [False, False]
+
+    def h2d(i):
+        j = i % 2
+        if used[j]:
+            s_in.wait_event(ev_comp[j])  # the call that last read buffer j has finished
+        with torch.cuda.stream(s_in):
+            dq[j].copy_(hq, non_blocking=True)
+            dbt[j].copy_(hbt, non_blocking=True)
+            dlens[j].copy_(hlens, non_blocking=True)
+        ev_in[j].record(s_in)
+
+    def run(n):
+        for j in range(2):
+            used[j] = False
+        h2d(0)
+        for i in range(n):
+            j = i % 2
+            if i + 1 < n:
+                h2d(i + 1)
+            comp.wait_event(ev_in[j])
+            if used[j]:
+                comp.wait_event(ev_out[j])  # out[j] of step i - 2 has reached the host
+            st = dw.fn(*args[j])
+            if st != 0:
+                raise dw.q8.Q8KVError(st, "q8kv_decode_attn")
+            used[j] = True
+            ev_comp[j].record(comp)
+            s_out.wait_event(ev_comp[j])
+            with torch.cuda.stream(s_out):
+                hout[j].copy_(dout[j], non_blocking=True)
+            ev_out[j].record(s_out)
+        for j in range(2):
+            comp.wait_event(ev_out[j])
+
+    run(3)
+    torch.cuda.synchronize(dev)
+    if pg is not None:
+        pg.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    s_in.wait_event(e0)
+    run(steps)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(e0.elapsed_time(e1) / steps, pg, dev)
+    return ms, {"h2d_bytes_per_step": int(w.q.nbytes + w.block_table.nbytes + w.seq_lens.nbytes),
+                "d2h_bytes_per_step": int(w.q.nbytes), "steps": steps,
+                "pipeline": "inputs of step i+1 copied during step i (copy streams, double "
+                            "buffers)"}
+
+
+def bench_leg(w, dev, stream, min_calls=50, target_s=0.25, parity_n=64, seed=0):
+    """One workload as an information leg of the line: µs per call (back to back, rotated
+    pools or flushed L2), bandwidth, fractions of the measured and the nominal HBM peak,
+    the clocks during its timed calls, and sampled-row parity against the oracle."""
+    import torch
+
+    dw = DeviceWorkload(w, dev, stream)
+    for i in range(5):
+        dw.call(i)
+    torch.cuda.synchronize(dev)
+    est = dw.time_calls(10)
+    n = max(min_calls, int(target_s / max(est * 1e-3, 1e-6)))
+    if dw.flush is not None:
+        n = min(n, 400)
+    sampler = ClockSampler(dev).start()
+    time.sleep(0.02)
+    h0 = time.monotonic()
+    ms = dw.time_calls(n)
+    h1 = time.monotonic()
+    sampler.stop()
+    algo = w.algorithmic_bytes()
+    peak, peak_kind = measured_peak()
+    gbs = algo / (ms * 1e-3) / 1e9
+    got = dw.result()
+    leg = {"config": workload_config(w, 1), "us_per_call": round(ms * 1e3, 3), "calls": n,
+           "GB/s": round(gbs, 2), "frac_of_measured_hbm": round(gbs / peak, 4),
+           "frac_of_8TBps_nominal": round(gbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
+           "clocks": sampler.summary(h0, h1),
+           "device_errors": dw.q8.q8kv_device_errors(clear=True),
+           "parity_vs_oracle": parity_rows(w, got, parity_n, seed)}
+    return leg, dw
+
+
+def cpu_sample_rate(w, seconds: float, seed: int = 0):
+    """The oracle as it stands, single-threaded, on random (sequence, head) rows of the
+    workload for about `seconds`; bytes counted pro rata to the rows done. Returns
+    (GB/s, rows done, rows in the workload, elapsed s)."""
+    import numpy as np
+
+    import oracle
+
+    cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
+                              w.cfg.n_q_heads, w.scale)
+    B, Hq = w.cfg.B, w.cfg.n_q_heads
+    pairs_all = [(b, h) for b in range(B) for h in range(Hq) if w.seq_lens[b] > 0]
+    rng = np.random.default_rng(seed)
+    done, t0 = 0, time.perf_counter()
+    chunk = 1
+    while True:
+        sel = rng.choice(len(pairs_all), min(chunk, len(pairs_all)), replace=False)
+        oracle.decode_pairs(cache, w.q, [pairs_all[j] for j in sel])
+        done += len(sel)
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+        chunk = min(len(pairs_all), max(1, chunk * 2 if dt < seconds / 4 else chunk))
+    gbs = w.algorithmic_bytes() * done / len(pairs_all) / dt / 1e9
+    return gbs, done, len(pairs_all), dt
+
+
+def cpu_baseline(w, seconds=12.0):
+    gbs, done, total, dt = cpu_sample_rate(w, seconds)
+    return {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} random (sequence, head) rows of {total} ({w.cfg.name}), "
+                      f"{dt:.1f} s, single-threaded C oracle; bytes counted pro rata"}
+
+
+def q8_vs_fp32(w, got, n_seqs=4, heads_per_seq=16, seed=0):
     """Information only: how far the q8 path's output is from attention over the unquantised
-    fp32 q, K, V (plain fp64 numpy softmax(q K^T * scale) V on a sample of (sequence, head)
-    rows). This measures the int8 quantisation itself, not the kernel's arithmetic."""
+    fp32 q, K, V (plain fp64 numpy softmax(q K^T * scale) V on sampled (sequence, head)
+    rows; each sampled sequence's fp32 rows are regenerated once from their random
+    streams). This measures the int8 quantisation itself, not the kernel's arithmetic."""
     import numpy as np
 
     from decode_attention_int8_b200 import inputs
 
     c = w.cfg
-    fp32_pool_bytes = 2 * 4 * w.k.size
-    if fp32_pool_bytes > (2 << 30):
-        return {"skipped": f"the unquantised fp32 pools would take {fp32_pool_bytes / 1e9:.1f} GB "
-                           "of host memory"}
-    w32 = inputs.make(c, keep_fp32=True)
-    P, bs, Hk, D = w32.k.shape
-    k32 = w32.k32.reshape(P * bs, Hk, D)
-    v32 = w32.v32.reshape(P * bs, Hk, D)
-    rng = np.random.default_rng(seed)
+    bs = c.block_size
     G = c.n_q_heads // c.n_kv_heads
+    rng = np.random.default_rng(seed)
+    live = np.flatnonzero(w.seq_lens > 0)
     diffs, refs = [], []
-    for _ in range(n_rows):
-        b = int(rng.integers(0, c.B))
-        h = int(rng.integers(0, c.n_q_heads))
-        L = int(w32.seq_lens[b])
-        if L == 0:
-            continue
+    for b in rng.choice(live, size=min(n_seqs, len(live)), replace=False):
+        L = int(w.seq_lens[b])
         t = np.arange(L)
-        slot = w32.block_table[b, t // bs].astype(np.int64) * bs + t % bs
-        kf = k32[slot, h // G].astype(np.float64)
-        vf = v32[slot, h // G].astype(np.float64)
-        sc = kf @ w32.q[b, h].astype(np.float64) * w32.scale
-        pr = np.exp(sc - sc.max())
-        ref = pr @ vf / pr.sum()
-        refs.append(ref)
-        diffs.append(np.asarray(got[b, h], np.float64) - ref)
+        slot = w.block_table[b, t // bs].astype(np.int64) * bs + t % bs
+        k32 = inputs.fp32_rows(w, "k", slot)
+        v32 = inputs.fp32_rows(w, "v", slot)
+        for h in rng.choice(c.n_q_heads, size=min(heads_per_seq, c.n_q_heads), replace=False):
+            kf = k32[:, h // G].astype(np.float64)
+            vf = v32[:, h // G].astype(np.float64)
+            sc = kf @ w.q[b, h].astype(np.float64) * w.scale
+            pr = np.exp(sc - sc.max())
+            ref = pr @ vf / pr.sum()
+            refs.append(ref)
+            diffs.append(np.asarray(got[b, h], np.float64) - ref)
     d, r = np.array(diffs), np.array(refs)
     return {"max_abs": float(np.abs(d).max()), "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(r)),
-            "rows": len(refs), "reference": "fp64 attention over the unquantised fp32 q, K, V"}
-
-
-def cpu_baseline(w, min_seconds=10.0):
-    """The oracle as it stands, single-threaded, on whole passes over the workload."""
-    import oracle
-
-    cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
-                              w.cfg.n_q_heads, w.scale)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle.decode_all(cache, w.q)
-        reps += 1
-        dt = time.perf_counter() - t0
-        if dt >= min_seconds:
-            break
-    gbs = w.algorithmic_bytes() * reps / dt / 1e9
-    return {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"whole workload ({w.cfg.B} sequences x {w.cfg.n_q_heads} heads), "
-                      f"{reps} passes, {dt:.1f} s, single-threaded C oracle"}
+            "rows": len(refs), "workload": c.name,
+            "reference": "fp64 attention over the unquantised fp32 q, K, V"}
 
 
 def _err_stats(got, ref):
@@ -356,13 +656,16 @@ def run_accuracy_study(args):
 
 
 def run_reference(args):
-    """--impl reference: the oracle on the host cores, on this arm's workload and metric."""
+    """--impl reference: the oracle on the host cores, on this arm's workload and metric.
+    Each step decodes a bounded random sample of (sequence, head) rows; the workload's
+    algorithmic bytes are counted pro rata to the rows done."""
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    from decode_attention_int8_b200 import inputs
     import numpy as np
+
     import oracle
+    from decode_attention_int8_b200 import inputs
 
     w = inputs.make(args.config)
     cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
@@ -377,29 +680,24 @@ def run_reference(args):
     n_pairs = int(max(1, min(len(pairs_all), budget / per_pair)))
     rng = np.random.default_rng(0)
 
-    def step(i):
-        # a random sample of (sequence, head) rows; the workload's algorithmic bytes are
-        # counted pro rata to the rows done
+    def step():
         sel = rng.choice(len(pairs_all), n_pairs, replace=False)
         oracle.decode_pairs(cache, w.q, [pairs_all[j] for j in sel])
         return n_pairs
 
-    for i in range(args.warmup):
-        step(i)
+    for _ in range(args.warmup):
+        step()
     t0 = time.perf_counter()
     done = 0
-    for i in range(args.steps):
-        done += step(i)
+    for _ in range(args.steps):
+        done += step()
     dt = time.perf_counter() - t0
-    frac = done / len(pairs_all)
-    gbs = w.algorithmic_bytes() * frac / dt / 1e9
+    gbs = w.algorithmic_bytes() * (done / len(pairs_all)) / dt / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.cfg.name, "B": B, "n_q_heads": Hq,
-                       "n_kv_heads": w.cfg.n_kv_heads, "head_dim": w.cfg.head_dim,
-                       "kv_block_size": w.cfg.block_size},
+            "config": workload_config(w, world),
             "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{n_pairs} random (sequence, head) rows per step of "
                                        f"{len(pairs_all)}; bytes counted pro rata"},
@@ -409,6 +707,15 @@ def run_reference(args):
     return 0
 
 
+# group-8 reading of the batched GQA workload's label: 64 q heads over its 8 KV heads
+def group8_workload():
+    from decode_attention_int8_b200 import inputs
+
+    c = inputs.WORKLOADS[1]
+    return inputs.make_custom(c.B, 64, c.n_kv_heads, c.head_dim, [c.seq_len] * c.B,
+                              c.block_size, seed=c.seed, name="gqa_batch_group8")
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -416,7 +723,6 @@ def main():
     if args.accuracy_study:
         return run_accuracy_study(args)
     world, rank, local = dist_env()
-    import numpy as np
     import torch
 
     import decode_attention_int8_b200 as q8
@@ -436,155 +742,106 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    w = inputs.make(args.config)
-    lib = q8.lib()
-    algo = w.algorithmic_bytes()
-    pool_bytes = w.k.nbytes + w.v.nbytes + w.ks.nbytes + w.vs.nbytes
-    n_copies = max(2, math.ceil(4 * L2_BYTES / pool_bytes) + 1) if pool_bytes < 8 * L2_BYTES else 1
-    n_copies = min(n_copies, 64)
-    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-    q = t(w.q)
-    bt = t(w.block_table)
-    lens = t(w.seq_lens)
-    pools = [(t(w.k), t(w.v), t(w.ks), t(w.vs)) for _ in range(n_copies)]
-    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    c = w.cfg
-    geo = (c.B, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block_size, w.max_blocks_per_seq,
-           w.num_blocks)
-    P = lambda x: ctypes.c_void_p(x.data_ptr())
-    argsets = [(P(out), P(q), P(k), P(v), P(ks), P(vs), P(bt), P(lens), *geo,
-                ctypes.c_float(w.scale), sp) for (k, v, ks, vs) in pools]
-    fn = lib.q8kv_decode_attn
-
-    def call(i):
-        st = fn(*argsets[i % n_copies])
-        if st != 0:
-            raise q8.Q8KVError(st, "q8kv_decode_attn")
+    w = inputs.make(args.config)
+    algo = w.algorithmic_bytes()
+    dw = DeviceWorkload(w, dev, stream)
+    q8.q8kv_device_errors(clear=True)
 
     # warm-up (also sizes the library workspace outside the timed region)
     for i in range(max(args.warmup, 1)):
-        call(i)
+        dw.call(i)
     torch.cuda.synchronize(dev)
 
     def barrier():
         if pg is not None:
             pg.barrier()
 
-    # timed region: K back-to-back calls between two CUDA events on the launching stream
-    # (events between the calls would sit between the kernels and break the programmatic
-    # dependent launch overlap of consecutive calls)
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
+    # timed region: K calls (back to back between two CUDA events on the launching stream,
+    # or one at a time after an L2 flush for a pool too small to rotate)
+    sampler = ClockSampler(dev).start()
+    time.sleep(0.05)
     barrier()
     torch.cuda.synchronize(dev)
     host_t0 = time.monotonic()
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_begin.record(stream)
-    for i in range(args.steps):
-        call(i)
-    t_end.record(stream)
+    ms_per_step = dw.time_calls(args.steps)
     torch.cuda.synchronize(dev)
     host_t1 = time.monotonic()
     barrier()
-    time.sleep(0.15)  # let the sampler deliver the last in-window line
-    sampler.mark(host_t0, host_t1)
-    clocks = sampler.stop()
-    total_ms = t_begin.elapsed_time(t_end)
-    total_ms = reduce_max(total_ms, pg, dev)
-    ms_per_step = total_ms / args.steps
-    kernel_ms = ms_per_step  # one step = the call's decode + combine kernels
-
-    # information only, outside the timed region: one call at a time between its own events
-    iso = []
-    for i in range(min(200, max(20, args.steps))):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        call(i)
-        e1.record(stream)
-        e1.synchronize()
-        iso.append(e0.elapsed_time(e1))
-    isolated_us = statistics.median(iso) * 1e3
+    sampler.stop()
+    clocks = sampler.summary(host_t0, host_t1)
+    ms_per_step = reduce_max(ms_per_step, pg, dev)
     value = whole_job_gbs(algo, world, ms_per_step)
+    isolated_us = dw.isolated_us(min(100, max(10, args.steps)))
+    got = dw.result()
+    dev_errors = q8.q8kv_device_errors(clear=True)
 
-    # end to end through the C ABI with host buffers: per step copy q / block table /
-    # seq_lens from pinned host memory, decode, copy out back (the KV cache stays resident)
     e2e = None
     if not args.no_e2e:
-        hq = torch.from_numpy(w.q).pin_memory()
-        hbt = torch.from_numpy(w.block_table).pin_memory()
-        hlens = torch.from_numpy(w.seq_lens).pin_memory()
-        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-        e2e_steps = max(10, min(args.steps, 2000))
-        for i in range(3):
-            q.copy_(hq, non_blocking=True)
-            call(i)
-            hout.copy_(out, non_blocking=True)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(e2e_steps):
-            q.copy_(hq, non_blocking=True)
-            bt.copy_(hbt, non_blocking=True)
-            lens.copy_(hlens, non_blocking=True)
-            call(i)
-            hout.copy_(out, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / e2e_steps
-        e2e_ms = reduce_max(e2e_ms, pg, dev)
+        e2e_ms, e2e_info = e2e_pipelined(dw, max(10, args.steps), pg)
         e2e = {"value": round(whole_job_gbs(algo, world, e2e_ms), 2), "unit": UNIT,
-               "h2d_bytes_per_step": int(w.q.nbytes + w.block_table.nbytes + w.seq_lens.nbytes),
-               "d2h_bytes_per_step": int(w.q.nbytes), "us_per_step": round(e2e_ms * 1e3, 3),
-               "steps": e2e_steps}
+               "us_per_step": round(e2e_ms * 1e3, 3), **e2e_info}
 
     peak, peak_kind = measured_peak()
-    achieved = algo / (kernel_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(c.name, "decode")
+    achieved = algo / (ms_per_step * 1e-3) / 1e9
+    traffic = recorded_traffic(w.cfg.name, "decode")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
         "us_per_call": round(ms_per_step * 1e3, 3),
         "us_per_call_isolated": round(isolated_us, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-        "config": workload_config(w, n_copies, {"parallelism": f"replicas{world}"}),
+        "config": workload_config(w, world),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
+                     "frac_of_8TBps_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                      "traffic": traffic,
                      "kernel": "q8kv::decode_kernel + q8kv::combine_kernel (one call)",
-                     "kernel_us": round(kernel_ms * 1e3, 3)},
+                     "kernel_us": round(ms_per_step * 1e3, 3)},
         "gpu_launches": LAUNCHES_PER_CALL * args.steps,
         "clocks": clocks,
+        "device_errors": dev_errors,
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if rank == 0:
+        line["parity_vs_oracle"] = parity_rows(w, got, 64, seed=args.config)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
-    if not args.no_multi_query:
-        # information, after the timed region: the same workload with n_queries new tokens
-        # per sequence (speculative decode), through q8kv_decode_attn_multi
-        line["multi_query"] = bench_multi_query(w, pools, bt, lens, dev, stream,
-                                                steps=max(10, min(args.steps, 2000)))
-    if not args.no_q4:
+    del dw
+    torch.cuda.empty_cache()
+
+    # information legs, after the timed region: every other workload (and the group-8
+    # reading of the batched one), each timed and checked against the oracle on its own
+    info = world == 1  # the scaling runs time the headline only
+    if info and not args.no_legs:
+        legs = {}
+        others = [i for i in range(len(inputs.WORKLOADS)) if i != args.config]
+        for i in others + ["group8"]:
+            wi = group8_workload() if i == "group8" else inputs.make(i)
+            leg, dwi = bench_leg(wi, dev, stream, seed=100 + (9 if i == "group8" else i))
+            if wi.cfg.name == "gqa_batch":
+                if not args.no_multi_query:
+                    # the same workload with n_queries new tokens per sequence (speculative
+                    # decode), through q8kv_decode_attn_multi
+                    line["multi_query"] = bench_multi_query(
+                        wi, dwi.pools, dwi.bt, dwi.lens, dev, stream,
+                        steps=max(10, min(args.steps, 2000)))
+                if rank == 0 and world == 1 and not args.no_accuracy:
+                    line["q8_vs_fp32"] = q8_vs_fp32(wi, dwi.result())
+            legs[wi.cfg.name] = leg
+            del dwi, wi
+            torch.cuda.empty_cache()
+        line["per_config"] = legs
+    if info and not args.no_q4:
         line["q4_0_decode"] = bench_q4(dev, stream, steps=max(10, min(args.steps, 2000)))
-    if not args.no_cache_write or not args.no_quest:
-        del pools, argsets
         torch.cuda.empty_cache()
-    if not args.no_cache_write:
-        # information, after the timed region: the write path that fills the cache
+    if info and not args.no_cache_write:
+        # the write path that fills the cache
         line["cache_write"] = bench_cache_write(dev, stream)
-    if not args.no_quest:
+        torch.cuda.empty_cache()
+    if info and not args.no_quest:
         line["quest_metadata"] = bench_quest(dev, stream)
-    if rank == 0 and world == 1 and not args.no_accuracy:
-        torch.cuda.synchronize(dev)
-        line["q8_vs_fp32"] = q8_vs_fp32(w, out.cpu().numpy())
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()

@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     q8kv_cache_write,
     q8kv_debug_block_dots,
     q8kv_debug_quantize_q,
+    q8kv_debug_stall_pipeline,
     q8kv_decode_attn,
     q8kv_decode_attn_multi,
     q8kv_decode_attn_q4,

@@ -37,6 +37,7 @@ EXPORTS = (
     "q8kv_quest_metadata",
     "q8kv_debug_quantize_q",
     "q8kv_debug_block_dots",
+    "q8kv_debug_stall_pipeline",
     "q8kv_device_errors",
     "q8kv_status_string",
     "q8kv_last_cuda_error",
@@ -79,6 +80,8 @@ def lib():
                 "q8kv_quest_metadata": ([P] * 7 + [I] * 8 + [P], I),
                 "q8kv_debug_quantize_q": ([P, P, P, I, I, P], I),
                 "q8kv_debug_block_dots": ([P, I] + [P] * 8 + [I] * 7 + [F, P], I),
+                "q8kv_debug_stall_pipeline": ([P] * 8 + [I] * 7 + [F, I, ctypes.c_ulonglong, P],
+                                              I),
                 "q8kv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
                 "q8kv_status_string": ([I], ctypes.c_char_p),
                 "q8kv_last_cuda_error": ([], I),
@@ -313,6 +316,18 @@ def q8kv_debug_block_dots(dots, out, q, k_blocks, v_blocks, kscale, vscale, bloc
                                        _ptr(k_blocks), _ptr(v_blocks), _ptr(kscale),
                                        _ptr(vscale), _ptr(block_table), _ptr(seq_lens), *geo,
                                        float(scale), _stream(stream)), "q8kv_debug_block_dots")
+
+
+def q8kv_debug_stall_pipeline(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+                              scale, stall_cta=0, limit_ns=100_000, stream=None):
+    """q8kv_decode_attn with CTA ``stall_cta``'s pipeline stalled on purpose: its waits run
+    out after ``limit_ns`` and set the time-out bit of the device error word."""
+    geo = _geometry(out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens)
+    _check(lib().q8kv_debug_stall_pipeline(_ptr(out), _ptr(q), _ptr(k_blocks), _ptr(v_blocks),
+                                           _ptr(kscale), _ptr(vscale), _ptr(block_table),
+                                           _ptr(seq_lens), *geo, float(scale), int(stall_cta),
+                                           int(limit_ns), _stream(stream)),
+           "q8kv_debug_stall_pipeline")
 
 
 def q8kv_device_errors(clear: bool = True) -> int:

@@ -332,6 +332,8 @@ struct Call {
     float scale;
     int32_t *dots;
     int dots_max_len;
+    int stall_cta = -1;                    // fault injection (q8kv_debug_stall_pipeline)
+    unsigned long long stall_limit_ns = 0;
 };
 
 q8kv_status check_call(const Call &c)
@@ -477,6 +479,8 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.heads_seg = pl.heads_seg;
     p.scratch_stride = pl.scratch_stride;
     p.scale_log2 = (float)((double)c.scale * 1.4426950408889634);
+    p.stall_cta = c.stall_cta;
+    p.stall_limit_ns = c.stall_limit_ns;
     p.lay = pl.lay;
 
     const bool dump = c.dots != nullptr;
@@ -492,8 +496,8 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
 
 } // namespace
 
-// Scratch of q8kv_decode_attn_static: split-KV counters and partial results at the same
-// offsets as a caller-owned workspace. A file-scope device array rather than an allocation,
+// Scratch of q8kv_decode_attn_static: split-segment descriptors and partial results at the
+// same offsets as a caller-owned workspace. A file-scope device array rather than an allocation,
 // so that a call of that entry point never allocates: its callers are ones that must not
 // allocate while serving (a pool allocator owns all device memory, or the step cannot take
 // cudaMalloc's latency or cudaFree's device-wide synchronisation). One instance exists per
@@ -686,6 +690,26 @@ q8kv_status q8kv_debug_block_dots(int32_t *dots, int max_seq_len, float *out, co
     return run(c, nullptr, 0, true, stream);
 }
 
+q8kv_status q8kv_debug_stall_pipeline(float *out, const float *q, const int8_t *k_blocks,
+                                      const int8_t *v_blocks, const float *kscale,
+                                      const float *vscale, const int32_t *block_table,
+                                      const int32_t *seq_lens, int B, int n_q_heads,
+                                      int n_kv_heads, int head_dim, int kv_block_size,
+                                      int max_blocks_per_seq, int num_kv_blocks, float scale,
+                                      int stall_cta, unsigned long long limit_ns,
+                                      cudaStream_t stream)
+{
+    if (stall_cta < 0 || limit_ns < 1000ull || limit_ns > 1000000000ull)
+        return Q8KV_ERR_INVALID_ARG;
+    Call c{out, q, k_blocks, v_blocks, kscale, vscale, block_table, seq_lens,
+           Shape{B, n_q_heads, n_kv_heads, head_dim, kv_block_size, max_blocks_per_seq,
+                 num_kv_blocks},
+           scale, nullptr, 0};
+    c.stall_cta = stall_cta;
+    c.stall_limit_ns = limit_ns;
+    return run(c, nullptr, 0, true, stream);
+}
+
 q8kv_status q8kv_device_errors(unsigned *flags, int clear)
 {
     if (!flags)
@@ -729,7 +753,7 @@ int q8kv_last_cuda_error(void)
 
 int q8kv_version(void)
 {
-    return 102;
+    return 103;
 }
 
 } // extern "C"

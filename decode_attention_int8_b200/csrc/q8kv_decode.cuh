@@ -172,8 +172,19 @@ struct DecodeParams {
     int heads_seg;       // query heads per segment (HPC * G)
     int scratch_stride;  // floats per (subtile, pair) merge region
     float scale_log2;    // softmax scale * log2(e)
+    // Pipeline fault injection (the wait time-out test; -1 = off): the producer of CTA
+    // stall_cta never arrives on, nor loads into, the stage of its second tile (its first
+    // when it has only one), and that CTA's waits give up after stall_limit_ns.
+    int stall_cta;
+    unsigned long long stall_limit_ns;
     SmemLayout lay;
 };
+
+// Wait limit of this CTA's pipeline waits.
+__device__ __forceinline__ unsigned long long wait_limit(const DecodeParams &p)
+{
+    return (int)blockIdx.x == p.stall_cta ? p.stall_limit_ns : kWaitLimitNs;
+}
 
 __device__ __forceinline__ void consumer_bar()
 {
@@ -350,6 +361,9 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
     int stage = 0;
     uint32_t phase = 0, issued = 0, issued_par = 0;
     bool aborted = false;
+    const unsigned long long limit = wait_limit(p);
+    // fault injection: the tile whose stage is never filled (-1: none)
+    const int x_stall = (int)blockIdx.x == p.stall_cta ? (t1 - t0 > 1 ? t0 + 1 : t0) : -1;
 
     int *ptab = reinterpret_cast<int *>(smem + p.lay.off_ptab);
 #pragma unroll 1
@@ -400,9 +414,12 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
             const int hci = __shfl_sync(kFullMask, hc, i);
             int ok = 1;
             if (lane == 0) {
-                if (!mbar_wait(&empty[stage], phase ^ 1u, kWaitLimitNs)) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
                     ok = 0;
                     atomicOr(p.errors, kErrTimeout);
+                } else if (xb + i == x_stall) {
+                    // injected fault: no arrive and no copies, so this stage's phase never
+                    // completes (nothing is in flight for it)
                 } else {
                     const int *sl = ptab + i * kMaxBoxes;
                     uint32_t bytes = 0;
@@ -461,7 +478,7 @@ __device__ void produce(const DecodeParams &p, const CUtensorMap *tmK, const CUt
 #pragma unroll 1
         for (int s = 0; s < p.n_stages; ++s)
             if ((issued >> s) & 1u)
-                mbar_wait(&full[s], (issued_par >> s) & 1u, kWaitLimitNs);
+                mbar_wait(&full[s], (issued_par >> s) & 1u, limit);
     }
 }
 
@@ -1304,6 +1321,7 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         fut[r] = hg < p.G ? p.nq - 1 - hg / p.Gq : 0;
     }
     bool dead = false; // set when a pipeline wait timed out: skip work, keep the barriers
+    const unsigned long long limit = wait_limit(p);
     int stage = 0;
     uint32_t phase = 0;
     const uint32_t smem_base = smem_addr(smem);
@@ -1353,7 +1371,7 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         for (; x < x_end; ++x) {
             const int tok0 = (x - cu.seg0) * p.TT;
             const int nvalid = min(p.TT, cu.L - tok0);
-            if (!dead && !mbar_wait(&full[stage], phase, kWaitLimitNs)) {
+            if (!dead && !mbar_wait(&full[stage], phase, limit)) {
                 dead = true;
                 atomicOr(p.errors, kErrTimeout);
             }

@@ -167,8 +167,9 @@ q8kv_status q8kv_decode_attn_q4(float *out, const float *q, const uint8_t *k4_bl
  * (0 if the sizes are invalid or unsupported). */
 size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim);
 
-/* Zero a caller-owned workspace. Optional: no part of the workspace needs an initial value
- * (every call rewrites the bookkeeping it reads). */
+/* Zero a caller-owned workspace. Optional and without effect on results: no part of the
+ * workspace needs an initial value (every call rewrites the split-segment descriptors it
+ * reads before reading them); it only gives a fresh workspace defined contents. */
 q8kv_status q8kv_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Same as q8kv_decode_attn with a caller-owned workspace (device memory of at least
@@ -186,9 +187,9 @@ q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_bloc
 #define Q8KV_STATIC_SCRATCH_BYTES (12u * 1024u * 1024u)
 
 /*
- * Same as q8kv_decode_attn, but the call allocates no device memory at all: the split-KV
- * counters and partial results live in a fixed device array inside the library,
- * Q8KV_STATIC_SCRATCH_BYTES bytes per device. None of the source pages has a counterpart
+ * Same as q8kv_decode_attn, but the call allocates no device memory at all: the
+ * split-segment descriptors and partial results live in a fixed device array inside the
+ * library, Q8KV_STATIC_SCRATCH_BYTES bytes per device. None of the source pages has a counterpart
  * to this entry point; they describe the computation, not where its scratch lives.
  *
  * Who needs it: a caller that must not allocate while it serves requests. Examples are a
@@ -315,6 +316,25 @@ q8kv_status q8kv_debug_block_dots(int32_t *dots, int max_seq_len, float *out, co
                                   int n_q_heads, int n_kv_heads, int head_dim,
                                   int kv_block_size, int max_blocks_per_seq, int num_kv_blocks,
                                   float scale, cudaStream_t stream);
+
+/* Debug: q8kv_decode_attn with one pipeline fault injected, to exercise the bounded waits.
+ * The producer warp of CTA stall_cta never arrives on, and never loads into, the stage of
+ * that CTA's second tile (its first when it has only one), so nothing is in flight for that
+ * stage and its phase never completes. That CTA's waits give up after limit_ns
+ * (1e3 <= limit_ns <= 1e9; other CTAs keep the normal limit of one second): its consumer
+ * warps stop computing and its producer stops issuing, Q8KV_DEVERR_TIMEOUT is set, and the
+ * kernel returns normally, so the context stays usable. Rows whose split segments that CTA
+ * contributes to are undefined; all other rows are what q8kv_decode_attn gives. A CTA
+ * index past the grid injects nothing. Library-managed workspace, asynchronous. Returns
+ * Q8KV_ERR_INVALID_ARG for stall_cta < 0 or limit_ns out of range. */
+q8kv_status q8kv_debug_stall_pipeline(float *out, const float *q, const int8_t *k_blocks,
+                                      const int8_t *v_blocks, const float *kscale,
+                                      const float *vscale, const int32_t *block_table,
+                                      const int32_t *seq_lens, int B, int n_q_heads,
+                                      int n_kv_heads, int head_dim, int kv_block_size,
+                                      int max_blocks_per_seq, int num_kv_blocks, float scale,
+                                      int stall_cta, unsigned long long limit_ns,
+                                      cudaStream_t stream);
 
 /* Read (and, if clear != 0, reset) the device-side error word of the current device.
  * Synchronises the device. */

@@ -6,10 +6,14 @@
  * FMA contraction: the fp32 Q quantisation must round every operation separately).
  *
  * Readings of the pages taken here (the garbled spots in the Kestrel-LLM walk-through,
- * trdm.cn/news/511694, section 2):
- *   - zero-block guard "if (qm 1e-6f) qm 1.0f" is read as  if (qm < 1e-6f) qm = 1.0f;
- *   - the cast "(int8_t)clamp(q*iq, -128, 127)" is replaced by round-half-to-even, then
- *     clamp to [-127, 127] (the rounding rule this library fixes);
+ * trdm.cn/news/511694, section 2 part 1):
+ *   - the walk-through guards a block whose largest magnitude is tiny, but the comparison
+ *     and assignment operators were lost in extraction; it is read as a less-than test
+ *     against 1e-6 that replaces that largest magnitude with 1, so the block quantises to
+ *     zeros;
+ *   - the walk-through turns the scaled value into a code by clamping to [-128, 127] and
+ *     truncating; this library instead rounds half to even and clamps to [-127, 127] (the
+ *     rounding rule it fixes; the two differ by at most one step per element);
  *   - the K/V scale arrays hold the dequantisation multiplier itself (no extra 1/127)
  *     and are indexed by the physical slot: scale[slot * n_kv_heads + kv_head];
  *   - the running max starts at -infinity (the page's -1e9 gives the same result when

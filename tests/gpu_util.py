@@ -46,3 +46,22 @@ def assert_close(got, ref, what=""):
     assert max_abs <= MAX_ABS_TOL and rel <= REL_L2_TOL, (
         f"{what}: max_abs={max_abs:.3e} (tol {MAX_ABS_TOL}) rel_l2={rel:.3e} (tol {REL_L2_TOL})")
     return max_abs, rel
+
+
+def without_block(block_table, seq_lens, b, j, bs):
+    """The table and lengths of the same cache with logical block j of sequence b left out:
+    the tokens a decode must attend to when that block's table entry is unusable (the
+    decode has no positional term, so skipping a block's tokens is attention over the
+    remaining ones)."""
+    bt = np.array(block_table, copy=True)
+    lens = np.array(seq_lens, copy=True)
+    L = int(lens[b])
+    nblk = -(-L // bs)
+    assert 0 <= j < nblk
+    dropped = min(bs, L - j * bs)
+    row = list(bt[b, :nblk])
+    del row[j]
+    bt[b, :] = -1
+    bt[b, :len(row)] = row
+    lens[b] = L - dropped
+    return bt, lens

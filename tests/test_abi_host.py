@@ -36,9 +36,11 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_library_is_built_for_sm100a():
-    out = subprocess.run(["cuobjdump", "--list-elf", q8.lib_path()], capture_output=True,
-                         text=True).stdout
-    assert "sm_100a" in out
+    from decode_attention_int8_b200 import build
+
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "-gencode arch=compute_100a,code=sm_100a" in flags
+    assert "compute_90" not in flags and "sm_90" not in flags
 
 
 def test_status_strings_and_version():
@@ -46,7 +48,7 @@ def test_status_strings_and_version():
     assert L.q8kv_status_string(0) == b"ok"
     assert L.q8kv_status_string(2) == b"unsupported shape"
     assert L.q8kv_status_string(99) == b"unknown status"
-    assert L.q8kv_version() == 102
+    assert L.q8kv_version() == 103
 
 
 def _call(**over):

@@ -12,7 +12,7 @@ import torch
 import decode_attention_int8_b200 as q8
 import oracle
 from decode_attention_int8_b200 import inputs
-from gpu_util import assert_close, oracle_cache, run_decode, to_device
+from gpu_util import assert_close, oracle_cache, run_decode, to_device, without_block
 
 pytestmark = pytest.mark.gpu
 
@@ -184,16 +184,24 @@ def test_device_side_checks_flag_bad_tables_without_faulting():
     assert q8.q8kv_device_errors(clear=True) == 0
     # an entry past the pool: that block's tokens are skipped, the flag is raised
     bad = inputs.make_custom(3, 8, 2, 128, [40, 70, 16], 16, seed=14, extra_blocks=2)
+    entry = int(bad.block_table[1, 2])
     bad.block_table[1, 2] = bad.num_blocks + 5
     got = run_decode(bad).cpu().numpy()
     assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
     np.testing.assert_array_equal(got[0], ref_ok[0])
     np.testing.assert_array_equal(got[2], ref_ok[2])
-    assert np.all(np.isfinite(got[1]))
-    # a negative entry
-    bad.block_table[1, 2] = -7
-    run_decode(bad)
+    # row 1 is attention over the tokens of its other blocks
+    bt, lens = without_block(bad.block_table, bad.seq_lens, 1, 2, 16)
+    kept = oracle.PagedCache(bad.k, bad.v, bad.ks, bad.vs, bt, lens, 8, bad.scale)
+    assert_close(got[1], oracle.decode_all(kept, bad.q)[1], "block skipped")
+    # a negative entry, here in the sequence's last (partial) block
+    bad.block_table[1, 2] = entry
+    bad.block_table[1, 4] = -7
+    got = run_decode(bad).cpu().numpy()
     assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
+    bt, lens = without_block(bad.block_table, bad.seq_lens, 1, 4, 16)
+    kept = oracle.PagedCache(bad.k, bad.v, bad.ks, bad.vs, bt, lens, 8, bad.scale)
+    assert_close(got[1], oracle.decode_all(kept, bad.q)[1], "last block skipped")
     # seq_len above max_blocks_per_seq * block_size is clamped and flagged
     long = inputs.make_custom(3, 8, 2, 128, [40, 70, 16], 16, seed=14, extra_blocks=2)
     long.seq_lens[0] = long.max_blocks_per_seq * 16 + 100

@@ -11,7 +11,7 @@ import torch
 import decode_attention_int8_b200 as q8
 import oracle
 from decode_attention_int8_b200 import inputs
-from gpu_util import assert_close
+from gpu_util import assert_close, without_block
 
 pytestmark = pytest.mark.gpu
 
@@ -101,8 +101,12 @@ def test_bad_block_table_entries_are_flagged_and_skipped():
     assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
     np.testing.assert_array_equal(got[0], ref[0])
     np.testing.assert_array_equal(got[2], ref[2])
-    assert np.all(np.isfinite(got[1]))
+    # row 1 is attention over the tokens of its other blocks
+    bt, lens = without_block(w.block_table, w.seq_lens, 1, 20, 16)
+    kept = oracle.PagedCacheQ4(w.k4, w.v4, w.kd, w.vd, bt, lens, w.cfg.n_q_heads, w.scale)
+    assert_close(got[1], oracle.decode_q4_all(kept, w.q)[1], "q4 block skipped")
     # a negative entry
     w.block_table[1, 20] = -3
-    run_q4(w)
+    got = run_q4(w)
     assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
+    assert_close(got[1], oracle.decode_q4_all(kept, w.q)[1], "q4 block skipped (negative)")
