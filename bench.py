@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run the workload's recipe with this many sequences instead (a "
+                         "smaller case of the same kernel, e.g. for an ncu capture)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -667,7 +670,7 @@ def run_reference(args):
     import oracle
     from decode_attention_int8_b200 import inputs
 
-    w = inputs.make(args.config)
+    w = make_workload(args)
     cache = oracle.PagedCache(w.k, w.v, w.ks, w.vs, w.block_table, w.seq_lens,
                               w.cfg.n_q_heads, w.scale)
     B, Hq = w.cfg.B, w.cfg.n_q_heads
@@ -707,6 +710,16 @@ def run_reference(args):
     return 0
 
 
+def make_workload(args):
+    """The workload of --config, or its recipe with --batch sequences."""
+    from decode_attention_int8_b200 import inputs
+
+    cfg = inputs.WORKLOADS[args.config]
+    if getattr(args, "batch", 0):
+        cfg = inputs.with_config(cfg, B=args.batch, name=f"{cfg.name}_b{args.batch}")
+    return inputs.make(cfg)
+
+
 # group-8 reading of the batched GQA workload's label: 64 q heads over its 8 KV heads
 def group8_workload():
     from decode_attention_int8_b200 import inputs
@@ -743,7 +756,7 @@ def main():
         pg = dist
 
     stream = torch.cuda.current_stream(dev)
-    w = inputs.make(args.config)
+    w = make_workload(args)
     algo = w.algorithmic_bytes()
     dw = DeviceWorkload(w, dev, stream)
     q8.q8kv_device_errors(clear=True)
@@ -1105,6 +1118,31 @@ def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):
     ms_fill = timed(kn, vn, slots)
     ms_step = timed(s_kn, s_vn, s_slots)
     errs = q8.q8kv_device_errors(clear=True)
+    # the same prompt fill into q4_0 pools (q8kv_cache_write_q4)
+    del k, v, ks, vs
+    k4 = torch.zeros((P, bs, Hk, D // 2), dtype=torch.uint8, device=dev)
+    v4 = torch.zeros_like(k4)
+    kd = torch.zeros((P, bs, Hk, D // 32), dtype=torch.int16, device=dev)
+    vd = torch.zeros_like(kd)
+    q8.q8kv_cache_write_q4(k4, v4, kd, vd, kn, vn, slots, stream=stream)
+    fn4 = q8.lib().q8kv_cache_write_q4
+    a4 = (P_(k4), P_(v4), P_(kd), P_(vd), P_(kn), P_(vn), P_(slots), n, Hk, D, bs, P, Hk * D, sp)
+    for _ in range(warmup):
+        fn4(*a4)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        st = fn4(*a4)
+        if st != 0:
+            raise q8.Q8KVError(st, "q8kv_cache_write_q4")
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_q4 = e0.elapsed_time(e1) / steps
+    errs |= q8.q8kv_device_errors(clear=True)
+    n_valid = int(np.count_nonzero(rows.slots >= 0))
+    algo_q4 = n_valid * Hk * 2 * (4 * D + D // 2 + 2 * (D // 32)) + 8 * n
     algo = rows.algorithmic_bytes()
     peak, peak_kind = measured_peak()
     achieved = algo / (ms_fill * 1e-3) / 1e9
@@ -1120,6 +1158,13 @@ def bench_cache_write(dev, stream, steps=50, warmup=5, step_B=16):
                          "traffic": recorded_traffic("gqa_prompt_fill", "cache_write"),
                          "kernel": "q8kv::cache_write_kernel<128>"},
             "l2": "inputs (537 MB of fp32 rows) and outputs (138 MB) larger than L2"},
+        "prompt_fill_q4": {
+            "workload": "the same prompt fill into q4_0 pools (q8kv_cache_write_q4)",
+            "us_per_call": round(ms_q4 * 1e3, 3), "calls": steps, "algorithmic_bytes": algo_q4,
+            "roofline": {"bound": "hbm", "achieved": round(algo_q4 / (ms_q4 * 1e-3) / 1e9, 2),
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(algo_q4 / (ms_q4 * 1e-3) / 1e9 / peak, 4),
+                         "traffic": None, "kernel": "q8kv::cache_write_q4_kernel<128>"}},
         "decode_step": {"workload": f"one new token per sequence: {step_B} x {Hk} rows",
                         "us_per_call": round(ms_step * 1e3, 3), "calls": steps,
                         "algorithmic_bytes": step_bytes,

@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     lib,
     lib_path,
     q8kv_cache_write,
+    q8kv_cache_write_q4,
     q8kv_debug_block_dots,
     q8kv_debug_quantize_q,
     q8kv_debug_stall_pipeline,

@@ -34,6 +34,7 @@ EXPORTS = (
     "q8kv_decode_attn_ws",
     "q8kv_decode_attn_static",
     "q8kv_cache_write",
+    "q8kv_cache_write_q4",
     "q8kv_quest_metadata",
     "q8kv_debug_quantize_q",
     "q8kv_debug_block_dots",
@@ -77,6 +78,7 @@ def lib():
                 "q8kv_decode_attn_ws": ([P] * 8 + [I] * 7 + [F, P, Z, P], I),
                 "q8kv_decode_attn_static": ([P] * 8 + [I] * 7 + [F, P], I),
                 "q8kv_cache_write": ([P] * 7 + [I] * 5 + [ctypes.c_longlong, P], I),
+                "q8kv_cache_write_q4": ([P] * 7 + [I] * 5 + [ctypes.c_longlong, P], I),
                 "q8kv_quest_metadata": ([P] * 7 + [I] * 8 + [P], I),
                 "q8kv_debug_quantize_q": ([P, P, P, I, I, P], I),
                 "q8kv_debug_block_dots": ([P, I] + [P] * 8 + [I] * 7 + [F, P], I),
@@ -261,6 +263,39 @@ def q8kv_cache_write(k_blocks, v_blocks, kscale, vscale, k_new, v_new, slot_mapp
     _check(lib().q8kv_cache_write(_ptr(k_blocks), _ptr(v_blocks), _ptr(kscale), _ptr(vscale),
                                   _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), n, Hk, D, bs, P,
                                   stride, _stream(stream)), "q8kv_cache_write")
+
+
+def q8kv_cache_write_q4(k4_blocks, v4_blocks, kd, vd, k_new, v_new, slot_mapping, stream=None):
+    """q4_0 cache write: quantise the new rows k_new, v_new [n_tokens][n_kv_heads][head_dim]
+    (fp32; the token dimension may be strided) per 32-channel block and store codes (uint8
+    [P][bs][Hk][D/2]) and binary16 scales (kd, vd [P][bs][Hk][D/32], torch.float16 or 16-bit
+    integers holding the bits) at the slots slot_mapping [n_tokens] (int64; negative =
+    padding)."""
+    _need(k4_blocks, "k4_blocks", torch.uint8, 4)
+    _need(v4_blocks, "v4_blocks", torch.uint8, 4)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    P, bs, Hk, half = k4_blocks.shape
+    D = 2 * half
+    if tuple(v4_blocks.shape) != (P, bs, Hk, half):
+        raise ValueError("k4/v4 shapes disagree")
+    for t, name in ((kd, "kd"), (vd, "vd")):
+        if t.dtype not in (torch.float16, torch.int16, torch.uint16) or not t.is_cuda or \
+                not t.is_contiguous() or tuple(t.shape) != (P, bs, Hk, D // 32):
+            raise ValueError(f"{name}: expected a contiguous CUDA 16-bit tensor "
+                             f"{(P, bs, Hk, D // 32)}")
+    n = int(slot_mapping.shape[0])
+    for t, name in ((k_new, "k_new"), (v_new, "v_new")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA float32 tensor")
+        if tuple(t.shape) != (n, Hk, D) or t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name}: expected shape {(n, Hk, D)} with contiguous rows, got "
+                             f"{tuple(t.shape)} strides {t.stride()}")
+    if n > 1 and k_new.stride(0) != v_new.stride(0):
+        raise ValueError("k_new and v_new must have the same token stride")
+    stride = int(k_new.stride(0)) if n > 1 else Hk * D
+    _check(lib().q8kv_cache_write_q4(_ptr(k4_blocks), _ptr(v4_blocks), _ptr(kd), _ptr(vd),
+                                     _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), n, Hk, D,
+                                     bs, P, stride, _stream(stream)), "q8kv_cache_write_q4")
 
 
 def q8kv_quest_metadata(maxblocks, minblocks, k_blocks, kscale, block_table, seq_lens,

@@ -31,6 +31,8 @@
 // depend on its slot, so they are issued together with the slot load.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include <cstdint>
 
 #include "q8kv_ptx.cuh"
@@ -204,6 +206,153 @@ __global__ void __launch_bounds__(kWriteThreads, write_blocks_per_sm(D))
             if (bad_k || bad_v)
                 err |= kErrNonFinite;
         }
+        tok += dtok;
+        h += dh;
+        if (h >= p.Hk) {
+            h -= p.Hk;
+            ++tok;
+        }
+    }
+    if (err)
+        atomicOr(p.errors, err);
+}
+
+// ------------------------------------------------------------------ q4_0 cache write
+//
+// The same write in llama.cpp's q4_0 format (one of the quantised KV-cache types of the
+// llama.cpp change on baguaai.com's FlashAttention page), into the pools the q4_0 decode
+// reads: per 32-channel block, m = the value of largest magnitude with its sign (the first
+// one on ties; +0 for an all-zero block), d = m / -8, id = d != 0 ? 1 / d : 0,
+// code = min(15, trunc(x * id + 8.5)), every operation rounded to fp32 on its own, d stored
+// as binary16 (round to nearest even); codes packed two per byte, channel 2i in the low
+// nibble of byte i. A block holding an infinity or a NaN is stored as codes 8 with a NaN
+// scale and sets a device error bit.
+//
+// Lanes as in the q8 write: chunk c of a lane holds 4 consecutive channels of one block, and
+// a block's 32 channels lie on 8 consecutive lanes, so the search for m is a 3-step
+// butterfly over a 64-bit key (|x| bits, then the reversed channel index, so that the
+// first channel wins a tie, then the sign); a lane stores the 2 code bytes of each of its
+// chunks (16 contiguous bytes per block and store instruction).
+struct CacheWriteQ4Params {
+    uint8_t *k4, *v4;
+    uint16_t *kd, *vd;
+    const float *k_new, *v_new;
+    const int64_t *slots;
+    long long n_tokens;
+    long long token_stride;
+    long long n_slots;
+    int Hk;
+    unsigned *errors;
+};
+
+// Key of element i (channel `ch` of its block) for the largest-magnitude search.
+__device__ __forceinline__ unsigned long long q4_key(float x, int ch)
+{
+    const uint32_t b = __float_as_uint(x);
+    return ((unsigned long long)(b & 0x7fffffffu) << 32) | ((uint32_t)(31 - ch) << 1) | (b >> 31);
+}
+
+__device__ __forceinline__ uint32_t q4_code(float x, float id)
+{
+    const int c = __float2int_rz(__fadd_rn(__fmul_rn(x, id), 8.5f));
+    return (uint32_t)(c > 15 ? 15 : c);
+}
+
+// One chunk of 4 channels (channel 4 * g8 .. 4 * g8 + 3 of its block, g8 = lane % 8 inside
+// the block's lane group): returns the chunk's two code bytes as 16 bits and the block's
+// binary16 scale; sets `bad` for a non-finite block.
+__device__ __forceinline__ uint32_t q4_chunk(float4 x, int g8, uint16_t &d16, bool &bad)
+{
+    unsigned long long k = q4_key(x.x, 4 * g8);
+    const unsigned long long k1 = q4_key(x.y, 4 * g8 + 1), k2 = q4_key(x.z, 4 * g8 + 2),
+                             k3 = q4_key(x.w, 4 * g8 + 3);
+    k = k1 > k ? k1 : k;
+    k = k2 > k ? k2 : k;
+    k = k3 > k ? k3 : k;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+        const unsigned long long t = __shfl_xor_sync(0xffffffffu, k, o);
+        k = t > k ? t : k;
+    }
+    const uint32_t abits = (uint32_t)(k >> 32);
+    bad = abits >= 0x7f800000u; // an infinity or a NaN in the block
+    if (bad) {
+        d16 = 0x7e00u;
+        return 0x8888u;
+    }
+    // m with its sign; an all-zero block keeps m = +0 (d = +0 / -8 = -0)
+    const float m = __uint_as_float(abits | (abits != 0u ? (uint32_t)(k & 1u) << 31 : 0u));
+    const float d = __fdiv_rn(m, -8.0f);
+    const float id = d != 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+    d16 = __half_as_ushort(__float2half_rn(d));
+    return q4_code(x.x, id) | (q4_code(x.y, id) << 4) | (q4_code(x.z, id) << 8) |
+           (q4_code(x.w, id) << 12);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kWriteThreads, write_blocks_per_sm(D))
+    cache_write_q4_kernel(const __grid_constant__ CacheWriteQ4Params p)
+{
+    constexpr int LPR = write_lanes_per_row(D);
+    constexpr int PPW = write_pairs_per_warp(D);
+    constexpr int C = RowFrag<D>::C;
+    // the new rows may come from the kernel before this one on the stream
+    grid_dep_wait();
+    grid_dep_launch();
+    const int lane = threadIdx.x & 31, sub = lane % LPR, g8 = sub & 7;
+    const long long n_pairs = p.n_tokens * p.Hk;
+    const long long step = (long long)gridDim.x * kWriteWarps * PPW;
+    const long long wbase = ((long long)blockIdx.x * kWriteWarps + (threadIdx.x >> 5)) * PPW;
+    const long long first = wbase + lane / LPR;
+    long long tok = first / p.Hk;
+    int h = (int)(first - tok * p.Hk);
+    const long long dtok = step / p.Hk;
+    const int dh = (int)(step - dtok * p.Hk);
+    unsigned err = 0;
+#pragma unroll 1
+    for (long long base = wbase; base < n_pairs; base += step) {
+        long long slot = -1;
+        RowFrag<D> fk, fv;
+        if (tok < p.n_tokens) {
+            const long long src = tok * p.token_stride + (long long)h * D;
+            slot = __ldg(p.slots + tok);
+            fk = load_frag<D>(p.k_new + src, sub);
+            fv = load_frag<D>(p.v_new + src, sub);
+        } else {
+#pragma unroll
+            for (int c = 0; c < C; ++c)
+                fk.x[c] = fv.x[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (slot >= p.n_slots) {
+            err |= kErrSlot;
+            slot = -1;
+        }
+        const bool store = slot >= 0;
+        const long long row = store ? slot * p.Hk + h : 0;
+        uint8_t *kc = p.k4 + row * (D / 2), *vc = p.v4 + row * (D / 2);
+        uint16_t *kdr = p.kd + row * (D / 32), *vdr = p.vd + row * (D / 32);
+        bool bad = false;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            // chunk c holds channels 4 * (sub + LPR * c) ..: block (sub + LPR * c) / 8
+            const int blk = (sub + LPR * c) >> 3;
+            uint16_t dk, dv;
+            bool bk, bv;
+            const uint32_t ck = q4_chunk(fk.x[c], g8, dk, bk);
+            const uint32_t cv = q4_chunk(fv.x[c], g8, dv, bv);
+            bad = bad || bk || bv;
+            if (store) {
+                reinterpret_cast<uint16_t *>(kc)[blk * 8 + g8] = (uint16_t)ck;
+                reinterpret_cast<uint16_t *>(vc)[blk * 8 + g8] = (uint16_t)cv;
+                // one lane per block writes its scales: K from g8 == c, V from g8 == 4 + c
+                if (g8 == c)
+                    kdr[blk] = dk;
+                else if (g8 == 4 + c)
+                    vdr[blk] = dv;
+            }
+        }
+        if (store && bad)
+            err |= kErrNonFinite;
         tok += dtok;
         h += dh;
         if (h >= p.Hk) {

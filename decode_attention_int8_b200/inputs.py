@@ -157,7 +157,8 @@ def quantize_q4_0_rows(x: np.ndarray):
     q = np.minimum(15, np.trunc(t.astype(np.float32)).astype(np.int32))
     q = q.reshape(x.shape)
     packed = (q[..., 0::2] | (q[..., 1::2] << 4)).astype(np.uint8)
-    return packed, d.astype(np.float16).view(np.uint16)
+    with np.errstate(over="ignore"):  # |d| > 65504 rounds to infinity, as binary16 does
+        return packed, d.astype(np.float16).view(np.uint16)
 
 
 def _fill_pool(seed, stream, dist, P, bs, Hk, D, bias, keep_fp32, threads, q4=False):

@@ -268,6 +268,37 @@ q8kv_status q8kv_cache_write(int8_t *k_blocks, int8_t *v_blocks, float *kscale, 
                              long long token_stride, cudaStream_t stream);
 
 /*
+ * KV-cache write in the q4_0 format (llama.cpp's q4_0 blocks, one of the quantised KV-cache
+ * types of the llama.cpp change on baguaai.com's FlashAttention page), into the pools
+ * q8kv_decode_attn_q4 reads: every (token, KV head) row of K and of V is quantised per
+ * 32-channel block, in IEEE fp32 with every operation rounded on its own:
+ *   m = the value of largest magnitude, sign kept (the first one on ties; +0 for an
+ *       all-zero block), d = m / -8, id = d != 0 ? 1 / d : 0,
+ *   code = min(15, trunc(x * id + 8.5))  (0..15; value = (code - 8) * d)
+ * d is stored as binary16 (round to nearest even; beyond 65504 it becomes infinity, as in
+ * the format). Codes are packed two per byte, channel 2i in the low nibble of byte i. A block
+ * holding an infinity or a NaN is stored as codes 8 with a NaN scale (0x7e00) and sets
+ * Q8KV_DEVERR_NONFINITE (a decode over it returns NaN); the row's other blocks are
+ * quantised as usual.
+ *
+ *   k4_blocks, v4_blocks  uint8 [num_kv_blocks][kv_block_size][n_kv_heads][head_dim / 2],
+ *                         16-byte aligned, written in place
+ *   kd, vd                binary16 bits [num_kv_blocks][kv_block_size][n_kv_heads]
+ *                         [head_dim / 32], 8-byte aligned, written in place
+ *   k_new, v_new, slot_mapping, n_tokens, token_stride: as q8kv_cache_write (the same slot
+ *                         rules: negative = padding, skipped; past the pool = skipped with
+ *                         Q8KV_DEVERR_SLOT; distinct slots within one call)
+ *   head_dim              64, 128 or 256 (the q4_0 decode reads head_dim 128)
+ * One kernel launch, asynchronous on `stream`, programmatic dependent launch as
+ * q8kv_cache_write.
+ */
+q8kv_status q8kv_cache_write_q4(uint8_t *k4_blocks, uint8_t *v4_blocks, uint16_t *kd,
+                                uint16_t *vd, const float *k_new, const float *v_new,
+                                const int64_t *slot_mapping, int n_tokens, int n_kv_heads,
+                                int head_dim, int kv_block_size, int num_kv_blocks,
+                                long long token_stride, cudaStream_t stream);
+
+/*
  * QUEST-style per-block K metadata (CANN quest_prefill_metadata guide, xdnf.cn/news/235188):
  * for every request r, KV block j < ceil(seq_lens[r] / kv_block_size) and KV head h, the
  * per-channel maximum and minimum of the dequantised K (code * kscale, one fp32 product)

@@ -113,6 +113,7 @@ def _load():
                 "q8kvo_decode_q4_all": [ctypes.POINTER(CacheQ4), P, P],
                 "q8kvo_decode_q4_pairs": [ctypes.POINTER(CacheQ4), P, P, l, P],
                 "q8kvo_cache_write": [P, P, P, P, P, P, P, l, i, i, i, i, l, P],
+                "q8kvo_cache_write_q4": [P, P, P, P, P, P, P, l, i, i, i, i, l, P],
             }
             for name, args in sigs.items():
                 fn = getattr(lib, name)
@@ -321,6 +322,34 @@ def cache_write(k, v, ks, vs, k_new, v_new, slot_mapping, token_stride=None) -> 
     _check(_load().q8kvo_cache_write(_ptr(k), _ptr(v), _ptr(ks), _ptr(vs), _ptr(k_new),
                                      _ptr(v_new), _ptr(slots), n, Hk, D, bs, P, stride,
                                      ctypes.byref(flags)), "cache_write")
+    return int(flags.value)
+
+
+def cache_write_q4(k4, v4, kd, vd, k_new, v_new, slot_mapping, token_stride=None) -> int:
+    """q4_0 KV-cache write into the host pools k4, v4 [P][bs][Hk][D/2] (uint8) and kd, vd
+    [P][bs][Hk][D/32] (uint16 binary16 bits), modified in place; k_new, v_new and the slots
+    as cache_write. Returns the flags."""
+    for a in (k4, v4, kd, vd):
+        if not a.flags.c_contiguous:
+            raise ValueError("pools must be C-contiguous")
+    if k4.dtype != np.uint8 or v4.dtype != np.uint8 or kd.dtype != np.uint16 or \
+            vd.dtype != np.uint16:
+        raise ValueError("q4_0 pools are uint8 codes and uint16 scales")
+    P, bs, Hk, D2 = k4.shape
+    D = 2 * D2
+    if v4.shape != k4.shape or kd.shape != (P, bs, Hk, D // 32) or vd.shape != kd.shape:
+        raise ValueError("pool shapes disagree")
+    slots = _c(slot_mapping, np.int64).reshape(-1)
+    n = slots.shape[0]
+    stride = Hk * D if token_stride is None else int(token_stride)
+    k_new = _c(k_new, np.float32).reshape(-1)
+    v_new = _c(v_new, np.float32).reshape(-1)
+    if n and (k_new.shape[0] < (n - 1) * stride + Hk * D or v_new.shape != k_new.shape):
+        raise ValueError("k_new / v_new too small for the token count and stride")
+    flags = ctypes.c_uint(0)
+    _check(_load().q8kvo_cache_write_q4(_ptr(k4), _ptr(v4), _ptr(kd), _ptr(vd), _ptr(k_new),
+                                        _ptr(v_new), _ptr(slots), n, Hk, D, bs, P, stride,
+                                        ctypes.byref(flags)), "cache_write_q4")
     return int(flags.value)
 
 

@@ -717,6 +717,60 @@ int q8kvo_quantize_q4_0(const float *x, long n, uint8_t *packed, uint16_t *d16)
     return Q8KVO_OK;
 }
 
+/* KV-cache write in the q4_0 format: every (token, KV head) row of k_new and v_new (fp32,
+ * row (i, h) at [i * token_stride + h * head_dim]) is quantised block by block with
+ * quantize_q4_block and stored at physical slot slot_mapping[i]: codes at
+ * k4[(slot * n_kv_heads + h) * head_dim / 2], block scales at
+ * kd[(slot * n_kv_heads + h) * head_dim / 32] (the same for V). The slot rules are those of
+ * q8kvo_cache_write (negative: skipped; at or past the pool: skipped, Q8KVO_FLAG_SLOT;
+ * tokens in order, so a repeated slot keeps the later token). A 32-channel block holding an
+ * infinity or a NaN has no q4_0 encoding: it is stored as codes 8 (value 0) with a NaN
+ * scale (binary16 0x7e00), so that the value reads back as NaN, and sets
+ * Q8KVO_FLAG_NONFINITE; the row's other blocks are quantised as usual. */
+int q8kvo_cache_write_q4(uint8_t *k4, uint8_t *v4, uint16_t *kd, uint16_t *vd,
+                         const float *k_new, const float *v_new, const int64_t *slot_mapping,
+                         long n_tokens, int n_kv_heads, int head_dim, int block_size,
+                         int num_blocks, long token_stride, unsigned *flags)
+{
+    if (!k4 || !v4 || !kd || !vd || !k_new || !v_new || !slot_mapping || !flags)
+        return Q8KVO_EINVAL;
+    if (n_tokens < 0 || n_kv_heads <= 0 || head_dim <= 0 || (head_dim % 32) != 0 ||
+        block_size <= 0 || num_blocks <= 0 || token_stride < (long)n_kv_heads * head_dim)
+        return Q8KVO_EINVAL;
+    const int64_t n_slots = (int64_t)num_blocks * block_size;
+    const int nb = head_dim / 32;
+    for (long i = 0; i < n_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        if (slot >= n_slots) {
+            *flags |= Q8KVO_FLAG_SLOT;
+            continue;
+        }
+        for (int h = 0; h < n_kv_heads; ++h) {
+            const long row = (long)slot * n_kv_heads + (MUT(28) ? (h + 1) % n_kv_heads : h);
+            for (int which = 0; which < 2; ++which) {
+                const float *x = (which ? v_new : k_new) + i * token_stride + (long)h * head_dim;
+                uint8_t *codes = (which ? v4 : k4) + row * (head_dim / 2);
+                uint16_t *d16 = (which ? vd : kd) + row * nb;
+                for (int j = 0; j < nb; ++j) {
+                    int finite = 1;
+                    for (int c = 0; c < 32; ++c)
+                        finite &= isfinite(x[32 * j + c]) ? 1 : 0;
+                    if (!finite) {
+                        memset(codes + 16 * j, 0x88, 16);
+                        d16[j] = 0x7e00u;
+                        *flags |= Q8KVO_FLAG_NONFINITE;
+                        continue;
+                    }
+                    quantize_q4_block(x + 32 * j, codes + 16 * j, d16 + j);
+                }
+            }
+        }
+    }
+    return Q8KVO_OK;
+}
+
 static int q4_code(const uint8_t *row, int i)
 {
     const uint8_t byte = row[i / 2];

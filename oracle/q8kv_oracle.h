@@ -164,6 +164,17 @@ int q8kvo_f32_to_f16(const float *x, long n, uint16_t *out);
  * d16 [n / 32] binary16 scales (rule in q8kv_oracle.c). */
 int q8kvo_quantize_q4_0(const float *x, long n, uint8_t *packed, uint16_t *d16);
 
+/* KV-cache write in the q4_0 format: the rows of k_new / v_new (as q8kvo_cache_write) are
+ * quantised per 32-channel block (q8kvo_quantize_q4_0's rule) and stored at their slots of
+ * k4, v4 [num_blocks][block_size][n_kv_heads][head_dim / 2] and kd, vd
+ * [num_blocks][block_size][n_kv_heads][head_dim / 32]; slot rules and flags as
+ * q8kvo_cache_write; a block holding inf or NaN is stored as codes 8 with a NaN scale
+ * (Q8KVO_FLAG_NONFINITE). */
+int q8kvo_cache_write_q4(uint8_t *k4, uint8_t *v4, uint16_t *kd, uint16_t *vd,
+                         const float *k_new, const float *v_new, const int64_t *slot_mapping,
+                         long n_tokens, int n_kv_heads, int head_dim, int block_size,
+                         int num_blocks, long token_stride, unsigned *flags);
+
 /* Single-query decode over a q4_0 cache (fp64 out [B][n_q_heads][head_dim], or the chosen
  * (b, h) pairs): the query quantisation and the online softmax of the q8 decode, with
  * the K and V values (code - 8) * d of their 32-channel blocks. */

@@ -38,6 +38,7 @@ MUTANTS = {
     25: "q4_0 decode without the code offset of 8",
     26: "q4_0 decode with block 0's K scale for every block",
     27: "q4_0 codes not clamped to 15",
+    28: "q4_0 cache row written under the next KV head",
 }
 
 
@@ -49,7 +50,8 @@ def test_planted_mistake_is_caught(mutant, tmp_path):
         [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
          "tests/test_oracle_qquant.py", "tests/test_oracle_attention.py",
          "tests/test_oracle_cache_write.py", "tests/test_oracle_multi_query.py",
-         "tests/test_oracle_quest.py", "tests/test_oracle_q4.py"],
+         "tests/test_oracle_quest.py", "tests/test_oracle_q4.py",
+         "tests/test_oracle_cache_write_q4.py"],
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {mutant} ({MUTANTS[mutant]}) passed every pin"
     assert "failed" in r.stdout, r.stdout[-2000:]
