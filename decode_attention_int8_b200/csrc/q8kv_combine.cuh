@@ -15,13 +15,17 @@
 // segment's first contributor: {b, hc, n contributors, first partial slot}; the other
 // contributors' slots are 2 * (first CTA + k), k = 1..n-1. This kernel runs next on the
 // stream (programmatic dependent launch: it is scheduled while the decode kernel drains
-// and waits for its completion before reading anything). The work is the list of units
-// (segment, query head, 32-channel quarter), split evenly over the CTAs; a CTA processes
-// up to 32 units at a time, giving each unit 32 / units-in-batch rows of 8 threads that
-// stride over the unit's inputs. A thread issues the loads of up to 8 inputs at once, so a
-// unit usually costs one round trip to L2 whatever its input count; maxima are taken
-// before any rescaling, so no exponential waits on another, and the rows of a unit are
-// merged through shared memory the same way.
+// and waits for its completion before reading anything). Its time is all latency (the
+// partials are a few MB in L2), so it is laid out for few dependent steps:
+//  * one load per thread of the descriptors and one block-wide scan compact them (the same
+//    order in every CTA);
+//  * the work is the list of units (segment, query head, 32-channel quarter), split evenly
+//    over the CTAs in 32-bit arithmetic; a CTA takes up to 32 units at a time and gives
+//    each unit 32 / units-in-batch rows of 8 threads that stride over the unit's inputs,
+//    a thread issuing the loads of up to 8 inputs at once;
+//  * a row merges its inputs with the maxima taken first, and the rows of a unit are then
+//    merged pairwise with the associative log-sum-exp merge, by shuffles inside a warp and
+//    one shared-memory step across warps.
 #pragma once
 
 #include <cstdint>
@@ -31,9 +35,11 @@
 namespace q8kv {
 
 constexpr int kCombineThreads = 256;
+constexpr int kCombineWarps = kCombineThreads / 32;
 constexpr int kCombineMaxDesc = 2048;  // 2 * decode grid (the grid is at most 1024 CTAs)
 constexpr int kCombineQuarter = 32;    // channels per unit
 constexpr int kCombineSlotRow = 132;   // floats per partial row: acc[128], M, S, A, pad
+constexpr int kCombineDescPerThread = kCombineMaxDesc / kCombineThreads;
 
 struct CombineParams {
     float *out;
@@ -47,72 +53,114 @@ struct CombineParams {
 
 constexpr int kCombineBatchIn = 8; // inputs a thread loads at once
 
+// A piece of one output row: the maxima M and A, the sum S (units 2^-M) and 4 channels of
+// the accumulator (units 2^-A).
+struct LsePiece {
+    float m, a, s;
+    float4 acc;
+};
+
+__device__ __forceinline__ float lse_factor(float from, float to)
+{
+    return from == -INFINITY ? 0.f : exp2f(from - to);
+}
+
+// Merge of two pieces (associative and commutative up to rounding).
+__device__ __forceinline__ LsePiece lse_merge(const LsePiece &x, const LsePiece &y)
+{
+    LsePiece r;
+    r.m = fmaxf(x.m, y.m);
+    r.a = fmaxf(x.a, y.a);
+    const float fx = lse_factor(x.m, r.m), fy = lse_factor(y.m, r.m);
+    const float gx = lse_factor(x.a, r.a), gy = lse_factor(y.a, r.a);
+    r.s = x.s * fx + y.s * fy;
+    r.acc = make_float4(x.acc.x * gx + y.acc.x * gy, x.acc.y * gx + y.acc.y * gy,
+                        x.acc.z * gx + y.acc.z * gy, x.acc.w * gx + y.acc.w * gy);
+    return r;
+}
+
+__device__ __forceinline__ LsePiece lse_shfl_xor(const LsePiece &x, int o)
+{
+    LsePiece r;
+    r.m = __shfl_xor_sync(0xffffffffu, x.m, o);
+    r.a = __shfl_xor_sync(0xffffffffu, x.a, o);
+    r.s = __shfl_xor_sync(0xffffffffu, x.s, o);
+    r.acc.x = __shfl_xor_sync(0xffffffffu, x.acc.x, o);
+    r.acc.y = __shfl_xor_sync(0xffffffffu, x.acc.y, o);
+    r.acc.z = __shfl_xor_sync(0xffffffffu, x.acc.z, o);
+    r.acc.w = __shfl_xor_sync(0xffffffffu, x.acc.w, o);
+    return r;
+}
+
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const __grid_constant__ CombineParams p)
 {
     __shared__ int4 sdesc[kCombineMaxDesc];
-    __shared__ int wcount[kCombineThreads / 32];
-    __shared__ float4 part_acc[32][8];
-    __shared__ float2 part_ma[32];
-    __shared__ float part_s[32];
+    __shared__ int wtot[kCombineWarps];
+    __shared__ LsePiece xw[kCombineWarps][8]; // cross-warp step of a unit's merge
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the decode kernel's partials and descriptors are complete and visible after this
     grid_dep_wait();
     grid_dep_launch();
 
-    // compact copy of the descriptors that start a split segment (same order in every
-    // CTA); all descriptor loads are issued before the first is used
-    constexpr int kDescPerThread = kCombineMaxDesc / kCombineThreads;
-    int4 dv[kDescPerThread];
+    // ---- the descriptors that start a split segment, compacted in order: thread t holds
+    // descriptors [t * per, (t + 1) * per)
+    const int per = (p.n_desc + kCombineThreads - 1) / kCombineThreads; // <= 8
+    int4 dv[kCombineDescPerThread];
+    int cnt = 0;
 #pragma unroll
-    for (int k = 0; k < kDescPerThread; ++k) {
-        const int i = k * kCombineThreads + tid;
-        dv[k] = i < p.n_desc ? __ldcg(&p.desc[i]) : make_int4(0, 0, 0, 0);
+    for (int k = 0; k < kCombineDescPerThread; ++k) {
+        const int i = tid * per + k;
+        dv[k] = (k < per && i < p.n_desc) ? __ldcg(&p.desc[i]) : make_int4(0, 0, 0, 0);
+        cnt += dv[k].z > 0 ? 1 : 0;
     }
-    int nvalid = 0;
+    int incl = cnt;
 #pragma unroll
-    for (int k = 0; k < kDescPerThread; ++k) {
-        if (k * kCombineThreads >= p.n_desc)
-            break;
-        const bool v = dv[k].z > 0;
-        const unsigned m = __ballot_sync(0xffffffffu, v);
-        if (lane == 0)
-            wcount[warp] = __popc(m);
-        __syncthreads();
-        int off = nvalid;
-        int total = 0;
-        for (int w = 0; w < kCombineThreads / 32; ++w) {
-            if (w < warp)
-                off += wcount[w];
-            total += wcount[w];
-        }
-        if (v)
-            sdesc[off + __popc(m & ((1u << lane) - 1u))] = dv[k];
-        nvalid += total;
-        __syncthreads();
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += t;
     }
+    if (lane == 31)
+        wtot[warp] = incl;
+    __syncthreads();
+    int off = incl - cnt, nvalid = 0;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+        off += w < warp ? wtot[w] : 0;
+        nvalid += wtot[w];
+    }
+#pragma unroll
+    for (int k = 0; k < kCombineDescPerThread; ++k)
+        if (dv[k].z > 0)
+            sdesc[off++] = dv[k];
+    __syncthreads();
+
     const int H = p.heads_seg;
     const int per_seg = H * (128 / kCombineQuarter);
-    const long long T = (long long)nvalid * per_seg;
-    const long long ubeg = T * blockIdx.x / gridDim.x, uend = T * (blockIdx.x + 1) / gridDim.x;
+    // T <= 2048 segments x 512 units < 2^21 and the grid is at most 1024 CTAs, so the
+    // products below stay under 2^31
+    const unsigned T = (unsigned)nvalid * (unsigned)per_seg;
+    const int ubeg = (int)(T * blockIdx.x / gridDim.x);
+    const int uend = (int)(T * (blockIdx.x + 1) / gridDim.x);
 
     const int fl = tid & 7, row = tid >> 3;
-    for (long long u0 = ubeg; u0 < uend; u0 += 32) {
-        const int U = (int)((uend - u0) < 32 ? (uend - u0) : 32);
+    for (int u0 = ubeg; u0 < uend; u0 += 32) {
+        const int U = (uend - u0) < 32 ? (uend - u0) : 32;
         int upow = 1;
         while (upow < U)
             upow <<= 1;
         const int IG = 32 / upow; // rows per unit; row ig takes inputs ig, ig + IG, ...
-        const int u = row / IG, ig = row % IG;
+        const int u = row / IG, ig = row - u * IG;
         const bool active = u < U;
         int b = 0, hc = 0, n = 0, first = 0, hl = 0, q = 0;
         if (active) {
-            const long long unit = u0 + u;
-            const int d = (int)(unit / per_seg);
-            const int rem = (int)(unit - (long long)d * per_seg);
-            hl = rem / (128 / kCombineQuarter);
-            q = rem % (128 / kCombineQuarter);
+            const int unit = u0 + u;
+            const int d = unit / per_seg;
+            const int rem = unit - d * per_seg;
+            hl = rem >> 2;
+            q = rem & 3;
             const int4 ds = sdesc[d];
             b = ds.x;
             hc = ds.y;
@@ -121,76 +169,63 @@ __global__ void __launch_bounds__(kCombineThreads)
         }
         // this row's inputs: per chunk of kCombineBatchIn, all loads first, then the
         // maxima, then the rescaled sums (no chain of dependent exponentials)
-        float m = -INFINITY, a = -INFINITY, s = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        LsePiece x;
+        x.m = -INFINITY;
+        x.a = -INFINITY;
+        x.s = 0.f;
+        x.acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int i0 = ig; i0 < n; i0 += kCombineBatchIn * IG) {
-            float4 hd[kCombineBatchIn], x[kCombineBatchIn];
+            float4 hd[kCombineBatchIn], v[kCombineBatchIn];
 #pragma unroll
             for (int k = 0; k < kCombineBatchIn; ++k) {
                 const int i = i0 + k * IG;
                 hd[k] = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-                x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (i < n) {
                     const int slot = i == 0 ? first : 2 * ((first >> 1) + i);
                     const float *rp = p.partials + ((size_t)slot * H + hl) * kCombineSlotRow;
                     hd[k] = __ldcg(reinterpret_cast<const float4 *>(rp + 128));
-                    x[k] = __ldcg(reinterpret_cast<const float4 *>(rp + q * kCombineQuarter + 4 * fl));
+                    v[k] = __ldcg(reinterpret_cast<const float4 *>(rp + q * kCombineQuarter + 4 * fl));
                 }
             }
-            float mn = m, an = a;
+            float mn = x.m, an = x.a;
 #pragma unroll
             for (int k = 0; k < kCombineBatchIn; ++k) {
                 mn = fmaxf(mn, hd[k].x);
                 an = fmaxf(an, hd[k].z);
             }
-            const float fo = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-            const float go = (a == -INFINITY) ? 0.f : exp2f(a - an);
-            s *= fo;
-            acc = make_float4(acc.x * go, acc.y * go, acc.z * go, acc.w * go);
+            const float fo = lse_factor(x.m, mn), go = lse_factor(x.a, an);
+            x.s *= fo;
+            x.acc = make_float4(x.acc.x * go, x.acc.y * go, x.acc.z * go, x.acc.w * go);
 #pragma unroll
             for (int k = 0; k < kCombineBatchIn; ++k) {
-                const float fm = (hd[k].x == -INFINITY) ? 0.f : exp2f(hd[k].x - mn);
-                const float ga = (hd[k].z == -INFINITY) ? 0.f : exp2f(hd[k].z - an);
-                s += hd[k].y * fm;
-                acc.x += x[k].x * ga;
-                acc.y += x[k].y * ga;
-                acc.z += x[k].z * ga;
-                acc.w += x[k].w * ga;
+                const float fm = lse_factor(hd[k].x, mn), ga = lse_factor(hd[k].z, an);
+                x.s += hd[k].y * fm;
+                x.acc.x += v[k].x * ga;
+                x.acc.y += v[k].y * ga;
+                x.acc.z += v[k].z * ga;
+                x.acc.w += v[k].w * ga;
             }
-            m = mn;
-            a = an;
+            x.m = mn;
+            x.a = an;
         }
-        // merge the unit's rows: maxima first, then every row rescales its own piece, then
-        // row 0 of the unit adds them up
-        if (fl == 0)
-            part_ma[row] = make_float2(m, a);
-        __syncthreads();
-        const int r0 = u * IG;
-        float um = -INFINITY, ua = -INFINITY;
-        if (active)
-            for (int k = 0; k < IG; ++k) {
-                const float2 o = part_ma[r0 + k];
-                um = fmaxf(um, o.x);
-                ua = fmaxf(ua, o.y);
-            }
-        const float fr = (m == -INFINITY) ? 0.f : exp2f(m - um);
-        const float gr = (a == -INFINITY) ? 0.f : exp2f(a - ua);
-        part_acc[row][fl] = make_float4(acc.x * gr, acc.y * gr, acc.z * gr, acc.w * gr);
-        if (fl == 0)
-            part_s[row] = s * fr;
-        __syncthreads();
+        // merge the unit's IG rows: rows r and r ^ 1 (lanes 8 apart) and r ^ 2 (16 apart)
+        // share a warp; a unit of more than 4 rows spans IG / 4 whole warps
+        if (IG >= 2)
+            x = lse_merge(x, lse_shfl_xor(x, 8));
+        if (IG >= 4)
+            x = lse_merge(x, lse_shfl_xor(x, 16));
+        if (IG >= 8) {
+            if (lane < 8)
+                xw[warp][lane] = x;
+            __syncthreads();
+            if (lane < 8 && (warp & (IG / 4 - 1)) == 0)
+                for (int w = 1; w < IG / 4; ++w)
+                    x = lse_merge(x, xw[warp + w][lane]);
+            __syncthreads(); // xw is reused by the next batch
+        }
         if (active && ig == 0) {
-            float4 t = part_acc[r0][fl];
-            float st = part_s[r0];
-            for (int k = 1; k < IG; ++k) {
-                const float4 o = part_acc[r0 + k][fl];
-                t.x += o.x;
-                t.y += o.y;
-                t.z += o.z;
-                t.w += o.w;
-                st += part_s[r0 + k];
-            }
-            const float f = st > 0.f ? exp2f(ua - um) / st : 0.f;
+            const float f = x.s > 0.f ? exp2f(x.a - x.m) / x.s : 0.f;
             // segment row hl is query row hl % G of KV head hc * HPC + hl / G; that row is
             // query token hg / Gq, head kvh * Gq + hg % Gq of the [B][nq][Hq] output
             const int kvh = hc * p.HPC + hl / p.G, hg = hl % p.G;
@@ -198,9 +233,9 @@ __global__ void __launch_bounds__(kCombineThreads)
             const long long orow =
                 ((long long)b * p.nq + ti) * p.Hq + (long long)kvh * p.Gq + (hg - ti * p.Gq);
             float *dst = p.out + orow * 128 + q * kCombineQuarter + 4 * fl;
-            *reinterpret_cast<float4 *>(dst) = make_float4(t.x * f, t.y * f, t.z * f, t.w * f);
+            *reinterpret_cast<float4 *>(dst) =
+                make_float4(x.acc.x * f, x.acc.y * f, x.acc.z * f, x.acc.w * f);
         }
-        __syncthreads(); // part_* are reused by the next batch
     }
 }
 

@@ -50,12 +50,13 @@ constexpr int kThreads = 12 * 32;
 constexpr int kLaunchRegs = 168;    // per-thread registers at launch (65536 / 384, rounded)
 // Per-thread registers after setmaxnreg: the producer warpgroup gives registers to the two
 // consumer warpgroups. One 8-row query tile (NT == 1) fits in 200 consumer registers with
-// 96 left to the producer (no spills); the packed path's int32 PV accumulators need 216, and
-// two query tiles 224.
+// 96 left to the producer (no spills); the packed path's int32 PV accumulators and two
+// query tiles take 224 (with 216 the packed path spilled 2.5x as much and ran 0.35 us
+// slower on the 16 x 4096-token workload).
 template <int NT, bool kPack>
 struct RegSplit {
-    static constexpr int producer = kPack ? 72 : (NT == 1 ? 96 : 56);
-    static constexpr int consumer = kPack ? 216 : (NT == 1 ? 200 : 224);
+    static constexpr int producer = kPack ? 56 : (NT == 1 ? 96 : 56);
+    static constexpr int consumer = kPack ? 224 : (NT == 1 ? 200 : 224);
     static_assert(4 * 32 * producer + 8 * 32 * consumer <= kThreads * kLaunchRegs,
                   "register split exceeds the launch allocation");
 };
@@ -84,6 +85,8 @@ constexpr unsigned kErrSeqLen = 0x1u;
 constexpr unsigned kErrBlockTable = 0x2u;
 constexpr unsigned kErrTimeout = 0x4u;
 
+constexpr int kPscanLen = 40; // >= 33 ints: prefix[0..32] of a batch of up to 32 sequences
+
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a)
 {
     return (x + a - 1) / a * a;
@@ -94,7 +97,7 @@ struct SmemLayout {
     uint32_t stage_bytes; // one ring slot: K | V | kscale | vscale
     uint32_t off_k, off_v, off_ks, off_vs; // within a slot
     uint32_t sc_gap;      // bytes from a stage's K scales to its V scales (TT * sc_heads * 4)
-    uint32_t off_full, off_empty, off_mbar, off_mask, off_misc, off_slots, off_ptab, off_cstart,
+    uint32_t off_full, off_empty, off_mask, off_misc, off_pscan, off_ptab, off_cstart,
         off_prefix, off_scratch;
     uint32_t off_nseq;  // prefix count of sequences with tokens (B <= kPenaltyMaxB), else 0
     uint32_t off_qbuf;  // quantised query of a CTA's second segment (0 bytes when it did not fit)
@@ -118,14 +121,12 @@ __host__ __device__ inline SmemLayout make_layout(int TT, int HPC, int sc_heads,
     o += 8 * kMaxStages;
     L.off_empty = o;
     o += 8 * kMaxStages;
-    L.off_mbar = o;
-    o += 8;
     L.off_mask = o;
     o += 4 * kMaxStages;
     L.off_misc = o; // 8-byte aligned: the prefix scan's per-warp 64-bit sums
     o += 128;
-    L.off_slots = o;
-    o += 4 * 32;
+    L.off_pscan = o; // producer's own copy of the tile and sequence prefixes (B <= 32)
+    o += 4 * 2 * kPscanLen;
     L.off_ptab = o; // producer: physical slot of every box of the next 32 tiles
     o += 4 * 32 * kMaxBoxes;
     L.off_cstart = o;
@@ -227,49 +228,57 @@ __device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
     return lo;
 }
 
-// Per-sequence tile prefix: prefix[b + 1] = sum over b' <= b of nhc * ceil(L_b' / TT).
-// Per-sequence prefixes, one block-wide scan of (tiles, has tokens) packed in 64 bits:
+// Per-sequence prefixes of (tiles, has tokens), packed in 64 bits for one scan:
 // prefix[b + 1] = sum over b' <= b of nhc * ceil(L_b' / TT); nseq[b + 1] (when nseq is
 // given) = number of sequences b' <= b with L_b' > 0.
-__device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
-                             volatile unsigned long long *wsum, int tid, int warp, int lane)
+__device__ __forceinline__ unsigned long long prefix_item(const DecodeParams &p, int b)
 {
     const int cap = p.mbps * p.bs;
-    auto item = [&](int b) -> unsigned long long {
-        int L = p.seq_lens[b];
-        if (L < 0 || L > cap) {
-            atomicOr(p.errors, kErrSeqLen);
-            L = L < 0 ? 0 : cap;
-        }
-        return ((unsigned long long)(((L + p.TT - 1) / p.TT) * p.nhc) << 32) | (L > 0 ? 1u : 0u);
-    };
-    if (p.B <= 32) { // one warp: no block-wide pass (the caller synchronises once)
-        if (warp == 0) {
-            unsigned long long v = lane < p.B ? item(lane) : 0ull;
+    int L = p.seq_lens[b];
+    if (L < 0 || L > cap) {
+        atomicOr(p.errors, kErrSeqLen);
+        L = L < 0 ? 0 : cap;
+    }
+    return ((unsigned long long)(((L + p.TT - 1) / p.TT) * p.nhc) << 32) | (L > 0 ? 1u : 0u);
+}
+
+// The prefixes of a batch of at most 32 sequences, by one warp (no block-wide step).
+__device__ void scan_one_warp(const DecodeParams &p, int *prefix, int *nseq, int lane)
+{
+    unsigned long long v = lane < p.B ? prefix_item(p, lane) : 0ull;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long t = __shfl_up_sync(kFullMask, v, o);
-                if (lane >= o)
-                    v += t;
-            }
-            if (lane < p.B) {
-                prefix[lane + 1] = (int)(v >> 32);
-                if (nseq)
-                    nseq[lane + 1] = (int)(v & 0xffffffffu);
-            }
-            if (lane == 0) {
-                prefix[0] = 0;
-                if (nseq)
-                    nseq[0] = 0;
-            }
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long t = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o)
+            v += t;
+    }
+    if (lane < p.B) {
+        prefix[lane + 1] = (int)(v >> 32);
+        if (nseq)
+            nseq[lane + 1] = (int)(v & 0xffffffffu);
+    }
+    if (lane == 0) {
+        prefix[0] = 0;
+        if (nseq)
+            nseq[0] = 0;
+    }
+}
+
+// The prefixes of any batch, by the consumer warps (ctid < kConsumerThreads); batches up
+// to 32 take one warp. The caller synchronises the consumers afterwards.
+__device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
+                             volatile unsigned long long *wsum, int ctid, int warp, int lane)
+{
+    if (p.B <= 32) {
+        if (warp == 0)
+            scan_one_warp(p, prefix, nseq, lane);
         return;
     }
     unsigned long long carry = 0;
 #pragma unroll 1
-    for (int base = 0; base < p.B; base += kThreads) {
-        const int b = base + tid;
-        unsigned long long v = b < p.B ? item(b) : 0ull;
+    for (int base = 0; base < p.B; base += kConsumerThreads) {
+        const int b = base + ctid;
+        unsigned long long v = b < p.B ? prefix_item(p, b) : 0ull;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const unsigned long long t = __shfl_up_sync(kFullMask, v, o);
@@ -278,10 +287,10 @@ __device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
         }
         if (lane == 31)
             wsum[warp] = v;
-        __syncthreads();
+        consumer_bar();
         unsigned long long off = carry, total = 0;
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) {
+        for (int w = 0; w < kConsumerWarps; ++w) {
             const unsigned long long ws = wsum[w];
             if (w < warp)
                 off += ws;
@@ -293,9 +302,9 @@ __device__ void build_prefix(const DecodeParams &p, int *prefix, int *nseq,
                 nseq[b + 1] = (int)((off + v) & 0xffffffffu);
         }
         carry += total;
-        __syncthreads();
+        consumer_bar();
     }
-    if (tid == 0) {
+    if (ctid == 0) {
         prefix[0] = 0;
         if (nseq)
             nseq[0] = 0;
@@ -336,6 +345,31 @@ __device__ int cta_start(const DecodeParams &p, const int *prefix, const int *ns
     const int r = off - hc * (ntb + P);
     const int x = prefix[lo] + (hc < p.nhc ? hc * ntb + (r > P ? r - P : 0) : p.nhc * ntb);
     return x < N ? x : N;
+}
+
+// Work split of the flat tile list (see kSegPenaltyTiles): penalised when the sequence
+// counts are at hand and every CTA's share is at least 2 penalties, so that no CTA's share
+// can fall inside one segment's penalty (an empty CTA in the middle of a split segment would
+// break the contributor numbering). The producer and the consumers compute it separately
+// from the same prefixes, so they agree.
+struct Split {
+    int N;    // tiles
+    int gcta; // CTAs with tiles
+    int pseg; // penalty units before each sequence with tokens (0: plain split)
+    int V;    // units of the virtual list
+};
+
+__device__ __forceinline__ Split split_of(const DecodeParams &p, const int *prefix,
+                                          const int *nseq)
+{
+    Split sp;
+    sp.N = prefix[p.B];
+    sp.gcta = sp.N < (int)gridDim.x ? sp.N : (int)gridDim.x;
+    const int nseg_units = nseq ? kSegPenaltyTiles * p.nhc * nseq[p.B] : 0;
+    const bool pen = nseq && sp.gcta > 0 && (sp.N + nseg_units) / sp.gcta >= 2 * kSegPenaltyTiles;
+    sp.pseg = pen ? kSegPenaltyTiles * p.nhc : 0;
+    sp.V = sp.N + (pen ? nseg_units : 0);
+    return sp;
 }
 
 __device__ __forceinline__ int clamp_len(int L, int cap)
@@ -1438,7 +1472,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
-        mbar_init(reinterpret_cast<uint64_t *>(smem + p.lay.off_mbar), 1);
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -1449,64 +1482,87 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmVs);
         }
     }
+    __syncthreads(); // the barrier initialisation is visible to every warp
     // Everything above touches only shared memory and kernel parameters; from here on the
     // previous kernel on the stream (another call's combine, which reads the workspace, or
     // a producer of the inputs) must be complete.
     grid_dep_wait();
     grid_dep_launch();
-    if (tid == 0) { // no split segment recorded yet in this CTA's descriptor slots
+    int *nseq = p.lay.off_nseq ? reinterpret_cast<int *>(smem + p.lay.off_nseq) : nullptr;
+    int *cstart = reinterpret_cast<int *>(smem + p.lay.off_cstart);
+    // Warp specialisation: the producer warpgroup hands most of its registers to the two
+    // consumer warpgroups (the sums match the launch allocation, checked by static_assert).
+    // From here on the roles synchronise separately (named barriers), so the producer does
+    // not wait for the consumers' prologue: for a batch of up to 32 sequences it scans the
+    // sequence lengths and computes its CTA's range itself and starts loading at once.
+    if (warp >= kConsumerWarps) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::producer));
+        if (warp != kProducerWarp)
+            return;
+        const int *pre = prefix;
+        const int *pns = nseq;
+        if (p.B <= 32) {
+            int *pp = reinterpret_cast<int *>(smem + p.lay.off_pscan);
+            scan_one_warp(p, pp, pp + kPscanLen, lane);
+            __syncwarp();
+            pre = pp;
+            pns = pp + kPscanLen;
+        } else {
+            // the consumers publish the prefixes and this CTA's range
+            asm volatile("bar.sync 2, %0;" ::"n"(kConsumerThreads + 32) : "memory");
+        }
+        const Split sp = split_of(p, pre, pns);
+        if (sp.gcta == 0 || (int)blockIdx.x >= sp.gcta)
+            return;
+        int t0, t1;
+        if (p.B <= 32) {
+            const int v = lane < 2 ? cta_start(p, pre, pns, sp.pseg, sp.V, sp.gcta,
+                                               (int)blockIdx.x + lane)
+                                   : 0;
+            t0 = __shfl_sync(kFullMask, v, 0);
+            t1 = __shfl_sync(kFullMask, v, 1);
+        } else {
+            t0 = cstart[blockIdx.x];
+            t1 = cstart[blockIdx.x + 1];
+        }
+        produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, pre, t0, t1, lane);
+        return;
+    }
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::consumer));
+    const int ctid = warp * 32 + lane;
+    if (ctid == 0) { // no split segment recorded yet in this CTA's descriptor slots
         p.split_desc[2 * blockIdx.x] = make_int4(0, 0, 0, 0);
         p.split_desc[2 * blockIdx.x + 1] = make_int4(0, 0, 0, 0);
     }
-    int *nseq = p.lay.off_nseq ? reinterpret_cast<int *>(smem + p.lay.off_nseq) : nullptr;
     build_prefix(p, prefix, nseq,
-                 reinterpret_cast<volatile unsigned long long *>(smem + p.lay.off_misc), tid,
+                 reinterpret_cast<volatile unsigned long long *>(smem + p.lay.off_misc), ctid,
                  warp, lane);
-    __syncthreads();
-
-    const int N = prefix[p.B];
-    int *cstart = reinterpret_cast<int *>(smem + p.lay.off_cstart);
-    const int gcta = N < (int)gridDim.x ? N : (int)gridDim.x;
-    // Work split (see kSegPenaltyTiles): penalised when the sequence counts are at hand and
-    // every CTA's share is at least 2 penalties, so that no CTA's share can fall inside one
-    // segment's penalty (an empty CTA in the middle of a split segment would break the
-    // contributor numbering). Only this CTA's own range is computed before the producer
-    // starts; the consumers fill in the rest of the table (needed at segment ends).
-    const int nseg_units = nseq ? kSegPenaltyTiles * p.nhc * nseq[p.B] : 0;
-    const bool pen = nseq && gcta > 0 && (N + nseg_units) / gcta >= 2 * kSegPenaltyTiles;
-    const int pseg = pen ? kSegPenaltyTiles * p.nhc : 0;
-    const int V = N + (pen ? nseg_units : 0);
+    consumer_bar();
+    const Split sp = split_of(p, prefix, nseq);
+    const int gcta = sp.gcta;
+    if (gcta > 0 && ctid < 2 && (int)blockIdx.x + ctid <= gcta)
+        cstart[blockIdx.x + ctid] =
+            cta_start(p, prefix, nseq, sp.pseg, sp.V, gcta, (int)blockIdx.x + ctid);
+    consumer_bar();
+    if (p.B > 32) // release the producer (it waits for the prefixes and the range)
+        asm volatile("bar.arrive 2, %0;" ::"n"(kConsumerThreads + 32) : "memory");
     if (gcta == 0) { // no sequence has tokens: every row is zero
 #pragma unroll 1
         for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
             float4 *row = reinterpret_cast<float4 *>(p.out + (long long)b * p.nq * p.Hq * kD);
 #pragma unroll 1
-            for (int i = tid; i < p.nq * p.Hq * kD / 4; i += kThreads)
+            for (int i = ctid; i < p.nq * p.Hq * kD / 4; i += kConsumerThreads)
                 row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
-    if (tid < 2 && (int)blockIdx.x + tid <= gcta)
-        cstart[blockIdx.x + tid] = cta_start(p, prefix, nseq, pseg, V, gcta, blockIdx.x + tid);
-    __syncthreads();
     if ((int)blockIdx.x >= gcta)
         return;
     const int t0 = cstart[blockIdx.x], t1 = cstart[blockIdx.x + 1];
-    // (the rest of the table and the zero rows of empty sequences: consumers, below)
-    // Warp specialisation: the producer warpgroup hands most of its registers to the two
-    // consumer warpgroups (the sums match the launch allocation, checked by static_assert).
-    if (warp >= kConsumerWarps) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::producer));
-        if (warp == kProducerWarp)
-            produce(p, &tmK, &tmV, &tmKs, &tmVs, smem, prefix, t0, t1, lane);
-        return;
-    }
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::consumer));
-    const int ctid = warp * 32 + lane;
 #pragma unroll 1
     for (int i = ctid; i <= gcta; i += kConsumerThreads)
         if (i != (int)blockIdx.x && i != (int)blockIdx.x + 1)
-            cstart[i] = cta_start(p, prefix, nseq, pseg, V, gcta, i);
+            cstart[i] = cta_start(p, prefix, nseq, sp.pseg, sp.V, gcta, i);
     // rows of empty sequences are zero (spread over the CTAs that have tiles)
 #pragma unroll 1
     for (int b = blockIdx.x; b < p.B; b += gcta) {
