@@ -10,15 +10,13 @@
 #include <mutex>
 
 #include "q8kv.h"
-#include "q8kv_combine.cuh"
-#include "q8kv_decode.cuh"
+#include "q8kv_combine.cuh" // (includes the decode kernel)
 #include "q8kv_qquant.cuh"
 
 namespace {
 
 using namespace q8kv;
 
-static_assert(kCombineSlotRow == kSlotRow, "partial row layout differs between the kernels");
 static_assert(kErrSeqLen == Q8KV_DEVERR_SEQ_LEN && kErrBlockTable == Q8KV_DEVERR_BLOCK_TABLE &&
                   kErrTimeout == Q8KV_DEVERR_TIMEOUT,
               "device error bits differ from the header");
@@ -48,6 +46,7 @@ struct DeviceInfo {
     int smem_optin = 0;
     unsigned *errors = nullptr;      // address of g_device_errors on this device
     bool attr_set[3][2] = {{false, false}, {false, false}, {false, false}};
+    bool combine_attr = false;
     void *ws = nullptr;              // library-managed workspace
     size_t ws_bytes = 0;
 };
@@ -101,7 +100,7 @@ struct Plan {
     int scale_bulk, sc_heads, heads_seg, scratch_stride, grid;
     SmemLayout lay;
     size_t smem_bytes;
-    size_t ws_desc_off, ws_part_off, ws_bytes;
+    size_t ws_bytes;
 };
 
 bool is_pow2(int x)
@@ -156,14 +155,11 @@ q8kv_status plan_heads(int Hq, int Hk, int D, Plan &pl)
     return Q8KV_OK;
 }
 
-// Workspace: the split-segment descriptors (2 per CTA, rewritten by every call, so no part
-// of the workspace needs an initial value), then the partial slots (2 per CTA).
+// Workspace: the partial slots (2 per CTA). Every call writes the slots its combine reads
+// (the combine derives which from the work split), so no part needs an initial value.
 void plan_workspace(int grid, Plan &pl)
 {
-    pl.ws_desc_off = 0;
-    pl.ws_part_off = align256(sizeof(int4) * 2 * (size_t)grid);
-    pl.ws_bytes = pl.ws_part_off +
-                  align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * kSlotRow);
+    pl.ws_bytes = align256(sizeof(float) * 2 * (size_t)grid * pl.heads_seg * kSlotRow);
 }
 
 q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
@@ -186,7 +182,8 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
     if (tiles_max >= (1LL << 30))
         return Q8KV_ERR_UNSUPPORTED; // tile indices (and the penalised split) are 32-bit
     pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
-    if (2 * pl.grid > kCombineMaxDesc)
+    // the combine kernel's dynamic shared memory (its static part is about 2 KB)
+    if (combine_layout(s.B, pl.grid).total + kCombineStaticSmemMax > (uint32_t)dev.smem_optin)
         return Q8KV_ERR_UNSUPPORTED;
     pl.box_tok = pl.TT < s.bs ? pl.TT : s.bs;
     pl.log2_box = ilog2(pl.box_tok);
@@ -384,22 +381,19 @@ q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl
     cfg.numAttrs = 1;
     Q8KV_CUDA(cudaLaunchKernelEx(&cfg, fn, p, mk, mv, mks, mvs));
 
-    CombineParams cp;
-    cp.out = p.out;
-    cp.partials = p.partials;
-    cp.desc = p.split_desc;
-    cp.n_desc = 2 * pl.grid;
-    cp.Hq = p.Hq;
-    cp.heads_seg = p.heads_seg;
-    cp.G = p.G;
-    cp.Gq = p.Gq;
-    cp.nq = p.nq;
-    cp.HPC = p.HPC;
+    if (!dev.combine_attr) {
+        // the dynamic part may use what the kernel's static shared memory leaves of the limit
+        cudaFuncAttributes fa;
+        Q8KV_CUDA(cudaFuncGetAttributes(&fa, combine_kernel));
+        Q8KV_CUDA(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev.smem_optin - (int)fa.sharedSizeBytes));
+        dev.combine_attr = true;
+    }
     cudaLaunchConfig_t cc = cfg;
     cc.gridDim = dim3((unsigned)dev.sms);
     cc.blockDim = dim3(kCombineThreads);
-    cc.dynamicSmemBytes = 0;
-    Q8KV_CUDA(cudaLaunchKernelEx(&cc, combine_kernel, cp));
+    cc.dynamicSmemBytes = combine_layout(p.B, pl.grid).total;
+    Q8KV_CUDA(cudaLaunchKernelEx(&cc, combine_kernel, p, pl.grid));
     return Q8KV_OK;
 }
 
@@ -450,8 +444,7 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.seq_lens = c.lens;
     p.kscale = c.ks;
     p.vscale = c.vs;
-    p.split_desc = reinterpret_cast<int4 *>(w + pl.ws_desc_off);
-    p.partials = reinterpret_cast<float *>(w + pl.ws_part_off);
+    p.partials = reinterpret_cast<float *>(w);
     p.errors = dev->errors;
     p.dbg_dots = c.dots;
     p.dbg_max_len = c.dots_max_len;
@@ -496,8 +489,8 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
 
 } // namespace
 
-// Scratch of q8kv_decode_attn_static: split-segment descriptors and partial results at the
-// same offsets as a caller-owned workspace. A file-scope device array rather than an allocation,
+// Scratch of q8kv_decode_attn_static: the partial results of split sequences, at the same
+// offsets as in a caller-owned workspace. A file-scope device array rather than an allocation,
 // so that a call of that entry point never allocates: its callers are ones that must not
 // allocate while serving (a pool allocator owns all device memory, or the step cannot take
 // cudaMalloc's latency or cudaFree's device-wide synchronisation). One instance exists per
@@ -514,8 +507,8 @@ struct StaticScratch {
 StaticScratch g_static[kMaxDevices];
 
 // Set-up, once per device, with that device current: look up the array's address on this
-// device. No part of the scratch needs an initial value (every call rewrites the
-// split-segment descriptors before the partial slots they point to are read).
+// device. No part of the scratch needs an initial value (every call's combine reads only
+// the partial slots the same call's decode kernel wrote).
 q8kv_status static_scratch(void **out)
 {
     std::lock_guard<std::mutex> lock(g_mutex);

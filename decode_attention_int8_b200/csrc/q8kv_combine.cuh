@@ -11,14 +11,20 @@
 // the Kestrel-LLM walk-through "flash_attn_single_q_q8_neon", trdm.cn/news/511694,
 // section 2 part 3, applied between pieces instead of between tokens).
 //
-// The decode kernel records, for every segment it split, a descriptor in the slot of the
-// segment's first contributor: {b, hc, n contributors, first partial slot}; the other
-// contributors' slots are 2 * (first CTA + k), k = 1..n-1. This kernel runs next on the
-// stream (programmatic dependent launch: it is scheduled while the decode kernel drains
-// and waits for its completion before reading anything). Its time is all latency (the
-// partials are a few MB in L2), so it is laid out for few dependent steps:
-//  * one load per thread of the descriptors and one block-wide scan compact them (the same
-//    order in every CTA);
+// Which segments the decode kernel split, and between which CTAs, follows from its work
+// split alone: the same prefixes of the sequence lengths and the same CTA ranges, which this
+// kernel recomputes (q8kv_decode.cuh) before it waits for the decode kernel. Reading the
+// sequence lengths that early is safe: the only kernel before this one on the stream is the
+// decode kernel of the same call, which never writes them, and this grid starts only after
+// every decode CTA has passed its own dependency wait. Decode CTA j owns partial slots 2j
+// (the segment its range starts in) and 2j + 1 (the segment it ends in); a split segment
+// whose first contributor is j sits in slot 2j (when it starts exactly at j's first tile)
+// or 2j + 1, and contributor k > 0 in slot 2 (j + k). This kernel runs next on the stream
+// (programmatic dependent launch: it is scheduled while the decode kernel drains and waits
+// for its completion before reading any partial). Its time is all latency (the partials
+// are a few MB in L2), so it is laid out for few dependent steps:
+//  * before the wait: the prefixes (one warp for up to 32 sequences), the CTA ranges, and
+//    the split segments in CTA order (a block-wide scan compacts them);
 //  * the work is the list of units (segment, query head, 32-channel quarter), split evenly
 //    over the CTAs in 32-bit arithmetic; a CTA takes up to 32 units at a time and gives
 //    each unit 32 / units-in-batch rows of 8 threads that stride over the unit's inputs,
@@ -30,26 +36,44 @@
 
 #include <cstdint>
 
+#include "q8kv_decode.cuh"
 #include "q8kv_ptx.cuh"
 
 namespace q8kv {
 
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 256; // = kConsumerThreads: the decode's split helpers
+                                     // synchronise 256 threads on named barrier 1
 constexpr int kCombineWarps = kCombineThreads / 32;
-constexpr int kCombineMaxDesc = 2048;  // 2 * decode grid (the grid is at most 1024 CTAs)
-constexpr int kCombineQuarter = 32;    // channels per unit
-constexpr int kCombineSlotRow = 132;   // floats per partial row: acc[128], M, S, A, pad
-constexpr int kCombineDescPerThread = kCombineMaxDesc / kCombineThreads;
+constexpr int kCombineQuarter = 32;  // channels per unit
+static_assert(kCombineThreads == kConsumerThreads, "the split helpers need 256 threads");
+constexpr uint32_t kCombineStaticSmemMax = 4096; // bound on the kernel's static shared memory
 
-struct CombineParams {
-    float *out;
-    const float *partials; // [n_desc slots] x heads_seg x kCombineSlotRow
-    const int4 *desc;      // [n_desc] {b, hc, n (0: none), first slot}
-    int n_desc;
-    int Hq, heads_seg;
-    int G, Gq, nq, HPC;    // query rows per KV head (nq tokens x Gq heads), tokens, KV heads
-                           // per segment
+// Dynamic shared memory of the combine kernel: split segments (one int4 per decode CTA),
+// CTA ranges, then the prefixes.
+struct CombineLayout {
+    uint32_t off_desc, off_cstart, off_prefix, off_nseq, off_wsum, total;
 };
+
+__host__ __device__ inline CombineLayout combine_layout(int B, int grid)
+{
+    CombineLayout L;
+    uint32_t o = 0;
+    L.off_desc = o;
+    o += 16u * (uint32_t)grid;
+    L.off_cstart = o;
+    o = align_up(o + 4u * (uint32_t)(grid + 1), 16);
+    L.off_prefix = o;
+    o = align_up(o + 4u * (uint32_t)(B + 1), 16);
+    L.off_nseq = 0;
+    if (B <= kPenaltyMaxB) {
+        L.off_nseq = o;
+        o = align_up(o + 4u * (uint32_t)(B + 1), 16);
+    }
+    L.off_wsum = o;
+    o += 8u * kConsumerWarps;
+    L.total = o;
+    return L;
+}
 
 constexpr int kCombineBatchIn = 8; // inputs a thread loads at once
 
@@ -93,49 +117,63 @@ __device__ __forceinline__ LsePiece lse_shfl_xor(const LsePiece &x, int o)
 }
 
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const __grid_constant__ CombineParams p)
+    combine_kernel(const __grid_constant__ DecodeParams p, int grid_dec)
 {
-    __shared__ int4 sdesc[kCombineMaxDesc];
+    extern __shared__ __align__(16) uint8_t csm[];
+    const CombineLayout cl = combine_layout(p.B, grid_dec);
+    int4 *sdesc = reinterpret_cast<int4 *>(csm + cl.off_desc);
+    int *cstart = reinterpret_cast<int *>(csm + cl.off_cstart);
+    int *prefix = reinterpret_cast<int *>(csm + cl.off_prefix);
+    int *nseq = cl.off_nseq ? reinterpret_cast<int *>(csm + cl.off_nseq) : nullptr;
     __shared__ int wtot[kCombineWarps];
     __shared__ LsePiece xw[kCombineWarps][8]; // cross-warp step of a unit's merge
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // the decode kernel's partials and descriptors are complete and visible after this
+    // ---- before the dependency wait: the decode kernel's work split (inputs only)
+    build_prefix(p, prefix, nseq,
+                 reinterpret_cast<volatile unsigned long long *>(csm + cl.off_wsum), tid, warp,
+                 lane);
+    consumer_bar();
+    const Split sp = split_of(p, prefix, nseq, grid_dec);
+    const int g = sp.gcta;
+    for (int i = tid; i <= g; i += kCombineThreads)
+        cstart[i] = cta_start(p, prefix, nseq, sp.pseg, sp.V, g, i);
+    consumer_bar();
+    // the split segment whose first contributor is decode CTA j (< g): the segment of its
+    // last tile, when it starts inside j's range and ends past it (thread t takes
+    // j = t, t + 256, ...; a block-wide scan compacts them in order)
+    int nvalid = 0;
+    for (int j0 = 0; j0 < g; j0 += kCombineThreads) {
+        const int j = j0 + tid;
+        int4 d = make_int4(0, 0, 0, 0);
+        bool v = false;
+        if (j < g) {
+            const int t0 = cstart[j], t1 = cstart[j + 1];
+            const SegCursor cu = cursor_at(p, prefix, t1 - 1);
+            if (cu.seg0 >= t0 && cu.seg1 > t1) {
+                const int last = cta_of_tile(cstart, g, cu.seg1 - 1);
+                d = make_int4(cu.b, cu.hc, last - j + 1, 2 * j + (cu.seg0 == t0 ? 0 : 1));
+                v = true;
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, v);
+        if (lane == 0)
+            wtot[warp] = __popc(m);
+        consumer_bar();
+        int off = nvalid, total = 0;
+#pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) {
+            off += w < warp ? wtot[w] : 0;
+            total += wtot[w];
+        }
+        if (v)
+            sdesc[off + __popc(m & ((1u << lane) - 1u))] = d;
+        nvalid += total;
+        consumer_bar();
+    }
+    // the decode kernel's partials are complete and visible after this
     grid_dep_wait();
     grid_dep_launch();
-
-    // ---- the descriptors that start a split segment, compacted in order: thread t holds
-    // descriptors [t * per, (t + 1) * per)
-    const int per = (p.n_desc + kCombineThreads - 1) / kCombineThreads; // <= 8
-    int4 dv[kCombineDescPerThread];
-    int cnt = 0;
-#pragma unroll
-    for (int k = 0; k < kCombineDescPerThread; ++k) {
-        const int i = tid * per + k;
-        dv[k] = (k < per && i < p.n_desc) ? __ldcg(&p.desc[i]) : make_int4(0, 0, 0, 0);
-        cnt += dv[k].z > 0 ? 1 : 0;
-    }
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o)
-            incl += t;
-    }
-    if (lane == 31)
-        wtot[warp] = incl;
-    __syncthreads();
-    int off = incl - cnt, nvalid = 0;
-#pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) {
-        off += w < warp ? wtot[w] : 0;
-        nvalid += wtot[w];
-    }
-#pragma unroll
-    for (int k = 0; k < kCombineDescPerThread; ++k)
-        if (dv[k].z > 0)
-            sdesc[off++] = dv[k];
-    __syncthreads();
 
     const int H = p.heads_seg;
     const int per_seg = H * (128 / kCombineQuarter);
@@ -183,7 +221,7 @@ __global__ void __launch_bounds__(kCombineThreads)
                 v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (i < n) {
                     const int slot = i == 0 ? first : 2 * ((first >> 1) + i);
-                    const float *rp = p.partials + ((size_t)slot * H + hl) * kCombineSlotRow;
+                    const float *rp = p.partials + ((size_t)slot * H + hl) * kSlotRow;
                     hd[k] = __ldcg(reinterpret_cast<const float4 *>(rp + 128));
                     v[k] = __ldcg(reinterpret_cast<const float4 *>(rp + q * kCombineQuarter + 4 * fl));
                 }

@@ -28,9 +28,9 @@
 //    spread of the V scales). Both are ordinary online maxima: rescale when they rise.
 //  * Per-warp states are merged in shared memory. A segment that one CTA covers whole is
 //    normalised and written out here; a CTA that covers only part of one leaves its
-//    partial (M, S, A, acc) in the workspace, and the first contributor records the
-//    segment in a descriptor for the log-sum-exp combine kernel (q8kv_combine.cuh) that
-//    runs next on the stream. No CTA ever waits for another.
+//    partial (M, S, A, acc) in the workspace for the log-sum-exp combine kernel
+//    (q8kv_combine.cuh) that runs next on the stream and recomputes the same work split to
+//    find the split segments. No CTA ever waits for another.
 #pragma once
 
 #include <cuda.h>
@@ -158,7 +158,6 @@ struct DecodeParams {
     const float *kscale;
     const float *vscale;
     float *partials;     // [2 * grid slots] x heads_seg x kSlotRow (kD acc, M, S, A, pad)
-    int4 *split_desc;    // [2 * grid] {b, hc, contributors, first slot}; rewritten every call
     unsigned *errors;    // device error word
     int32_t *dbg_dots;   // [B][Hq][dbg_max_len][kNB] (debug instantiation only)
     int dbg_max_len;
@@ -234,7 +233,7 @@ __device__ __forceinline__ int cta_of_tile(const int *cstart, int g, int x)
 __device__ __forceinline__ unsigned long long prefix_item(const DecodeParams &p, int b)
 {
     const int cap = p.mbps * p.bs;
-    int L = p.seq_lens[b];
+    int L = __ldcg(p.seq_lens + b);
     if (L < 0 || L > cap) {
         atomicOr(p.errors, kErrSeqLen);
         L = L < 0 ? 0 : cap;
@@ -360,11 +359,11 @@ struct Split {
 };
 
 __device__ __forceinline__ Split split_of(const DecodeParams &p, const int *prefix,
-                                          const int *nseq)
+                                          const int *nseq, int grid)
 {
     Split sp;
     sp.N = prefix[p.B];
-    sp.gcta = sp.N < (int)gridDim.x ? sp.N : (int)gridDim.x;
+    sp.gcta = sp.N < grid ? sp.N : grid;
     const int nseg_units = nseq ? kSegPenaltyTiles * p.nhc * nseq[p.B] : 0;
     const bool pen = nseq && sp.gcta > 0 && (sp.N + nseg_units) / sp.gcta >= 2 * kSegPenaltyTiles;
     sp.pseg = pen ? kSegPenaltyTiles * p.nhc : 0;
@@ -1144,8 +1143,7 @@ template <int NT, bool kPack>
 __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpState<NT> &st,
                                                  uint8_t *smem, int b,
                                  int hc, int kl, int slice, int pair, int ts, int g, int c,
-                                 int ctid, const int *prefix, const int *cstart, int gcta,
-                                 int t0, int t1)
+                                 const int *prefix, int t0, int t1)
 {
     // complete this lane's row sums
 #pragma unroll
@@ -1256,8 +1254,8 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
     }
 
     // partial: this CTA's share of the segment goes to its workspace slot (0: the segment
-    // this CTA's range starts in, 1: the one it ends in); the first contributor describes
-    // the segment for the combine kernel
+    // this CTA's range starts in, 1: the one it ends in); the combine kernel finds the
+    // split segments and their contributors from the same work split
     const int which = (seg0 <= t0) ? 0 : 1;
     const int H = p.heads_seg;
     if (ts == 0) {
@@ -1281,11 +1279,6 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams &p, WarpStat
                         make_float4(st.M[r], st.S[r], st.A[r], 0.f);
             }
         }
-    }
-    if (ctid == 0 && seg0 >= t0) {
-        const int last = cta_of_tile(cstart, gcta, seg1 - 1);
-        const int slot = 2 * (int)blockIdx.x + which;
-        p.split_desc[slot] = make_int4(b, hc, last - (int)blockIdx.x + 1, slot);
     }
 }
 
@@ -1318,9 +1311,34 @@ __device__ __forceinline__ SegCursor cursor_at(const DecodeParams &p, const int 
     return cu;
 }
 
+// Does this CTA's range [t0, t1) reach into a second segment whose query fits the buffer?
+__device__ __forceinline__ bool has_second_query(const DecodeParams &p, const int *prefix, int t0,
+                                                 int t1)
+{
+    return p.lay.qbuf_rows != 0 && cursor_at(p, prefix, t0).seg1 < t1;
+}
+
+// Warp 9: the quantised query rows of the CTA's second segment, for every (KV head, slice)
+// pair, in the buffer's lane-fragment order (what the consumers' load_query would produce).
+template <int NT, bool kPack>
+__device__ void prepare_second_query(const DecodeParams &p, uint8_t *smem, const int *prefix,
+                                     int t0, int lane)
+{
+    const SegCursor c1 = cursor_at(p, prefix, cursor_at(p, prefix, t0).seg1);
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll 1
+    for (int pair = 0; pair < p.pairs; ++pair) {
+        const int kl = pair / p.slices, slice = pair % p.slices;
+        const QueryFrag<NT> qf = load_query<NT, kPack>(p, c1.b, c1.hc, kl, slice, g, c);
+        store_query<NT, kPack>(smem_addr(smem) + p.lay.off_qbuf +
+                                   (uint32_t)pair * p.lay.qbuf_rows * kQRowBytes,
+                               qf, g, c);
+    }
+}
+
 template <int NT, bool kPack, bool kDump>
 __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
-                        const int *cstart, int t0, int t1, int gcta, int warp, int lane)
+                        int t0, int t1, int warp, int lane)
 {
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
     uint64_t *empty = reinterpret_cast<uint64_t *>(smem + p.lay.off_empty);
@@ -1365,20 +1383,12 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
     const int all_boxes = (1 << p.n_boxes) - 1;
     const uint32_t qbuf = smem_base + p.lay.off_qbuf +
                           (uint32_t)pair * p.lay.qbuf_rows * kQRowBytes;
-    // The quantised query of the CTA's second segment is prepared before the first stage
-    // (while the first loads are in flight) and kept in shared memory, so that switching
-    // segments in the middle of the stream costs neither a global round trip nor the
-    // quantisation code. Warps of one (KV head, slice) pair hold the same rows; the ts == 0
-    // warp writes them.
-    const SegCursor first = cursor_at(p, prefix, t0);
-    const bool prefetch_q = p.lay.qbuf_rows != 0 && first.seg1 < t1;
-    if (prefetch_q) {
-        const SegCursor c1 = cursor_at(p, prefix, first.seg1);
-        const QueryFrag<NT> qf = load_query<NT, kPack>(p, c1.b, c1.hc, kl, slice, g, c);
-        if (ts == 0)
-            store_query<NT, kPack>(qbuf, qf, g, c);
-        consumer_bar();
-    }
+    // The quantised query of the CTA's second segment is prepared by warp 9 (otherwise idle)
+    // while the first segment streams and kept in shared memory, so that switching segments
+    // in the middle of the stream costs neither a global round trip nor the quantisation
+    // code, and the first stage is not held up by it; the consumers take it at the switch
+    // after named barrier 4.
+    const bool prefetch_q = has_second_query(p, prefix, t0, t1);
     int seg_index = 0;
     // Outer loop: one segment (this CTA's tiles of one sequence and head chunk) per pass.
     for (int x = t0; x < t1;) {
@@ -1386,6 +1396,8 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
         const int x_end = cu.seg1 < t1 ? cu.seg1 : t1;
         const uint32_t scol4 = 4u * (uint32_t)((cu.hc * p.HPC) % p.sc_heads);
         {
+            if (prefetch_q && seg_index == 1) // warp 9 has written the buffer
+                asm volatile("bar.sync 4, %0;" ::"n"(kConsumerThreads + 32) : "memory");
             const QueryFrag<NT> qf = (prefetch_q && seg_index == 1)
                                          ? load_query_smem<NT, kPack>(qbuf, g, c)
                                          : load_query<NT, kPack>(p, cu.b, cu.hc, kl, slice, g, c);
@@ -1449,7 +1461,7 @@ __device__ void consume(const DecodeParams &p, uint8_t *smem, const int *prefix,
                 packed_fold(st, pa, k0, k1, 1.f, 1.f);
         }
         finalize_segment<NT, kPack>(p, st, smem, cu.b, cu.hc, kl, slice, pair, ts, g, c,
-                                    warp * 32 + lane, prefix, cstart, gcta, t0, t1);
+                                    prefix, t0, t1);
     }
 }
 
@@ -1497,6 +1509,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // sequence lengths and computes its CTA's range itself and starts loading at once.
     if (warp >= kConsumerWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::producer));
+        if (warp == kProducerWarp + 1) {
+            // the second segment's query, once the consumers have published the split
+            asm volatile("bar.sync 3, %0;" ::"n"(kConsumerThreads + 32) : "memory");
+            const Split sp = split_of(p, prefix, nseq, (int)gridDim.x);
+            if (sp.gcta == 0 || (int)blockIdx.x >= sp.gcta)
+                return;
+            const int t0 = cstart[blockIdx.x], t1 = cstart[blockIdx.x + 1];
+            if (has_second_query(p, prefix, t0, t1)) {
+                prepare_second_query<NT, kPack>(p, smem, prefix, t0, lane);
+                asm volatile("bar.arrive 4, %0;" ::"n"(kConsumerThreads + 32) : "memory");
+            }
+            return;
+        }
         if (warp != kProducerWarp)
             return;
         const int *pre = prefix;
@@ -1511,7 +1536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the consumers publish the prefixes and this CTA's range
             asm volatile("bar.sync 2, %0;" ::"n"(kConsumerThreads + 32) : "memory");
         }
-        const Split sp = split_of(p, pre, pns);
+        const Split sp = split_of(p, pre, pns, (int)gridDim.x);
         if (sp.gcta == 0 || (int)blockIdx.x >= sp.gcta)
             return;
         int t0, t1;
@@ -1530,15 +1555,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<NT, kPack>::consumer));
     const int ctid = warp * 32 + lane;
-    if (ctid == 0) { // no split segment recorded yet in this CTA's descriptor slots
-        p.split_desc[2 * blockIdx.x] = make_int4(0, 0, 0, 0);
-        p.split_desc[2 * blockIdx.x + 1] = make_int4(0, 0, 0, 0);
-    }
     build_prefix(p, prefix, nseq,
                  reinterpret_cast<volatile unsigned long long *>(smem + p.lay.off_misc), ctid,
                  warp, lane);
     consumer_bar();
-    const Split sp = split_of(p, prefix, nseq);
+    const Split sp = split_of(p, prefix, nseq, (int)gridDim.x);
     const int gcta = sp.gcta;
     if (gcta > 0 && ctid < 2 && (int)blockIdx.x + ctid <= gcta)
         cstart[blockIdx.x + ctid] =
@@ -1546,6 +1567,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     consumer_bar();
     if (p.B > 32) // release the producer (it waits for the prefixes and the range)
         asm volatile("bar.arrive 2, %0;" ::"n"(kConsumerThreads + 32) : "memory");
+    // and warp 9 (the second segment's query)
+    asm volatile("bar.arrive 3, %0;" ::"n"(kConsumerThreads + 32) : "memory");
     if (gcta == 0) { // no sequence has tokens: every row is zero
 #pragma unroll 1
         for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
@@ -1559,10 +1582,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if ((int)blockIdx.x >= gcta)
         return;
     const int t0 = cstart[blockIdx.x], t1 = cstart[blockIdx.x + 1];
-#pragma unroll 1
-    for (int i = ctid; i <= gcta; i += kConsumerThreads)
-        if (i != (int)blockIdx.x && i != (int)blockIdx.x + 1)
-            cstart[i] = cta_start(p, prefix, nseq, sp.pseg, sp.V, gcta, i);
     // rows of empty sequences are zero (spread over the CTAs that have tiles)
 #pragma unroll 1
     for (int b = blockIdx.x; b < p.B; b += gcta) {
@@ -1574,7 +1593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             row[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     consumer_bar();
-    consume<NT, kPack, kDump>(p, smem, prefix, cstart, t0, t1, gcta, warp, lane);
+    consume<NT, kPack, kDump>(p, smem, prefix, t0, t1, warp, lane);
 }
 
 } // namespace q8kv

@@ -168,8 +168,9 @@ q8kv_status q8kv_decode_attn_q4(float *out, const float *q, const uint8_t *k4_bl
 size_t q8kv_workspace_bytes(int B, int n_q_heads, int n_kv_heads, int head_dim);
 
 /* Zero a caller-owned workspace. Optional and without effect on results: no part of the
- * workspace needs an initial value (every call rewrites the split-segment descriptors it
- * reads before reading them); it only gives a fresh workspace defined contents. */
+ * workspace needs an initial value (every call writes the partial results its combine
+ * step reads before that step reads them); it only gives a fresh workspace defined
+ * contents. */
 q8kv_status q8kv_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Same as q8kv_decode_attn with a caller-owned workspace (device memory of at least
@@ -187,9 +188,9 @@ q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_bloc
 #define Q8KV_STATIC_SCRATCH_BYTES (12u * 1024u * 1024u)
 
 /*
- * Same as q8kv_decode_attn, but the call allocates no device memory at all: the
- * split-segment descriptors and partial results live in a fixed device array inside the
- * library, Q8KV_STATIC_SCRATCH_BYTES bytes per device. None of the source pages has a counterpart
+ * Same as q8kv_decode_attn, but the call allocates no device memory at all: the partial
+ * results of the split sequences live in a fixed device array inside the library,
+ * Q8KV_STATIC_SCRATCH_BYTES bytes per device. None of the source pages has a counterpart
  * to this entry point; they describe the computation, not where its scratch lives.
  *
  * Who needs it: a caller that must not allocate while it serves requests. Examples are a
@@ -203,9 +204,9 @@ q8kv_status q8kv_decode_attn_ws(float *out, const float *q, const int8_t *k_bloc
  * address (cudaGetSymbolAddress) and the kernels' attributes; later calls reuse them.
  * Make that first call before any stream capture begins.
  *
- * Initial state: nothing in the array needs to start at zero. Every call first rewrites
- * the split-segment descriptors (2 per CTA), then the partial results they point to, and
- * the combine kernel reads only what the same call wrote.
+ * Initial state: nothing in the array needs to start at zero. Every call's decode kernel
+ * writes the partial results (2 slots per CTA) that the same call's combine kernel reads,
+ * and the combine reads no other slot.
  *
  * Races: every call on one device uses the same array. Two calls that may run at the
  * same time on the GPU (different streams with no ordering between them, or threads
