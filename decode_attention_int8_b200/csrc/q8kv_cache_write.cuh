@@ -282,8 +282,11 @@ __device__ __forceinline__ uint32_t q4_chunk(float4 x, int g8, uint16_t &d16, bo
     }
     // m with its sign; an all-zero block keeps m = +0 (d = +0 / -8 = -0)
     const float m = __uint_as_float(abits | (abits != 0u ? (uint32_t)(k & 1u) << 31 : 0u));
-    const float d = __fdiv_rn(m, -8.0f);
-    const float id = d != 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+    // m / -8 and 1 / d, each correctly rounded: the quotient by a power of two is the product
+    // by its reciprocal (the same exact value, so the same rounding), and the correctly
+    // rounded reciprocal is the correctly rounded quotient 1 / d
+    const float d = __fmul_rn(m, -0.125f);
+    const float id = d != 0.0f ? __frcp_rn(d) : 0.0f;
     d16 = __half_as_ushort(__float2half_rn(d));
     return q4_code(x.x, id) | (q4_code(x.y, id) << 4) | (q4_code(x.z, id) << 8) |
            (q4_code(x.w, id) << 12);
