@@ -127,6 +127,28 @@ def test_many_short_sequences():
     check_full(w, "700 short")
 
 
+@pytest.mark.parametrize("B", [2049, 3000])
+def test_batches_past_the_charged_split(B):
+    # above 2048 sequences the work split charges no segment starts and the sequence
+    # counts are not kept; both the decode kernel and the combine kernel (which recomputes
+    # the split) take that path. Every 7th sequence is long enough to be split over CTAs,
+    # some are empty.
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 60, B)
+    lens[::7] = rng.integers(800, 2500, len(lens[::7]))
+    w = inputs.make_custom(B, 8, 2, 128, lens, 32, seed=B)
+    got = run_decode(w).cpu().numpy()
+    assert np.all(got[lens == 0] == 0)
+    assert_close(got, oracle.decode_all(oracle_cache(w), w.q), f"B={B}")
+
+
+def test_batch_limit_is_rejected_on_host():
+    w = inputs.make_custom(16385, 8, 2, 128, np.ones(16385, np.int64), 16, seed=2)
+    with pytest.raises(q8.Q8KVError) as e:
+        run_decode(w)
+    assert e.value.status == 2
+
+
 # ------------------------------------------------------------------ API behaviour
 
 def test_repeat_calls_identical_and_workspace_variant():
