@@ -11,6 +11,7 @@
 
 #include "q8kv.h"
 #include "q8kv_combine.cuh" // (includes the decode kernel)
+#include "q8kv_mq_tc.cuh"
 #include "q8kv_qquant.cuh"
 
 namespace {
@@ -46,6 +47,7 @@ struct DeviceInfo {
     int smem_optin = 0;
     unsigned *errors = nullptr;      // address of g_device_errors on this device
     bool attr_set[3][2] = {{false, false}, {false, false}, {false, false}};
+    bool tc_attr[2] = {false, false}; // mq_tc_kernel<16>, <32>
     bool combine_attr = false;
     void *ws = nullptr;              // library-managed workspace
     size_t ws_bytes = 0;
@@ -98,6 +100,8 @@ struct Shape {
 struct Plan {
     int G, slices, NT, HPC, nhc, pairs, subtiles, TT, box_tok, log2_box, n_boxes, n_stages;
     int scale_bulk, sc_heads, heads_seg, scratch_stride, grid;
+    int box_heads = 0; // KV heads per TMA box of the K / V tensor maps
+    int tc_rows = 0;   // > 0: the tensor-memory kernel for this many rows per KV head
     SmemLayout lay;
     size_t smem_bytes;
     size_t ws_bytes;
@@ -211,7 +215,75 @@ q8kv_status make_plan(const Shape &s, const DeviceInfo &dev, Plan &pl)
         }
     }
     pl.smem_bytes = (size_t)pl.lay.total + 1024;
+    pl.box_heads = pl.HPC;
     plan_workspace(dev.sms, pl); // sized for the full grid so one size fits all calls
+    return Q8KV_OK;
+}
+
+// Rows per KV head the tensor-memory kernel (q8kv_mq_tc.cuh) takes this shape with: several
+// query tokens per sequence, 9 to 32 rows (padded to 16 or 32), K / V scales that load as
+// a bulk copy (one KV head) or 16-byte boxes (KV heads a multiple of 4). 0: not taken.
+int tc_rows(const Shape &s)
+{
+    if (s.nq < 2 || s.D != kD || s.Hk <= 0 || s.Hq % s.Hk != 0)
+        return 0;
+    const long long rows = (long long)s.nq * (s.Hq / s.Hk);
+    if (rows <= 8 || rows > 32)
+        return 0;
+    if (s.Hk != 1 && s.Hk % 4 != 0)
+        return 0;
+    return rows <= 16 ? 16 : 32;
+}
+
+// The tiling of the tensor-memory kernel: tiles of 128 tokens of one KV head, the same
+// work split and partial-result slots as the single-query kernel.
+q8kv_status make_plan_tc(const Shape &s, const DeviceInfo &dev, int R, Plan &pl)
+{
+    if (s.B <= 0 || s.bs <= 0 || s.mbps <= 0 || s.P <= 0)
+        return Q8KV_ERR_INVALID_ARG;
+    if (!is_pow2(s.bs) || s.bs < 16 || s.bs > 256)
+        return Q8KV_ERR_UNSUPPORTED;
+    if (s.B > 16384 || (long long)s.P * s.bs >= (1LL << 31) ||
+        (long long)s.mbps * s.bs >= (1LL << 31))
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.G = s.nq * (s.Hq / s.Hk);
+    pl.slices = 1;
+    pl.NT = 1;
+    pl.HPC = 1;
+    pl.nhc = s.Hk;
+    pl.pairs = 1;
+    pl.subtiles = 1;
+    pl.TT = kTcTT;
+    pl.heads_seg = pl.G;
+    pl.scratch_stride = 0;
+    pl.scale_bulk = (s.Hk == 1) ? 1 : 0;
+    pl.sc_heads = pl.scale_bulk ? 1 : 4;
+    pl.box_heads = 1;
+    pl.tc_rows = R;
+    const long long tiles_per_seq = ((long long)s.mbps * s.bs + pl.TT - 1) / pl.TT;
+    const long long tiles_max = (long long)s.B * pl.nhc * tiles_per_seq;
+    if (tiles_max >= (1LL << 30))
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.grid = (int)(tiles_max < dev.sms ? tiles_max : dev.sms);
+    if (combine_layout(s.B, pl.grid).total + kCombineStaticSmemMax > (uint32_t)dev.smem_optin)
+        return Q8KV_ERR_UNSUPPORTED;
+    pl.box_tok = pl.TT < s.bs ? pl.TT : s.bs;
+    pl.log2_box = ilog2(pl.box_tok);
+    pl.n_boxes = pl.TT / pl.box_tok;
+    pl.n_stages = 0;
+    for (int n = kMaxStages; n >= 2; --n) {
+        SmemLayout Lb = make_layout(pl.TT, pl.HPC, pl.sc_heads, n, s.B, 0, pl.grid);
+        const TcLayout Lt = tc_layout(Lb.total, R);
+        if ((size_t)Lt.total + 1024 <= (size_t)dev.smem_optin) {
+            pl.n_stages = n;
+            pl.lay = Lb;
+            pl.smem_bytes = (size_t)Lt.total + 1024;
+            break;
+        }
+    }
+    if (pl.n_stages == 0)
+        return Q8KV_ERR_UNSUPPORTED;
+    plan_workspace(dev.sms, pl);
     return Q8KV_OK;
 }
 
@@ -233,7 +305,7 @@ q8kv_status encode_maps_uncached(const Shape &s, const Plan &pl, const int8_t *k
     // [kv head][token][128 channels], 128-byte swizzled.
     cuuint64_t dims[3] = {(cuuint64_t)kD, slots, (cuuint64_t)s.Hk};
     cuuint64_t strides[2] = {(cuuint64_t)s.Hk * kD, (cuuint64_t)kD};
-    cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)pl.box_tok, (cuuint32_t)pl.HPC};
+    cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)pl.box_tok, (cuuint32_t)pl.box_heads};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t *>(k), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -270,12 +342,12 @@ q8kv_status encode_maps_uncached(const Shape &s, const Plan &pl, const int8_t *k
 // cache reuse them (a small round-robin cache, guarded by g_mutex).
 struct MapKey {
     const void *k, *v, *ks, *vs;
-    int Hk, bs, P, HPC, box_tok, scale_bulk, sc_heads;
+    int Hk, bs, P, HPC, box_heads, box_tok, scale_bulk, sc_heads;
     bool operator==(const MapKey &o) const
     {
         return k == o.k && v == o.v && ks == o.ks && vs == o.vs && Hk == o.Hk && bs == o.bs &&
-               P == o.P && HPC == o.HPC && box_tok == o.box_tok && scale_bulk == o.scale_bulk &&
-               sc_heads == o.sc_heads;
+               P == o.P && HPC == o.HPC && box_heads == o.box_heads && box_tok == o.box_tok &&
+               scale_bulk == o.scale_bulk && sc_heads == o.sc_heads;
     }
 };
 
@@ -293,8 +365,8 @@ q8kv_status encode_maps(const Shape &s, const Plan &pl, const int8_t *k, const i
                         const float *ks, const float *vs, CUtensorMap *mk, CUtensorMap *mv,
                         CUtensorMap *mks, CUtensorMap *mvs)
 {
-    const MapKey key{k, v, ks, vs, s.Hk, s.bs, s.P, pl.HPC, pl.box_tok, pl.scale_bulk,
-                     pl.sc_heads};
+    const MapKey key{k, v, ks, vs, s.Hk, s.bs, s.P, pl.HPC, pl.box_heads, pl.box_tok,
+                     pl.scale_bulk, pl.sc_heads};
     std::lock_guard<std::mutex> lock(g_mutex);
     for (auto &e : g_maps) {
         if (e.used && e.key == key) {
@@ -348,6 +420,27 @@ q8kv_status check_call(const Call &c)
     return Q8KV_OK;
 }
 
+// The log-sum-exp combine after a decode kernel launched with cfg (same stream, programmatic
+// dependent launch).
+q8kv_status launch_combine(DeviceInfo &dev, const DecodeParams &p, const Plan &pl,
+                           const cudaLaunchConfig_t &cfg)
+{
+    if (!dev.combine_attr) {
+        // the dynamic part may use what the kernel's static shared memory leaves of the limit
+        cudaFuncAttributes fa;
+        Q8KV_CUDA(cudaFuncGetAttributes(&fa, combine_kernel));
+        Q8KV_CUDA(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev.smem_optin - (int)fa.sharedSizeBytes));
+        dev.combine_attr = true;
+    }
+    cudaLaunchConfig_t cc = cfg;
+    cc.gridDim = dim3((unsigned)dev.sms);
+    cc.blockDim = dim3(kCombineThreads);
+    cc.dynamicSmemBytes = combine_layout(p.B, pl.grid).total;
+    Q8KV_CUDA(cudaLaunchKernelEx(&cc, combine_kernel, p, pl.grid));
+    return Q8KV_OK;
+}
+
 template <int NT, bool kPack, bool kDump>
 q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl,
                           const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mks,
@@ -380,21 +473,38 @@ q8kv_status launch_kernel(DeviceInfo &dev, const DecodeParams &p, const Plan &pl
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     Q8KV_CUDA(cudaLaunchKernelEx(&cfg, fn, p, mk, mv, mks, mvs));
+    return launch_combine(dev, p, pl, cfg);
+}
 
-    if (!dev.combine_attr) {
-        // the dynamic part may use what the kernel's static shared memory leaves of the limit
-        cudaFuncAttributes fa;
-        Q8KV_CUDA(cudaFuncGetAttributes(&fa, combine_kernel));
-        Q8KV_CUDA(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       dev.smem_optin - (int)fa.sharedSizeBytes));
-        dev.combine_attr = true;
+// The tensor-memory kernel for R rows per KV head, then the combine.
+template <int R>
+q8kv_status launch_tc(DeviceInfo &dev, const DecodeParams &p, const Plan &pl,
+                      const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mks,
+                      const CUtensorMap &mvs, cudaStream_t stream)
+{
+    auto fn = mq_tc_kernel<R>;
+    bool &set = dev.tc_attr[R == 16 ? 0 : 1];
+    if (!set) {
+        cudaFuncAttributes attr;
+        Q8KV_CUDA(cudaFuncGetAttributes(&attr, fn));
+        if (attr.numRegs != kTcLaunchRegs)
+            return Q8KV_ERR_UNSUPPORTED;
+        Q8KV_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev.smem_optin));
+        set = true;
     }
-    cudaLaunchConfig_t cc = cfg;
-    cc.gridDim = dim3((unsigned)dev.sms);
-    cc.blockDim = dim3(kCombineThreads);
-    cc.dynamicSmemBytes = combine_layout(p.B, pl.grid).total;
-    Q8KV_CUDA(cudaLaunchKernelEx(&cc, combine_kernel, p, pl.grid));
-    return Q8KV_OK;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.grid);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    Q8KV_CUDA(cudaLaunchKernelEx(&cfg, fn, p, mk, mv, mks, mvs));
+    return launch_combine(dev, p, pl, cfg);
 }
 
 q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaStream_t stream)
@@ -410,7 +520,8 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     if (st != Q8KV_OK)
         return st;
     Plan pl;
-    st = make_plan(c.s, *dev, pl);
+    const int R = (c.dots || c.stall_cta >= 0) ? 0 : tc_rows(c.s);
+    st = R ? make_plan_tc(c.s, *dev, R, pl) : make_plan(c.s, *dev, pl);
     if (st != Q8KV_OK)
         return st;
     if (managed_ws) {
@@ -476,6 +587,10 @@ q8kv_status run(const Call &c, void *ws, size_t ws_bytes, bool managed_ws, cudaS
     p.stall_limit_ns = c.stall_limit_ns;
     p.lay = pl.lay;
 
+    if (pl.tc_rows == 16)
+        return launch_tc<16>(*dev, p, pl, mk, mv, mks, mvs, stream);
+    if (pl.tc_rows == 32)
+        return launch_tc<32>(*dev, p, pl, mk, mv, mks, mvs, stream);
     const bool dump = c.dots != nullptr;
     if (pl.G <= 4) // heads fill at most half of the 8 MMA columns: pack the split halves
         return dump ? launch_kernel<1, true, true>(*dev, p, pl, mk, mv, mks, mvs, stream)

@@ -128,8 +128,11 @@ q8kv_status q8kv_decode_attn(float *out, const float *q, const int8_t *k_blocks,
  * with the single-query arithmetic of q8kv_decode_attn per (b, i, head); a query that sees
  * no token (seq_lens[b] < n_queries - i) gets a zero row. n_queries = 1 is
  * q8kv_decode_attn. Supported shapes: as above with R = n_queries * n_q_heads /
- * n_kv_heads rows per KV head. Other arguments, errors and asynchrony as
- * q8kv_decode_attn.
+ * n_kv_heads rows per KV head. With n_queries > 1, 9 <= R <= 32 and n_kv_heads 1 or a
+ * multiple of 4, the call runs on the fifth-generation tensor cores (tcgen05.mma with
+ * int32 accumulators in tensor memory; rows padded to 16 or 32); other shapes on the warp
+ * MMAs of q8kv_decode_attn. Both give the same results within the documented tolerance.
+ * Other arguments, errors and asynchrony as q8kv_decode_attn.
  */
 q8kv_status q8kv_decode_attn_multi(float *out, const float *q, const int8_t *k_blocks,
                                    const int8_t *v_blocks, const float *kscale,
