@@ -26,11 +26,13 @@
 //    maxima per row come from redux.sync over order-preserving integer keys and one exchange
 //    across the warpgroup's 4 warps. The row state (running max M of the scores, running
 //    max A of score + log2 V scale) is kept by one thread per row.
-//  * PV: the weight w * vs * 2^(M - A + 19) of (token, row) is an exact integer below 2^23
-//    (A: the largest score + log2 vs, moved only when exceeded by 3), split into 3 byte
-//    planes. O^T = V^T . P: M = 128 channels (V^T read straight from the
-//    swizzled tile: MN-major int8), N = 3 R (plane, row) columns, K = 32 tokens, int32
-//    accumulators in TMEM. A warpgroup recombines its rows' planes in fp32 into per-thread
+//  * PV: the weight w * vs * 2^(M - A + 19) of (token, row) is an exact integer P below
+//    2^23 (A: the largest score + log2 vs, moved only when exceeded by 3); the fp32 bits
+//    of P + 2^23 hold it in their low three bytes. Those 32-bit words are the B operand as
+//    they are: O^T = V^T . W with M = 128 channels (V^T read straight from the swizzled
+//    tile: MN-major int8), N = 4 R columns (row, byte), K = 32 tokens, int32 accumulators in
+//    TMEM; byte k of a row's column group is plane k of P, the fourth (the constant exponent
+//    byte) is never read. A warpgroup recombines its rows' planes in fp32 into per-thread
 //    accumulators (thread t owns channel t) when A rises, every 256 tiles (int32 headroom)
 //    and at segment end, and zeroes those columns again.
 //  * Warp 17 issues the QK MMAs, warp 18 the PV MMAs (one thread each, in fixed orders with
@@ -44,6 +46,7 @@ namespace q8kv {
 
 constexpr int kTcTT = 128;           // tokens per tile: the QK MMA's M, the TMEM lanes
 constexpr uint32_t kTcCols = 512;    // TMEM columns allocated: [S buffer 0 | S buffer 1 | O]
+                                     // = [4 R | 4 R | 4 R]
 constexpr int kTcFoldEvery = 256;    // tiles between forced folds: 256*128*255*127 < 2^31
 constexpr float kTwo23F = 8388608.0f;
 // Headroom of the weights' reference A (log2 units): a weight is w vs 2^(M - A + 22 - h), at
@@ -143,8 +146,11 @@ __device__ __forceinline__ void tc_wait_st()
 template <int N>
 __device__ __forceinline__ void tc_ld(uint32_t taddr, uint32_t *v)
 {
-    static_assert(N == 4 || N == 8 || N == 16, "4, 8 or 16 columns");
-    if constexpr (N == 4)
+    static_assert(N == 4 || N == 8 || N == 16 || N == 32, "4, 8, 16 or 32 columns");
+    if constexpr (N == 32) {
+        tc_ld<16>(taddr, v);
+        tc_ld<16>(taddr + 16, v + 16);
+    } else if constexpr (N == 4)
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
                      : "r"(taddr));
@@ -166,8 +172,11 @@ __device__ __forceinline__ void tc_ld(uint32_t taddr, uint32_t *v)
 template <int N>
 __device__ __forceinline__ void tc_fill(uint32_t taddr, uint32_t x)
 {
-    static_assert(N == 4 || N == 8 || N == 16, "4, 8 or 16 columns");
-    if constexpr (N == 4)
+    static_assert(N == 4 || N == 8 || N == 16 || N == 32, "4, 8, 16 or 32 columns");
+    if constexpr (N == 32) {
+        tc_fill<16>(taddr, x);
+        tc_fill<16>(taddr + 16, x);
+    } else if constexpr (N == 4)
         asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%1,%1,%1};" ::"r"(taddr),
                      "r"(x)
                      : "memory");
@@ -200,10 +209,10 @@ __host__ __device__ constexpr uint32_t idesc_qk(int R)
 {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(R >> 3) << 17) | (8u << 24);
 }
-// PV: A = V^T (signed, MN-major), B = weight planes (unsigned, MN-major), N = 3 R.
+// PV: A = V^T (signed, MN-major), B = weight words (unsigned bytes, MN-major), N = 4 R.
 __host__ __device__ constexpr uint32_t idesc_pv(int R)
 {
-    return (2u << 4) | (1u << 7) | (1u << 15) | (1u << 16) | ((uint32_t)((3 * R) >> 3) << 17) |
+    return (2u << 4) | (1u << 7) | (1u << 15) | (1u << 16) | ((uint32_t)((4 * R) >> 3) << 17) |
            (8u << 24);
 }
 
@@ -233,14 +242,14 @@ __device__ __forceinline__ void wg_bar(int w)
 // ------------------------------------------------------------------ shared memory
 
 // Bytes of a query slot's operand (4 blocks of R rows x 32 codes in 8-row core matrices)
-// and of one 32-token K-step of a weight-plane buffer ((3 R / 16) groups of 16 columns).
+// and of one 32-token K-step of a weight buffer (R / 4 groups of 16 byte columns).
 __host__ __device__ constexpr uint32_t tc_q_bytes(int R)
 {
     return 4u * (uint32_t)R * 32u;
 }
 __host__ __device__ constexpr uint32_t tc_p_kstep_bytes(int R)
 {
-    return (3u * (uint32_t)R / 16u) * 512u;
+    return ((uint32_t)R / 4u) * 512u;
 }
 
 struct TcLayout {
@@ -249,7 +258,7 @@ struct TcLayout {
     uint32_t off_flag;   // int[4]: a row of warpgroup w rose this tile (fold)
     uint32_t off_q;      // Q operands [slot 2]
     uint32_t off_qs;     // Q block scales x softmax scale x log2 e [slot][block][row]
-    uint32_t off_p;      // weight planes [buffer 2][K-step 4]
+    uint32_t off_p;      // weight words [buffer 2][K-step 4]
     uint32_t off_xch;    // per-warp row maxima / sums [warpgroup 4][warp 4][row] float2
     uint32_t off_row;    // row factors [warpgroup][row] float4 (M, S factor, weight factor,
                          // fold factor)
@@ -402,8 +411,8 @@ __device__ void tc_issue_qk(const DecodeParams &p, uint8_t *smem, const TcLayout
     tc_commit(&bars[kFinal]);
 }
 
-// Warp 18, lane 0: PV of tile k once every warpgroup has written its weight planes into
-// plane buffer k & 1; its completion frees the stage and the plane buffer.
+// Warp 18, lane 0: PV of tile k once every warpgroup has written its weight words into
+// weight buffer k & 1; its completion frees the stage and the weight buffer.
 template <int R>
 __device__ void tc_issue_pv(const DecodeParams &p, uint8_t *smem, const TcLayout &L,
                             uint32_t tbase, int n)
@@ -418,7 +427,7 @@ __device__ void tc_issue_pv(const DecodeParams &p, uint8_t *smem, const TcLayout
 #pragma unroll 1
     for (int k = 0; k < n; ++k) {
         const int slot = k % p.n_stages, buf = k & 1;
-        // (the stage has landed once the planes are written; the wait on it makes the TMA
+        // (the stage has landed once the weights are written; the wait on it makes the TMA
         // writes visible to this thread's MMAs directly)
         if (!mbar_wait(&bars[kPReady + buf], (uint32_t)(k >> 1) & 1u, limit) ||
             !mbar_wait(&full[slot], (uint32_t)(k / p.n_stages) & 1u, limit)) {
@@ -462,7 +471,7 @@ __device__ __forceinline__ float tc_row_sums(float (&v)[N], int lane)
     return v[0];
 }
 
-// This warpgroup's columns of the PV accumulators: plane p of row i at tOw + p R + i.
+// This warpgroup's columns of the PV accumulators: byte plane k of row i at tOw + 4 i + k.
 // Fold them into acc (units of 2^A: the weights carry 2^(22 - h)) when add_o, scale every
 // row by its fold factor when rescale, and zero the columns (the next PV starts from zero).
 template <int R>
@@ -471,15 +480,13 @@ __device__ __forceinline__ void tc_fold(float (&acc)[R / kTcWGs], uint32_t tOw, 
 {
     constexpr int RH = R / kTcWGs;
     if (add_o) {
-        uint32_t o0[RH], o1[RH], o2[RH];
-        tc_ld<RH>(tOw, o0);
-        tc_ld<RH>(tOw + R, o1);
-        tc_ld<RH>(tOw + 2 * R, o2);
+        uint32_t o[4 * RH];
+        tc_ld<4 * RH>(tOw, o);
         tc_wait_ld();
 #pragma unroll
         for (int i = 0; i < RH; ++i) {
-            const float c = fmaf((float)(int)o2[i], 65536.f,
-                                 fmaf((float)(int)o1[i], 256.f, (float)(int)o0[i]));
+            const float c = fmaf((float)(int)o[4 * i + 2], 65536.f,
+                                 fmaf((float)(int)o[4 * i + 1], 256.f, (float)(int)o[4 * i]));
             acc[i] = fmaf(c, 1.f / 524288.f, acc[i]); // 2^-(22 - kTcAHead)
         }
     }
@@ -488,9 +495,7 @@ __device__ __forceinline__ void tc_fold(float (&acc)[R / kTcWGs], uint32_t tOw, 
         for (int i = 0; i < RH; ++i)
             acc[i] *= lds_f32(rowi + 16u * i + 12u);
     }
-#pragma unroll
-    for (int pl = 0; pl < 3; ++pl)
-        tc_fill<RH>(tOw + (uint32_t)(pl * R), 0u);
+    tc_fill<4 * RH>(tOw, 0u);
 }
 
 template <int R>
@@ -506,10 +511,10 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
     const bool owner = q4 == 0 && lane < RH;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t tlane = tbase + ((uint32_t)(q4 * 32) << 16);
-    const uint32_t tOw = tlane + (uint32_t)(8 * R + r0);
+    const uint32_t tOw = tlane + (uint32_t)(8 * R + 4 * r0);
     const uint32_t pofs = L.off_p + (uint32_t)q4 * tc_p_kstep_bytes(R) +
                           (uint32_t)(lane >> 3) * 128u + (uint32_t)(lane & 7) * 16u +
-                          (uint32_t)(r0 & 15);
+                          (uint32_t)(r0 / 4) * 512u;
     static_assert(RH == 4 || RH == 8 || RH == 16, "rows per warpgroup: 4, 8 or 16");
     const uint32_t xch = sbase + L.off_xch + (uint32_t)w * 4u * RH * 8u;
     const uint32_t rowi = sbase + L.off_row + (uint32_t)w * RH * 16u;
@@ -525,9 +530,7 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
 #pragma unroll
     for (int bj = 0; bj < 8; ++bj)
         tc_fill<RH>(tlane + (uint32_t)(bj * R + r0), (uint32_t)kDotBias);
-#pragma unroll
-    for (int pl = 0; pl < 3; ++pl)
-        tc_fill<RH>(tOw + (uint32_t)(pl * R), 0u);
+    tc_fill<4 * RH>(tOw, 0u);
     tc_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -691,7 +694,7 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                 Spart[i] = fmaf(Spart[i], ri.y, wv);
                 bits[i] = __float_as_uint(fmaf(wv * vsv, ri.z, kTwo23F));
             }
-            // plane buffer k & 1 was read by tile k - 2's PV; a fold also needs tile k - 1's
+            // weight buffer k & 1 was read by tile k - 2's PV; a fold also needs tile k - 1's
             if (!dead && kst >= 2 &&
                 !mbar_wait(&bars[kPvDone + buf], ((kst >> 1) - 1u) & 1u, limit)) {
                 dead = true;
@@ -709,26 +712,13 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                     since_fold = 0;
                 }
             }
-            // planes: byte k of P for this warpgroup's rows (MN-major, 8-token core rows)
+            // the weight words of this warpgroup's rows: 4 rows (16 byte columns) per 16-byte
+            // store (MN-major, 8-token core rows)
             const uint32_t pb = sbase + pofs + (uint32_t)buf * 4u * tc_p_kstep_bytes(R);
 #pragma unroll
-            for (int pl = 0; pl < 3; ++pl) {
-                const uint32_t sel = (uint32_t)pl | ((uint32_t)(4 + pl) << 4);
-                uint32_t wd[RH / 4];
-#pragma unroll
-                for (int m = 0; m < RH / 4; ++m) {
-                    const uint32_t a = prmt(bits[4 * m], bits[4 * m + 1], sel);
-                    const uint32_t b = prmt(bits[4 * m + 2], bits[4 * m + 3], sel);
-                    wd[m] = prmt(a, b, 0x5410u);
-                }
-                const uint32_t addr = pb + (uint32_t)((pl * R + r0) / 16) * 512u;
-                if constexpr (RH == 16)
-                    sts128(addr, wd[0], wd[1], wd[2], wd[3]);
-                else if constexpr (RH == 8)
-                    sts64(addr, wd[0], wd[1]);
-                else
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(wd[0]) : "memory");
-            }
+            for (int c = 0; c < RH / 4; ++c)
+                sts128(pb + (uint32_t)c * 512u, bits[4 * c], bits[4 * c + 1], bits[4 * c + 2],
+                       bits[4 * c + 3]);
             ofresh = false;
             ++since_fold;
             fence_proxy_async_smem();
