@@ -22,10 +22,12 @@
 //    the bit pattern of 1.5 * 2^23 (tcgen05.st), so an int32 dot read as fp32 minus
 //    1.5 * 2^23 is the exact dot.
 //  * Softmax: thread t of a consumer warpgroup owns token t (TMEM lane t); warpgroup w of
-//    the four owns rows [w R/4, (w + 1) R/4). Each thread forms its token's scores for its rows; the tile
-//    maxima per row come from redux.sync over order-preserving integer keys and one exchange
-//    across the warpgroup's 4 warps. The row state (running max M of the scores, running
-//    max A of score + log2 V scale) is kept by one thread per row.
+//    the four owns rows [w R/4, (w + 1) R/4). Each thread forms its token's scores for its
+//    rows; the tile maxima per row come from fp32 redux.sync and one exchange across the
+//    warpgroup's 4 warps (one named barrier per tile). The row state (running max M of the
+//    scores, running max A of score + log2 V scale) is kept by lane r of every warp of the
+//    warpgroup, each computing it from the same exchanged maxima, and broadcast with
+//    shuffles.
 //  * PV: the weight w * vs * 2^(M - A + 19) of (token, row) is an exact integer P below
 //    2^23 (A: the largest score + log2 vs, moved only when exceeded by 3); the fp32 bits
 //    of P + 2^23 hold it in their low three bytes. Those 32-bit words are the B operand as
@@ -255,13 +257,14 @@ __host__ __device__ constexpr uint32_t tc_p_kstep_bytes(int R)
 struct TcLayout {
     uint32_t off_tmem;   // TMEM base address written by tcgen05.alloc
     uint32_t off_bar;    // mbarriers, see TcBar
-    uint32_t off_flag;   // int[4]: a row of warpgroup w rose this tile (fold)
+    uint32_t off_flag;   // (unused, 16 bytes)
     uint32_t off_q;      // Q operands [slot 2]
     uint32_t off_qs;     // Q block scales x softmax scale x log2 e [slot][block][row]
     uint32_t off_p;      // weight words [buffer 2][K-step 4]
-    uint32_t off_xch;    // per-warp row maxima / sums [warpgroup 4][warp 4][row] float2
-    uint32_t off_row;    // row factors [warpgroup][row] float4 (M, S factor, weight factor,
-                         // fold factor)
+    uint32_t off_xch;    // per-warp row maxima [tile parity 2][warpgroup 4][warp 4][row]
+                         // float2 (and the row sums at segment end)
+    uint32_t off_row;    // output factor per row at segment end [warpgroup][row] (float4
+                         // stride)
     uint32_t total;
 };
 
@@ -285,7 +288,7 @@ __host__ __device__ inline TcLayout tc_layout(uint32_t base_total, int R)
     L.off_p = align_up(o, 128);
     o = L.off_p + 2u * 4u * tc_p_kstep_bytes(R);
     L.off_xch = o;
-    o += 4u * (uint32_t)R * 8u; // 4 warpgroups x 4 warps x R/4 rows
+    o += 2u * 4u * (uint32_t)R * 8u; // 2 x 4 warpgroups x 4 warps x R/4 rows
     L.off_row = align_up(o, 16);
     o = L.off_row + (uint32_t)R * 16u;
     L.total = o;
@@ -473,9 +476,10 @@ __device__ __forceinline__ float tc_row_sums(float (&v)[N], int lane)
 
 // This warpgroup's columns of the PV accumulators: byte plane k of row i at tOw + 4 i + k.
 // Fold them into acc (units of 2^A: the weights carry 2^(22 - h)) when add_o, scale every
-// row by its fold factor when rescale, and zero the columns (the next PV starts from zero).
+// row by its fold factor (lane i holds row i's) when rescale, and zero the columns (the next
+// PV starts from zero).
 template <int R>
-__device__ __forceinline__ void tc_fold(float (&acc)[R / kTcWGs], uint32_t tOw, uint32_t rowi,
+__device__ __forceinline__ void tc_fold(float (&acc)[R / kTcWGs], uint32_t tOw, float fa_lane,
                                         bool add_o, bool rescale)
 {
     constexpr int RH = R / kTcWGs;
@@ -493,7 +497,7 @@ __device__ __forceinline__ void tc_fold(float (&acc)[R / kTcWGs], uint32_t tOw, 
     if (rescale) {
 #pragma unroll
         for (int i = 0; i < RH; ++i)
-            acc[i] *= lds_f32(rowi + 16u * i + 12u);
+            acc[i] *= __shfl_sync(kFullMask, fa_lane, i);
     }
     tc_fill<4 * RH>(tOw, 0u);
 }
@@ -505,10 +509,9 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
     constexpr int RH = R / kTcWGs;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.lay.off_full);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.off_bar);
-    volatile int *flags = reinterpret_cast<volatile int *>(smem + L.off_flag);
     const int w = warp >> 2, q4 = warp & 3, tt = q4 * 32 + lane;
     const int r0 = w * RH; // this warpgroup's first row
-    const bool owner = q4 == 0 && lane < RH;
+    const bool owner = q4 == 0 && lane < RH; // writes the row's results at segment end
     const uint32_t sbase = smem_addr(smem);
     const uint32_t tlane = tbase + ((uint32_t)(q4 * 32) << 16);
     const uint32_t tOw = tlane + (uint32_t)(8 * R + 4 * r0);
@@ -520,8 +523,8 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
     const uint32_t rowi = sbase + L.off_row + (uint32_t)w * RH * 16u;
     // the tables read in the per-tile loop, as plain shared-memory pointers (ordinary loads
     // the compiler can batch; the named barriers order them against the writers)
-    const float4 *rowt = reinterpret_cast<const float4 *>(smem + L.off_row + w * RH * 16);
     const float2 *xcht = reinterpret_cast<const float2 *>(smem + L.off_xch + w * 4 * RH * 8);
+    constexpr int kXchParity = kTcWGs * 4 * RH; // float2 entries per tile parity
     const unsigned long long limit = wait_limit(p);
     bool dead = false;
 
@@ -540,7 +543,7 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
     }
 
     float Spart[RH], acc[RH];
-    float Mrow = -INFINITY, Arow = -INFINITY; // the owner's row state
+    float Mrow = -INFINITY, Arow = -INFINITY; // row `lane`'s state (lanes < RH, every warp)
     bool seed_pending = false; // this tile's score columns re-seeded, sfree not yet signalled
     int seed_buf = 0;
     int stage = 0;
@@ -642,20 +645,23 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                 km[i] = warp_max(s[i]);
                 ka[i] = warp_max(s[i] + lvs);
             }
+            const int xp = buf * kXchParity; // tile parity: a warp is at most one tile ahead
             if (lane == 0) {
-                float2 *xw = reinterpret_cast<float2 *>(smem + L.off_xch + (w * 4 + q4) * RH * 8);
+                float2 *xw = reinterpret_cast<float2 *>(smem + L.off_xch) + xp + (w * 4 + q4) * RH;
 #pragma unroll
                 for (int i = 0; i < RH; ++i)
                     xw[i] = make_float2(km[i], ka[i]);
             }
             wg_bar(w);
-            if (q4 == 0) {
-                bool rose = false;
-                if (owner) {
+            // every warp updates the row state from the same maxima (lane i: row i)
+            float Ms = 0.f, cM = 1.f, g = 0.f, fa = 1.f;
+            bool rose = false;
+            {
+                if (lane < RH) {
                     float mst = -INFINITY, ast = -INFINITY;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float2 v = xcht[q * RH + lane];
+                        const float2 v = xcht[xp + q * RH + lane];
                         mst = fmaxf(mst, v.x);
                         ast = fmaxf(ast, v.y);
                     }
@@ -668,31 +674,25 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                     // M - 104 (the weights of that row then keep fewer significant bits)
                     if (An != -INFINITY && Mn - An > 104.f)
                         An = Mn - 104.f;
-                    const float cM = Mrow == -INFINITY ? 1.f : fast_exp2(Mrow - Mn);
-                    const float fa = Arow == -INFINITY ? 1.f : fast_exp2(Arow - An);
-                    const float g = An == -INFINITY ? 0.f : fast_exp2(Mn - An + (22.f - kTcAHead));
+                    cM = Mrow == -INFINITY ? 1.f : fast_exp2(Mrow - Mn);
+                    fa = Arow == -INFINITY ? 1.f : fast_exp2(Arow - An);
+                    g = An == -INFINITY ? 0.f : fast_exp2(Mn - An + (22.f - kTcAHead));
+                    Ms = Mn == -INFINITY ? 0.f : Mn;
                     rose = An != Arow && Arow != -INFINITY;
-                    sts128(rowi + 16u * lane, __float_as_uint(Mn == -INFINITY ? 0.f : Mn),
-                           __float_as_uint(cM), __float_as_uint(g), __float_as_uint(fa));
                     Mrow = Mn;
                     Arow = An;
                 }
-                const unsigned any = __ballot_sync(kFullMask, rose);
-                if (lane == 0)
-                    flags[w] = any != 0u;
             }
-            wg_bar(w);
-            const bool fold = flags[w] != 0 || since_fold >= kTcFoldEvery;
+            const bool fold = __any_sync(kFullMask, rose) || since_fold >= kTcFoldEvery;
 
             // weights: w = 2^(s - M) into the row sums, P = w vs 2^(M - A + 19) < 2^23 as an
             // integer in the low mantissa bits of P + 2^23
             uint32_t bits[RH];
 #pragma unroll
             for (int i = 0; i < RH; ++i) {
-                const float4 ri = rowt[i];
-                const float wv = fast_exp2(s[i] - ri.x);
-                Spart[i] = fmaf(Spart[i], ri.y, wv);
-                bits[i] = __float_as_uint(fmaf(wv * vsv, ri.z, kTwo23F));
+                const float wv = fast_exp2(s[i] - __shfl_sync(kFullMask, Ms, i));
+                Spart[i] = fmaf(Spart[i], __shfl_sync(kFullMask, cM, i), wv);
+                bits[i] = __float_as_uint(fmaf(wv * vsv, __shfl_sync(kFullMask, g, i), kTwo23F));
             }
             // weight buffer k & 1 was read by tile k - 2's PV; a fold also needs tile k - 1's
             if (!dead && kst >= 2 &&
@@ -707,7 +707,7 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                     atomicOr(p.errors, kErrTimeout);
                 } else {
                     tc_fence_after();
-                    tc_fold<R>(acc, tOw, rowi, !ofresh, true);
+                    tc_fold<R>(acc, tOw, fa, !ofresh, true);
                     ofresh = true;
                     since_fold = 0;
                 }
@@ -748,7 +748,7 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                 atomicOr(p.errors, kErrTimeout);
             } else if (!ofresh) {
                 tc_fence_after();
-                tc_fold<R>(acc, tOw, rowi, true, false);
+                tc_fold<R>(acc, tOw, 1.f, true, false);
                 tc_wait_st();
                 tc_fence_before();
             }
@@ -790,7 +790,7 @@ __device__ void tc_consume(const DecodeParams &p, uint8_t *smem, const TcLayout 
                 }
             }
         }
-        wg_bar(w); // the row table is rewritten by the next tile
+        wg_bar(w); // the sums and the row table are rewritten at the next segment end
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&bars[kQFree + qslot]);
