@@ -73,6 +73,10 @@ def parse():
                     help="skip the QUEST block-metadata information report")
     ap.add_argument("--no-q4", action="store_true",
                     help="skip the q4_0-cache decode information report")
+    ap.add_argument("--multi-query-only", type=int, default=0, metavar="NQ",
+                    help="instead of the headline: only the multi-query report on the 16 x "
+                         "4096-token GQA workload with NQ query tokens per sequence (one "
+                         "JSON line; e.g. for an ncu capture of that call's kernels)")
     ap.add_argument("--accuracy-study", action="store_true",
                     help="instead of timing: the q8-vs-fp32 output error study over the "
                          "workloads and K/V distributions (one JSON line)")
@@ -735,6 +739,8 @@ def main():
         return run_reference(args)
     if args.accuracy_study:
         return run_accuracy_study(args)
+    if args.multi_query_only:
+        return run_multi_query_only(args)
     world, rank, local = dist_env()
     import torch
 
@@ -906,6 +912,26 @@ def recorded_traffic(name: str, kernel: str = "decode"):
             if len(parts) == 3 and not ln.startswith("#") and parts[0] == name and parts[1] == h:
                 return int(parts[2])
     return None
+
+
+def run_multi_query_only(args):
+    """--multi-query-only NQ: the multi-query report alone (one GPU, one JSON line)."""
+    import torch
+
+    from decode_attention_int8_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = inputs.make(1)
+    _, dw = bench_leg(w, dev, stream, min_calls=3, target_s=0.0, parity_n=8, seed=101)
+    res = bench_multi_query(w, dw.pools, dw.bt, dw.lens, dev, stream,
+                            steps=max(args.steps, 1), warmup=max(args.warmup, 1),
+                            nqs=(args.multi_query_only,))
+    print(json.dumps({"metric": METRIC, "unit": UNIT, "multi_query": res}), flush=True)
+    return 0
 
 
 def bench_multi_query(w, pools, bt, lens, dev, stream, steps, warmup=20, nqs=(2, 4, 8)):
