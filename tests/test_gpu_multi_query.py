@@ -101,3 +101,51 @@ def test_unsupported_row_counts(nq, Hq, Hk):
     with pytest.raises(q8.Q8KVError) as e:
         run_multi(w, q)
     assert e.value.status == 2
+
+
+# ------------------------------------------------------------------ tensor-memory kernel
+# (9-32 query rows per KV head with n_queries > 1 run on q8kv_mq_tc.cuh)
+
+@pytest.mark.parametrize("nq,Hq,Hk,bs", [
+    (16, 1, 1, 64),    # 16 rows, one KV head: scales by bulk copy
+    (12, 2, 1, 128),   # 24 rows padded to 32, a 128-token block per tile
+    (10, 4, 4, 256),   # 10 rows padded to 16, a tile covers half a block
+    (9, 16, 4, 16),    # 36 rows: above 32, the warp-MMA kernel
+])
+def test_tensor_memory_shapes(nq, Hq, Hk, bs):
+    lens = [1, nq - 1, nq, 15, 127, 128, 129, 1000, 5000]
+    w = inputs.make_custom(len(lens), Hq, Hk, 128, lens, bs, seed=nq + Hq + bs)
+    q = inputs.multi_queries(len(lens), nq, Hq, 128, seed=bs)
+    assert_close(run_multi(w, q), oracle.decode_multi(oracle_cache(w), q, nq),
+                 f"nq={nq} Hq={Hq} Hk={Hk} bs={bs}")
+
+
+def test_many_segments_per_cta():
+    # 400 short sequences x 8 KV heads: each CTA switches segments many times, so the query
+    # slots alternate and the later segments' rows are quantised by the helper warp
+    rng = np.random.default_rng(21)
+    lens = rng.integers(1, 300, 400)
+    nq, Hq, Hk = 4, 32, 8
+    w = inputs.make_custom(len(lens), Hq, Hk, 128, lens, 16, seed=21)
+    q = inputs.multi_queries(len(lens), nq, Hq, 128, seed=21)
+    assert_close(run_multi(w, q), oracle.decode_multi(oracle_cache(w), q, nq), "400 x nq=4")
+
+
+@pytest.mark.parametrize("nq,Hq,Hk", [(8, 32, 8), (4, 32, 8)])
+def test_tiny_and_huge_v_scales(nq, Hq, Hk):
+    # V scales over 60 decades: each row's weights and its reference move with them; the
+    # tolerance is relative to each output row's own magnitude
+    lens = [500, 64, 3000]
+    w = inputs.make_custom(len(lens), Hq, Hk, 128, lens, 32, seed=9 + nq)
+    rng = np.random.default_rng(nq)
+    w.vs *= (10.0 ** rng.uniform(-30, 30, w.vs.shape)).astype(np.float32)
+    w.ks *= (10.0 ** rng.uniform(-2, 1, w.ks.shape)).astype(np.float32)
+    q = inputs.multi_queries(len(lens), nq, Hq, 128, seed=nq)
+    got = run_multi(w, q)
+    ref = oracle.decode_multi(oracle_cache(w), q, nq)
+    for b in range(len(lens)):
+        for i in range(nq):
+            for h in range(Hq):
+                r = ref[b, i, h]
+                assert np.linalg.norm(got[b, i, h] - r) <= 1e-5 * np.linalg.norm(r) + 1e-30, \
+                    (b, i, h)
