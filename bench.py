@@ -473,6 +473,34 @@ def bench_leg(w, dev, stream, min_calls=50, target_s=0.25, parity_n=64, seed=0):
     return leg, dw
 
 
+def read_floor(nbytes: int, dev, stream, calls: int = 200) -> dict:
+    """Context for a leg: a library kernel (torch's fp32 sum) reading the same number of
+    bytes, timed like the leg (back-to-back calls, rotated over copies larger than 4x L2).
+    What one call of that size costs a plain streaming read, launch and tail included."""
+    import torch
+
+    n = max(1, nbytes // 4)
+    copies = max(1, n_pool_copies(4 * n))
+    bufs = [torch.ones(n, dtype=torch.float32, device=dev) for _ in range(copies)]
+    out = torch.empty((), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(10):
+            torch.sum(bufs[i % copies], dim=0, out=out)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(calls):
+            torch.sum(bufs[i % copies], dim=0, out=out)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) / calls * 1e3
+    peak, _ = measured_peak()
+    del bufs
+    return {"kernel": "torch.sum over fp32 (library)", "bytes": 4 * n,
+            "us_per_call": round(us, 3), "frac_of_measured_hbm": round(4 * n / (us * 1e-6) / 1e9 / peak, 4)}
+
+
 def cpu_sample_rate(w, seconds: float, seed: int = 0):
     """The oracle as it stands, single-threaded, on random (sequence, head) rows of the
     workload for about `seconds`; bytes counted pro rata to the rows done. Returns
@@ -839,6 +867,9 @@ def main():
         for i in others + ["group8"]:
             wi = group8_workload() if i == "group8" else inputs.make(i)
             leg, dwi = bench_leg(wi, dev, stream, seed=100 + (9 if i == "group8" else i))
+            if wi.cfg.name in ("gqa_batch", "long_context"):
+                # how close one call of this size can get: a plain read of the same bytes
+                leg["read_floor"] = read_floor(wi.algorithmic_bytes(), dev, stream)
             if wi.cfg.name == "gqa_batch":
                 if not args.no_multi_query:
                     # the same workload with n_queries new tokens per sequence (speculative
