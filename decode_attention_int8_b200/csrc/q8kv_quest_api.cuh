@@ -36,7 +36,8 @@ q8kv_status q8kv_quest_metadata(float *maxblocks, float *minblocks, const int8_t
         return Q8KV_ERR_UNSUPPORTED;
     if ((long long)max_blocks_per_seq * kv_block_size >= (1LL << 31) ||
         (long long)num_kv_blocks * kv_block_size >= (1LL << 31) ||
-        (long long)num_meta_blocks * kv_block_size >= (1LL << 31))
+        (long long)num_meta_blocks * kv_block_size >= (1LL << 31) ||
+        (long long)max_meta_blocks_per_seq * kv_block_size >= (1LL << 31))
         return Q8KV_ERR_UNSUPPORTED;
     DeviceInfo *dev = nullptr;
     q8kv_status st;
@@ -75,7 +76,15 @@ q8kv_status q8kv_quest_metadata(float *maxblocks, float *minblocks, const int8_t
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel, p));
+    switch (n_kv_heads) { // head counts whose batch offsets compile to immediates
+    case 1: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<1>, p)); break;
+    case 2: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<2>, p)); break;
+    case 4: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<4>, p)); break;
+    case 8: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<8>, p)); break;
+    case 16: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<16>, p)); break;
+    case 32: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<32>, p)); break;
+    default: Q8KV_CUDA(cudaLaunchKernelEx(&cfg, quest_metadata_kernel<0>, p)); break;
+    }
     return Q8KV_OK;
 }
 

@@ -323,7 +323,9 @@ q8kv_status q8kv_cache_write_q4(uint8_t *k4_blocks, uint8_t *v4_blocks, uint16_t
  * (Q8KV_DEVERR_SEQ_LEN); a block-table entry outside the pool skips its row
  * (Q8KV_DEVERR_BLOCK_TABLE); a metadata-table entry outside [0, num_meta_blocks), or a
  * request needing more than max_meta_blocks_per_seq metadata blocks, sets
- * Q8KV_DEVERR_META (the rows it cannot place are skipped). One kernel launch, asynchronous
+ * Q8KV_DEVERR_META (the rows it cannot place are skipped). Host-side: Q8KV_ERR_UNSUPPORTED
+ * for head_dim != 128, or when max_blocks_per_seq, num_kv_blocks, num_meta_blocks or
+ * max_meta_blocks_per_seq times kv_block_size reaches 2^31. One kernel launch, asynchronous
  * on `stream`, programmatic dependent launch as the other kernels.
  */
 q8kv_status q8kv_quest_metadata(float *maxblocks, float *minblocks, const int8_t *k_blocks,

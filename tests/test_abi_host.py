@@ -152,6 +152,10 @@ def test_quest_metadata_bad_arguments_rejected():
     odd = list(sizes)
     odd[2] = 64
     assert L.q8kv_quest_metadata(*ptrs, *odd, None) == UNSUPPORTED
+    for i in (4, 5, 6, 7):  # a table or pool of 2^31 tokens or more (bs 16 x 2^27 entries)
+        big = list(sizes)
+        big[i] = 1 << 27
+        assert L.q8kv_quest_metadata(*ptrs, *big, None) == UNSUPPORTED
 
 
 def test_q4_decode_bad_arguments_rejected():

@@ -82,3 +82,36 @@ def test_metadata_table_too_short_is_flagged():
     # the block that fits is still written
     rx, rn = oracle.quest_metadata(oracle_cache(w), np.array([[0, 1]], np.int32), 2)
     assert np.array_equal(mx[0], rx[0]) and np.array_equal(mn[0], rn[0])
+
+
+@pytest.mark.parametrize("Hk", [8, 3])
+def test_scales_at_the_edges_of_fp32(Hk):
+    """Subnormal (down to the smallest), zero, tiny, huge and overflowing scales, with codes
+    at -128, -127, 0 and 127: each product is one correctly rounded fp32 multiply with no
+    flush to zero, and max and min equal the oracle's bit for bit (8 heads: the head count
+    compiled in; 3 heads: read at run time). Zero scales carry non-negative codes only, so
+    no product is -0: the oracle keeps the first of two equal zeros, and the sign of a zero
+    extreme is not what this checks."""
+    bs = 16
+    lens = [300, 129, 17]
+    w = inputs.make_custom(3, Hk, Hk, 128, lens, bs, seed=77, extra_blocks=3)
+    rng = np.random.default_rng(77)
+    special = np.array([1.4e-45, 1e-42, 1.1754942e-38, 2.0 ** -126, 0.0, 1e-30, 1.0, 3e36,
+                        3.4e38], np.float32)
+    ks, k = w.ks, w.k
+    pick = rng.integers(0, len(special), ks.shape)
+    on = rng.random(ks.shape) < 0.5
+    ks[on] = special[pick[on]]
+    edge = np.array([-128, -127, 0, 127], np.int8)
+    kon = rng.random(k.shape) < 0.1
+    k[kon] = edge[rng.integers(0, 4, k.shape)[kon]]
+    zero = ks == 0
+    k[zero] = np.abs(k[zero].astype(np.int16)).clip(0, 127).astype(np.int8)
+    meta, n_meta = inputs.quest_meta_table(lens, bs, seed=77)
+    mx, mn, err = run(w, meta, n_meta)
+    rx, rn = oracle.quest_metadata(oracle_cache(w), meta, n_meta)
+    assert err == 0
+    assert np.isinf(rx).any() and (np.abs(rx[rx != 0]) < 1.1754944e-38).any()  # both edges hit
+    for got, ref, name in ((mx, rx, "max"), (mn, rn, "min")):
+        bad = np.argwhere(got.view(np.uint32) != ref.view(np.uint32))
+        assert bad.size == 0, f"{name}: {len(bad)} mismatches, first {bad[0].tolist()}"
