@@ -110,3 +110,29 @@ def test_bad_block_table_entries_are_flagged_and_skipped():
     got = run_q4(w)
     assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
     assert_close(got[1], oracle.decode_q4_all(kept, w.q)[1], "q4 block skipped (negative)")
+
+
+@pytest.mark.parametrize("G", [1, 4, 8, 16])
+def test_many_ragged_sequences_with_empty_ones(G):
+    # 40 ragged sequences (some empty) x 4 KV heads: about 1800 chunks of 256 tokens, more
+    # than one wave of CTAs, with the chunks past each sequence's end left out of the merge,
+    # and a bad block-table entry in the middle of the longest sequence
+    rng = np.random.default_rng(40 + G)
+    lens = rng.integers(0, 2700, 40)
+    lens[[3, 17, 18, 30]] = 0
+    lens[7] = 2700
+    w = inputs.make_q4_custom(40, 4 * G, 4, 128, lens.tolist(), 32, seed=G)
+    ref = oracle.decode_q4_all(oracle_q4(w), w.q)
+    q8.q8kv_device_errors(clear=True)
+    got = run_q4(w)
+    assert q8.q8kv_device_errors(clear=True) == 0
+    assert np.all(got[lens == 0] == 0.0)
+    assert_close(got, ref, f"G={G} many chunks")
+    w.block_table[7, 40] = -1  # tokens 1280-1311 of sequence 7 (its sixth chunk)
+    got = run_q4(w)
+    assert q8.q8kv_device_errors(clear=True) & q8.DEVERR_BLOCK_TABLE
+    bt, kept_lens = without_block(w.block_table, w.seq_lens, 7, 40, 32)
+    kept = oracle.PagedCacheQ4(w.k4, w.v4, w.kd, w.vd, bt, kept_lens, w.cfg.n_q_heads, w.scale)
+    assert_close(got[7], oracle.decode_q4_all(kept, w.q)[7], f"G={G} bad entry mid-run")
+    others = np.arange(40) != 7
+    assert_close(got[others], ref[others], f"G={G} other rows")
