@@ -173,17 +173,23 @@ __device__ __forceinline__ float half_of(uint2 w, int j)
     return half_bits_to_float((uint16_t)(x >> ((j & 1) * 16)));
 }
 
-// Physical slot of token t of sequence b, or -1 (and an error bit) for a bad table entry.
-__device__ __forceinline__ long long q4_slot(const Q4Params &p, int b, int t, unsigned &err)
+// Block-table entry of token t of sequence b (t below the table's capacity), read before
+// the sequence's length is known so that both reads share one round trip.
+__device__ __forceinline__ int q4_entry(const Q4Params &p, int b, int t)
 {
     const int blk = p.log2_bs >= 0 ? t >> p.log2_bs : t / p.bs;
-    const int off = t - blk * p.bs;
-    const int ph = __ldg(p.block_table + (long long)b * p.mbps + blk);
+    return __ldg(p.block_table + (long long)b * p.mbps + blk);
+}
+
+// Physical slot of token t given its table entry, or -1 (and an error bit) for a bad entry.
+__device__ __forceinline__ long long q4_slot(const Q4Params &p, int t, int ph, unsigned &err)
+{
     if (ph < 0 || ph >= p.num_blocks) {
         err |= kErrBlockTable;
         return -1;
     }
-    return (long long)ph * p.bs + off;
+    const int blk = p.log2_bs >= 0 ? t >> p.log2_bs : t / p.bs;
+    return (long long)ph * p.bs + (t - blk * p.bs);
 }
 
 // Block of QK row r_base + g (r_base a multiple of 8, g < 8); compile-time for GT >= 8.
@@ -217,25 +223,28 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
 
     grid_dep_wait(); // q, the cache and the tables may come from the previous kernel
     grid_dep_launch();
-    int L = __ldg(p.seq_lens + b);
     const int cap = p.mbps * p.bs;
+    const int t0 = blockIdx.x * kQ4Chunk;
+    const int tl = warp * 32 + lane; // this thread's token of the chunk
+    // the length and this token's table entry in one round trip (the entry is used only if
+    // the token turns out to be below the length)
+    const int ph = t0 + tl < cap ? q4_entry(p, b, t0 + tl) : -1;
+    int L = __ldg(p.seq_lens + b);
     unsigned err = 0;
     if (L < 0 || L > cap) {
         if (blockIdx.x == 0 && tid == 0)
             atomicOr(p.errors, kErrSeqLen);
         L = L < 0 ? 0 : cap;
     }
-    const int t0 = blockIdx.x * kQ4Chunk;
     if (t0 >= L)
         return; // the combine only reads the chunks that hold tokens
     const int nt = min(kQ4Chunk, L - t0);
 
     // ---- loads: lane = token of this warp's slice; tokens without data are zero-filled
     {
-        const int tl = warp * 32 + lane;
         long long slot = -1;
         if (tl < nt)
-            slot = q4_slot(p, b, t0 + tl, err);
+            slot = q4_slot(p, t0 + tl, ph, err);
         const bool ok = slot >= 0;
         const long long row = ok ? slot * p.Hk + kvh : 0;
         const uint32_t n16 = ok ? 16u : 0u, n8 = ok ? 8u : 0u;
@@ -283,7 +292,6 @@ __global__ void __launch_bounds__(kQ4Threads, GT <= 4 ? 4 : (GT <= 8 ? 3 : 2))
     // lane's own copies are visible to it after the wait)
     asm volatile("cp.async.wait_all;" ::: "memory");
     {
-        const int tl = warp * 32 + lane;
         const uint2 kd = sm.u.raw.kd[tl], vd = sm.u.raw.vd[tl];
         *reinterpret_cast<float4 *>(&sm.kdf[tl][0]) =
             make_float4(half_of(kd, 0), half_of(kd, 1), half_of(kd, 2), half_of(kd, 3));
